@@ -1,0 +1,163 @@
+"""fp64 CPU oracle of the Mixtral-style sparse MoE feed-forward layer.
+
+TEST INFRASTRUCTURE: only the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package.  The product path never
+does, and this package never imports the product package.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, double precision, no BLAS);
+this file only compiles it with gcc and marshals numpy arrays.  Which passage
+of the pages each step follows is stated in the C file's header:
+"Mistral/Mixtral architecture" page, section "MoEの数学 — ルーターとゲーティング機構"
+(score, Top-2, gate, expert and output equations).
+
+Parity status of each function (what pins it is in tests/test_oracle_pins.py):
+  scores / route / select  pinned: brute force over all k-subsets, closed
+                           form of the k=2 gate, invariants, hand example
+  expert                   pinned: E=1 dense SwiGLU against torch fp64, hand example
+  moe                      pinned: k=E uniform average, E=1 dense FFN, hand
+                           example, permutation/relabelling invariances
+  counts                   pinned: sums to k*T, brute-force histogram
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+DTYPE_CODE = {"f32": 0, "bf16": 1}
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle.so (gcc -O2, OpenMP; no -ffast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            vp, ci = ctypes.c_void_p, ctypes.c_int
+            lib.oracle_scores.argtypes = [ci, ci, ci, vp, vp, ci, vp, ci]
+            lib.oracle_select.argtypes = [ci, ci, ci, vp, vp, vp, vp, vp]
+            lib.oracle_route.argtypes = [ci, ci, ci, ci, vp, vp, ci, vp, vp, vp, vp, ci]
+            lib.oracle_expert.argtypes = [ci, ci, vp, vp, vp, vp, ci, ci, ci, vp]
+            lib.oracle_moe.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, ci, vp, vp, vp, vp,
+                                       vp, ci]
+            lib.oracle_counts.argtypes = [ci, ci, ci, vp, vp]
+            lib.oracle_max_threads.restype = ci
+            _lib = lib
+    return _lib
+
+
+def _arr(a, dtype):
+    want = np.uint16 if dtype == "bf16" else np.float32
+    a = np.ascontiguousarray(a)
+    if a.dtype != want:
+        raise TypeError(f"expected {want} storage for dtype {dtype}, got {a.dtype}")
+    return a
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (code {rc})")
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def scores(x, Wg, dtype: str, nthreads: int = 0) -> np.ndarray:
+    x, Wg = _arr(x, dtype), _arr(Wg, dtype)
+    T, d = x.shape
+    E = Wg.shape[0]
+    out = np.empty((T, E), dtype=np.float64)
+    _check(_load().oracle_scores(T, d, E, x.ctypes.data, Wg.ctypes.data, DTYPE_CODE[dtype],
+                                 out.ctypes.data, nthreads), "scores")
+    return out
+
+
+def select(logits, k: int):
+    """Top-k selection + gate softmax from given fp64 scores [T][E]."""
+    s = np.ascontiguousarray(logits, dtype=np.float64)
+    T, E = s.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    g = np.empty((T, k), dtype=np.float64)
+    margin = np.empty(T, dtype=np.float64)
+    mingap = np.empty(T, dtype=np.float64)
+    _check(_load().oracle_select(T, E, k, s.ctypes.data, idx.ctypes.data, g.ctypes.data, margin.ctypes.data,
+                                 mingap.ctypes.data), "select")
+    return idx, g, margin, mingap
+
+
+def route(x, Wg, k: int, dtype: str, nthreads: int = 0):
+    """Steps 1-3 for every token: (idx [T][k] int32, g [T][k] f64, margin [T], mingap [T])."""
+    x, Wg = _arr(x, dtype), _arr(Wg, dtype)
+    T, d = x.shape
+    E = Wg.shape[0]
+    idx = np.empty((T, k), dtype=np.int32)
+    g = np.empty((T, k), dtype=np.float64)
+    margin = np.empty(T, dtype=np.float64)
+    mingap = np.empty(T, dtype=np.float64)
+    _check(_load().oracle_route(T, d, E, k, x.ctypes.data, Wg.ctypes.data, DTYPE_CODE[dtype], idx.ctypes.data,
+                                g.ctypes.data, margin.ctypes.data, mingap.ctypes.data, nthreads), "route")
+    return idx, g, margin, mingap
+
+
+def expert(x, W1, W3, W2, e: int, t: int, dtype: str) -> np.ndarray:
+    """Step 4 alone: expert e applied to token row t of x, in double."""
+    x, W1, W3, W2 = (_arr(a, dtype) for a in (x, W1, W3, W2))
+    d = x.shape[1]
+    F = W1.shape[1]
+    y = np.empty(d, dtype=np.float64)
+    _check(_load().oracle_expert(d, F, x.ctypes.data, W1.ctypes.data, W3.ctypes.data, W2.ctypes.data,
+                                 DTYPE_CODE[dtype], e, t, y.ctypes.data), "expert")
+    return y
+
+
+def moe(x, Wg, W1, W3, W2, k: int, dtype: str, tokens=None, nthreads: int = 0) -> dict:
+    """The whole layer for all tokens, or for the listed token ids only.
+
+    Returns dict(out [n][d] f64, idx [n][k], g [n][k], margin [n], mingap [n], tokens [n]).
+    """
+    x, Wg, W1, W3, W2 = (_arr(a, dtype) for a in (x, Wg, W1, W3, W2))
+    T, d = x.shape
+    E, F = W1.shape[0], W1.shape[1]
+    if tokens is None:
+        tok = None
+        n = T
+    else:
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = tok.size
+    out = np.empty((n, d), dtype=np.float64)
+    idx = np.empty((n, k), dtype=np.int32)
+    g = np.empty((n, k), dtype=np.float64)
+    margin = np.empty(n, dtype=np.float64)
+    mingap = np.empty(n, dtype=np.float64)
+    _check(_load().oracle_moe(T, d, F, E, k, x.ctypes.data, Wg.ctypes.data, W1.ctypes.data, W3.ctypes.data,
+                              W2.ctypes.data, DTYPE_CODE[dtype], None if tok is None else tok.ctypes.data, n,
+                              out.ctypes.data, idx.ctypes.data, g.ctypes.data, margin.ctypes.data,
+                              mingap.ctypes.data, nthreads), "moe")
+    return dict(out=out, idx=idx, g=g, margin=margin, mingap=mingap,
+                tokens=np.arange(T, dtype=np.int32) if tok is None else tok)
+
+
+def counts(idx, E: int) -> np.ndarray:
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    c = np.empty(E, dtype=np.int64)
+    _check(_load().oracle_counts(T, k, E, idx.ctypes.data, c.ctypes.data), "counts")
+    return c

@@ -1,0 +1,246 @@
+/*
+ * fp64 CPU oracle of the Mixtral-style sparse MoE feed-forward layer.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the bench's CPU
+ * baseline leg may load or call this.  It shares no code with the CUDA path:
+ * no headers, helpers, tables or constants.  It is plain and slow on purpose:
+ * every sum runs in double, index ascending, with no blocking or reordering.
+ *
+ * What it computes, per token x (a row of the input), following the
+ * "Mistral/Mixtral architecture" page (disassemble-channel.com,
+ * "Mistral/Mixtralのアーキテクチャ — Sliding Window AttentionとMoEの融合"),
+ * section "MoEの数学 — ルーターとゲーティング機構":
+ *
+ *   1. router scores   s = Wg x, Wg in R^{E x d}, no bias
+ *                      (subsection "Top-2ゲーティングの定式化", score equation;
+ *                       the "Mixtral of Experts" summary page writes the same
+ *                       thing as H(x)_i = (x . Wg)_i)
+ *   2. top-k selection of the k largest scores, ordered by descending score
+ *                      (same subsection, Top-2 equation with s_i1 >= s_i2);
+ *                      equal scores go to the lower expert index
+ *   3. gate weights    g_j = exp(s_ij) / sum_m exp(s_im) over the k selected
+ *                      only (same subsection, gate equation; the summary page's
+ *                      Softmax(KeepTopK(H, 2)) with the others at -inf is the
+ *                      same thing).  Evaluated as exp(s_ij - s_i1) / sum, which
+ *                      is the same number, to keep exp() in range.
+ *   4. experts         E_i(x) = W2_i (SiLU(W1_i x) * W3_i x), SiLU(a) = a sigmoid(a)
+ *                      (subsection "各エキスパートの構造"; the page's code
+ *                       "MoEレイヤー全体の実装" applies w2 on the left, so
+ *                       W2_i in R^{d x F} multiplies the F-vector)
+ *   5. output          MoE(x) = sum_j g_j E_ij(x), j = 0 .. k-1 in selection
+ *                      order (subsection "Top-2ゲーティングの定式化", output
+ *                      equation; the page's code adds slot 0 of every expert
+ *                      first, then slot 1, which is the same per-token order)
+ *
+ * Only selected experts are evaluated: an unselected expert has gate weight
+ * exactly zero, so it adds nothing.
+ *
+ * Operands are row-major: x[T][d], Wg[E][d], W1[E][F][d], W3[E][F][d],
+ * W2[E][d][F].  dtype 0 = float32 storage, 1 = bfloat16 bit patterns; every
+ * element is widened exactly to double before use.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* exact widening of one stored element to double */
+static double elem(const void* base, int dtype, size_t i) {
+    if (dtype == 0) return (double)((const float*)base)[i];
+    uint32_t bits = ((uint32_t)((const uint16_t*)base)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, 4);
+    return (double)f;
+}
+
+/* step 1 for one token: s[e] = sum_j x[j] * Wg[e][j], j ascending */
+static void token_scores(int d, int E, const void* x, const void* Wg, int dtype, size_t t, double* s) {
+    for (int e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int j = 0; j < d; ++j)
+            acc += elem(x, dtype, t * (size_t)d + j) * elem(Wg, dtype, (size_t)e * d + j);
+        s[e] = acc;
+    }
+}
+
+/* e beats f in the selection order: higher score, or equal score and lower index */
+static int beats(const double* s, int e, int f) {
+    return s[e] > s[f] || (s[e] == s[f] && e < f);
+}
+
+/*
+ * steps 2-3 for one token.  idx[0..k) and g[0..k) in selection order.
+ * margin = s_(k) - s_(k+1) (k-th minus (k+1)-th largest score, +inf when k == E)
+ * mingap = smallest gap between consecutive selected scores (+inf when k == 1)
+ */
+static void token_select(int E, int k, const double* s, int32_t* idx, double* g,
+                         double* margin, double* mingap) {
+    int chosen[64] = {0};
+    int order[65];
+    int n_order = (k < E) ? k + 1 : k;       /* also find the best unselected one */
+    for (int r = 0; r < n_order; ++r) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            if (chosen[e]) continue;
+            if (best < 0 || beats(s, e, best)) best = e;
+        }
+        chosen[best] = 1;
+        order[r] = best;
+    }
+    for (int j = 0; j < k; ++j) idx[j] = order[j];
+    double top = s[order[0]];
+    double denom = 0.0;
+    for (int j = 0; j < k; ++j) denom += exp(s[order[j]] - top);
+    for (int j = 0; j < k; ++j) g[j] = exp(s[order[j]] - top) / denom;
+    if (margin) *margin = (k < E) ? s[order[k - 1]] - s[order[k]] : INFINITY;
+    if (mingap) {
+        double m = INFINITY;
+        for (int j = 0; j + 1 < k; ++j) {
+            double gap = s[order[j]] - s[order[j + 1]];
+            if (gap < m) m = gap;
+        }
+        *mingap = m;
+    }
+}
+
+/* step 4 for one token vector xv (already widened): y = W2_e (SiLU(W1_e xv) * W3_e xv) */
+static void expert_apply(int d, int F, const double* xv, const void* W1, const void* W3, const void* W2,
+                         int dtype, int e, double* h, double* y) {
+    size_t w13 = (size_t)e * F * d;
+    for (int f = 0; f < F; ++f) {
+        double a = 0.0, b = 0.0;
+        for (int j = 0; j < d; ++j) {
+            a += elem(W1, dtype, w13 + (size_t)f * d + j) * xv[j];
+            b += elem(W3, dtype, w13 + (size_t)f * d + j) * xv[j];
+        }
+        double silu = a / (1.0 + exp(-a));
+        h[f] = silu * b;
+    }
+    size_t w2 = (size_t)e * d * F;
+    for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int f = 0; f < F; ++f) acc += elem(W2, dtype, w2 + (size_t)i * F + f) * h[f];
+        y[i] = acc;
+    }
+}
+
+/* router scores for all tokens: logits[T][E] */
+int oracle_scores(int T, int d, int E, const void* x, const void* Wg, int dtype, double* logits,
+                  int nthreads) {
+    if (T < 0 || d <= 0 || E <= 0 || E > 64) return 1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int t = 0; t < T; ++t) token_scores(d, E, x, Wg, dtype, (size_t)t, logits + (size_t)t * E);
+    return 0;
+}
+
+/* selection + gates from given scores (used by tests to pin the selection) */
+int oracle_select(int T, int E, int k, const double* logits, int32_t* idx, double* g, double* margin,
+                  double* mingap) {
+    if (T < 0 || E <= 0 || E > 64 || k <= 0 || k > E) return 1;
+    for (int t = 0; t < T; ++t)
+        token_select(E, k, logits + (size_t)t * E, idx + (size_t)t * k, g + (size_t)t * k,
+                     margin ? margin + t : NULL, mingap ? mingap + t : NULL);
+    return 0;
+}
+
+/* routing of all tokens (steps 1-3) */
+int oracle_route(int T, int d, int E, int k, const void* x, const void* Wg, int dtype, int32_t* idx,
+                 double* g, double* margin, double* mingap, int nthreads) {
+    if (T < 0 || d <= 0 || E <= 0 || E > 64 || k <= 0 || k > E) return 1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int t = 0; t < T; ++t) {
+        double s[64];
+        token_scores(d, E, x, Wg, dtype, (size_t)t, s);
+        token_select(E, k, s, idx + (size_t)t * k, g + (size_t)t * k, margin + t, mingap + t);
+    }
+    return 0;
+}
+
+/* one expert on one token row of x (step 4 alone) */
+int oracle_expert(int d, int F, const void* x, const void* W1, const void* W3, const void* W2, int dtype,
+                  int e, int t, double* y) {
+    if (d <= 0 || F <= 0) return 1;
+    double* xv = (double*)malloc(sizeof(double) * d);
+    double* h = (double*)malloc(sizeof(double) * F);
+    if (!xv || !h) { free(xv); free(h); return 2; }
+    for (int j = 0; j < d; ++j) xv[j] = elem(x, dtype, (size_t)t * d + j);
+    expert_apply(d, F, xv, W1, W3, W2, dtype, e, h, y);
+    free(xv);
+    free(h);
+    return 0;
+}
+
+/*
+ * The whole layer for the tokens listed in tokens[0..n) (all tokens when
+ * tokens == NULL, n == T).  out[n][d] in double; idx/g [n][k]; margin/mingap [n].
+ */
+int oracle_moe(int T, int d, int F, int E, int k, const void* x, const void* Wg, const void* W1,
+               const void* W3, const void* W2, int dtype, const int32_t* tokens, int n, double* out,
+               int32_t* idx, double* g, double* margin, double* mingap, int nthreads) {
+    if (T < 0 || d <= 0 || F <= 0 || E <= 0 || E > 64 || k <= 0 || k > E || n < 0) return 1;
+    if (!tokens && n != T) return 1;
+    for (int r = 0; r < n; ++r)
+        if (tokens && (tokens[r] < 0 || tokens[r] >= T)) return 1;
+    int fail = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        double* xv = (double*)malloc(sizeof(double) * d);
+        double* h = (double*)malloc(sizeof(double) * F);
+        double* y = (double*)malloc(sizeof(double) * d);
+        if (!xv || !h || !y) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int r = 0; r < n; ++r) {
+                size_t t = tokens ? (size_t)tokens[r] : (size_t)r;
+                double s[64];
+                token_scores(d, E, x, Wg, dtype, t, s);
+                int32_t* ir = idx + (size_t)r * k;
+                double* gr = g + (size_t)r * k;
+                token_select(E, k, s, ir, gr, margin + r, mingap + r);
+                for (int j = 0; j < d; ++j) xv[j] = elem(x, dtype, t * d + j);
+                double* o = out + (size_t)r * d;
+                for (int i = 0; i < d; ++i) o[i] = 0.0;
+                for (int j = 0; j < k; ++j) {
+                    expert_apply(d, F, xv, W1, W3, W2, dtype, ir[j], h, y);
+                    for (int i = 0; i < d; ++i) o[i] += gr[j] * y[i];
+                }
+            }
+        }
+        free(xv);
+        free(h);
+        free(y);
+    }
+    return fail ? 2 : 0;
+}
+
+/* per-expert assignment counts: counts[e] = #{(t, j) : idx[t][j] == e} */
+int oracle_counts(int T, int k, int E, const int32_t* idx, int64_t* counts) {
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (size_t a = 0; a < (size_t)T * k; ++a) {
+        if (idx[a] < 0 || idx[a] >= E) return 1;
+        counts[idx[a]] += 1;
+    }
+    return 0;
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
