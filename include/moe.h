@@ -1,0 +1,201 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse mixture-of-experts feed-forward layer.
+ *
+ * The layer is the Mixtral-style top-k MoE FFN described on the page
+ * "Mistral/Mixtralのアーキテクチャ — Sliding Window AttentionとMoEの融合"
+ * (disassemble-channel.com/mistral-mixtral-architecture), section
+ * "MoEの数学 — ルーターとゲーティング機構".  Per token x (a row of length d):
+ *
+ *   s   = Wg x                      router scores, Wg in R^{E x d}, no bias
+ *                                   (subsection "Top-2ゲーティングの定式化")
+ *   i_1..i_k = the k largest scores, s_i1 >= s_i2 >= ...; equal scores go to
+ *                                   the lower expert index
+ *   g_j = exp(s_ij) / sum_m exp(s_im)   softmax over the selected k only
+ *   E_i(x) = W2_i (SiLU(W1_i x) * W3_i x),  SiLU(a) = a sigmoid(a)
+ *                                   (subsection "各エキスパートの構造")
+ *   out = g_1 E_i1(x) + ... + g_k E_ik(x), summed in that order
+ *
+ * Layouts (row-major, the nn.Linear weight convention of the page's
+ * "MoEレイヤー全体の実装" code; every GEMM operand is contiguous along its
+ * reduction axis):
+ *   x   [T][d]          Wg [E][d]
+ *   W1  [E][F][d]       W3 [E][F][d]       W2 [E][d][F]      (F = ffn)
+ *   out [T][d]
+ *   topk_idx [T][k] int32, topk_w [T][k] float   (slot j = j-th largest score)
+ *
+ * Element types: the plain entry points take bfloat16 tensors (bit patterns,
+ * IEEE bfloat16, passed as void*), accumulate in fp32 and round the output to
+ * bfloat16 (round to nearest even).  The *_f32 entry points take and return
+ * float and compute in fp32 throughout (no TF32).
+ *
+ * Pointers: "device" means memory the current CUDA device can address
+ * (cudaMalloc, cudaMallocAsync, torch CUDA tensors); "host" means ordinary or
+ * pinned host memory.  Every pointer must be 16-byte aligned.  The caller owns
+ * every buffer; the library keeps no pointer past the call.  Outputs are fully
+ * overwritten, never accumulated into.
+ *
+ * Streams: every call is stream-ordered on `stream` (0 = legacy default
+ * stream) and returns without synchronising, except moe_forward_host and
+ * moe_get_device_status, which synchronise `stream`.  Calls are reentrant;
+ * calls on different streams may run concurrently, each with its own
+ * workspace.
+ *
+ * Errors: argument checks run on the host before anything is launched and
+ * return MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED with nothing launched.  A
+ * failed launch or allocation returns MOE_ERR_CUDA / MOE_ERR_WORKSPACE.  Faults
+ * found on the device while kernels run (an expert index out of range, a
+ * pipeline wait that ran past its time limit) do not trap: the kernel records
+ * the first one in a per-device status word, stops its own work, releases what
+ * it holds and returns; read the word with moe_get_device_status.  Outputs of a
+ * call that recorded a device fault are unspecified.  Inputs are assumed
+ * finite: the layer's definition says nothing about NaN or Inf.
+ *
+ * Supported sizes: 1 <= k <= E <= 32, T >= 0 (T == 0 is a no-op returning
+ * MOE_OK).  bfloat16 entry points: d % 64 == 0, F % 128 == 0.  fp32 entry
+ * points: d % 4 == 0, F >= 1.  T * k must stay below 2^31.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* null pointer, negative size, k > E, misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid layer, but a size this build does not handle */
+    MOE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    MOE_ERR_TIMEOUT = 4,      /* device: a pipeline wait ran past its time limit */
+    MOE_ERR_WORKSPACE = 5,    /* workspace missing or smaller than moe_workspace_size() */
+    MOE_ERR_DEVICE = 6        /* device: an input failed a kernel's own check (index range) */
+} moe_status;
+
+/* path selection for moe_forward_ws */
+enum {
+    MOE_PATH_AUTO = 0,    /* decode path for small T, grouped-GEMM path otherwise */
+    MOE_PATH_PREFILL = 1, /* gather + tensor-core grouped GEMMs */
+    MOE_PATH_DECODE = 2   /* expert-weight streaming (bfloat16 only) */
+};
+
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+
+/*
+ * Routing alone (router scores, top-k, softmax over the selected k): steps
+ * "s = Wg x", "Top-2(s)" and the gate equation of subsection
+ * "Top-2ゲーティングの定式化"; the page's MoERouter.forward in
+ * "簡易MoEルーターの実装" returns the same (weights, indices) pair.
+ *   x [T][d] bf16 (device), Wg [E][d] bf16 (device)
+ *   topk_idx [T][k] int32 (device, out), topk_w [T][k] float (device, out)
+ * Scores are accumulated in fp32 and never rounded to bf16.
+ */
+MOE_API moe_status moe_route(const void* x, const void* Wg, int T, int d, int E, int k,
+                     int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+
+/* moe_route for float x [T][d] and Wg [E][d] (device). */
+MOE_API moe_status moe_route_f32(const float* x, const float* Wg, int T, int d, int E, int k,
+                         int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+
+/*
+ * Number of rows of the expert-contiguous buffers that moe_dispatch fills:
+ * each expert's segment is padded up to a multiple of 128 rows, so this is
+ * T*k + E*127 rounded up to a multiple of 128.
+ */
+MOE_API size_t moe_slots_capacity(int T, int E, int k);
+
+/*
+ * Counting-sort dispatch of the routed tokens: the per-expert batching that
+ * the page's "MoEレイヤー全体の実装" code does with one mask per expert
+ * (x[mask] for the tokens that chose expert i), done as one stable pass.
+ *   topk_idx [T][k] int32 (device, in): expert ids in [0, E)
+ *   counts   [E]   int32 (device, out): assignments per expert
+ *   offsets  [E+1] int32 (device, out): start row of each expert's segment;
+ *                  offsets[e+1] - offsets[e] = counts[e] rounded up to 128
+ *   perm     [moe_slots_capacity(T,E,k)] int32 (device, out): for each row of
+ *                  a segment, the assignment t*k + j it holds, or -1 on a
+ *                  padding row; rows past offsets[E] are left untouched
+ *   inv      [T][k] int32 (device, out): the row that assignment (t, j) went to
+ * Within a segment, rows are in increasing token order (stable).  Scratch
+ * memory comes from the library's stream-ordered pool on `stream`.  An
+ * expert id out of range records MOE_ERR_DEVICE in the status word.
+ */
+MOE_API moe_status moe_dispatch(const int32_t* topk_idx, int T, int E, int k, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, int32_t* inv, cudaStream_t stream);
+
+/*
+ * The whole layer (route, dispatch, experts, combine) with bfloat16 tensors
+ * (all device): x [T][d], Wg [E][d], W1/W3 [E][F][d], W2 [E][d][F], out [T][d].
+ * The workspace comes from the library's stream-ordered pool on `stream`
+ * (cudaMallocAsync semantics: no host synchronisation).
+ */
+MOE_API moe_status moe_forward(const void* x, const void* Wg, const void* W1, const void* W3,
+                       const void* W2, void* out, int T, int d, int ffn, int E, int k,
+                       cudaStream_t stream);
+
+/* moe_forward with float tensors (all device), fp32 arithmetic throughout. */
+MOE_API moe_status moe_forward_f32(const float* x, const float* Wg, const float* W1, const float* W3,
+                           const float* W2, float* out, int T, int d, int ffn, int E, int k,
+                           cudaStream_t stream);
+
+/* Bytes of workspace moe_forward_ws needs for this layer (dtype: MOE_DTYPE_*). */
+MOE_API size_t moe_workspace_size(int T, int d, int ffn, int E, int k, int dtype);
+
+/*
+ * moe_forward / moe_forward_f32 with a caller-provided device workspace of
+ * at least moe_workspace_size() bytes (256-byte aligned), and an explicit
+ * path (MOE_PATH_*; the decode path needs dtype == MOE_DTYPE_BF16).  The
+ * workspace must not be in use by another call in flight.
+ */
+MOE_API moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1, const void* W3,
+                          const void* W2, void* out, int T, int d, int ffn, int E, int k,
+                          int dtype, int path, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
+
+/*
+ * End-to-end call from host memory: copies x_host [T][d] (host, bf16) to the
+ * device, runs moe_forward with the device-resident weights (device), copies
+ * the result back into out_host [T][d] (host, bf16) and synchronises
+ * `stream`.  Pinned host buffers give full copy bandwidth; pageable ones work.
+ */
+MOE_API moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3,
+                            const void* W2, void* out_host, int T, int d, int ffn, int E, int k,
+                            cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status
+ * word: MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE (the first fault recorded
+ * since the last read), or MOE_ERR_CUDA if the synchronisation itself failed.
+ */
+MOE_API moe_status moe_get_device_status(cudaStream_t stream);
+
+/*
+ * Self-test of the device fault path: launches one CTA that waits on a
+ * shared-memory barrier that nothing ever arrives at, with a time limit of
+ * limit_ns nanoseconds (1e3 <= limit_ns <= 1e10).  The wait gives up, records
+ * MOE_ERR_TIMEOUT in the status word and the kernel returns normally; read
+ * the result with moe_get_device_status.  Nothing faults or hangs.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(long long limit_ns, cudaStream_t stream);
+
+/* Static description of a status code. */
+MOE_API const char* moe_status_string(moe_status status);
+
+/* Token count at or below which MOE_PATH_AUTO takes the decode path. */
+MOE_API int moe_decode_max_tokens(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

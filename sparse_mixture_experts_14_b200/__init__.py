@@ -1,0 +1,214 @@
+"""B200 (sm_100a) sparse mixture-of-experts feed-forward layer: Python binding.
+
+A thin ctypes layer over ``libmoe.so`` (the C ABI declared in include/moe.h):
+the functions below carry the C names, check shapes/dtypes/devices, pass raw
+device pointers and torch's current CUDA stream, and turn a non-zero status
+into ``MoEError``.  Every step of the layer runs in the library's CUDA
+kernels.  There is no fallback: if the library is missing or cannot load,
+importing this package raises.
+
+bf16 tensors are torch.bfloat16; the layer's operand layouts are
+    x [T][d], Wg [E][d], W1 [E][F][d], W3 [E][F][d], W2 [E][d][F], out [T][d].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_14_b200.build` "
+                      f"(or __graft_entry__.build())")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_WORKSPACE, \
+    MOE_ERR_DEVICE = range(7)
+MOE_PATH_AUTO, MOE_PATH_PREFILL, MOE_PATH_DECODE = 0, 1, 2
+MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
+
+# every symbol include/moe.h declares, with its ctypes signature
+_vp, _ci, _sz, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
+SIGNATURES = {
+    "moe_route": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _vp, _vp, _vp]),
+    "moe_route_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _vp, _vp, _vp]),
+    "moe_slots_capacity": (_sz, [_ci, _ci, _ci]),
+    "moe_dispatch": (_ci, [_vp, _ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp]),
+    "moe_forward": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _vp]),
+    "moe_forward_f32": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _vp]),
+    "moe_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
+    "moe_forward_ws": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _vp, _sz, _vp]),
+    "moe_forward_host": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _vp]),
+    "moe_get_device_status": (_ci, [_vp]),
+    "moe_selftest_wait_timeout": (_ci, [_ll, _vp]),
+    "moe_status_string": (ctypes.c_char_p, [_ci]),
+    "moe_decode_max_tokens": (_ci, []),
+}
+for _name, (_res, _args) in SIGNATURES.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {moe_status_string(status)} (status {status})")
+
+
+def moe_status_string(status: int) -> str:
+    return _lib.moe_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoEError(status, what)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _dev(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return MOE_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return MOE_DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _layer_shapes(x, Wg, W1, W3, W2):
+    T, d = x.shape
+    E, F, d1 = W1.shape
+    if Wg.shape != (E, d) or d1 != d or W3.shape != (E, F, d) or W2.shape != (E, d, F):
+        raise ValueError(f"inconsistent shapes x{tuple(x.shape)} Wg{tuple(Wg.shape)} W1{tuple(W1.shape)} "
+                         f"W3{tuple(W3.shape)} W2{tuple(W2.shape)}")
+    return T, d, F, E
+
+
+def moe_route(x, Wg, k, topk_idx=None, topk_w=None, stream=None):
+    """Router scores, top-k (lowest index on ties), softmax over the k: (topk_idx int32 [T][k], topk_w f32 [T][k])."""
+    code = _dtype_code(x)
+    _dev(x, x.dtype, "x")
+    _dev(Wg, x.dtype, "Wg")
+    T, d = x.shape
+    E = Wg.shape[0]
+    if topk_idx is None:
+        topk_idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    _dev(topk_idx, torch.int32, "topk_idx")
+    _dev(topk_w, torch.float32, "topk_w")
+    fn = _lib.moe_route if code == MOE_DTYPE_BF16 else _lib.moe_route_f32
+    _check(fn(_ptr(x), _ptr(Wg), T, d, E, k, _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
+    return topk_idx, topk_w
+
+
+def moe_slots_capacity(T, E, k) -> int:
+    return int(_lib.moe_slots_capacity(T, E, k))
+
+
+def moe_dispatch(topk_idx, E, stream=None):
+    """Stable counting sort of assignments into 128-padded expert segments: (counts, offsets, perm, inv)."""
+    _dev(topk_idx, torch.int32, "topk_idx")
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(moe_slots_capacity(T, E, k), 1), dtype=torch.int32, device=dev)
+    inv = torch.empty((T, k), dtype=torch.int32, device=dev)
+    _check(_lib.moe_dispatch(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
+                             _stream(stream)), "moe_dispatch")
+    return counts, offsets, perm, inv
+
+
+def moe_forward(x, Wg, W1, W3, W2, k, out=None, stream=None):
+    """The whole layer; bf16 tensors use moe_forward, float32 tensors moe_forward_f32."""
+    code = _dtype_code(x)
+    for t, n in ((x, "x"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2")):
+        _dev(t, x.dtype, n)
+    T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
+    if out is None:
+        out = torch.empty((T, d), dtype=x.dtype, device=x.device)
+    _dev(out, x.dtype, "out")
+    fn = _lib.moe_forward if code == MOE_DTYPE_BF16 else _lib.moe_forward_f32
+    _check(fn(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, _stream(stream)),
+           "moe_forward")
+    return out
+
+
+moe_forward_f32 = moe_forward
+
+
+def moe_workspace_size(T, d, ffn, E, k, dtype=MOE_DTYPE_BF16) -> int:
+    return int(_lib.moe_workspace_size(T, d, ffn, E, k, dtype))
+
+
+def moe_forward_ws(x, Wg, W1, W3, W2, k, path=MOE_PATH_AUTO, workspace=None, out=None, stream=None):
+    """moe_forward with an explicit workspace (a uint8 CUDA tensor) and path."""
+    code = _dtype_code(x)
+    for t, n in ((x, "x"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2")):
+        _dev(t, x.dtype, n)
+    T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
+    need = moe_workspace_size(T, d, F, E, k, code)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _dev(workspace, torch.uint8, "workspace")
+    if out is None:
+        out = torch.empty((T, d), dtype=x.dtype, device=x.device)
+    _dev(out, x.dtype, "out")
+    _check(_lib.moe_forward_ws(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, code,
+                               path, _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward_ws")
+    return out
+
+
+def moe_forward_host(x_host, Wg, W1, W3, W2, k, out_host=None, stream=None):
+    """End to end from host memory: x_host / out_host are CPU bf16 tensors (pinned for full speed)."""
+    if x_host.is_cuda or x_host.dtype != torch.bfloat16 or not x_host.is_contiguous():
+        raise TypeError("x_host must be a contiguous CPU bfloat16 tensor")
+    for t, n in ((Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2")):
+        _dev(t, torch.bfloat16, n)
+    T, d = x_host.shape
+    E, F, _ = W1.shape
+    if out_host is None:
+        out_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
+    _check(_lib.moe_forward_host(_ptr(x_host), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out_host), T, d, F, E,
+                                 k, _stream(stream)), "moe_forward_host")
+    return out_host
+
+
+def moe_get_device_status(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device fault word (MOE_OK if none)."""
+    return int(_lib.moe_get_device_status(_stream(stream)))
+
+
+def moe_selftest_wait_timeout(limit_ns: int, stream=None):
+    _check(_lib.moe_selftest_wait_timeout(int(limit_ns), _stream(stream)), "moe_selftest_wait_timeout")
+
+
+def moe_decode_max_tokens() -> int:
+    return int(_lib.moe_decode_max_tokens())
+
+
+def loaded_library_path() -> str:
+    return LIB_PATH

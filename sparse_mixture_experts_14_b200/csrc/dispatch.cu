@@ -1,0 +1,188 @@
+// Dispatch: a deterministic, stable counting sort of the routed assignments
+// into expert-contiguous segments, then a gather of token rows into them.
+//
+// This is the per-expert batching of the page's "MoEレイヤー全体の実装" code
+// (one mask per expert, x[mask] for the tokens that chose it), done in one
+// integer-only pass instead of E masked passes.  Assignment (t, j) of a token
+// that chose expert e lands in row
+//     offsets[e] + #{t' < t : e is among the experts t' chose}
+// so rows inside a segment follow token order.  Segments are padded to 128
+// rows (one tensor-core tile); padding rows carry perm = -1 and zero inputs.
+//
+// Kernels: histogram (per 1024-token block), scan (one block: totals, padded
+// offsets, per-block bases), scatter (per-block stable ranks by warp ballots),
+// gather (one warp per row, 16-byte copies).
+#include "moe_common.cuh"
+
+namespace moe {
+namespace {
+
+__global__ void __launch_bounds__(kDispatchTokens) hist_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                                                               int32_t* __restrict__ blk_counts, int* status) {
+    __shared__ int cnt[kMaxExperts];
+    if (threadIdx.x < kMaxExperts) cnt[threadIdx.x] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * kDispatchTokens + threadIdx.x;
+    if (t < T) {
+        uint32_t mask = 0;
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[(size_t)t * k + j];
+            if (e < 0 || e >= E || ((mask >> e) & 1u)) {
+                record_status(status, MOE_ERR_DEVICE);   // out of range or chosen twice: dropped
+                continue;
+            }
+            mask |= 1u << e;
+            atomicAdd(&cnt[e], 1);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < E) blk_counts[(size_t)blockIdx.x * E + threadIdx.x] = cnt[threadIdx.x];
+}
+
+// One block of 32 warps; warp e owns expert e.  In place: blk_counts[b][e]
+// becomes the first row of block b's assignments to expert e.
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ blk, int NB, int E, Meta* __restrict__ meta,
+                                                    int32_t* __restrict__ perm, size_t slots, int* status) {
+    __shared__ int tot[kMaxExperts];
+    __shared__ int offs[kMaxExperts + 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < E) {
+        int s = 0;
+        for (int b = lane; b < NB; b += 32) s += blk[(size_t)b * E + warp];
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+        if (lane == 0) tot[warp] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        offs[0] = 0;
+        for (int e = 0; e < E; ++e) offs[e + 1] = offs[e] + (tot[e] + kSegRows - 1) / kSegRows * kSegRows;
+        if ((size_t)offs[E] > slots) record_status(status, MOE_ERR_DEVICE);
+        for (int e = 0; e < E; ++e) meta->counts[e] = tot[e];
+        for (int e = 0; e <= E; ++e) meta->offsets[e] = offs[e];
+    }
+    __syncthreads();
+    if (warp < E) {
+        int carry = offs[warp];
+        for (int b0 = 0; b0 < NB; b0 += 32) {
+            const int b = b0 + lane;
+            const int v = (b < NB) ? blk[(size_t)b * E + warp] : 0;
+            int incl = v;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, m);
+                if (lane >= m) incl += o;
+            }
+            if (b < NB) blk[(size_t)b * E + warp] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    // padding rows of every segment
+    for (int e = 0; e < E; ++e) {
+        const int beg = offs[e] + tot[e], end = offs[e + 1];
+        for (int r = beg + threadIdx.x; r < end; r += blockDim.x)
+            if ((size_t)r < slots) perm[r] = -1;
+    }
+}
+
+__global__ void __launch_bounds__(kDispatchTokens) scatter_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                                                                  const int32_t* __restrict__ blk_base,
+                                                                  int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                  size_t slots, int* status) {
+    __shared__ int wcnt[32][kMaxExperts + 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kDispatchTokens + threadIdx.x;
+    uint32_t mask = 0;
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[(size_t)t * k + j];
+            if (e >= 0 && e < E) mask |= 1u << e;
+        }
+    }
+    const uint32_t lt = (1u << lane) - 1u;
+    int rank[kMaxExperts];   // in-warp rank of this token among the warp's tokens that chose e
+    for (int e = 0; e < E; ++e) {
+        const uint32_t bal = __ballot_sync(0xffffffffu, (mask >> e) & 1u);
+        rank[e] = __popc(bal & lt);
+        if (lane == 0) wcnt[warp][e] = __popc(bal);
+    }
+    __syncthreads();
+    if (threadIdx.x < E) {
+        const int e = threadIdx.x;
+        int run = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int c = wcnt[w][e];
+            wcnt[w][e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    if (t < T) {
+        uint32_t seen = 0;
+        for (int j = 0; j < k; ++j) {
+            const int a = t * k + j;
+            const int e = idx[a];
+            if (e < 0 || e >= E || ((seen >> e) & 1u)) {
+                inv[a] = -1;
+                continue;
+            }
+            seen |= 1u << e;
+            const int slot = blk_base[(size_t)blockIdx.x * E + e] + wcnt[warp][e] + rank[e];
+            if (slot < 0 || (size_t)slot >= slots) {
+                record_status(status, MOE_ERR_DEVICE);
+                inv[a] = -1;
+                continue;
+            }
+            perm[slot] = a;
+            inv[a] = slot;
+        }
+    }
+}
+
+// One warp per row of the padded buffer; rows past offsets[E] are left alone.
+__global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ x, size_t row_bytes, int T, int k,
+                                                     const Meta* __restrict__ meta, int E,
+                                                     const int32_t* __restrict__ perm, uint8_t* __restrict__ xp,
+                                                     size_t slots) {
+    const int lane = threadIdx.x & 31;
+    const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
+    const size_t total = (size_t)meta->offsets[E];
+    const size_t nvec = row_bytes / 16;
+    const long long TK = (long long)T * k;
+    for (size_t r = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < total && r < slots;
+         r += warps) {
+        const int a = perm[r];
+        uint4* dst = reinterpret_cast<uint4*>(xp + r * row_bytes);
+        if (a >= 0 && a < TK) {
+            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(a / k) * row_bytes);
+            for (size_t v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+        } else {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            for (size_t v = lane; v < nvec; v += 32) dst[v] = z;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* blk_counts, Meta* meta, int32_t* perm,
+                            int32_t* inv, int* status, cudaStream_t s) {
+    const int NB = dispatch_blocks(T);
+    const size_t slots = slots_capacity(T, E, k);
+    hist_kernel<<<NB, kDispatchTokens, 0, s>>>(idx, T, E, k, blk_counts, status);
+    scan_kernel<<<1, 1024, 0, s>>>(blk_counts, NB, E, meta, perm, slots, status);
+    scatter_kernel<<<NB, kDispatchTokens, 0, s>>>(idx, T, E, k, blk_counts, perm, inv, slots, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
+                          const int32_t* perm, void* xp, size_t slots, cudaStream_t s) {
+    const size_t rows_per_block = 8;
+    size_t blocks = (slots + rows_per_block - 1) / rows_per_block;
+    if (blocks > 65535 * 4) blocks = 65535 * 4;
+    gather_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), (size_t)d * elem_bytes, T, k,
+                                                  meta, E, perm, static_cast<uint8_t*>(xp), slots);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,386 @@
+// Tensor-core grouped GEMMs of the experts (bf16 in, fp32 accumulate in tensor
+// memory), sm_100a: tcgen05.mma fed by TMA, accumulators in TMEM.
+//
+// Subsection "各エキスパートの構造" of the "Mistral/Mixtral architecture" page:
+//     E_i(x) = W2_i (SiLU(W1_i x) * W3_i x)
+// computed per expert over its expert-contiguous rows Xp_e (from dispatch):
+//     GEMM1  acc = Xp_e [W1_e ; W3_e]^T,   H = SiLU(acc[:, :128]) * acc[:, 128:]  -> bf16
+//     GEMM2  Y   = H_e W2_e^T                                              -> fp32
+//
+// Tile: 128 rows x 256 accumulator columns x 64-deep K steps.  In GEMM1 the
+// 256 columns are 128 rows of W1_e followed by the same 128 rows of W3_e, so
+// one MMA of N = 256 yields both halves of the SwiGLU for a 128 x 128 block of
+// H, and the gating runs in the epilogue straight out of TMEM.
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0     TMA producer (one thread): A and B tiles into a 4-stage ring
+//   warp 1     MMA issuer (one thread) + TMEM owner (512 columns = two
+//              128 x 256 fp32 accumulators, so the epilogue of one tile
+//              overlaps the MMAs of the next)
+//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, gating / fp32
+//              stores
+// Tiles are (expert, n-block, m-block) with m fastest, so CTAs working at the
+// same time share one block of expert weights through L2.  The tile list is
+// derived on the device from the dispatch offsets: no host synchronisation.
+#include <cuda.h>
+
+#include "moe_common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int BN = 256;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;          // 16 KiB
+constexpr int B_BYTES = BN * BK * 2;          // 32 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int NUM_THREADS = 192;
+constexpr int NUM_EPI_THREADS = 128;
+constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN);
+
+struct Ctrl {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int total;
+    int tile_base[kMaxExperts + 1];
+    int mt[kMaxExperts];
+    int row0[kMaxExperts];
+};
+
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + (int)sizeof(Ctrl) + 1024;
+
+__device__ __forceinline__ void decode_tile(const Ctrl* c, int tile, int& e, int& m_blk, int& n_blk) {
+    e = 0;
+    while (tile >= c->tile_base[e + 1]) ++e;
+    const int local = tile - c->tile_base[e];
+    n_blk = local / c->mt[e];
+    m_blk = local - n_blk * c->mt[e];
+}
+
+// SWIGLU: GEMM1 (B = W1/W3 row blocks of 128, out = H bf16 [slots][N]).
+// !SWIGLU: GEMM2 (B = W2 row block of 256, out = Y fp32 [slots][N]).
+template <bool SWIGLU>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB1,
+                   const __grid_constant__ CUtensorMap mapB3, const Meta* __restrict__ meta, int E, int K, int N,
+                   size_t slots, void* __restrict__ out, int* status, long long wait_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    constexpr int N_PER_TILE = SWIGLU ? BN / 2 : BN;   // output columns per tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(&ctrl->full[s], 1);
+            ptx::mbar_init(&ctrl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&ctrl->tfull[b], 1);
+            ptx::mbar_init(&ctrl->tempty[b], NUM_EPI_THREADS);
+        }
+        ptx::mbar_init(&ctrl->drain, 1);
+        ctrl->abort = 0;
+        const int ntn = (N + N_PER_TILE - 1) / N_PER_TILE;
+        ctrl->tile_base[0] = 0;
+        bool ok = true;
+        for (int e = 0; e < E; ++e) {
+            const int r0 = meta->offsets[e], r1 = meta->offsets[e + 1];
+            if (r1 < r0 || (r1 - r0) % BM != 0 || (size_t)r1 > slots) ok = false;
+            const int mt = ok ? (r1 - r0) / BM : 0;
+            ctrl->mt[e] = mt;
+            ctrl->row0[e] = r0;
+            ctrl->tile_base[e + 1] = ctrl->tile_base[e] + mt * ntn;
+        }
+        ctrl->total = ok ? ctrl->tile_base[E] : 0;
+        if (!ok) record_status(status, MOE_ERR_DEVICE);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::tma_prefetch_desc(&mapA);
+        ptx::tma_prefetch_desc(&mapB1);
+        if (SWIGLU) ptx::tma_prefetch_desc(&mapB3);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+
+    const uint32_t tmem_base = ctrl->tmem_base;
+    const int total = ctrl->total;
+    const int nk = (K + BK - 1) / BK;
+    const ptx::WaitCtl wc{&ctrl->abort, status, (uint64_t)wait_ns};
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol_act = ptx::policy_evict_last();
+            const uint64_t pol_w = ptx::policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool armed[STAGES];
+            uint32_t armed_phase[STAGES];
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s) {
+                armed[s] = false;
+                armed_phase[s] = 0;
+            }
+            bool aborted = false;
+            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+                int e, m_blk, n_blk;
+                decode_tile(ctrl, tile, e, m_blk, n_blk);
+                const int rowA = ctrl->row0[e] + m_blk * BM;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!ptx::mbar_wait(&ctrl->empty[stage], phase ^ 1u, wc)) {
+                        aborted = true;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    ptx::mbar_arrive_expect_tx(&ctrl->full[stage], STAGE_BYTES);
+                    ptx::tma_load_2d(sa, &mapA, &ctrl->full[stage], kb * BK, rowA, pol_act);
+                    if (SWIGLU) {
+                        ptx::tma_load_3d(sb, &mapB1, &ctrl->full[stage], kb * BK, n_blk * (BN / 2), e, pol_w);
+                        ptx::tma_load_3d(sb + B_BYTES / 2, &mapB3, &ctrl->full[stage], kb * BK, n_blk * (BN / 2), e,
+                                         pol_w);
+                    } else {
+                        ptx::tma_load_3d(sb, &mapB1, &ctrl->full[stage], kb * BK, n_blk * BN, e, pol_w);
+                    }
+#pragma unroll
+                    for (int s = 0; s < STAGES; ++s)
+                        if (s == stage) {
+                            armed[s] = true;
+                            armed_phase[s] = phase;
+                        }
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (aborted || ctrl->abort) {
+                // let every copy still in flight land before the CTA's shared memory is released
+#pragma unroll
+                for (int s = 0; s < STAGES; ++s)
+                    if (armed[s]) ptx::mbar_wait_drain(&ctrl->full[s], armed_phase[s], 2000000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool issued = false, aborted = false;
+            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+                if (!ptx::mbar_wait(&ctrl->tempty[acc], acc_phase ^ 1u, wc)) {
+                    aborted = true;
+                    break;
+                }
+                ptx::tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!ptx::mbar_wait(&ctrl->full[stage], phase, wc)) {
+                        aborted = true;
+                        break;
+                    }
+                    ptx::tc_fence_after_sync();
+                    const uint32_t a0 = ptx::smem_addr(smem + stage * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        ptx::tc_mma_bf16(d_tmem, ptx::desc_kmajor_sw128(a0 + kk * 32),
+                                         ptx::desc_kmajor_sw128(b0 + kk * 32), IDESC, (kb | kk) != 0);
+                    }
+                    ptx::tc_commit(&ctrl->empty[stage]);
+                    issued = true;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (aborted) break;
+                ptx::tc_commit(&ctrl->tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if ((aborted || ctrl->abort) && issued) {
+                ptx::tc_commit(&ctrl->drain);
+                ptx::mbar_wait_drain(&ctrl->drain, 0, 2000000000ull);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            int e, m_blk, n_blk;
+            decode_tile(ctrl, tile, e, m_blk, n_blk);
+            bool ok = ptx::mbar_wait(&ctrl->tfull[acc], acc_phase, wc);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
+            const size_t row = (size_t)ctrl->row0[e] + (size_t)m_blk * BM + q * 32 + lane;
+            const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+            if (SWIGLU) {
+                __nv_bfloat16* H = static_cast<__nv_bfloat16*>(out);
+#pragma unroll 1
+                for (int c = 0; c < BN / 2; c += 32) {
+                    uint32_t ra[32], rb[32];
+                    ptx::tmem_ld_32x32b_x32(taddr + c, ra);
+                    ptx::tmem_ld_32x32b_x32(taddr + BN / 2 + c, rb);
+                    ptx::tmem_ld_wait();
+                    uint32_t hp[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float h0 = silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i]));
+                        const float h1 = silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1]));
+                        hp[i] = pack_bf16x2(h0, h1);
+                    }
+                    const int col = n_blk * (BN / 2) + c;
+                    uint4* dst = reinterpret_cast<uint4*>(H + row * (size_t)N + col);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+                }
+            } else {
+                float* Y = static_cast<float*>(out);
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t r[32];
+                    ptx::tmem_ld_32x32b_x32(taddr + c, r);
+                    ptx::tmem_ld_wait();
+                    const int col = n_blk * BN + c;
+                    if (col < N) {
+                        float4* dst = reinterpret_cast<float4*>(Y + row * (size_t)N + col);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                 __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                    }
+                }
+            }
+            ptx::tc_fence_before_sync();
+            ptx::mbar_arrive(&ctrl->tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after_sync();
+        ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes.
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+              const cuuint32_t* box) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// rows x K matrix, K contiguous: box 64 x box_rows
+bool map_rows(CUtensorMap* m, const void* base, size_t rows, int K, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    return make_map(m, base, 2, dims, strides, box);
+}
+
+// E x R x K weights, K contiguous: box 64 x box_rows x 1
+bool map_weights(CUtensorMap* m, const void* base, int E, int R, int K, int box_rows) {
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)R, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)R * K * 2};
+    cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)box_rows, 1};
+    return make_map(m, base, 3, dims, strides, box);
+}
+
+template <bool SWIGLU>
+cudaError_t ensure_smem_attr() {
+    static bool done = false;
+    if (!done) {
+        cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        done = true;
+    }
+    return cudaSuccess;
+}
+
+int grid_for(size_t slots, int n_tiles_per_m, int num_sms) {
+    const size_t upper = (slots / BM) * (size_t)n_tiles_per_m;
+    int g = num_sms > 0 ? num_sms : 148;
+    if ((size_t)g > upper) g = (int)upper;
+    return g < 1 ? 1 : g;
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s) {
+    CUtensorMap mA, mB1, mB3;
+    if (!map_rows(&mA, a.xp, a.slots, a.d, BM) || !map_weights(&mB1, a.W1, a.E, a.F, a.d, BN / 2) ||
+        !map_weights(&mB3, a.W3, a.E, a.F, a.d, BN / 2))
+        return cudaErrorInvalidValue;
+    cudaError_t e = ensure_smem_attr<true>();
+    if (e != cudaSuccess) return e;
+    const int grid = grid_for(a.slots, (a.F + BN / 2 - 1) / (BN / 2), a.num_sms);
+    tc_gemm_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB1, mB3, a.meta, a.E, a.d, a.F, a.slots, a.H,
+                                                               a.status, a.wait_ns);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s) {
+    CUtensorMap mA, mB;
+    if (!map_rows(&mA, a.H, a.slots, a.F, BM) || !map_weights(&mB, a.W2, a.E, a.d, a.F, BN))
+        return cudaErrorInvalidValue;
+    cudaError_t e = ensure_smem_attr<false>();
+    if (e != cudaSuccess) return e;
+    const int grid = grid_for(a.slots, (a.d + BN - 1) / BN, a.num_sms);
+    tc_gemm_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mB, a.meta, a.E, a.F, a.d, a.slots, a.Y,
+                                                                a.status, a.wait_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,376 @@
+// C ABI of the MoE layer: argument checks, workspace, launch orchestration.
+// Every step of the layer runs in this library's kernels; nothing here
+// computes on the host.  See include/moe.h for the contract of each call.
+#include <climits>
+#include <cstdlib>
+#include <mutex>
+
+#include "moe_common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace moe {
+
+__device__ int g_status;   // per-device sticky fault word (first fault wins)
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kDecodeMaxTokens = 64;
+
+std::mutex g_mu;
+cudaMemPool_t g_pools[kMaxDevices] = {};
+int* g_status_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+
+long long wait_limit_ns() {
+    static long long v = [] {
+        const char* s = std::getenv("MOE_WAIT_LIMIT_MS");
+        long long ms = s ? std::atoll(s) : 1000;
+        if (ms < 1) ms = 1;
+        return ms * 1000000LL;
+    }();
+    return v;
+}
+
+// Make the device that owns `p` current in this library's runtime; returns its id.
+int select_device(const void* p) {
+    int dev = 0;
+    cudaPointerAttributes at;
+    if (p && cudaPointerGetAttributes(&at, p) == cudaSuccess &&
+        (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged)) {
+        dev = at.device;
+        int cur = -1;
+        if (cudaGetDevice(&cur) != cudaSuccess || cur != dev) cudaSetDevice(dev);
+    } else {
+        cudaGetLastError();
+        cudaGetDevice(&dev);
+    }
+    return dev;
+}
+
+struct DeviceState {
+    cudaMemPool_t pool;
+    int* status;
+    int num_sms;
+};
+
+bool device_state(int dev, DeviceState* st) {
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return false;
+        uint64_t thr = UINT64_MAX;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+        void* sp = nullptr;
+        if (cudaGetSymbolAddress(&sp, g_status) != cudaSuccess) return false;
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        g_status_ptr[dev] = static_cast<int*>(sp);
+        g_num_sms[dev] = n;
+        g_pools[dev] = pool;
+    }
+    st->pool = g_pools[dev];
+    st->status = g_status_ptr[dev];
+    st->num_sms = g_num_sms[dev];
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Sizes every entry point shares.
+moe_status check_sizes(int T, int d, int E, int k) {
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if ((long long)T * k + (long long)E * kSegRows >= INT_MAX) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status check_layer(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2, const void* out,
+                       int T, int d, int F, int E, int k, int dtype) {
+    moe_status st = check_sizes(T, d, E, k);
+    if (st != MOE_OK) return st;
+    if (F <= 0) return MOE_ERR_INVALID_ARG;
+    if (dtype == MOE_DTYPE_BF16) {
+        if (d % 64 != 0 || F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    } else if (dtype == MOE_DTYPE_F32) {
+        if (d % 4 != 0) return MOE_ERR_UNSUPPORTED;
+    } else {
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (T == 0) return MOE_OK;
+    const void* ptrs[6] = {x, Wg, W1, W3, W2, out};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+struct Plan {
+    size_t idx, w, blk, meta, perm, inv, xp, h, y, total;
+    size_t slots;
+};
+
+Plan make_plan(int T, int d, int F, int E, int k, int dtype) {
+    Plan p{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + (bytes ? bytes : 1), 256);
+        return o;
+    };
+    const size_t es = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+    const size_t tk = (size_t)T * k;
+    p.slots = slots_capacity(T, E, k);
+    p.idx = take(tk * 4);
+    p.w = take(tk * 4);
+    p.blk = take((size_t)dispatch_blocks(T) * E * 4);
+    p.meta = take(sizeof(Meta));
+    p.perm = take(p.slots * 4);
+    p.inv = take(tk * 4);
+    p.xp = take(p.slots * (size_t)d * es);
+    p.h = take(p.slots * (size_t)F * es);
+    p.y = take(p.slots * (size_t)d * 4);
+    p.total = off;
+    return p;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(call)                                  \
+    do {                                               \
+        cudaError_t _e = (call);                       \
+        if (_e != cudaSuccess) return MOE_ERR_CUDA;    \
+    } while (0)
+
+moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2, void* out, int T,
+                     int d, int F, int E, int k, int dtype, int path, uint8_t* ws, const DeviceState& dev,
+                     cudaStream_t s) {
+    const Plan p = make_plan(T, d, F, E, k, dtype);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + p.idx);
+    float* w = reinterpret_cast<float*>(ws + p.w);
+    int32_t* blk = reinterpret_cast<int32_t*>(ws + p.blk);
+    Meta* meta = reinterpret_cast<Meta*>(ws + p.meta);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + p.perm);
+    int32_t* inv = reinterpret_cast<int32_t*>(ws + p.inv);
+    void* xp = ws + p.xp;
+    void* h = ws + p.h;
+    float* y = reinterpret_cast<float*>(ws + p.y);
+
+    if (dtype == MOE_DTYPE_BF16) {
+        MOE_TRY(launch_router_bf16(x, Wg, T, d, E, k, idx, w, dev.num_sms, s));
+    } else {
+        MOE_TRY(launch_router_f32(static_cast<const float*>(x), static_cast<const float*>(Wg), T, d, E, k, idx, w,
+                                  dev.num_sms, s));
+    }
+    MOE_TRY(launch_dispatch(idx, T, E, k, blk, meta, perm, inv, dev.status, s));
+    MOE_TRY(launch_gather(x, dtype == MOE_DTYPE_BF16 ? 2 : 4, T, d, E, k, meta, perm, xp, p.slots, s));
+    if (dtype == MOE_DTYPE_BF16) {
+        TcGemmArgs a{xp, W1, W3, W2, h, y, meta, E, d, F, p.slots, dev.num_sms, dev.status, wait_limit_ns()};
+        (void)path;
+        MOE_TRY(launch_tc_gemm1(a, s));
+        MOE_TRY(launch_tc_gemm2(a, s));
+        MOE_TRY(launch_combine_bf16(y, w, inv, T, d, k, out, s));
+    } else {
+        MOE_TRY(launch_simt_gemm1_f32(static_cast<const float*>(xp), static_cast<const float*>(W1),
+                                      static_cast<const float*>(W3), meta, E, d, F, static_cast<float*>(h), p.slots,
+                                      s));
+        MOE_TRY(launch_simt_gemm2_f32(static_cast<const float*>(h), static_cast<const float*>(W2), meta, E, d, F, y,
+                                      p.slots, s));
+        MOE_TRY(launch_combine_f32(y, w, inv, T, d, k, static_cast<float*>(out), s));
+    }
+    return MOE_OK;
+}
+
+moe_status forward_pooled(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2, void* out,
+                          int T, int d, int F, int E, int k, int dtype, cudaStream_t s) {
+    moe_status st = check_layer(x, Wg, W1, W3, W2, out, T, d, F, E, k, dtype);
+    if (st != MOE_OK || T == 0) return st;
+    DeviceState dev;
+    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const Plan p = make_plan(T, d, F, E, k, dtype);
+    void* ws = nullptr;
+    if (cudaMallocFromPoolAsync(&ws, p.total, dev.pool, s) != cudaSuccess) return MOE_ERR_WORKSPACE;
+    st = run_layer(x, Wg, W1, W3, W2, out, T, d, F, E, k, dtype, MOE_PATH_AUTO, static_cast<uint8_t*>(ws), dev, s);
+    if (cudaFreeAsync(ws, s) != cudaSuccess && st == MOE_OK) st = MOE_ERR_CUDA;
+    return st;
+}
+
+__global__ void wait_selftest_kernel(int* status, long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);   // nothing ever arrives on this barrier
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const ptx::WaitCtl wc{&abort_flag, status, (uint64_t)limit_ns};
+        ptx::mbar_wait(&bar, 0, wc);
+    }
+    __syncthreads();
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_route(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* topk_idx, float* topk_w,
+                     cudaStream_t stream) {
+    moe_status st = check_sizes(T, d, E, k);
+    if (st != MOE_OK) return st;
+    if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!x || !Wg || !topk_idx || !topk_w || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
+    DeviceState dev;
+    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    return cuda_status(launch_router_bf16(x, Wg, T, d, E, k, topk_idx, topk_w, dev.num_sms, stream));
+}
+
+moe_status moe_route_f32(const float* x, const float* Wg, int T, int d, int E, int k, int32_t* topk_idx,
+                         float* topk_w, cudaStream_t stream) {
+    moe_status st = check_sizes(T, d, E, k);
+    if (st != MOE_OK) return st;
+    if (d % 4 != 0) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!x || !Wg || !topk_idx || !topk_w || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
+    DeviceState dev;
+    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    return cuda_status(launch_router_f32(x, Wg, T, d, E, k, topk_idx, topk_w, dev.num_sms, stream));
+}
+
+size_t moe_slots_capacity(int T, int E, int k) {
+    if (check_sizes(T, 1, E, k) != MOE_OK) return 0;
+    return slots_capacity(T, E, k);
+}
+
+moe_status moe_dispatch(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                        int32_t* perm, int32_t* inv, cudaStream_t stream) {
+    moe_status st = check_sizes(T, 1, E, k);
+    if (st != MOE_OK) return st;
+    if (!counts || !offsets || (T > 0 && (!topk_idx || !perm || !inv))) return MOE_ERR_INVALID_ARG;
+    DeviceState dev;
+    if (!device_state(select_device(counts), &dev)) return MOE_ERR_CUDA;
+    const size_t blk_bytes = align_up((size_t)dispatch_blocks(T) * E * 4 + 1, 256);
+    void* scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, blk_bytes + sizeof(Meta), dev.pool, stream) != cudaSuccess)
+        return MOE_ERR_WORKSPACE;
+    int32_t* blk = static_cast<int32_t*>(scratch);
+    Meta* meta = reinterpret_cast<Meta*>(static_cast<uint8_t*>(scratch) + blk_bytes);
+    cudaError_t e = cudaSuccess;
+    if (T == 0) {
+        e = cudaMemsetAsync(meta, 0, sizeof(Meta), stream);
+    } else {
+        e = launch_dispatch(topk_idx, T, E, k, blk, meta, perm, inv, dev.status, stream);
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(counts, meta->counts, E * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(offsets, meta->offsets, (E + 1) * 4, cudaMemcpyDeviceToDevice, stream);
+    cudaError_t f = cudaFreeAsync(scratch, stream);
+    return (e == cudaSuccess && f == cudaSuccess) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_forward(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2, void* out, int T,
+                       int d, int ffn, int E, int k, cudaStream_t stream) {
+    return forward_pooled(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, MOE_DTYPE_BF16, stream);
+}
+
+moe_status moe_forward_f32(const float* x, const float* Wg, const float* W1, const float* W3, const float* W2,
+                           float* out, int T, int d, int ffn, int E, int k, cudaStream_t stream) {
+    return forward_pooled(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, MOE_DTYPE_F32, stream);
+}
+
+size_t moe_workspace_size(int T, int d, int ffn, int E, int k, int dtype) {
+    if (check_sizes(T, d, E, k) != MOE_OK || ffn <= 0) return 0;
+    if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_F32) return 0;
+    return make_plan(T, d, ffn, E, k, dtype).total;
+}
+
+moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2, void* out,
+                          int T, int d, int ffn, int E, int k, int dtype, int path, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
+    moe_status st = check_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype);
+    if (st != MOE_OK) return st;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE) return MOE_ERR_INVALID_ARG;
+    if (path == MOE_PATH_DECODE && dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
+    DeviceState dev;
+    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    return run_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
+                     stream);
+}
+
+moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3, const void* W2,
+                            void* out_host, int T, int d, int ffn, int E, int k, cudaStream_t stream) {
+    moe_status st = check_layer(x_host, Wg, W1, W3, W2, out_host, T, d, ffn, E, k, MOE_DTYPE_BF16);
+    if (st != MOE_OK || T == 0) return st;
+    DeviceState dev;
+    if (!device_state(select_device(Wg), &dev)) return MOE_ERR_CUDA;
+    const size_t act = (size_t)T * d * 2;
+    const size_t act_al = align_up(act, 256);
+    const Plan p = make_plan(T, d, ffn, E, k, MOE_DTYPE_BF16);
+    void* buf = nullptr;
+    if (cudaMallocFromPoolAsync(&buf, 2 * act_al + p.total, dev.pool, stream) != cudaSuccess)
+        return MOE_ERR_WORKSPACE;
+    uint8_t* xd = static_cast<uint8_t*>(buf);
+    uint8_t* od = xd + act_al;
+    uint8_t* ws = od + act_al;
+    cudaError_t e = cudaMemcpyAsync(xd, x_host, act, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) {
+        st = run_layer(xd, Wg, W1, W3, W2, od, T, d, ffn, E, k, MOE_DTYPE_BF16, MOE_PATH_AUTO, ws, dev, stream);
+        if (st == MOE_OK) e = cudaMemcpyAsync(out_host, od, act, cudaMemcpyDeviceToHost, stream);
+    }
+    cudaError_t f = cudaFreeAsync(buf, stream);
+    cudaError_t g = cudaStreamSynchronize(stream);
+    if (st != MOE_OK) return st;
+    return (e == cudaSuccess && f == cudaSuccess && g == cudaSuccess) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    DeviceState st;
+    if (!device_state(dev, &st)) return MOE_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, st.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(st.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    return static_cast<moe_status>(v);
+}
+
+moe_status moe_selftest_wait_timeout(long long limit_ns, cudaStream_t stream) {
+    if (limit_ns < 1000 || limit_ns > 10000000000LL) return MOE_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    DeviceState st;
+    if (!device_state(dev, &st)) return MOE_ERR_CUDA;
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(st.status, limit_ns);
+    return cuda_status(cudaGetLastError());
+}
+
+const char* moe_status_string(moe_status status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported size";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_DEVICE: return "device-side input check failed";
+    }
+    return "unknown status";
+}
+
+int moe_decode_max_tokens(void) { return kDecodeMaxTokens; }
+
+}  // extern "C"

@@ -1,0 +1,99 @@
+// Shared device/host definitions of the MoE layer's kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Rows per expert segment granule: every expert's rows are padded to this, so
+// a 128-row tensor-core tile never straddles two experts.
+constexpr int kSegRows = 128;
+constexpr int kMaxExperts = 32;
+// Tokens handled by one dispatch block (histogram / scatter).
+constexpr int kDispatchTokens = 1024;
+
+// Small per-call table written by the dispatch scan, read by every later kernel.
+struct Meta {
+    int32_t counts[kMaxExperts];        // assignments per expert
+    int32_t offsets[kMaxExperts + 1];   // padded segment start rows; offsets[E] = padded total
+};
+
+// Per-device sticky status word (first fault wins).
+__device__ __forceinline__ void record_status(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// SiLU(a) * b with SiLU(a) = a / (1 + e^-a).
+__device__ __forceinline__ float silu_mul(float a, float b) {
+    return a / (1.0f + __expf(-a)) * b;
+}
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Rows of the padded expert-contiguous buffers.
+inline size_t slots_capacity(int T, int E, int k) {
+    return align_up((size_t)T * k + (size_t)E * (kSegRows - 1), kSegRows);
+}
+
+inline int dispatch_blocks(int T) { return (T + kDispatchTokens - 1) / kDispatchTokens; }
+
+// ---- kernel launchers (one per translation unit) ----
+cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx,
+                               float* w, int num_sms, cudaStream_t s);
+cudaError_t launch_router_f32(const float* x, const float* Wg, int T, int d, int E, int k, int32_t* idx,
+                              float* w, int num_sms, cudaStream_t s);
+
+cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* blk_counts, Meta* meta,
+                            int32_t* perm, int32_t* inv, int* status, cudaStream_t s);
+cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
+                          const int32_t* perm, void* xp, size_t slots, cudaStream_t s);
+
+cudaError_t launch_combine_bf16(const float* Y, const float* w, const int32_t* inv, int T, int d, int k,
+                                void* out, cudaStream_t s);
+cudaError_t launch_combine_f32(const float* Y, const float* w, const int32_t* inv, int T, int d, int k,
+                               float* out, cudaStream_t s);
+
+cudaError_t launch_simt_gemm1_f32(const float* xp, const float* W1, const float* W3, const Meta* meta, int E,
+                                  int d, int F, float* H, size_t slots, cudaStream_t s);
+cudaError_t launch_simt_gemm2_f32(const float* H, const float* W2, const Meta* meta, int E, int d, int F,
+                                  float* Y, size_t slots, cudaStream_t s);
+
+struct TcGemmArgs {
+    const void* xp;     // [slots][d] bf16, expert-contiguous
+    const void* W1;
+    const void* W3;
+    const void* W2;
+    void* H;            // [slots][F] bf16
+    float* Y;           // [slots][d] fp32
+    const Meta* meta;
+    int E, d, F;
+    size_t slots;
+    int num_sms;
+    int* status;
+    long long wait_ns;
+};
+cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s);
+cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const TcGemmArgs& a, cudaStream_t s);
+
+cudaError_t launch_wait_selftest(int* status, long long limit_ns, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,108 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol, and
+rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_mixture_experts_14_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_symbols())
+    for must in ("moe_route", "moe_forward", "moe_forward_f32", "moe_dispatch", "moe_forward_ws",
+                 "moe_forward_host", "moe_get_device_status", "moe_status_string"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in moe.h but not exported"
+
+
+def test_binding_signatures_cover_header():
+    import sparse_mixture_experts_14_b200 as m
+    assert set(declared_symbols()) == set(m.SIGNATURES)
+
+
+def _vp(v=0x1000):
+    return ctypes.c_void_p(v)
+
+
+def _fwd(lib, T=8, d=128, F=256, E=8, k=2, x=0x1000, out=0x2000, f32=False):
+    fn = lib.moe_forward_f32 if f32 else lib.moe_forward
+    fn.restype = ctypes.c_int
+    return fn(_vp(x), _vp(), _vp(), _vp(), _vp(), _vp(out), T, d, F, E, k, ctypes.c_void_p(0))
+
+
+def test_forward_argument_checks(lib):
+    assert _fwd(lib, k=9) == 1                 # k > E
+    assert _fwd(lib, k=0) == 1
+    assert _fwd(lib, T=-1) == 1
+    assert _fwd(lib, E=33, k=2) == 2           # more experts than supported
+    assert _fwd(lib, d=100) == 2               # bf16 path wants d % 64 == 0
+    assert _fwd(lib, F=200) == 2               # and F % 128 == 0
+    assert _fwd(lib, d=102, f32=True) == 2     # fp32 path wants d % 4 == 0
+    assert _fwd(lib, x=0) == 1                 # null pointer
+    assert _fwd(lib, x=0x1008) == 1            # not 16-byte aligned
+    assert _fwd(lib, T=0, x=0, out=0) == 0     # empty batch: no-op
+
+
+def test_route_argument_checks(lib):
+    f = lib.moe_route
+    f.restype = ctypes.c_int
+    assert f(_vp(), _vp(), 4, 128, 8, 9, _vp(), _vp(), None) == 1
+    assert f(_vp(), _vp(), 4, 100, 8, 2, _vp(), _vp(), None) == 2
+    assert f(None, _vp(), 4, 128, 8, 2, _vp(), _vp(), None) == 1
+    assert f(_vp(), _vp(), 0, 128, 8, 2, _vp(), _vp(), None) == 0
+
+
+def test_workspace_and_slots(lib):
+    lib.moe_workspace_size.restype = ctypes.c_size_t
+    lib.moe_slots_capacity.restype = ctypes.c_size_t
+    assert lib.moe_slots_capacity(16, 8, 2) == 32 + 8 * 127 + (128 - (32 + 8 * 127) % 128) % 128
+    assert lib.moe_slots_capacity(16, 8, 2) % 128 == 0
+    assert lib.moe_slots_capacity(4, 2, 3) == 0              # k > E
+    ws = lib.moe_workspace_size(4096, 4096, 14336, 8, 2, 1)
+    slots = lib.moe_slots_capacity(4096, 8, 2)
+    assert ws >= slots * (4096 * 2 + 14336 * 2 + 4096 * 4)
+    assert lib.moe_workspace_size(4096, 4096, 14336, 8, 2, 7) == 0
+
+
+def test_forward_ws_checks(lib):
+    f = lib.moe_forward_ws
+    f.restype = ctypes.c_int
+    args = [_vp(), _vp(), _vp(), _vp(), _vp(), _vp(), 8, 128, 256, 8, 2]
+    assert f(*args, 1, 5, _vp(0x10000), ctypes.c_size_t(1 << 30), None) == 1    # unknown path
+    assert f(*args, 0, 2, _vp(0x10000), ctypes.c_size_t(1 << 30), None) == 2    # decode path is bf16 only
+    assert f(*args, 1, 0, None, ctypes.c_size_t(1 << 30), None) == 5            # no workspace
+    assert f(*args, 1, 0, _vp(0x10000), ctypes.c_size_t(16), None) == 5         # too small
+
+
+def test_status_strings(lib):
+    lib.moe_status_string.restype = ctypes.c_char_p
+    for code in range(7):
+        assert lib.moe_status_string(code)
+    assert lib.moe_status_string(4) == b"device wait timed out"
+
+
+def test_selftest_rejects_bad_limit(lib):
+    f = lib.moe_selftest_wait_timeout
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_longlong, ctypes.c_void_p]
+    assert f(10, None) == 1
+    assert f(10 ** 12, None) == 1

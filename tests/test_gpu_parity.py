@@ -1,0 +1,223 @@
+"""CUDA path against the fp64 oracle, through the C ABI (sm_100a, B200).
+
+Small shapes compare every output element; the full-size workloads compare
+sampled tokens (the oracle evaluates them one by one) in the same launch
+configuration the bench times.  Rules are in moe_testlib.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+from moe_testlib import compare_outputs, compare_routing, out_to_f64, sample_tokens, upload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import sparse_mixture_experts_14_b200 as m
+    return m
+
+
+def _status_clear(moe):
+    assert moe.moe_get_device_status() == moe.MOE_OK
+
+
+# ---------------------------------------------------------------- routing
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 256), ("f32", 128)])
+@pytest.mark.parametrize("E,k", [(1, 1), (3, 2), (8, 1), (8, 2), (8, 8), (16, 4), (32, 2)])
+def test_route_small(moe, dtype, d, E, k):
+    inp = moe_inputs.make_inputs(300, d, 128, E, k, dtype, seed=100 + E * 7 + k, weights=False)
+    x, Wg = upload(inp)[:2]
+    idx, w = moe.moe_route(x, Wg, k)
+    ref = oracle.route(inp.x, inp.Wg, k, dtype)
+    compare_routing(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    _status_clear(moe)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+def test_route_configs(moe, cfg):
+    inp = moe_inputs.make_config(cfg, weights=False)
+    x, Wg = upload(inp)[:2]
+    idx, w = moe.moe_route(x, Wg, inp.k)
+    ref = oracle.route(inp.x, inp.Wg, inp.k, inp.dtype)
+    keep = compare_routing(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    assert keep.mean() > 0.99
+    _status_clear(moe)
+
+
+def test_route_tie_break_lowest_index(moe):
+    # every score equal: the k lowest expert ids in ascending order, uniform gates
+    x = torch.randn(50, 128, device="cuda").to(torch.bfloat16)
+    Wg = torch.zeros(8, 128, device="cuda", dtype=torch.bfloat16)
+    idx, w = moe.moe_route(x, Wg, 3)
+    assert torch.equal(idx.cpu(), torch.tensor([[0, 1, 2]] * 50, dtype=torch.int32))
+    assert torch.allclose(w.cpu(), torch.full((50, 3), 1 / 3), atol=1e-7)
+
+
+# ---------------------------------------------------------------- dispatch
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (1000, 8, 2), (2500, 5, 3), (4097, 32, 4), (300, 1, 1)])
+def test_dispatch_stable_counting_sort(moe, T, E, k):
+    rng = np.random.default_rng(T + E)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    counts, offsets, perm, inv = moe.moe_dispatch(torch.from_numpy(idx).cuda(), E)
+    counts, offsets, perm, inv = (a.cpu().numpy() for a in (counts, offsets, perm, inv))
+    assert np.array_equal(counts, oracle.counts(idx, E))
+    seg = (counts + 127) // 128 * 128
+    assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(seg)]))
+    for e in range(E):
+        rows = perm[offsets[e]:offsets[e] + counts[e]]
+        toks = rows // k
+        assert np.all(idx.reshape(-1)[rows] == e)
+        assert np.all(np.diff(toks) > 0)                        # stable: token order kept
+        assert np.all(perm[offsets[e] + counts[e]:offsets[e + 1]] == -1)
+    assert np.array_equal(perm[inv.reshape(-1)], np.arange(T * k))   # inverse permutation
+    _status_clear(moe)
+
+
+def test_dispatch_bad_expert_id_is_reported(moe):
+    idx = torch.tensor([[0, 1], [2, 99], [3, 4]], dtype=torch.int32, device="cuda")
+    moe.moe_dispatch(idx, 8)
+    assert moe.moe_get_device_status() == moe.MOE_ERR_DEVICE
+    _status_clear(moe)                                          # cleared, context still usable
+    counts, _, _, _ = moe.moe_dispatch(idx.clamp(max=7), 8)
+    assert int(counts.sum()) == 6
+
+
+# ---------------------------------------------------------------- whole layer, small shapes
+
+SMALL_BF16 = [
+    (1, 128, 256, 8, 2),
+    (7, 128, 256, 4, 2),
+    (130, 128, 256, 8, 2),
+    (300, 256, 512, 8, 2),
+    (1000, 128, 256, 8, 2),
+    (257, 192, 384, 5, 3),
+    (64, 128, 128, 1, 1),
+    (100, 128, 256, 4, 4),
+    (333, 320, 256, 32, 2),
+]
+
+
+@pytest.mark.parametrize("T,d,F,E,k", SMALL_BF16)
+def test_forward_bf16_small(moe, T, d, F, E, k):
+    inp = moe_inputs.make_inputs(T, d, F, E, k, "bf16", seed=T + d + E)
+    dev = upload(inp)
+    out = moe.moe_forward(*dev, k)
+    _status_clear(moe)
+    ref = oracle.moe(*inp.arrays(), k=k, dtype="bf16")
+    idx, w = moe.moe_route(dev[0], dev[1], k)
+    keep = compare_routing(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    compare_outputs(out_to_f64(out), ref["out"], keep, "bf16")
+
+
+@pytest.mark.parametrize("T,d,F,E,k", [(64, 128, 256, 8, 2), (1, 4, 1, 1, 1), (37, 12, 20, 3, 2),
+                                       (200, 64, 100, 8, 8), (129, 132, 70, 6, 1)])
+def test_forward_f32_small(moe, T, d, F, E, k):
+    inp = moe_inputs.make_inputs(T, d, F, E, k, "f32", seed=T + d + F)
+    dev = upload(inp)
+    out = moe.moe_forward(*dev, k)
+    _status_clear(moe)
+    ref = oracle.moe(*inp.arrays(), k=k, dtype="f32")
+    idx, w = moe.moe_route(dev[0], dev[1], k)
+    keep = compare_routing(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    compare_outputs(out_to_f64(out), ref["out"], keep, "f32")
+
+
+def test_forward_zero_tokens(moe):
+    inp = moe_inputs.make_inputs(1, 128, 256, 4, 2, "bf16", seed=1)
+    dev = upload(inp)
+    x0 = dev[0][:0]
+    out = moe.moe_forward(x0, *dev[1:], 2)
+    assert out.shape == (0, 128)
+    _status_clear(moe)
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled tokens
+
+
+@pytest.mark.parametrize("cfg,n", [(1, 64), (2, 16), (3, 24), (4, 24), (5, 12)])
+def test_forward_configs(moe, cfg, n):
+    inp = moe_inputs.make_config(cfg)
+    dev = upload(inp)
+    out = moe.moe_forward(*dev, inp.k)
+    _status_clear(moe)
+    toks = sample_tokens(inp.T, n, seed=cfg) if cfg != 1 else None
+    ref = oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks)
+    sel = ref["tokens"]
+    idx, w = moe.moe_route(dev[0], dev[1], inp.k)
+    keep = compare_routing(idx.cpu().numpy()[sel], w.cpu().numpy()[sel], ref)
+    got = out_to_f64(out)[sel]
+    rel = compare_outputs(got, ref["out"], keep, inp.dtype)
+    print(f"config {cfg}: max|err|/RMS = {rel:.3e} over {keep.sum()} tokens")
+    del dev, out
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- invariants of the CUDA path
+
+
+@pytest.fixture(scope="module")
+def mid():
+    inp = moe_inputs.make_inputs(700, 256, 512, 8, 2, "bf16", seed=77)
+    return inp, upload(inp)
+
+
+def test_run_to_run_bitwise(moe, mid):
+    _, dev = mid
+    a = moe.moe_forward(*dev, 2)
+    b = moe.moe_forward(*dev, 2)
+    assert torch.equal(a, b)
+
+
+def test_token_permutation_equivariance(moe, mid):
+    _, dev = mid
+    out = moe.moe_forward(*dev, 2)
+    p = torch.randperm(dev[0].shape[0], generator=torch.Generator().manual_seed(0)).cuda()
+    out_p = moe.moe_forward(dev[0][p].contiguous(), *dev[1:], 2)
+    assert torch.equal(out_p, out[p])
+
+
+def test_expert_relabelling_invariance(moe, mid):
+    _, dev = mid
+    out = moe.moe_forward(*dev, 2)
+    r = torch.tensor([3, 7, 0, 5, 1, 6, 2, 4], device="cuda")
+    out_r = moe.moe_forward(dev[0], *[t[r].contiguous() for t in dev[1:]], 2)
+    assert torch.equal(out_r, out)
+
+
+def test_w2_scaling_by_two_is_exact(moe, mid):
+    _, dev = mid
+    out = moe.moe_forward(*dev, 2)
+    out2 = moe.moe_forward(*dev[:4], (dev[4].float() * 2).to(torch.bfloat16), 2)
+    assert torch.equal(out2, (out.float() * 2).to(torch.bfloat16))
+
+
+def test_workspace_entry_matches_pooled(moe, mid):
+    _, dev = mid
+    a = moe.moe_forward(*dev, 2)
+    b = moe.moe_forward_ws(*dev, 2, path=moe.MOE_PATH_PREFILL)
+    assert torch.equal(a, b)
+
+
+def test_host_entry_matches_device(moe, mid):
+    _, dev = mid
+    a = moe.moe_forward(*dev, 2)
+    x_host = dev[0].cpu().pin_memory()
+    b = moe.moe_forward_host(x_host, *dev[1:], 2)
+    assert torch.equal(a.cpu(), b)
+
+
+def test_wait_timeout_is_reported_not_hung(moe):
+    moe.moe_selftest_wait_timeout(2_000_000)          # 2 ms on a barrier nobody arrives at
+    assert moe.moe_get_device_status() == moe.MOE_ERR_TIMEOUT
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    x = torch.randn(8, 128, device="cuda").to(torch.bfloat16)   # context still usable
+    idx, _ = moe.moe_route(x, torch.randn(4, 128, device="cuda").to(torch.bfloat16), 2)
+    assert idx.shape == (8, 2)
