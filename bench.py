@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Throughput of the sparse MoE feed-forward layer on B200: tokens/s of whole layer calls.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+A step is one call of the whole layer (route, dispatch, gather, expert GEMMs,
+combine) over one batch of T tokens of the chosen workload, with inputs and
+weights already resident in HBM.  The timed region is K steps bracketed by a
+barrier and a device synchronise; times come from CUDA events on the stream
+the kernels run on, max over ranks.  With N > 1 (torchrun, one process per
+GPU) every rank runs an independent replica of the layer on its own batch:
+tokens are independent and the layer needs no exchange, so there is no
+collective on the data path ("replicas", weak scaling).
+
+One JSON line is printed by rank 0.  Besides the base keys it carries:
+  stages_ms     mean device time of each stage (events recorded between launches)
+  roofline      the dominant kernel: algorithmic bytes or FLOPs per launch over its
+                measured mean duration, against MEASURED_PEAKS.json
+  layer_roofline  the whole layer against max(FLOPs / tensor peak, bytes / HBM)
+  e2e           the same metric through moe_forward_host: x copied from pinned host
+                memory and out copied back inside every timed step (wall clock)
+  cpu_baseline  the fp64 CPU oracle on the host cores, on a bounded token sample
+  clocks        NVML samples taken during the timed region
+--impl reference times the fp64 CPU oracle (there is no other implementation
+of this layer to run) on the same workload and prints the same line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from datetime import timedelta
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec at 1 B200; achieved % of roofline (tensor TFLOPS or HBM GB/s)"
+L2_BYTES = 126 * 1000 * 1000
+DEFAULT_CONFIG = 2   # the Mixtral-shape decode layer (T=16, d=4096, ffn=14336, E=8, k=2)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(moe_inputs.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            doc = json.load(f)
+        return {k: float(doc[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+           0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x10: "sync_boost",
+           0x1: "gpu_idle"}
+
+
+class ClockSampler:
+    """NVML samples of SM clock, throttle reasons and power every 10 ms while running."""
+
+    def __init__(self, device_index):
+        self.samples = []
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            handle = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                handle = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.h = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.err = str(e)
+
+    def _sample(self):
+        nv = self.nv
+        sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        power = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+        self.samples.append((sm, reasons, power))
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if not self.ok:
+            return None
+        self._sample()
+        self._stop.set()
+        self._thread.join()
+        sms = [s[0] for s in self.samples]
+        mask = 0
+        for s in self.samples:
+            mask |= int(s[1])
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in sorted(REASONS.items()) if mask & b and n != "gpu_idle"],
+                "samples": len(sms), "power_w_max": round(max(s[2] for s in self.samples), 1)}
+
+
+# ------------------------------------------------------------------ work accounting
+
+
+def accounting(inp, counts):
+    """Algorithmic FLOPs and bytes of the layer and of each expert GEMM (padding rows excluded)."""
+    T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
+    es = 2 if inp.dtype == "bf16" else 4
+    touched = int((np.asarray(counts) > 0).sum())
+    kT = k * T
+    return {
+        "touched": touched,
+        "layer_flops": 2.0 * T * d * E + 6.0 * kT * d * F,
+        "layer_bytes": touched * 3.0 * d * F * es + 2.0 * T * d * es + E * d * es,
+        "expert1_flops": 4.0 * kT * d * F,
+        "expert1_bytes": touched * 2.0 * F * d * es + kT * d * es + kT * F * es,
+        "expert2_flops": 2.0 * kT * d * F,
+        "expert2_bytes": touched * 1.0 * d * F * es + kT * F * es + kT * d * 4.0,
+    }
+
+
+def source_sha(files):
+    h = hashlib.sha1()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(kernel, workload):
+    """dram read+write bytes per launch from a committed ncu capture, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        doc = json.load(f)
+    ent = doc.get(f"{kernel}@{workload}")
+    if not ent:
+        return None
+    if ent.get("source_sha") != source_sha(ent.get("sources", [])):
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+
+def cpu_oracle_run(inp, target_s, threads):
+    """Time the fp64 oracle on a token sample sized for about target_s seconds; returns (tokens/s, sample text)."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=[0], nthreads=1)
+    per_tok = max(time.perf_counter() - t0, 1e-5)
+    n = int(max(1, min(inp.T, round(target_s * threads / per_tok))))
+    toks = np.unique(np.linspace(0, inp.T - 1, n).astype(np.int32))
+    reps = max(1, int(target_s * threads / (per_tok * len(toks)))) if len(toks) == inp.T else 1
+    reps = min(reps, 50)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=threads)
+    dt = time.perf_counter() - t0
+    sample = (f"{len(toks)} of {inp.T} tokens (evenly spaced), x{reps}, full layer per token "
+              f"(routing over all E, k SwiGLU experts, weighted sum) in fp64")
+    return reps * len(toks) / dt, sample, dt
+
+
+# ------------------------------------------------------------------ reference arm
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    c = moe_inputs.CONFIGS[args.config]
+    inp = moe_inputs.make_config(args.config)
+    threads = len(os.sched_getaffinity(0))
+    total_steps = args.steps + args.warmup
+    per_step = max(0.5, min(30.0, 150.0 / max(total_steps, 1)))
+    import oracle
+    t0 = time.perf_counter()
+    oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=[0], nthreads=1)
+    per_tok = max(time.perf_counter() - t0, 1e-5)
+    n = int(max(1, min(inp.T, round(per_step * threads / per_tok))))
+    toks = np.unique(np.linspace(0, inp.T - 1, n).astype(np.int32))
+    for _ in range(args.warmup):
+        oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=threads)
+    dt = time.perf_counter() - t0
+    value = args.steps * len(toks) / dt
+    sample = f"{len(toks)} of {inp.T} tokens per step (evenly spaced), fp64 oracle, {threads} threads"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": c["name"], "T": inp.T, "d": inp.d, "ffn": inp.F, "E": inp.E, "k": inp.k,
+                   "seed": c["seed"], "sample_tokens_per_step": int(len(toks))},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+
+def to_dev(a, dtype, device):
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def run_ours(args, rank, world, local):
+    import sparse_mixture_experts_14_b200 as moe
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    c = moe_inputs.CONFIGS[args.config]
+    inp = moe_inputs.make_config(args.config)
+    dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
+    tdt = dev[0].dtype
+    T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
+    code = moe.MOE_DTYPE_BF16 if inp.dtype == "bf16" else moe.MOE_DTYPE_F32
+    ws = torch.empty(moe.moe_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
+    out = torch.empty((T, d), dtype=tdt, device=device)
+
+    idx, _ = moe.moe_route(dev[0], dev[1], k)
+    counts = moe.moe_dispatch(idx, E)[0].cpu().numpy()
+    acc = accounting(inp, counts)
+    flush = acc["layer_bytes"] < 3 * L2_BYTES
+    flush_buf = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if flush else None
+
+    ns = moe.MOE_NUM_STAGES
+    K, W = args.steps, args.warmup
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(K)]
+    stream = torch.cuda.current_stream()
+    for row in events:          # create the CUDA events before the library records them
+        for e in row:
+            e.record(stream)
+    for _ in range(W):
+        moe.moe_forward_profiled(*dev, k, ws, out)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    launches = 0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(K):
+        if flush:
+            flush_buf.zero_()
+            events[i][0].record(stream)
+        launches += moe.moe_forward_profiled(*dev, k, ws, out, events=events[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    status = moe.moe_get_device_status()
+    if status != moe.MOE_OK:
+        raise RuntimeError(f"device fault during the timed region: {moe.moe_status_string(status)}")
+
+    if flush:
+        total_ms = sum(events[i][0].elapsed_time(events[i][ns]) for i in range(K))
+    else:
+        total_ms = start.elapsed_time(end)
+    stage_ms = [statistics.mean(events[i][s].elapsed_time(events[i][s + 1]) for i in range(K)) for s in range(ns)]
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    value = world * T * K / (total_ms / 1000.0)
+
+    # e2e: host buffers, copies inside every step
+    e2e = None
+    if not args.no_e2e:
+        x_host = dev[0].cpu().pin_memory() if inp.dtype == "bf16" else None
+        if x_host is not None:
+            out_host = torch.empty((T, d), dtype=tdt, pin_memory=True)
+            for _ in range(max(1, min(W, 3))):
+                moe.moe_forward_host(x_host, *dev[1:], k, out_host)
+            if world > 1:
+                torch.distributed.barrier()
+            t0 = time.perf_counter()
+            for _ in range(K):
+                moe.moe_forward_host(x_host, *dev[1:], k, out_host)
+            wall = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=device)
+            if world > 1:
+                torch.distributed.all_reduce(wall, op=torch.distributed.ReduceOp.MAX)
+            e2e = {"value": world * T * K / float(wall.item()), "unit": "tokens/s",
+                   "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
+                   "timing": "host wall clock around moe_forward_host (synchronises every step)"}
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    long_run = total_ms > 1000.0
+    tflops_peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
+    hbm = peaks["hbm_gbs"]
+    stages = dict(zip(moe.STAGE_NAMES, stage_ms))
+
+    layer_t_tensor = acc["layer_flops"] / (tflops_peak * 1e12)
+    layer_t_hbm = acc["layer_bytes"] / (hbm * 1e9)
+    layer_bound = "tensor" if layer_t_tensor >= layer_t_hbm else "hbm"
+    roof_tps = T / max(layer_t_tensor, layer_t_hbm)
+    layer_roof = {"bound": layer_bound, "roofline_tokens_per_s": roof_tps, "frac": (value / world) / roof_tps,
+                  "flops": acc["layer_flops"], "bytes": acc["layer_bytes"], "touched_experts": acc["touched"]}
+
+    dom = max(("expert1", "expert2"), key=lambda s: stages[s])
+    fl, by = acc[f"{dom}_flops"], acc[f"{dom}_bytes"]
+    sec = stages[dom] / 1000.0
+    if inp.dtype == "bf16" and fl / (tflops_peak * 1e12) >= by / (hbm * 1e9):
+        roof = {"bound": "tensor", "achieved": fl / sec / 1e12, "peak": tflops_peak, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    kname = {"expert1": "tc_gemm_kernel<true>", "expert2": "tc_gemm_kernel<false>"}[dom] if inp.dtype == "bf16" \
+        else {"expert1": "simt_gemm_kernel<true>", "expert2": "simt_gemm_kernel<false>"}[dom]
+    roof["traffic"] = recorded_traffic(kname, c["name"])
+    roof["kernel"] = kname
+    roof["per_launch"] = {"flops": fl, "bytes": by, "ms": stages[dom]}
+    roof["peak_source"] = f"{peak_src} ({'sustained' if long_run and roof['unit'] == 'TFLOP/s' else 'burst'})"
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        threads = len(os.sched_getaffinity(0))
+        v, sample, _ = cpu_oracle_run(inp, args.cpu_seconds, threads)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": inp.dtype, "data": "synthetic",
+        "config": {"workload": c["name"], "T": T, "d": d, "ffn": F, "E": E, "k": k, "seed": c["seed"],
+                   "routing": "zipf1.2-skewed" if c["skew"] else "near-uniform",
+                   "l2": "L2 flushed between steps" if flush else "touched weights larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "layer_roofline": layer_roof,
+        "stages_ms": stages,
+        "expert_counts": [int(v) for v in counts],
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -162,6 +162,30 @@ MOE_API moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1,
                           int dtype, int path, void* workspace, size_t workspace_bytes,
                           cudaStream_t stream);
 
+/* Stages of one layer call, in launch order (moe_forward_profiled). */
+enum {
+    MOE_STAGE_ROUTE = 0,    /* scores, top-k, gates */
+    MOE_STAGE_DISPATCH = 1, /* histogram, scan, stable scatter */
+    MOE_STAGE_GATHER = 2,   /* token rows into expert segments */
+    MOE_STAGE_EXPERT1 = 3,  /* W1/W3 GEMM with SwiGLU (or the decode pass over W1/W3) */
+    MOE_STAGE_EXPERT2 = 4,  /* W2 GEMM (or the decode pass over W2) */
+    MOE_STAGE_COMBINE = 5,  /* gate-weighted sum */
+    MOE_NUM_STAGES = 6
+};
+
+/*
+ * moe_forward_ws that also records stage_events[i] (cudaEvent_t, created by
+ * the caller with timing enabled, device-side only) on `stream` just before
+ * stage i is launched, and stage_events[MOE_NUM_STAGES] after the last stage,
+ * so cudaEventElapsedTime of consecutive events gives each stage's device
+ * time.  stage_events may be NULL.  If `launches` is not NULL it receives the
+ * number of kernels the call launched.
+ */
+MOE_API moe_status moe_forward_profiled(const void* x, const void* Wg, const void* W1, const void* W3,
+                                        const void* W2, void* out, int T, int d, int ffn, int E, int k,
+                                        int dtype, int path, void* workspace, size_t workspace_bytes,
+                                        cudaEvent_t* stage_events, int* launches, cudaStream_t stream);
+
 /*
  * End-to-end call from host memory: copies x_host [T][d] (host, bf16) to the
  * device, runs moe_forward with the device-resident weights (device), copies

@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_14_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python sparse_mixture_experts_14_b200/build.py` "
                       f"(or __graft_entry__.build())")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -30,6 +30,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT,
     MOE_ERR_DEVICE = range(7)
 MOE_PATH_AUTO, MOE_PATH_PREFILL, MOE_PATH_DECODE = 0, 1, 2
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
+MOE_NUM_STAGES = 6
+STAGE_NAMES = ("route", "dispatch", "gather", "expert1", "expert2", "combine")
 
 # every symbol include/moe.h declares, with its ctypes signature
 _vp, _ci, _sz, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
@@ -42,6 +44,8 @@ SIGNATURES = {
     "moe_forward_f32": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _vp]),
     "moe_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
     "moe_forward_ws": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _vp, _sz, _vp]),
+    "moe_forward_profiled": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _vp, _sz, _vp,
+                                   _vp, _vp]),
     "moe_forward_host": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _vp]),
     "moe_get_device_status": (_ci, [_vp]),
     "moe_selftest_wait_timeout": (_ci, [_ll, _vp]),
@@ -180,6 +184,23 @@ def moe_forward_ws(x, Wg, W1, W3, W2, k, path=MOE_PATH_AUTO, workspace=None, out
     _check(_lib.moe_forward_ws(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, code,
                                path, _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward_ws")
     return out
+
+
+def moe_forward_profiled(x, Wg, W1, W3, W2, k, workspace, out, events=None, path=MOE_PATH_AUTO, stream=None):
+    """moe_forward_ws recording torch.cuda.Event objects (MOE_NUM_STAGES + 1 of them, timing enabled)
+    at the stage boundaries; returns the number of kernels launched."""
+    code = _dtype_code(x)
+    T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
+    ev_arr = None
+    if events is not None:
+        if len(events) != MOE_NUM_STAGES + 1:
+            raise ValueError(f"need {MOE_NUM_STAGES + 1} events")
+        ev_arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    n = ctypes.c_int(0)
+    _check(_lib.moe_forward_profiled(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, code,
+                                     path, _ptr(workspace), workspace.numel(), ev_arr, ctypes.byref(n),
+                                     _stream(stream)), "moe_forward_profiled")
+    return n.value
 
 
 def moe_forward_host(x_host, Wg, W1, W3, W2, k, out_host=None, stream=None):

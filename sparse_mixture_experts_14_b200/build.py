@@ -1,6 +1,9 @@
 """Build libmoe.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m sparse_mixture_experts_14_b200.build [--force]
+    python sparse_mixture_experts_14_b200/build.py [--force] [-v]
+
+(Run it as a script or load it by file path: importing it as a submodule
+would first import the package, which loads the library being rebuilt.)
 
 Each csrc/*.cu compiles to an object under _build/ (parallel nvcc
 processes); the objects link into sparse_mixture_experts_14_b200/libmoe.so.

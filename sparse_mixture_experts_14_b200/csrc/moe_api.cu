@@ -148,7 +148,7 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 
 moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2, void* out, int T,
                      int d, int F, int E, int k, int dtype, int path, uint8_t* ws, const DeviceState& dev,
-                     cudaStream_t s) {
+                     cudaStream_t s, cudaEvent_t* ev = nullptr, int* launches = nullptr) {
     const Plan p = make_plan(T, d, F, E, k, dtype);
     int32_t* idx = reinterpret_cast<int32_t*>(ws + p.idx);
     float* w = reinterpret_cast<float*>(ws + p.w);
@@ -160,28 +160,45 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
     void* h = ws + p.h;
     float* y = reinterpret_cast<float*>(ws + p.y);
 
+    auto mark = [&](int stage) -> cudaError_t { return ev ? cudaEventRecord(ev[stage], s) : cudaSuccess; };
+    int n = 0;
+    MOE_TRY(mark(MOE_STAGE_ROUTE));
     if (dtype == MOE_DTYPE_BF16) {
         MOE_TRY(launch_router_bf16(x, Wg, T, d, E, k, idx, w, dev.num_sms, s));
     } else {
         MOE_TRY(launch_router_f32(static_cast<const float*>(x), static_cast<const float*>(Wg), T, d, E, k, idx, w,
                                   dev.num_sms, s));
     }
+    n += 1;
+    MOE_TRY(mark(MOE_STAGE_DISPATCH));
     MOE_TRY(launch_dispatch(idx, T, E, k, blk, meta, perm, inv, dev.status, s));
+    n += 3;
+    MOE_TRY(mark(MOE_STAGE_GATHER));
     MOE_TRY(launch_gather(x, dtype == MOE_DTYPE_BF16 ? 2 : 4, T, d, E, k, meta, perm, xp, p.slots, s));
+    n += 1;
     if (dtype == MOE_DTYPE_BF16) {
         TcGemmArgs a{xp, W1, W3, W2, h, y, meta, E, d, F, p.slots, dev.num_sms, dev.status, wait_limit_ns()};
         (void)path;
+        MOE_TRY(mark(MOE_STAGE_EXPERT1));
         MOE_TRY(launch_tc_gemm1(a, s));
+        MOE_TRY(mark(MOE_STAGE_EXPERT2));
         MOE_TRY(launch_tc_gemm2(a, s));
+        MOE_TRY(mark(MOE_STAGE_COMBINE));
         MOE_TRY(launch_combine_bf16(y, w, inv, T, d, k, out, s));
     } else {
+        MOE_TRY(mark(MOE_STAGE_EXPERT1));
         MOE_TRY(launch_simt_gemm1_f32(static_cast<const float*>(xp), static_cast<const float*>(W1),
                                       static_cast<const float*>(W3), meta, E, d, F, static_cast<float*>(h), p.slots,
                                       s));
+        MOE_TRY(mark(MOE_STAGE_EXPERT2));
         MOE_TRY(launch_simt_gemm2_f32(static_cast<const float*>(h), static_cast<const float*>(W2), meta, E, d, F, y,
                                       p.slots, s));
+        MOE_TRY(mark(MOE_STAGE_COMBINE));
         MOE_TRY(launch_combine_f32(y, w, inv, T, d, k, static_cast<float*>(out), s));
     }
+    n += 3;
+    MOE_TRY(mark(MOE_NUM_STAGES));
+    if (launches) *launches = n;
     return MOE_OK;
 }
 
@@ -307,6 +324,24 @@ moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1, const v
     if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
     return run_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
                      stream);
+}
+
+moe_status moe_forward_profiled(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2,
+                                void* out, int T, int d, int ffn, int E, int k, int dtype, int path, void* workspace,
+                                size_t workspace_bytes, cudaEvent_t* stage_events, int* launches,
+                                cudaStream_t stream) {
+    if (launches) *launches = 0;
+    moe_status st = check_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype);
+    if (st != MOE_OK) return st;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE) return MOE_ERR_INVALID_ARG;
+    if (path == MOE_PATH_DECODE && dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
+    DeviceState dev;
+    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    return run_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
+                     stream, stage_events, launches);
 }
 
 moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3, const void* W2,

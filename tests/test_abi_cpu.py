@@ -12,8 +12,8 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 
 @pytest.fixture(scope="module")
 def lib():
-    from sparse_mixture_experts_14_b200 import build
-    path = build.build()
+    import __graft_entry__
+    path = __graft_entry__._builder().build()
     return ctypes.CDLL(path)
 
 
