@@ -357,8 +357,12 @@ def run_ours(args, rank, world, local):
     else:
         roof = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": hbm, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    kname = {"expert1": "tc_gemm_kernel<true>", "expert2": "tc_gemm_kernel<false>"}[dom] if inp.dtype == "bf16" \
-        else {"expert1": "simt_gemm_kernel<true>", "expert2": "simt_gemm_kernel<false>"}[dom]
+    if inp.dtype != "bf16":
+        kname = {"expert1": "simt_gemm_kernel<true>", "expert2": "simt_gemm_kernel<false>"}[dom]
+    elif T <= moe.moe_decode_max_tokens():
+        kname = {"expert1": "decode_kernel<true>", "expert2": "decode_kernel<false>"}[dom]
+    else:
+        kname = {"expert1": "tc_gemm_kernel<true>", "expert2": "tc_gemm_kernel<false>"}[dom]
     roof["traffic"] = recorded_traffic(kname, c["name"])
     roof["kernel"] = kname
     roof["per_launch"] = {"flops": fl, "bytes": by, "ms": stages[dom]}

@@ -84,9 +84,10 @@ typedef enum {
 
 /* path selection for moe_forward_ws */
 enum {
-    MOE_PATH_AUTO = 0,    /* decode path for small T, grouped-GEMM path otherwise */
-    MOE_PATH_PREFILL = 1, /* gather + tensor-core grouped GEMMs */
-    MOE_PATH_DECODE = 2   /* expert-weight streaming (bfloat16 only) */
+    MOE_PATH_AUTO = 0,    /* decode path when T <= moe_decode_max_tokens(), else grouped GEMMs */
+    MOE_PATH_PREFILL = 1, /* gather + tensor-core grouped GEMMs (CTA pairs, 256-row tiles) */
+    MOE_PATH_DECODE = 2   /* expert-weight streaming, weights as the MMA's M side
+                             (bfloat16 only, T <= moe_decode_max_tokens()) */
 };
 
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };

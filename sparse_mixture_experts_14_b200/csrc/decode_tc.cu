@@ -1,0 +1,339 @@
+// Decode path (few tokens): expert-weight streaming on the tensor cores.
+//
+// Same mathematics as the grouped GEMMs (subsection "各エキスパートの構造" of the
+// "Mistral/Mixtral architecture" page, E_i(x) = W2_i (SiLU(W1_i x) * W3_i x)),
+// arranged for the case where each expert sees a handful of tokens and the
+// cost is reading its weights once from HBM: the weights are the M side of
+// the MMA and the tokens the N side ("swap AB"),
+//     stage 1   D1 = W1_e[f0:f0+128] Xp_e^T,  D3 = W3_e[f0:f0+128] Xp_e^T,
+//               H[slot][f] = SiLU(D1[f][t]) * D3[f][t]          (bf16)
+//     stage 2   D  = W2_e[r0:r0+128] H_e^T,   Y[slot][r] = D[r][t]  (fp32)
+// Only experts with at least one token are read (a page section "推論効率の
+// 観点" point: a small batch touches few experts).  N = the expert's token
+// count rounded up to 16 (at most 64), set per tile in the MMA instruction
+// descriptor; TMA streams 128-row x 64-column weight boxes through a 5-stage
+// ring (160 KiB of weights in flight per SM) with an evict-first L2 policy,
+// since every weight byte is used once.
+//
+// One CTA per SM, 6 warps: warp 0 TMA producer, warp 1 MMA issuer + TMEM
+// owner (256 columns: two accumulator sets of 2 x 64), warps 2-5 epilogue
+// (thread = weight row; for each token the warp's 32 lanes store 32
+// consecutive H or Y elements).
+#include <cuda.h>
+
+#include "moe_common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int DM = 128;                     // weight rows per tile (MMA M)
+constexpr int DK = 64;                      // K per stage
+constexpr int DNMAX = 64;                   // tokens per expert on this path (MMA N <= 64)
+constexpr int DSTAGES = 5;
+constexpr int W_BYTES = DM * DK * 2;        // 16 KiB
+constexpr int X_BYTES = DNMAX * DK * 2;     // 8 KiB
+constexpr int DSTAGE_BYTES = 2 * W_BYTES + X_BYTES;
+constexpr int DTMEM_COLS = 256;
+constexpr int DTHREADS = 192;
+
+struct DCtrl {
+    uint64_t full[DSTAGES];
+    uint64_t empty[DSTAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int total;
+    int tile_base[kMaxExperts + 1];
+    int ntok[kMaxExperts];
+    int row0[kMaxExperts];
+};
+
+constexpr int DSMEM_BYTES = DSTAGES * DSTAGE_BYTES + (int)sizeof(DCtrl) + 1024;
+
+// GATE: stage 1 (mapWa = W1, mapWb = W3, mapX = Xp, out = H bf16 [slots][R]).
+// !GATE: stage 2 (mapWa = W2, mapX = H, out = Y fp32 [slots][R]).
+// R = weight rows per expert (F in stage 1, d in stage 2), K = reduction length.
+template <bool GATE>
+__global__ void __launch_bounds__(DTHREADS, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap mapWa, const __grid_constant__ CUtensorMap mapWb,
+                  const __grid_constant__ CUtensorMap mapX, const Meta* __restrict__ meta, int E, int K, int R,
+                  void* __restrict__ out, int* status, long long wait_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    DCtrl* ctrl = reinterpret_cast<DCtrl*>(smem + DSTAGES * DSTAGE_BYTES);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    constexpr uint32_t STAGE_TX = GATE ? (uint32_t)DSTAGE_BYTES : (uint32_t)(W_BYTES + X_BYTES);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < DSTAGES; ++s) {
+            ptx::mbar_init(&ctrl->full[s], 1);
+            ptx::mbar_init(&ctrl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&ctrl->tfull[b], 1);
+            ptx::mbar_init(&ctrl->tempty[b], 4);
+        }
+        ptx::mbar_init(&ctrl->drain, 1);
+        ctrl->abort = 0;
+        const int blocks = (R + DM - 1) / DM;
+        ctrl->tile_base[0] = 0;
+        bool ok = true;
+        for (int e = 0; e < E; ++e) {
+            const int n = meta->counts[e];
+            if (n < 0 || n > DNMAX) ok = false;
+            ctrl->ntok[e] = n;
+            ctrl->row0[e] = meta->offsets[e];
+            ctrl->tile_base[e + 1] = ctrl->tile_base[e] + (n > 0 ? blocks : 0);
+        }
+        ctrl->total = ok ? ctrl->tile_base[E] : 0;
+        if (!ok) record_status(status, MOE_ERR_DEVICE);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::tma_prefetch_desc(&mapWa);
+        if (GATE) ptx::tma_prefetch_desc(&mapWb);
+        ptx::tma_prefetch_desc(&mapX);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&ctrl->tmem_base, DTMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+
+    const uint32_t tmem_base = ctrl->tmem_base;
+    const int total = ctrl->total;
+    const int nk = (K + DK - 1) / DK;
+    const ptx::WaitCtl wc{&ctrl->abort, status, (uint64_t)wait_ns};
+
+    auto decode_tile = [&](int tile, int& e, int& blk) {
+        e = 0;
+        while (tile >= ctrl->tile_base[e + 1]) ++e;
+        blk = tile - ctrl->tile_base[e];
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_w = ptx::policy_evict_first();
+            const uint64_t pol_x = ptx::policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool armed[DSTAGES];
+            uint32_t armed_phase[DSTAGES];
+#pragma unroll
+            for (int s = 0; s < DSTAGES; ++s) {
+                armed[s] = false;
+                armed_phase[s] = 0;
+            }
+            bool aborted = false;
+            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+                int e, blk;
+                decode_tile(tile, e, blk);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!ptx::mbar_wait(&ctrl->empty[stage], phase ^ 1u, wc)) {
+                        aborted = true;
+                        break;
+                    }
+                    uint8_t* sw = smem + stage * DSTAGE_BYTES;
+                    ptx::mbar_arrive_expect_tx(&ctrl->full[stage], STAGE_TX);
+                    ptx::tma_load_3d(sw, &mapWa, &ctrl->full[stage], kb * DK, blk * DM, e, pol_w);
+                    if (GATE) ptx::tma_load_3d(sw + W_BYTES, &mapWb, &ctrl->full[stage], kb * DK, blk * DM, e, pol_w);
+                    ptx::tma_load_2d(sw + 2 * W_BYTES, &mapX, &ctrl->full[stage], kb * DK, ctrl->row0[e], pol_x);
+#pragma unroll
+                    for (int s = 0; s < DSTAGES; ++s)
+                        if (s == stage) {
+                            armed[s] = true;
+                            armed_phase[s] = phase;
+                        }
+                    if (++stage == DSTAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (aborted || ctrl->abort) {
+#pragma unroll
+                for (int s = 0; s < DSTAGES; ++s)
+                    if (armed[s]) ptx::mbar_wait_drain(&ctrl->full[s], armed_phase[s], 100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool issued = false, aborted = false;
+            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+                int e, blk;
+                decode_tile(tile, e, blk);
+                const int nn = (ctrl->ntok[e] + 15) / 16 * 16;
+                const uint32_t idesc = ptx::idesc_bf16_f32(DM, nn);
+                if (!ptx::mbar_wait(&ctrl->tempty[acc], acc_phase ^ 1u, wc)) {
+                    aborted = true;
+                    break;
+                }
+                ptx::tc_fence_after_sync();
+                const uint32_t d1 = tmem_base + (uint32_t)(acc * 128);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!ptx::mbar_wait(&ctrl->full[stage], phase, wc)) {
+                        aborted = true;
+                        break;
+                    }
+                    ptx::tc_fence_after_sync();
+                    const uint32_t w0 = ptx::smem_addr(smem + stage * DSTAGE_BYTES);
+                    const uint32_t x0 = w0 + 2 * W_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint64_t bx = ptx::desc_kmajor_sw128(x0 + kk * 32);
+                        ptx::tc_mma_bf16(d1, ptx::desc_kmajor_sw128(w0 + kk * 32), bx, idesc, (kb | kk) != 0);
+                        if (GATE)
+                            ptx::tc_mma_bf16(d1 + 64, ptx::desc_kmajor_sw128(w0 + W_BYTES + kk * 32), bx, idesc,
+                                             (kb | kk) != 0);
+                    }
+                    ptx::tc_commit(&ctrl->empty[stage]);
+                    issued = true;
+                    if (++stage == DSTAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (aborted) break;
+                ptx::tc_commit(&ctrl->tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if ((aborted || ctrl->abort) && issued) {
+                ptx::tc_commit(&ctrl->drain);
+                ptx::mbar_wait_drain(&ctrl->drain, 0, 100000000ull);
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            int e, blk;
+            decode_tile(tile, e, blk);
+            const int n = ctrl->ntok[e];
+            bool ok = ptx::mbar_wait(&ctrl->tfull[acc], acc_phase, wc);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
+            const int r = blk * DM + q * 32 + lane;      // weight row = output column
+            const size_t row0 = (size_t)ctrl->row0[e];
+            const uint32_t taddr = tmem_base + (uint32_t)(acc * 128) + ((uint32_t)(q * 32) << 16);
+            for (int t0 = 0; t0 < n; t0 += 16) {
+                uint32_t a[16];
+                ptx::tmem_ld_32x32b_x16(taddr + t0, a);
+                if (GATE) {
+                    uint32_t b[16];
+                    ptx::tmem_ld_32x32b_x16(taddr + 64 + t0, b);
+                    ptx::tmem_ld_wait();
+                    __nv_bfloat16* H = static_cast<__nv_bfloat16*>(out);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (t0 + i < n && r < R)
+                            H[(row0 + t0 + i) * (size_t)R + r] =
+                                __float2bfloat16_rn(silu_mul(__uint_as_float(a[i]), __uint_as_float(b[i])));
+                    }
+                } else {
+                    ptx::tmem_ld_wait();
+                    float* Y = static_cast<float*>(out);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (t0 + i < n && r < R) Y[(row0 + t0 + i) * (size_t)R + r] = __uint_as_float(a[i]);
+                    }
+                }
+            }
+            ptx::tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ctrl->tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after_sync();
+        ptx::tmem_dealloc(tmem_base, DTMEM_COLS);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// E x R x K weights, K contiguous, box 64 x 128 x 1
+bool map_w(CUtensorMap* m, const void* base, int E, int R, int K) {
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)R, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)R * K * 2};
+    cuuint32_t box[3] = {(cuuint32_t)DK, (cuuint32_t)DM, 1};
+    return encode(m, base, 3, dims, strides, box);
+}
+
+// rows x K token matrix, box 64 x 64
+bool map_x(CUtensorMap* m, const void* base, size_t rows, int K) {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)DK, (cuuint32_t)DNMAX};
+    return encode(m, base, 2, dims, strides, box);
+}
+
+template <bool GATE>
+cudaError_t launch_stage(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& x, const TcGemmArgs& g, int K,
+                         int R, void* out, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e =
+            cudaFuncSetAttribute(decode_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, DSMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    int grid = g.num_sms > 0 ? g.num_sms : 148;
+    const int upper = g.E * ((R + DM - 1) / DM);
+    if (grid > upper) grid = upper;
+    if (grid < 1) grid = 1;
+    decode_kernel<GATE><<<grid, DTHREADS, DSMEM_BYTES, s>>>(a, b, x, g.meta, g.E, K, R, out, g.status, g.wait_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const TcGemmArgs& g, int stage, cudaStream_t s) {
+    if (stage == 1) {
+        CUtensorMap w1, w3, xp;
+        if (!map_w(&w1, g.W1, g.E, g.F, g.d) || !map_w(&w3, g.W3, g.E, g.F, g.d) || !map_x(&xp, g.xp, g.slots, g.d))
+            return cudaErrorInvalidValue;
+        return launch_stage<true>(w1, w3, xp, g, g.d, g.F, g.H, s);
+    }
+    CUtensorMap w2, h;
+    if (!map_w(&w2, g.W2, g.E, g.d, g.F) || !map_x(&h, g.H, g.slots, g.F)) return cudaErrorInvalidValue;
+    return launch_stage<false>(w2, w2, h, g, g.F, g.d, g.Y, s);
+}
+
+}  // namespace moe

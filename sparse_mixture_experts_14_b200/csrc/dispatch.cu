@@ -9,9 +9,10 @@
 // so rows inside a segment follow token order.  Segments are padded to 128
 // rows (one tensor-core tile); padding rows carry perm = -1 and zero inputs.
 //
-// Kernels: histogram (per 1024-token block), scan (one block: totals, padded
-// offsets, per-block bases), scatter (per-block stable ranks by warp ballots),
-// gather (one warp per row, 16-byte copies).
+// Kernels: up to 1024 tokens, one block does it all; above that, histogram
+// (per 1024-token block), scan (one block: totals, padded offsets, per-block
+// bases) and scatter (per-block stable ranks by warp ballots).  Then gather
+// (one warp per row, 16-byte copies).
 #include "moe_common.cuh"
 
 namespace moe {
@@ -139,6 +140,82 @@ __global__ void __launch_bounds__(kDispatchTokens) scatter_kernel(const int32_t*
     }
 }
 
+// Whole dispatch in one block when every token fits one 1024-thread block:
+// histogram, padded offsets and stable ranks without global scratch.
+__global__ void __launch_bounds__(kDispatchTokens) dispatch_single_kernel(const int32_t* __restrict__ idx, int T,
+                                                                          int E, int k, Meta* __restrict__ meta,
+                                                                          int32_t* __restrict__ perm,
+                                                                          int32_t* __restrict__ inv, size_t slots,
+                                                                          int* status) {
+    __shared__ int wcnt[32][kMaxExperts + 1];
+    __shared__ int offs[kMaxExperts + 1];
+    __shared__ int tot[kMaxExperts];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = threadIdx.x;
+    uint32_t mask = 0;
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[(size_t)t * k + j];
+            if (e < 0 || e >= E || ((mask >> e) & 1u)) {
+                record_status(status, MOE_ERR_DEVICE);
+                continue;
+            }
+            mask |= 1u << e;
+        }
+    }
+    const uint32_t lt = (1u << lane) - 1u;
+    int rank[kMaxExperts];
+    for (int e = 0; e < E; ++e) {
+        const uint32_t bal = __ballot_sync(0xffffffffu, (mask >> e) & 1u);
+        rank[e] = __popc(bal & lt);
+        if (lane == 0) wcnt[warp][e] = __popc(bal);
+    }
+    __syncthreads();
+    if (threadIdx.x < E) {
+        const int e = threadIdx.x;
+        int run = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int c = wcnt[w][e];
+            wcnt[w][e] = run;
+            run += c;
+        }
+        tot[e] = run;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        offs[0] = 0;
+        for (int e = 0; e < E; ++e) offs[e + 1] = offs[e] + (tot[e] + kSegRows - 1) / kSegRows * kSegRows;
+        if ((size_t)offs[E] > slots) record_status(status, MOE_ERR_DEVICE);
+        for (int e = 0; e < E; ++e) meta->counts[e] = tot[e];
+        for (int e = 0; e <= E; ++e) meta->offsets[e] = offs[e];
+    }
+    __syncthreads();
+    if (t < T) {
+        uint32_t seen = 0;
+        for (int j = 0; j < k; ++j) {
+            const int a = t * k + j;
+            const int e = idx[a];
+            if (e < 0 || e >= E || ((seen >> e) & 1u)) {
+                inv[a] = -1;
+                continue;
+            }
+            seen |= 1u << e;
+            const int slot = offs[e] + wcnt[warp][e] + rank[e];
+            if ((size_t)slot >= slots) {
+                inv[a] = -1;
+                continue;
+            }
+            perm[slot] = a;
+            inv[a] = slot;
+        }
+    }
+    for (int e = 0; e < E; ++e) {
+        const int beg = offs[e] + tot[e], end = offs[e + 1];
+        for (int r = beg + threadIdx.x; r < end; r += blockDim.x)
+            if ((size_t)r < slots) perm[r] = -1;
+    }
+}
+
 // One warp per row of the padded buffer; rows past offsets[E] are left alone.
 __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ x, size_t row_bytes, int T, int k,
                                                      const Meta* __restrict__ meta, int E,
@@ -169,6 +246,10 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* bl
                             int32_t* inv, int* status, cudaStream_t s) {
     const int NB = dispatch_blocks(T);
     const size_t slots = slots_capacity(T, E, k);
+    if (NB == 1) {
+        dispatch_single_kernel<<<1, kDispatchTokens, 0, s>>>(idx, T, E, k, meta, perm, inv, slots, status);
+        return cudaGetLastError();
+    }
     hist_kernel<<<NB, kDispatchTokens, 0, s>>>(idx, T, E, k, blk_counts, status);
     scan_kernel<<<1, 1024, 0, s>>>(blk_counts, NB, E, meta, perm, slots, status);
     scatter_kernel<<<NB, kDispatchTokens, 0, s>>>(idx, T, E, k, blk_counts, perm, inv, slots, status);

@@ -1,5 +1,5 @@
 // Tensor-core grouped GEMMs of the experts (bf16 in, fp32 accumulate in tensor
-// memory), sm_100a: tcgen05.mma fed by TMA, accumulators in TMEM.
+// memory), sm_100a: tcgen05.mma on CTA pairs, fed by TMA, accumulators in TMEM.
 //
 // Subsection "各エキスパートの構造" of the "Mistral/Mixtral architecture" page:
 //     E_i(x) = W2_i (SiLU(W1_i x) * W3_i x)
@@ -7,21 +7,31 @@
 //     GEMM1  acc = Xp_e [W1_e ; W3_e]^T,   H = SiLU(acc[:, :128]) * acc[:, 128:]  -> bf16
 //     GEMM2  Y   = H_e W2_e^T                                              -> fp32
 //
-// Tile: 128 rows x 256 accumulator columns x 64-deep K steps.  In GEMM1 the
-// 256 columns are 128 rows of W1_e followed by the same 128 rows of W3_e, so
-// one MMA of N = 256 yields both halves of the SwiGLU for a 128 x 128 block of
-// H, and the gating runs in the epilogue straight out of TMEM.
+// A cluster of two CTAs (one SM pair) computes a 256 x 256 accumulator tile
+// with tcgen05.mma.cta_group::2: each CTA holds 128 of the 256 rows (one
+// 128-row m-tile of the expert) and 128 of the 256 B rows, so each SM moves
+// 32 KiB of operands per 64-deep K step instead of 48 KiB for a 1-SM tile of
+// the same per-SM work.  In GEMM1 the leader's B half is a 128-row block of
+// W1_e and the peer's the same block of W3_e: the pair MMA gives each CTA
+// both halves of the SwiGLU for its rows, and the gating runs in the epilogue
+// straight out of TMEM.
 //
-// Persistent kernel, one CTA per SM, 6 warps:
-//   warp 0     TMA producer (one thread): A and B tiles into a 4-stage ring
-//   warp 1     MMA issuer (one thread) + TMEM owner (512 columns = two
-//              128 x 256 fp32 accumulators, so the epilogue of one tile
+// Persistent kernel, one CTA per SM, 6 warps per CTA:
+//   warp 0     TMA producer (one thread per CTA): own A rows and own B half
+//              into a 6-stage ring; completion bytes of both CTAs are counted
+//              on the leader's barrier
+//   warp 1     leader: MMA issuer (one thread); commits arrive on both CTAs'
+//              barriers (multicast).  Both CTAs: TMEM owner (512 columns =
+//              two 128 x 256 fp32 accumulators, so the epilogue of one tile
 //              overlaps the MMAs of the next)
-//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, gating / fp32
-//              stores
-// Tiles are (expert, n-block, m-block) with m fastest, so CTAs working at the
-// same time share one block of expert weights through L2.  The tile list is
-// derived on the device from the dispatch offsets: no host synchronisation.
+//   warps 2-5  epilogue of the CTA's own rows: tcgen05.ld of their 32-lane
+//              quarter, gating / fp32 stores; then one arrival per warp on the
+//              leader's "accumulator free" barrier
+// Pair tiles are (expert, n-block, m-tile pair) with pairs fastest, so the
+// CTAs at work share one block of expert weights through L2.  When an expert
+// has an odd number of m-tiles, the peer of its last pair computes rows past
+// the expert's segment and stores nothing.  The tile list is derived on the
+// device from the dispatch offsets: no host synchronisation.
 #include <cuda.h>
 
 #include "moe_common.cuh"
@@ -30,44 +40,47 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BK = 64;
-constexpr int BN = 256;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;          // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;          // 32 KiB
+constexpr int BM = 128;                        // rows per CTA (256 per pair)
+constexpr int BK = 64;                         // K per stage (one 128-byte swizzle row)
+constexpr int BN = 256;                        // accumulator columns of the pair MMA
+constexpr int BNH = BN / 2;                    // B rows held by each CTA
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;           // 16 KiB
+constexpr int B_BYTES = BNH * BK * 2;          // 16 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t PAIR_TX_BYTES = 2 * STAGE_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int NUM_THREADS = 192;
-constexpr int NUM_EPI_THREADS = 128;
-constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN);
+constexpr int NUM_EPI_WARPS = 4;
+constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BM, BN);
 
 struct Ctrl {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t full[STAGES];      // leader: both CTAs' bytes of a stage landed
+    uint64_t empty[STAGES];     // each CTA: the pair MMAs reading a stage are done
+    uint64_t tfull[2];          // each CTA: accumulator b holds a finished tile
+    uint64_t tempty[2];         // leader: both CTAs' epilogues released accumulator b
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
     int total;
     int tile_base[kMaxExperts + 1];
-    int mt[kMaxExperts];
+    int mt[kMaxExperts];        // 128-row m-tiles of expert e
+    int pt[kMaxExperts];        // pairs of m-tiles of expert e
     int row0[kMaxExperts];
 };
 
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + (int)sizeof(Ctrl) + 1024;
 
-__device__ __forceinline__ void decode_tile(const Ctrl* c, int tile, int& e, int& m_blk, int& n_blk) {
+__device__ __forceinline__ void decode_tile(const Ctrl* c, int tile, int& e, int& pair, int& n_blk) {
     e = 0;
     while (tile >= c->tile_base[e + 1]) ++e;
     const int local = tile - c->tile_base[e];
-    n_blk = local / c->mt[e];
-    m_blk = local - n_blk * c->mt[e];
+    n_blk = local / c->pt[e];
+    pair = local - n_blk * c->pt[e];
 }
 
-// SWIGLU: GEMM1 (B = W1/W3 row blocks of 128, out = H bf16 [slots][N]).
-// !SWIGLU: GEMM2 (B = W2 row block of 256, out = Y fp32 [slots][N]).
+// SWIGLU: GEMM1 (B halves = 128-row blocks of W1 and W3, out = H bf16 [slots][N]).
+// !SWIGLU: GEMM2 (B halves = the two 128-row halves of a 256-row W2 block, out = Y fp32 [slots][N]).
 template <bool SWIGLU>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB1,
@@ -78,7 +91,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    constexpr int N_PER_TILE = SWIGLU ? BN / 2 : BN;   // output columns per tile
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1;
+    const int nclusters = gridDim.x >> 1;
+    constexpr int N_PER_TILE = SWIGLU ? BNH : BN;   // output columns per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -87,7 +104,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&ctrl->tfull[b], 1);
-            ptx::mbar_init(&ctrl->tempty[b], NUM_EPI_THREADS);
+            ptx::mbar_init(&ctrl->tempty[b], 2 * NUM_EPI_WARPS);
         }
         ptx::mbar_init(&ctrl->drain, 1);
         ctrl->abort = 0;
@@ -99,8 +116,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (r1 < r0 || (r1 - r0) % BM != 0 || (size_t)r1 > slots) ok = false;
             const int mt = ok ? (r1 - r0) / BM : 0;
             ctrl->mt[e] = mt;
+            ctrl->pt[e] = (mt + 1) / 2;
             ctrl->row0[e] = r0;
-            ctrl->tile_base[e + 1] = ctrl->tile_base[e] + mt * ntn;
+            ctrl->tile_base[e + 1] = ctrl->tile_base[e] + ctrl->pt[e] * ntn;
         }
         ctrl->total = ok ? ctrl->tile_base[E] : 0;
         if (!ok) record_status(status, MOE_ERR_DEVICE);
@@ -112,11 +130,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (SWIGLU) ptx::tma_prefetch_desc(&mapB3);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
-        ptx::tmem_relinquish();
+        ptx::tmem_alloc_pair(&ctrl->tmem_base, TMEM_COLS);
+        ptx::tmem_relinquish_pair();
     }
     ptx::tc_fence_before_sync();
-    __syncthreads();
+    ptx::cluster_sync();
     ptx::tc_fence_after_sync();
 
     const uint32_t tmem_base = ctrl->tmem_base;
@@ -125,10 +143,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const ptx::WaitCtl wc{&ctrl->abort, status, (uint64_t)wait_ns};
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer
+        // ---------------------------------------------------------------- TMA producer (both CTAs)
         if (lane == 0) {
-            const uint64_t pol_act = ptx::policy_evict_last();
-            const uint64_t pol_w = ptx::policy_evict_first();
+            const uint64_t pol = ptx::policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
             bool armed[STAGES];
@@ -139,10 +156,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 armed_phase[s] = 0;
             }
             bool aborted = false;
-            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
-                int e, m_blk, n_blk;
-                decode_tile(ctrl, tile, e, m_blk, n_blk);
-                const int rowA = ctrl->row0[e] + m_blk * BM;
+            for (int tile = cluster; tile < total && !aborted; tile += nclusters) {
+                int e, pair, n_blk;
+                decode_tile(ctrl, tile, e, pair, n_blk);
+                const int rowA = ctrl->row0[e] + (2 * pair + (int)rank) * BM;
+                const CUtensorMap* mapB = (SWIGLU && !leader) ? &mapB3 : &mapB1;
+                const int rowB = SWIGLU ? n_blk * BNH : n_blk * BN + (int)rank * BNH;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!ptx::mbar_wait(&ctrl->empty[stage], phase ^ 1u, wc)) {
                         aborted = true;
@@ -150,15 +169,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     uint8_t* sa = smem + stage * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
-                    ptx::mbar_arrive_expect_tx(&ctrl->full[stage], STAGE_BYTES);
-                    ptx::tma_load_2d(sa, &mapA, &ctrl->full[stage], kb * BK, rowA, pol_act);
-                    if (SWIGLU) {
-                        ptx::tma_load_3d(sb, &mapB1, &ctrl->full[stage], kb * BK, n_blk * (BN / 2), e, pol_w);
-                        ptx::tma_load_3d(sb + B_BYTES / 2, &mapB3, &ctrl->full[stage], kb * BK, n_blk * (BN / 2), e,
-                                         pol_w);
-                    } else {
-                        ptx::tma_load_3d(sb, &mapB1, &ctrl->full[stage], kb * BK, n_blk * BN, e, pol_w);
-                    }
+                    const uint32_t full_leader = ptx::map_to_rank(ptx::smem_addr(&ctrl->full[stage]), 0);
+                    if (leader) ptx::mbar_arrive_expect_tx(&ctrl->full[stage], PAIR_TX_BYTES);
+                    ptx::tma_load_2d_pair(sa, &mapA, full_leader, kb * BK, rowA, pol);
+                    ptx::tma_load_3d_pair(sb, mapB, full_leader, kb * BK, rowB, e, pol);
 #pragma unroll
                     for (int s = 0; s < STAGES; ++s)
                         if (s == stage) {
@@ -171,22 +185,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             }
-            if (aborted || ctrl->abort) {
-                // let every copy still in flight land before the CTA's shared memory is released
+            if (leader && (aborted || ctrl->abort)) {
+                // let copies still in flight land before shared memory is released
 #pragma unroll
                 for (int s = 0; s < STAGES; ++s)
-                    if (armed[s]) ptx::mbar_wait_drain(&ctrl->full[s], armed_phase[s], 2000000000ull);
+                    if (armed[s]) ptx::mbar_wait_drain(&ctrl->full[s], armed_phase[s], 100000000ull);
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // ---------------------------------------------------------------- MMA issuer (leader)
+        if (lane == 0 && leader) {
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool issued = false, aborted = false;
-            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+            for (int tile = cluster; tile < total && !aborted; tile += nclusters) {
                 if (!ptx::mbar_wait(&ctrl->tempty[acc], acc_phase ^ 1u, wc)) {
                     aborted = true;
                     break;
@@ -203,10 +217,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        ptx::tc_mma_bf16(d_tmem, ptx::desc_kmajor_sw128(a0 + kk * 32),
-                                         ptx::desc_kmajor_sw128(b0 + kk * 32), IDESC, (kb | kk) != 0);
+                        ptx::tc_mma_bf16_pair(d_tmem, ptx::desc_kmajor_sw128(a0 + kk * 32),
+                                              ptx::desc_kmajor_sw128(b0 + kk * 32), IDESC, (kb | kk) != 0);
                     }
-                    ptx::tc_commit(&ctrl->empty[stage]);
+                    ptx::tc_commit_pair_multicast(&ctrl->empty[stage], 0x3);
                     issued = true;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -214,78 +228,85 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
                 if (aborted) break;
-                ptx::tc_commit(&ctrl->tfull[acc]);
+                ptx::tc_commit_pair_multicast(&ctrl->tfull[acc], 0x3);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             }
             if ((aborted || ctrl->abort) && issued) {
-                ptx::tc_commit(&ctrl->drain);
-                ptx::mbar_wait_drain(&ctrl->drain, 0, 2000000000ull);
+                ptx::tc_commit_pair(&ctrl->drain);
+                ptx::mbar_wait_drain(&ctrl->drain, 0, 100000000ull);
             }
         }
     } else {
-        // ---------------------------------------------------------------- epilogue
+        // ---------------------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;   // TMEM lane quarter this warp may access
+        const uint64_t pol_out = ptx::policy_evict_first();
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            int e, m_blk, n_blk;
-            decode_tile(ctrl, tile, e, m_blk, n_blk);
+        for (int tile = cluster; tile < total; tile += nclusters) {
+            int e, pair, n_blk;
+            decode_tile(ctrl, tile, e, pair, n_blk);
+            const int m_tile = 2 * pair + (int)rank;
             bool ok = ptx::mbar_wait(&ctrl->tfull[acc], acc_phase, wc);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             ptx::tc_fence_after_sync();
-            const size_t row = (size_t)ctrl->row0[e] + (size_t)m_blk * BM + q * 32 + lane;
-            const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-            if (SWIGLU) {
-                __nv_bfloat16* H = static_cast<__nv_bfloat16*>(out);
+            if (m_tile < ctrl->mt[e]) {
+                const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
+                const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+                if (SWIGLU) {
+                    __nv_bfloat16* H = static_cast<__nv_bfloat16*>(out);
 #pragma unroll 1
-                for (int c = 0; c < BN / 2; c += 32) {
-                    uint32_t ra[32], rb[32];
-                    ptx::tmem_ld_32x32b_x32(taddr + c, ra);
-                    ptx::tmem_ld_32x32b_x32(taddr + BN / 2 + c, rb);
-                    ptx::tmem_ld_wait();
-                    uint32_t hp[16];
+                    for (int c = 0; c < BNH; c += 32) {
+                        uint32_t ra[32], rb[32];
+                        ptx::tmem_ld_32x32b_x32(taddr + c, ra);
+                        ptx::tmem_ld_32x32b_x32(taddr + BNH + c, rb);
+                        ptx::tmem_ld_wait();
+                        uint32_t hp[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float h0 = silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i]));
-                        const float h1 = silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1]));
-                        hp[i] = pack_bf16x2(h0, h1);
+                        for (int i = 0; i < 16; ++i) {
+                            const float h0 = silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i]));
+                            const float h1 = silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1]));
+                            hp[i] = pack_bf16x2(h0, h1);
+                        }
+                        uint8_t* dst = reinterpret_cast<uint8_t*>(H + row * (size_t)N + n_blk * BNH + c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            ptx::st_global_v4_hint(dst + 16 * v, hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3],
+                                                   pol_out);
                     }
-                    const int col = n_blk * (BN / 2) + c;
-                    uint4* dst = reinterpret_cast<uint4*>(H + row * (size_t)N + col);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
-                }
-            } else {
-                float* Y = static_cast<float*>(out);
+                } else {
+                    float* Y = static_cast<float*>(out);
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t r[32];
-                    ptx::tmem_ld_32x32b_x32(taddr + c, r);
-                    ptx::tmem_ld_wait();
-                    const int col = n_blk * BN + c;
-                    if (col < N) {
-                        float4* dst = reinterpret_cast<float4*>(Y + row * (size_t)N + col);
+                    for (int c = 0; c < BN; c += 32) {
+                        uint32_t r[32];
+                        ptx::tmem_ld_32x32b_x32(taddr + c, r);
+                        ptx::tmem_ld_wait();
+                        const int col = n_blk * BN + c;
+                        if (col < N) {
+                            uint8_t* dst = reinterpret_cast<uint8_t*>(Y + row * (size_t)N + col);
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                                 __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                            for (int v = 0; v < 8; ++v)
+                                ptx::st_global_v4_hint(dst + 16 * v, r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3],
+                                                       pol_out);
+                        }
                     }
                 }
             }
             ptx::tc_fence_before_sync();
-            ptx::mbar_arrive(&ctrl->tempty[acc]);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&ctrl->tempty[acc]), 0));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
     }
 
     ptx::tc_fence_before_sync();
-    __syncthreads();
+    __syncwarp();
+    ptx::cluster_sync();
     if (warp == 1) {
         ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+        ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 
@@ -349,38 +370,79 @@ cudaError_t ensure_smem_attr() {
     return cudaSuccess;
 }
 
+// Persistent grid: as many CTA pairs as fit at once, no more than there are pair tiles.
+template <bool SWIGLU>
 int grid_for(size_t slots, int n_tiles_per_m, int num_sms) {
-    const size_t upper = (slots / BM) * (size_t)n_tiles_per_m;
-    int g = num_sms > 0 ? num_sms : 148;
-    if ((size_t)g > upper) g = (int)upper;
-    return g < 1 ? 1 : g;
+    static int max_clusters = -1;
+    if (max_clusters < 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * 74, 1, 1);
+        cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_kernel<SWIGLU>, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = (num_sms > 0 ? num_sms : 148) / 2;
+        }
+        max_clusters = n;
+    }
+    const size_t pair_rows = (slots / BM + 1) / 2;
+    const size_t upper = pair_rows * (size_t)n_tiles_per_m;
+    size_t clusters = (size_t)max_clusters;
+    if (clusters > upper) clusters = upper;
+    if (clusters < 1) clusters = 1;
+    return (int)(2 * clusters);
+}
+
+template <bool SWIGLU>
+cudaError_t launch_pair(int grid, const CUtensorMap& mA, const CUtensorMap& mB1, const CUtensorMap& mB3,
+                        const TcGemmArgs& a, int K, int N, void* out, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<SWIGLU>, mA, mB1, mB3, a.meta, a.E, K, N, a.slots, out, a.status,
+                              a.wait_ns);
 }
 
 }  // namespace
 
 cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s) {
     CUtensorMap mA, mB1, mB3;
-    if (!map_rows(&mA, a.xp, a.slots, a.d, BM) || !map_weights(&mB1, a.W1, a.E, a.F, a.d, BN / 2) ||
-        !map_weights(&mB3, a.W3, a.E, a.F, a.d, BN / 2))
+    if (!map_rows(&mA, a.xp, a.slots, a.d, BM) || !map_weights(&mB1, a.W1, a.E, a.F, a.d, BNH) ||
+        !map_weights(&mB3, a.W3, a.E, a.F, a.d, BNH))
         return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_attr<true>();
     if (e != cudaSuccess) return e;
-    const int grid = grid_for(a.slots, (a.F + BN / 2 - 1) / (BN / 2), a.num_sms);
-    tc_gemm_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB1, mB3, a.meta, a.E, a.d, a.F, a.slots, a.H,
-                                                               a.status, a.wait_ns);
-    return cudaGetLastError();
+    const int grid = grid_for<true>(a.slots, (a.F + BNH - 1) / BNH, a.num_sms);
+    e = launch_pair<true>(grid, mA, mB1, mB3, a, a.d, a.F, a.H, s);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s) {
     CUtensorMap mA, mB;
-    if (!map_rows(&mA, a.H, a.slots, a.F, BM) || !map_weights(&mB, a.W2, a.E, a.d, a.F, BN))
+    if (!map_rows(&mA, a.H, a.slots, a.F, BM) || !map_weights(&mB, a.W2, a.E, a.d, a.F, BNH))
         return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_attr<false>();
     if (e != cudaSuccess) return e;
-    const int grid = grid_for(a.slots, (a.d + BN - 1) / BN, a.num_sms);
-    tc_gemm_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mB, a.meta, a.E, a.F, a.d, a.slots, a.Y,
-                                                                a.status, a.wait_ns);
-    return cudaGetLastError();
+    const int grid = grid_for<false>(a.slots, (a.d + BN - 1) / BN, a.num_sms);
+    e = launch_pair<false>(grid, mA, mB, mB, a, a.F, a.d, a.Y, s);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -15,7 +15,6 @@ __device__ int g_status;   // per-device sticky fault word (first fault wins)
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kDecodeMaxTokens = 64;
 
 std::mutex g_mu;
 cudaMemPool_t g_pools[kMaxDevices] = {};
@@ -172,17 +171,17 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
     n += 1;
     MOE_TRY(mark(MOE_STAGE_DISPATCH));
     MOE_TRY(launch_dispatch(idx, T, E, k, blk, meta, perm, inv, dev.status, s));
-    n += 3;
+    n += dispatch_launches(T);
     MOE_TRY(mark(MOE_STAGE_GATHER));
     MOE_TRY(launch_gather(x, dtype == MOE_DTYPE_BF16 ? 2 : 4, T, d, E, k, meta, perm, xp, p.slots, s));
     n += 1;
     if (dtype == MOE_DTYPE_BF16) {
         TcGemmArgs a{xp, W1, W3, W2, h, y, meta, E, d, F, p.slots, dev.num_sms, dev.status, wait_limit_ns()};
-        (void)path;
+        const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxTokens);
         MOE_TRY(mark(MOE_STAGE_EXPERT1));
-        MOE_TRY(launch_tc_gemm1(a, s));
+        MOE_TRY(decode ? launch_decode(a, 1, s) : launch_tc_gemm1(a, s));
         MOE_TRY(mark(MOE_STAGE_EXPERT2));
-        MOE_TRY(launch_tc_gemm2(a, s));
+        MOE_TRY(decode ? launch_decode(a, 2, s) : launch_tc_gemm2(a, s));
         MOE_TRY(mark(MOE_STAGE_COMBINE));
         MOE_TRY(launch_combine_bf16(y, w, inv, T, d, k, out, s));
     } else {
@@ -316,7 +315,7 @@ moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1, const v
     moe_status st = check_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype);
     if (st != MOE_OK) return st;
     if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE) return MOE_ERR_INVALID_ARG;
-    if (path == MOE_PATH_DECODE && dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (path == MOE_PATH_DECODE && (dtype != MOE_DTYPE_BF16 || T > kDecodeMaxTokens)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
@@ -334,7 +333,7 @@ moe_status moe_forward_profiled(const void* x, const void* Wg, const void* W1, c
     moe_status st = check_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype);
     if (st != MOE_OK) return st;
     if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE) return MOE_ERR_INVALID_ARG;
-    if (path == MOE_PATH_DECODE && dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (path == MOE_PATH_DECODE && (dtype != MOE_DTYPE_BF16 || T > kDecodeMaxTokens)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;

@@ -61,6 +61,8 @@ cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int 
 cudaError_t launch_router_f32(const float* x, const float* Wg, int T, int d, int E, int k, int32_t* idx,
                               float* w, int num_sms, cudaStream_t s);
 
+// Launches 1 kernel when T <= kDispatchTokens, else 3.
+inline int dispatch_launches(int T) { return T <= kDispatchTokens ? 1 : 3; }
 cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* blk_counts, Meta* meta,
                             int32_t* perm, int32_t* inv, int* status, cudaStream_t s);
 cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
@@ -92,7 +94,9 @@ struct TcGemmArgs {
 };
 cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s);
 cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s);
-cudaError_t launch_decode(const TcGemmArgs& a, cudaStream_t s);
+// Decode path: stage 1 (W1/W3 -> H) or stage 2 (W2 -> Y); at most 64 tokens per expert.
+constexpr int kDecodeMaxTokens = 64;
+cudaError_t launch_decode(const TcGemmArgs& a, int stage, cudaStream_t s);
 
 cudaError_t launch_wait_selftest(int* status, long long limit_ns, cudaStream_t s);
 

@@ -3,11 +3,11 @@
 // "Mistral/Mixtral architecture" page (score, Top-2 and gate equations) and its
 // MoERouter.forward in "簡易MoEルーターの実装", fused into one pass over x.
 //
-// One warp owns TPW tokens.  Lanes stride over 16-byte chunks of the rows;
-// each Wg chunk loaded once is applied to all TPW tokens.  Partial sums are
-// reduced with a fixed xor-butterfly, so every lane ends with the same,
-// run-to-run identical fp32 scores.  Scores are never rounded to bf16.
-// The pass is bound by reading x once from HBM.
+// Large batches: one warp owns TPW tokens and each Wg chunk it loads serves
+// all of them.  Small batches: one block per token, its warps split the row.
+// Partial sums are reduced in a fixed order (xor-butterfly, then warp order),
+// so the fp32 scores are identical run to run for a given batch size; they
+// are never rounded to bf16.  The pass is bound by reading x once from HBM.
 #include "moe_common.cuh"
 
 namespace moe {
@@ -19,8 +19,12 @@ struct Chunk;
 template <>
 struct Chunk<__nv_bfloat16> {
     static constexpr int N = 8;
-    __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
-        uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    using Raw = uint4;
+    __device__ __forceinline__ static Raw load(const __nv_bfloat16* p) {
+        return __ldg(reinterpret_cast<const uint4*>(p));
+    }
+    __device__ __forceinline__ static Raw zero() { return make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ static void widen(const Raw& u, float (&v)[8]) {
         v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
         v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
         v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z);
@@ -31,8 +35,10 @@ struct Chunk<__nv_bfloat16> {
 template <>
 struct Chunk<float> {
     static constexpr int N = 4;
-    __device__ __forceinline__ static void load(const float* p, float (&v)[4]) {
-        float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    using Raw = float4;
+    __device__ __forceinline__ static Raw load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+    __device__ __forceinline__ static Raw zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ static void widen(const Raw& u, float (&v)[4]) {
         v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
     }
 };
@@ -64,10 +70,38 @@ __device__ __forceinline__ void select_and_gate(const float (&s)[EB], int E, int
     for (int j = 0; j < k; ++j) w[j] = expf(sel[j] - sel[0]) / denom;
 }
 
+// acc[t][e] += x_t[chunk] . Wg_e[chunk] for one 16-byte chunk; rows of Wg
+// past E alias row E-1 (their sums are never read), so every load is
+// unconditional and issues before the arithmetic.
 template <typename In, int EB, int TPW>
-__global__ void __launch_bounds__(256) router_kernel(const In* __restrict__ x, const In* __restrict__ Wg, int T,
-                                                     int d, int E, int k, int32_t* __restrict__ idx,
-                                                     float* __restrict__ w) {
+__device__ __forceinline__ void chunk_dot(const typename Chunk<In>::Raw (&xr)[TPW], const In* __restrict__ Wg, int d,
+                                          int E, int c, float (&acc)[TPW][EB]) {
+    constexpr int CN = Chunk<In>::N;
+    typename Chunk<In>::Raw wr[EB];
+#pragma unroll
+    for (int e = 0; e < EB; ++e) wr[e] = Chunk<In>::load(Wg + (size_t)(e < E ? e : E - 1) * d + (size_t)c * CN);
+    float xv[TPW][CN];
+#pragma unroll
+    for (int t = 0; t < TPW; ++t) Chunk<In>::widen(xr[t], xv[t]);
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+        float wv[CN];
+        Chunk<In>::widen(wr[e], wv);
+#pragma unroll
+        for (int t = 0; t < TPW; ++t)
+#pragma unroll
+            for (int i = 0; i < CN; ++i) acc[t][e] = fmaf(xv[t][i], wv[i], acc[t][e]);
+    }
+}
+
+// Large T: one warp owns TPW tokens, lanes stride over the chunks of the rows
+// (the next x chunks are fetched while the current ones are used); a fixed
+// xor-butterfly reduces the lanes' partial sums.
+template <typename In, int EB, int TPW>
+__global__ void __launch_bounds__(256) router_warp_kernel(const In* __restrict__ x, const In* __restrict__ Wg, int T,
+                                                          int d, int E, int k, int32_t* __restrict__ idx,
+                                                          float* __restrict__ w) {
+    using Raw = typename Chunk<In>::Raw;
     constexpr int CN = Chunk<In>::N;
     const int lane = threadIdx.x & 31;
     const int warps_per_block = blockDim.x >> 5;
@@ -81,29 +115,20 @@ __global__ void __launch_bounds__(256) router_kernel(const In* __restrict__ x, c
         for (int t = 0; t < TPW; ++t)
 #pragma unroll
             for (int e = 0; e < EB; ++e) acc[t][e] = 0.f;
-
+        Raw xn[TPW];
+#pragma unroll
+        for (int t = 0; t < TPW; ++t)
+            xn[t] = (lane < nchunks && t0 + t < T) ? Chunk<In>::load(x + (size_t)(t0 + t) * d + (size_t)lane * CN)
+                                                   : Chunk<In>::zero();
         for (int c = lane; c < nchunks; c += 32) {
-            float xv[TPW][CN];
+            Raw xc[TPW];
 #pragma unroll
-            for (int t = 0; t < TPW; ++t) {
-                if (t0 + t < T) {
-                    Chunk<In>::load(x + (size_t)(t0 + t) * d + (size_t)c * CN, xv[t]);
-                } else {
+            for (int t = 0; t < TPW; ++t) xc[t] = xn[t];
+            const int cn = c + 32;
 #pragma unroll
-                    for (int i = 0; i < CN; ++i) xv[t][i] = 0.f;
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < EB; ++e) {
-                if (e < E) {
-                    float wv[CN];
-                    Chunk<In>::load(Wg + (size_t)e * d + (size_t)c * CN, wv);
-#pragma unroll
-                    for (int t = 0; t < TPW; ++t)
-#pragma unroll
-                        for (int i = 0; i < CN; ++i) acc[t][e] = fmaf(xv[t][i], wv[i], acc[t][e]);
-                }
-            }
+            for (int t = 0; t < TPW; ++t)
+                if (cn < nchunks && t0 + t < T) xn[t] = Chunk<In>::load(x + (size_t)(t0 + t) * d + (size_t)cn * CN);
+            chunk_dot<In, EB, TPW>(xc, Wg, d, E, c, acc);
         }
 #pragma unroll
         for (int t = 0; t < TPW; ++t)
@@ -121,22 +146,72 @@ __global__ void __launch_bounds__(256) router_kernel(const In* __restrict__ x, c
     }
 }
 
+// Small T: one block per token, its 8 warps split the row; warp sums meet in
+// shared memory and are added in warp order.
+template <typename In, int EB>
+__global__ void __launch_bounds__(256) router_split_kernel(const In* __restrict__ x, const In* __restrict__ Wg, int T,
+                                                           int d, int E, int k, int32_t* __restrict__ idx,
+                                                           float* __restrict__ w) {
+    using Raw = typename Chunk<In>::Raw;
+    constexpr int CN = Chunk<In>::N;
+    __shared__ float part[8][EB];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nchunks = d / CN;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        float acc[1][EB];
+#pragma unroll
+        for (int e = 0; e < EB; ++e) acc[0][e] = 0.f;
+        for (int c = threadIdx.x; c < nchunks; c += 256) {
+            Raw xr[1] = {Chunk<In>::load(x + (size_t)t * d + (size_t)c * CN)};
+            chunk_dot<In, EB, 1>(xr, Wg, d, E, c, acc);
+        }
+#pragma unroll
+        for (int e = 0; e < EB; ++e)
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) acc[0][e] += __shfl_xor_sync(0xffffffffu, acc[0][e], m);
+        if (lane == 0) {
+#pragma unroll
+            for (int e = 0; e < EB; ++e) part[warp][e] = acc[0][e];
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float s[EB];
+#pragma unroll
+            for (int e = 0; e < EB; ++e) {
+                float v = 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v += part[q][e];
+                s[e] = v;
+            }
+            select_and_gate<EB>(s, E, k, idx + (size_t)t * k, w + (size_t)t * k);
+        }
+        __syncthreads();
+    }
+}
+
+// Tokens at or below which one block handles one token.
+constexpr int kSplitMaxTokens = 512;
+
 template <typename In, int EB, int TPW>
 cudaError_t launch_router_t(const In* x, const In* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
                             int num_sms, cudaStream_t s) {
+    if (T <= kSplitMaxTokens) {
+        router_split_kernel<In, EB><<<T, 256, 0, s>>>(x, Wg, T, d, E, k, idx, w);
+        return cudaGetLastError();
+    }
     const int warps = (T + TPW - 1) / TPW;
     int blocks = (warps + 7) / 8;
-    const int cap = num_sms * 8;
+    const int cap = num_sms * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    router_kernel<In, EB, TPW><<<blocks, 256, 0, s>>>(x, Wg, T, d, E, k, idx, w);
+    router_warp_kernel<In, EB, TPW><<<blocks, 256, 0, s>>>(x, Wg, T, d, E, k, idx, w);
     return cudaGetLastError();
 }
 
 template <typename In>
 cudaError_t launch_router_any(const In* x, const In* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
                               int num_sms, cudaStream_t s) {
-    if (E <= 8) return launch_router_t<In, 8, 4>(x, Wg, T, d, E, k, idx, w, num_sms, s);
+    if (E <= 8) return launch_router_t<In, 8, 2>(x, Wg, T, d, E, k, idx, w, num_sms, s);
     if (E <= 16) return launch_router_t<In, 16, 2>(x, Wg, T, d, E, k, idx, w, num_sms, s);
     return launch_router_t<In, 32, 1>(x, Wg, T, d, E, k, idx, w, num_sms, s);
 }

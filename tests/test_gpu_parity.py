@@ -221,3 +221,30 @@ def test_wait_timeout_is_reported_not_hung(moe):
     x = torch.randn(8, 128, device="cuda").to(torch.bfloat16)   # context still usable
     idx, _ = moe.moe_route(x, torch.randn(4, 128, device="cuda").to(torch.bfloat16), 2)
     assert idx.shape == (8, 2)
+
+
+# ---------------------------------------------------------------- both expert paths
+
+
+@pytest.mark.parametrize("T,d,F,E,k", [(1, 128, 256, 8, 2), (16, 256, 512, 8, 2), (40, 192, 384, 5, 3),
+                                       (64, 128, 256, 4, 1), (64, 320, 256, 32, 2), (9, 128, 128, 1, 1)])
+@pytest.mark.parametrize("path", ["prefill", "decode"])
+def test_forward_paths_match_oracle(moe, T, d, F, E, k, path):
+    inp = moe_inputs.make_inputs(T, d, F, E, k, "bf16", seed=900 + T + E)
+    dev = upload(inp)
+    code = moe.MOE_PATH_DECODE if path == "decode" else moe.MOE_PATH_PREFILL
+    out = moe.moe_forward_ws(*dev, k, path=code)
+    _status_clear(moe)
+    ref = oracle.moe(*inp.arrays(), k=k, dtype="bf16")
+    idx, w = moe.moe_route(dev[0], dev[1], k)
+    keep = compare_routing(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    compare_outputs(out_to_f64(out), ref["out"], keep, "bf16")
+
+
+def test_decode_path_rejects_large_batches(moe):
+    inp = moe_inputs.make_inputs(65, 128, 256, 4, 2, "bf16", seed=3)
+    dev = upload(inp)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_forward_ws(*dev, 2, path=moe.MOE_PATH_DECODE)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
+    assert moe.moe_decode_max_tokens() == 64
