@@ -8,8 +8,10 @@
 //     stage 1   D1 = W1_e[f0:f0+128] Xp_e^T,  D3 = W3_e[f0:f0+128] Xp_e^T,
 //               H[slot][f] = SiLU(D1[f][t]) * D3[f][t]          (bf16)
 //     stage 2   D  = W2_e[r0:r0+128] H_e^T,   Y[slot][r] = D[r][t]  (fp32)
-// Only experts with at least one token are read (a page section "推論効率の
-// 観点" point: a small batch touches few experts).  N = the expert's token
+// Only experts with at least one token are read (the "Mixtral of Experts"
+// summary page lists, among its limitations, that small-batch inference
+// benefits from the small active parameter count while a large batch makes
+// every expert active).  N = the expert's token
 // count rounded up to 16 (at most 64), set per tile in the MMA instruction
 // descriptor; TMA streams 128-row x 64-column weight boxes through a 5-stage
 // ring (160 KiB of weights in flight per SM) with an evict-first L2 policy,
