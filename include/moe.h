@@ -135,6 +135,30 @@ MOE_API moe_status moe_dispatch(const int32_t* topk_idx, int T, int E, int k, in
                         int32_t* offsets, int32_t* perm, int32_t* inv, cudaStream_t stream);
 
 /*
+ * moe_dispatch for callers that cannot allocate device memory (no
+ * counterpart on the pages: an interface addition of this library).
+ *
+ * Some callers may not request device memory at call time: a plugin inside
+ * an inference runtime that is handed fixed buffers and forbidden to
+ * allocate, or a service that reserves all its memory at start-up.
+ * moe_dispatch takes its scratch from the library's memory pool, and creating
+ * or growing that pool allocates; this call never allocates.  Arguments,
+ * outputs and results are those of moe_dispatch, bit for bit.
+ *
+ * Scratch: one 16 KiB array compiled into the library, on every device that
+ * loads it, held until the process exits.  Limit: ceil(T / 1024) * E <= 3968
+ * (for example T <= 507,904 with E = 8, T <= 126,976 with E = 32); above it
+ * the call returns MOE_ERR_UNSUPPORTED and launches nothing.  Every call
+ * shares that array and finds the previous call's contents in it (each call
+ * writes every entry before reading it); calls whose kernels overlap on the
+ * GPU (other streams, other host threads) race on it.  The first call on a
+ * device, with that device current, looks up the array's device address
+ * once; make that call before any stream capture begins.
+ */
+MOE_API moe_status moe_dispatch_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* counts,
+                                        int32_t* offsets, int32_t* perm, int32_t* inv, cudaStream_t stream);
+
+/*
  * The whole layer (route, dispatch, experts, combine) with bfloat16 tensors
  * (all device): x [T][d], Wg [E][d], W1/W3 [E][F][d], W2 [E][d][F], out [T][d].
  * The workspace comes from the library's stream-ordered pool on `stream`

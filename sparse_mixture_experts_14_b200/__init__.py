@@ -40,6 +40,7 @@ SIGNATURES = {
     "moe_route_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _vp, _vp, _vp]),
     "moe_slots_capacity": (_sz, [_ci, _ci, _ci]),
     "moe_dispatch": (_ci, [_vp, _ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp]),
+    "moe_dispatch_noalloc": (_ci, [_vp, _ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp]),
     "moe_forward": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _vp]),
     "moe_forward_f32": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _vp]),
     "moe_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
@@ -143,6 +144,18 @@ def moe_dispatch(topk_idx, E, stream=None):
     inv = torch.empty((T, k), dtype=torch.int32, device=dev)
     _check(_lib.moe_dispatch(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
                              _stream(stream)), "moe_dispatch")
+    return counts, offsets, perm, inv
+
+
+def moe_dispatch_noalloc(topk_idx, E, counts, offsets, perm, inv, stream=None):
+    """moe_dispatch into caller-provided outputs, using the library's fixed scratch array instead of
+    any allocation (for callers that may not allocate device memory); raises MoEError above its limit."""
+    _dev(topk_idx, torch.int32, "topk_idx")
+    for t, n in ((counts, "counts"), (offsets, "offsets"), (perm, "perm"), (inv, "inv")):
+        _dev(t, torch.int32, n)
+    T, k = topk_idx.shape
+    _check(_lib.moe_dispatch_noalloc(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
+                                     _stream(stream)), "moe_dispatch_noalloc")
     return counts, offsets, perm, inv
 
 

@@ -232,6 +232,21 @@ __global__ void wait_selftest_kernel(int* status, long long limit_ns) {
 }
 
 }  // namespace
+
+// Address of the status word on device `dev` (current), resolved once; creates no memory pool.
+int* status_word(int dev) {
+    static std::mutex mu;
+    static int* ptrs[kMaxDevices] = {};
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int*>(p);
+    }
+    return ptrs[dev];
+}
+
 }  // namespace moe
 
 using namespace moe;
