@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ blk, i
         if ((size_t)offs[E] > slots) record_status(status, MOE_ERR_DEVICE);
         for (int e = 0; e < E; ++e) meta->counts[e] = tot[e];
         for (int e = 0; e <= E; ++e) meta->offsets[e] = offs[e];
+        meta->waves[0] = meta->waves[1] = 0;
     }
     __syncthreads();
     if (warp < E) {
@@ -188,6 +189,7 @@ __global__ void __launch_bounds__(kDispatchTokens) dispatch_single_kernel(const 
         if ((size_t)offs[E] > slots) record_status(status, MOE_ERR_DEVICE);
         for (int e = 0; e < E; ++e) meta->counts[e] = tot[e];
         for (int e = 0; e <= E; ++e) meta->offsets[e] = offs[e];
+        meta->waves[0] = meta->waves[1] = 0;
     }
     __syncthreads();
     if (t < T) {

@@ -79,12 +79,29 @@ __device__ __forceinline__ void decode_tile(const Ctrl* c, int tile, int& e, int
     pair = local - n_blk * c->pt[e];
 }
 
+// Soft per-wave alignment of the clusters.  CTA pairs that share a block of
+// expert weights run tiles of the same wave; if the clusters drift apart over
+// many waves, a shared block leaves L2 between its first and last reader and
+// is fetched from HBM again.  Each leader announces the start of its wave on a
+// device counter and waits, for at most 20 us, until every cluster with a
+// tile in that wave has announced it.  The wait is only a hint: on expiry the
+// cluster goes on, so nothing can deadlock on it.
+__device__ __forceinline__ void wave_sync(int* counter, int target) {
+    atomicAdd(counter, 1);
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+        if (v >= target || global_timer_ns() - t0 > 20000ull) break;
+    }
+}
+
 // SWIGLU: GEMM1 (B halves = 128-row blocks of W1 and W3, out = H bf16 [slots][N]).
 // !SWIGLU: GEMM2 (B halves = the two 128-row halves of a 256-row W2 block, out = Y fp32 [slots][N]).
 template <bool SWIGLU>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB1,
-                   const __grid_constant__ CUtensorMap mapB3, const Meta* __restrict__ meta, int E, int K, int N,
+                   const __grid_constant__ CUtensorMap mapB3, Meta* __restrict__ meta, int E, int K, int N,
                    size_t slots, void* __restrict__ out, int* status, long long wait_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -156,10 +173,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 armed_phase[s] = 0;
             }
             bool aborted = false;
-            for (int tile = cluster; tile < total && !aborted; tile += nclusters) {
+            int wave = 0;
+            for (int tile = cluster; tile < total && !aborted; tile += nclusters, ++wave) {
                 int e, pair, n_blk;
                 decode_tile(ctrl, tile, e, pair, n_blk);
                 const int rowA = ctrl->row0[e] + (2 * pair + (int)rank) * BM;
+                if (leader) wave_sync(&meta->waves[SWIGLU ? 0 : 1], min(total, (wave + 1) * nclusters));
                 const CUtensorMap* mapB = (SWIGLU && !leader) ? &mapB3 : &mapB1;
                 const int rowB = SWIGLU ? n_blk * BNH : n_blk * BN + (int)rank * BNH;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -416,8 +435,8 @@ cudaError_t launch_pair(int grid, const CUtensorMap& mA, const CUtensorMap& mB1,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<SWIGLU>, mA, mB1, mB3, a.meta, a.E, K, N, a.slots, out, a.status,
-                              a.wait_ns);
+    return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<SWIGLU>, mA, mB1, mB3, const_cast<Meta*>(a.meta), a.E, K, N,
+                              a.slots, out, a.status, a.wait_ns);
 }
 
 }  // namespace

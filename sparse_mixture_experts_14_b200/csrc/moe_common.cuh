@@ -20,6 +20,7 @@ constexpr int kDispatchTokens = 1024;
 struct Meta {
     int32_t counts[kMaxExperts];        // assignments per expert
     int32_t offsets[kMaxExperts + 1];   // padded segment start rows; offsets[E] = padded total
+    int32_t waves[2];                   // wave counters of the two expert GEMMs (zeroed by dispatch)
 };
 
 // Per-device sticky status word (first fault wins).
