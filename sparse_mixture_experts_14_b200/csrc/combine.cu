@@ -13,6 +13,8 @@ template <bool BF16_OUT>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ Y, const float* __restrict__ w,
                                                       const int32_t* __restrict__ inv, int T, int d, int k,
                                                       void* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     const int q = d / 4;   // float4 columns per row
     const size_t n = (size_t)T * q;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
@@ -47,8 +49,7 @@ cudaError_t launch_combine_t(const float* Y, const float* w, const int32_t* inv,
     size_t blocks = (n + 255) / 256;
     if (blocks > 148 * 32) blocks = 148 * 32;
     if (blocks < 1) blocks = 1;
-    combine_kernel<BF16_OUT><<<(unsigned)blocks, 256, 0, s>>>(Y, w, inv, T, d, k, out);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel<BF16_OUT>, dim3((unsigned)blocks), dim3(256), 0, s, Y, w, inv, T, d, k, out);
 }
 
 }  // namespace

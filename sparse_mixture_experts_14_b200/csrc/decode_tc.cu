@@ -13,9 +13,9 @@
 // benefits from the small active parameter count while a large batch makes
 // every expert active).  N = the expert's token
 // count rounded up to 16 (at most 64), set per tile in the MMA instruction
-// descriptor; TMA streams 128-row x 64-column weight boxes through a 5-stage
-// ring (160 KiB of weights in flight per SM) with an evict-first L2 policy,
-// since every weight byte is used once.
+// descriptor; TMA streams 128-row x 64-column weight boxes through a ring of
+// 5 (stage 1) or 8 (stage 2) steps, 128-160 KiB of weights in flight per SM,
+// with an evict-first L2 policy, since every weight byte is used once.
 //
 // One CTA per SM, 6 warps: warp 0 TMA producer, warp 1 MMA issuer + TMEM
 // owner (256 columns: two accumulator sets of 2 x 64), warps 2-5 epilogue
@@ -32,16 +32,26 @@ namespace {
 constexpr int DM = 128;                     // weight rows per tile (MMA M)
 constexpr int DK = 64;                      // K per stage
 constexpr int DNMAX = 64;                   // tokens per expert on this path (MMA N <= 64)
-constexpr int DSTAGES = 5;
 constexpr int W_BYTES = DM * DK * 2;        // 16 KiB
 constexpr int X_BYTES = DNMAX * DK * 2;     // 8 KiB
-constexpr int DSTAGE_BYTES = 2 * W_BYTES + X_BYTES;
+constexpr int DSTAGES_MAX = 8;
+
+// Ring geometry per stage kind: stage 1 streams two weight boxes (W1, W3) per
+// step in 5 x 40 KiB, stage 2 one box (W2) in 8 x 24 KiB; both keep 128-160 KiB
+// of weights in flight per SM.
+template <bool GATE>
+struct Ring {
+    static constexpr int STAGES = GATE ? 5 : 8;
+    static constexpr int W_BOXES = GATE ? 2 : 1;
+    static constexpr int STAGE_BYTES = W_BOXES * W_BYTES + X_BYTES;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES;
+};
 constexpr int DTMEM_COLS = 256;
 constexpr int DTHREADS = 192;
 
 struct DCtrl {
-    uint64_t full[DSTAGES];
-    uint64_t empty[DSTAGES];
+    uint64_t full[DSTAGES_MAX];
+    uint64_t empty[DSTAGES_MAX];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -53,7 +63,8 @@ struct DCtrl {
     int row0[kMaxExperts];
 };
 
-constexpr int DSMEM_BYTES = DSTAGES * DSTAGE_BYTES + (int)sizeof(DCtrl) + 1024;
+template <bool GATE>
+constexpr int dsmem_bytes() { return Ring<GATE>::SMEM_BYTES + (int)sizeof(DCtrl) + 1024; }
 
 // GATE: stage 1 (mapWa = W1, mapWb = W3, mapX = Xp, out = H bf16 [slots][R]).
 // !GATE: stage 2 (mapWa = W2, mapX = H, out = Y fp32 [slots][R]).
@@ -65,11 +76,15 @@ __global__ void __launch_bounds__(DTHREADS, 1)
                   void* __restrict__ out, int* status, long long wait_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    DCtrl* ctrl = reinterpret_cast<DCtrl*>(smem + DSTAGES * DSTAGE_BYTES);
+    constexpr int DSTAGES = Ring<GATE>::STAGES;
+    constexpr int DSTAGE_BYTES = Ring<GATE>::STAGE_BYTES;
+    constexpr int X_OFF = Ring<GATE>::W_BOXES * W_BYTES;
+    DCtrl* ctrl = reinterpret_cast<DCtrl*>(smem + Ring<GATE>::SMEM_BYTES);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    constexpr uint32_t STAGE_TX = GATE ? (uint32_t)DSTAGE_BYTES : (uint32_t)(W_BYTES + X_BYTES);
+    constexpr uint32_t STAGE_TX = (uint32_t)DSTAGE_BYTES;
 
+    pdl_trigger();
     if (threadIdx.x == 0) {
         for (int s = 0; s < DSTAGES; ++s) {
             ptx::mbar_init(&ctrl->full[s], 1);
@@ -81,6 +96,20 @@ __global__ void __launch_bounds__(DTHREADS, 1)
         }
         ptx::mbar_init(&ctrl->drain, 1);
         ctrl->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::tma_prefetch_desc(&mapWa);
+        if (GATE) ptx::tma_prefetch_desc(&mapWb);
+        ptx::tma_prefetch_desc(&mapX);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&ctrl->tmem_base, DTMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    // everything above overlaps the previous kernel; global memory only after this
+    pdl_wait();
+    if (threadIdx.x == 0) {
         const int blocks = (R + DM - 1) / DM;
         ctrl->tile_base[0] = 0;
         bool ok = true;
@@ -93,16 +122,6 @@ __global__ void __launch_bounds__(DTHREADS, 1)
         }
         ctrl->total = ok ? ctrl->tile_base[E] : 0;
         if (!ok) record_status(status, MOE_ERR_DEVICE);
-        ptx::fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        ptx::tma_prefetch_desc(&mapWa);
-        if (GATE) ptx::tma_prefetch_desc(&mapWb);
-        ptx::tma_prefetch_desc(&mapX);
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc(&ctrl->tmem_base, DTMEM_COLS);
-        ptx::tmem_relinquish();
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
@@ -145,7 +164,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
                     ptx::mbar_arrive_expect_tx(&ctrl->full[stage], STAGE_TX);
                     ptx::tma_load_3d(sw, &mapWa, &ctrl->full[stage], kb * DK, blk * DM, e, pol_w);
                     if (GATE) ptx::tma_load_3d(sw + W_BYTES, &mapWb, &ctrl->full[stage], kb * DK, blk * DM, e, pol_w);
-                    ptx::tma_load_2d(sw + 2 * W_BYTES, &mapX, &ctrl->full[stage], kb * DK, ctrl->row0[e], pol_x);
+                    ptx::tma_load_2d(sw + X_OFF, &mapX, &ctrl->full[stage], kb * DK, ctrl->row0[e], pol_x);
 #pragma unroll
                     for (int s = 0; s < DSTAGES; ++s)
                         if (s == stage) {
@@ -189,7 +208,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
                     }
                     ptx::tc_fence_after_sync();
                     const uint32_t w0 = ptx::smem_addr(smem + stage * DSTAGE_BYTES);
-                    const uint32_t x0 = w0 + 2 * W_BYTES;
+                    const uint32_t x0 = w0 + X_OFF;
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk) {
                         const uint64_t bx = ptx::desc_kmajor_sw128(x0 + kk * 32);
@@ -312,7 +331,7 @@ cudaError_t launch_stage(const CUtensorMap& a, const CUtensorMap& b, const CUten
     static bool attr = false;
     if (!attr) {
         cudaError_t e =
-            cudaFuncSetAttribute(decode_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, DSMEM_BYTES);
+            cudaFuncSetAttribute(decode_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsmem_bytes<GATE>());
         if (e != cudaSuccess) return e;
         attr = true;
     }
@@ -320,8 +339,8 @@ cudaError_t launch_stage(const CUtensorMap& a, const CUtensorMap& b, const CUten
     const int upper = g.E * ((R + DM - 1) / DM);
     if (grid > upper) grid = upper;
     if (grid < 1) grid = 1;
-    decode_kernel<GATE><<<grid, DTHREADS, DSMEM_BYTES, s>>>(a, b, x, g.meta, g.E, K, R, out, g.status, g.wait_ns);
-    return cudaGetLastError();
+    return launch_pdl(decode_kernel<GATE>, dim3(grid), dim3(DTHREADS), dsmem_bytes<GATE>(), s, a, b, x, g.meta, g.E, K, R, out,
+                      g.status, g.wait_ns);
 }
 
 }  // namespace

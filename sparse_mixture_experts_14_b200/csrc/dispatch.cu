@@ -20,6 +20,8 @@ namespace {
 
 __global__ void __launch_bounds__(kDispatchTokens) hist_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
                                                                int32_t* __restrict__ blk_counts, int* status) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ int cnt[kMaxExperts];
     if (threadIdx.x < kMaxExperts) cnt[threadIdx.x] = 0;
     __syncthreads();
@@ -44,6 +46,8 @@ __global__ void __launch_bounds__(kDispatchTokens) hist_kernel(const int32_t* __
 // becomes the first row of block b's assignments to expert e.
 __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ blk, int NB, int E, Meta* __restrict__ meta,
                                                     int32_t* __restrict__ perm, size_t slots, int* status) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ int tot[kMaxExperts];
     __shared__ int offs[kMaxExperts + 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -91,6 +95,8 @@ __global__ void __launch_bounds__(kDispatchTokens) scatter_kernel(const int32_t*
                                                                   const int32_t* __restrict__ blk_base,
                                                                   int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                                                                   size_t slots, int* status) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ int wcnt[32][kMaxExperts + 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * kDispatchTokens + threadIdx.x;
@@ -148,6 +154,8 @@ __global__ void __launch_bounds__(kDispatchTokens) dispatch_single_kernel(const 
                                                                           int32_t* __restrict__ perm,
                                                                           int32_t* __restrict__ inv, size_t slots,
                                                                           int* status) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ int wcnt[32][kMaxExperts + 1];
     __shared__ int offs[kMaxExperts + 1];
     __shared__ int tot[kMaxExperts];
@@ -223,6 +231,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__
                                                      const Meta* __restrict__ meta, int E,
                                                      const int32_t* __restrict__ perm, uint8_t* __restrict__ xp,
                                                      size_t slots) {
+    pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
     const size_t total = (size_t)meta->offsets[E];
@@ -234,7 +244,20 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__
         uint4* dst = reinterpret_cast<uint4*>(xp + r * row_bytes);
         if (a >= 0 && a < TK) {
             const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(a / k) * row_bytes);
-            for (size_t v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+            // 8 loads in flight per lane before their stores
+            for (size_t v0 = lane; v0 < nvec; v0 += 32 * 8) {
+                uint4 buf[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const size_t v = v0 + (size_t)u * 32;
+                    if (v < nvec) buf[u] = __ldg(src + v);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const size_t v = v0 + (size_t)u * 32;
+                    if (v < nvec) dst[v] = buf[u];
+                }
+            }
         } else {
             const uint4 z = make_uint4(0, 0, 0, 0);
             for (size_t v = lane; v < nvec; v += 32) dst[v] = z;
@@ -249,13 +272,15 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* bl
     const int NB = dispatch_blocks(T);
     const size_t slots = slots_capacity(T, E, k);
     if (NB == 1) {
-        dispatch_single_kernel<<<1, kDispatchTokens, 0, s>>>(idx, T, E, k, meta, perm, inv, slots, status);
-        return cudaGetLastError();
+        return launch_pdl(dispatch_single_kernel, dim3(1), dim3(kDispatchTokens), 0, s, idx, T, E, k, meta, perm, inv,
+                          slots, status);
     }
-    hist_kernel<<<NB, kDispatchTokens, 0, s>>>(idx, T, E, k, blk_counts, status);
-    scan_kernel<<<1, 1024, 0, s>>>(blk_counts, NB, E, meta, perm, slots, status);
-    scatter_kernel<<<NB, kDispatchTokens, 0, s>>>(idx, T, E, k, blk_counts, perm, inv, slots, status);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(hist_kernel, dim3(NB), dim3(kDispatchTokens), 0, s, idx, T, E, k, blk_counts, status);
+    if (e == cudaSuccess) e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, blk_counts, NB, E, meta, perm, slots, status);
+    if (e == cudaSuccess)
+        e = launch_pdl(scatter_kernel, dim3(NB), dim3(kDispatchTokens), 0, s, idx, T, E, k, blk_counts, perm, inv, slots,
+                       status);
+    return e;
 }
 
 cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
@@ -263,9 +288,8 @@ cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E,
     const size_t rows_per_block = 8;
     size_t blocks = (slots + rows_per_block - 1) / rows_per_block;
     if (blocks > 65535 * 4) blocks = 65535 * 4;
-    gather_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), (size_t)d * elem_bytes, T, k,
-                                                  meta, E, perm, static_cast<uint8_t*>(xp), slots);
-    return cudaGetLastError();
+    return launch_pdl(gather_kernel, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const uint8_t*>(x),
+                      (size_t)d * elem_bytes, T, k, meta, E, perm, static_cast<uint8_t*>(xp), slots);
 }
 
 }  // namespace moe

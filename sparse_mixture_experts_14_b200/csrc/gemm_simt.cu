@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
                                                         const float* __restrict__ B3, const Meta* __restrict__ meta,
                                                         int E, int K, int N, size_t b_expert_stride,
                                                         float* __restrict__ C) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ float As[TK][TM + 4];
     __shared__ float B1s[TK][TN + 4];
     __shared__ float B3s[SWIGLU ? TK : 1][TN + 4];
@@ -97,15 +99,14 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
 cudaError_t launch_simt_gemm1_f32(const float* xp, const float* W1, const float* W3, const Meta* meta, int E, int d,
                                   int F, float* H, size_t slots, cudaStream_t s) {
     dim3 grid((unsigned)(slots / TM), (unsigned)((F + TN - 1) / TN));
-    simt_gemm_kernel<true><<<grid, 256, 0, s>>>(xp, W1, W3, meta, E, d, F, (size_t)F * d, H);
-    return cudaGetLastError();
+    return launch_pdl(simt_gemm_kernel<true>, grid, dim3(256), 0, s, xp, W1, W3, meta, E, d, F, (size_t)F * d, H);
 }
 
 cudaError_t launch_simt_gemm2_f32(const float* H, const float* W2, const Meta* meta, int E, int d, int F, float* Y,
                                   size_t slots, cudaStream_t s) {
     dim3 grid((unsigned)(slots / TM), (unsigned)((d + TN - 1) / TN));
-    simt_gemm_kernel<false><<<grid, 256, 0, s>>>(H, W2, nullptr, meta, E, F, d, (size_t)d * F, Y);
-    return cudaGetLastError();
+    return launch_pdl(simt_gemm_kernel<false>, grid, dim3(256), 0, s, H, W2, static_cast<const float*>(nullptr), meta,
+                      E, F, d, (size_t)d * F, Y);
 }
 
 }  // namespace moe

@@ -18,7 +18,7 @@
 //
 // Persistent kernel, one CTA per SM, 6 warps per CTA:
 //   warp 0     TMA producer (one thread per CTA): own A rows and own B half
-//              into a 6-stage ring; completion bytes of both CTAs are counted
+//              into a 7-stage ring; completion bytes of both CTAs are counted
 //              on the leader's barrier
 //   warp 1     leader: MMA issuer (one thread); commits arrive on both CTAs'
 //              barriers (multicast).  Both CTAs: TMEM owner (512 columns =
@@ -44,7 +44,7 @@ constexpr int BM = 128;                        // rows per CTA (256 per pair)
 constexpr int BK = 64;                         // K per stage (one 128-byte swizzle row)
 constexpr int BN = 256;                        // accumulator columns of the pair MMA
 constexpr int BNH = BN / 2;                    // B rows held by each CTA
-constexpr int STAGES = 6;
+constexpr int STAGES = 7;
 constexpr int A_BYTES = BM * BK * 2;           // 16 KiB
 constexpr int B_BYTES = BNH * BK * 2;          // 16 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int nclusters = gridDim.x >> 1;
     constexpr int N_PER_TILE = SWIGLU ? BNH : BN;   // output columns per tile
 
+    pdl_trigger();
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             ptx::mbar_init(&ctrl->full[s], 1);
@@ -125,6 +126,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::mbar_init(&ctrl->drain, 1);
         ctrl->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::tma_prefetch_desc(&mapA);
+        ptx::tma_prefetch_desc(&mapB1);
+        if (SWIGLU) ptx::tma_prefetch_desc(&mapB3);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(&ctrl->tmem_base, TMEM_COLS);
+        ptx::tmem_relinquish_pair();
+    }
+    // everything above overlaps the previous kernel; global memory only after this
+    pdl_wait();
+    if (threadIdx.x == 0) {
         const int ntn = (N + N_PER_TILE - 1) / N_PER_TILE;
         ctrl->tile_base[0] = 0;
         bool ok = true;
@@ -139,16 +154,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ctrl->total = ok ? ctrl->tile_base[E] : 0;
         if (!ok) record_status(status, MOE_ERR_DEVICE);
-        ptx::fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        ptx::tma_prefetch_desc(&mapA);
-        ptx::tma_prefetch_desc(&mapB1);
-        if (SWIGLU) ptx::tma_prefetch_desc(&mapB3);
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc_pair(&ctrl->tmem_base, TMEM_COLS);
-        ptx::tmem_relinquish_pair();
     }
     ptx::tc_fence_before_sync();
     ptx::cluster_sync();
@@ -428,13 +433,15 @@ cudaError_t launch_pair(int grid, const CUtensorMap& mA, const CUtensorMap& mB1,
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<SWIGLU>, mA, mB1, mB3, const_cast<Meta*>(a.meta), a.E, K, N,
                               a.slots, out, a.status, a.wait_ns);
 }

@@ -49,6 +49,32 @@ __device__ __forceinline__ float silu_mul(float a, float b) {
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Programmatic dependent launch.  Every kernel of the layer is launched with
+// programmatic stream serialisation: it lets the next kernel in the stream be
+// scheduled once all of its own CTAs have started (pdl_trigger at entry),
+// and it does no global-memory access before pdl_wait, which returns once
+// the previous grid in the stream has completed and its writes are visible.
+// The next kernel's launch latency and prologue (barrier set-up, tensor
+// memory allocation) thereby overlap the tail of the current one.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 // Rows of the padded expert-contiguous buffers.
 inline size_t slots_capacity(int T, int E, int k) {
     return align_up((size_t)T * k + (size_t)E * (kSegRows - 1), kSegRows);
