@@ -226,6 +226,120 @@ __global__ void __launch_bounds__(kDispatchTokens) dispatch_single_kernel(const 
     }
 }
 
+// Few tokens (T <= 64, the decode path): dispatch and gather in one launch.
+// Every block recomputes the (tiny) stable counting sort in shared memory, so
+// the blocks need no communication; block 0 publishes the segment table, perm
+// and inv, and all blocks copy their share of token rows into the segments.
+constexpr int kSmallTokens = 64;
+constexpr int kSmallMaxRows = kSmallTokens * kMaxExperts + kMaxExperts * kSegRows;
+
+__global__ void __launch_bounds__(256) dispatch_gather_small_kernel(const int32_t* __restrict__ idx, int T, int E,
+                                                                    int k, const uint8_t* __restrict__ x,
+                                                                    size_t row_bytes, Meta* __restrict__ meta,
+                                                                    int32_t* __restrict__ perm,
+                                                                    int32_t* __restrict__ inv,
+                                                                    uint8_t* __restrict__ xp, size_t slots,
+                                                                    int* status) {
+    pdl_trigger();
+    pdl_wait();
+    __shared__ int offs[kMaxExperts + 1];
+    __shared__ int cnt[kMaxExperts];
+    __shared__ int sidx[kSmallTokens * kMaxExperts];     // the assignments
+    __shared__ int row_of[kSmallTokens * kMaxExperts];   // slot of assignment (t, j), -1 if dropped
+    __shared__ int owner[kSmallMaxRows];                  // assignment held by each row, -1 on padding
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int a = tid; a < T * k; a += blockDim.x) {
+        sidx[a] = idx[a];
+        row_of[a] = -1;
+    }
+    __syncthreads();
+    // warp 0: stable counting sort; lane owns tokens lane and lane + 32
+    if (warp == 0) {
+        uint32_t mask[2] = {0u, 0u};
+        for (int h = 0; h < 2; ++h) {
+            const int t = lane + 32 * h;
+            if (t < T) {
+                for (int j = 0; j < k; ++j) {
+                    const int e = sidx[t * k + j];
+                    if (e < 0 || e >= E || ((mask[h] >> e) & 1u)) {
+                        if (blockIdx.x == 0) record_status(status, MOE_ERR_DEVICE);
+                        continue;
+                    }
+                    mask[h] |= 1u << e;
+                }
+            }
+        }
+        const uint32_t lt = (1u << lane) - 1u;
+        int base = 0;
+        for (int e = 0; e < E; ++e) {
+            const uint32_t b0 = __ballot_sync(0xffffffffu, (mask[0] >> e) & 1u);
+            const uint32_t b1 = __ballot_sync(0xffffffffu, (mask[1] >> e) & 1u);
+            const int n = __popc(b0) + __popc(b1);
+            for (int h = 0; h < 2; ++h) {
+                if ((mask[h] >> e) & 1u) {
+                    const int t = lane + 32 * h;
+                    const int r = h == 0 ? __popc(b0 & lt) : __popc(b0) + __popc(b1 & lt);
+                    for (int j = 0; j < k; ++j)
+                        if (sidx[t * k + j] == e) {
+                            row_of[t * k + j] = base + r;   // first occurrence; duplicates stay dropped
+                            break;
+                        }
+                }
+            }
+            if (lane == 0) {
+                cnt[e] = n;
+                offs[e] = base;
+            }
+            base += (n + kSegRows - 1) / kSegRows * kSegRows;
+        }
+        if (lane == 0) offs[E] = base;
+    }
+    __syncthreads();
+    const int total = offs[E];
+    for (int r = tid; r < total; r += blockDim.x) owner[r] = -1;
+    __syncthreads();
+    for (int a = tid; a < T * k; a += blockDim.x)
+        if (row_of[a] >= 0) owner[row_of[a]] = a;
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        if (tid == 0) {
+            if ((size_t)total > slots) record_status(status, MOE_ERR_DEVICE);
+            for (int e = 0; e < E; ++e) meta->counts[e] = cnt[e];
+            for (int e = 0; e <= E; ++e) meta->offsets[e] = offs[e];
+            meta->waves[0] = meta->waves[1] = 0;
+        }
+        for (int a = tid; a < T * k; a += blockDim.x) inv[a] = row_of[a];
+        for (int r = tid; r < total; r += blockDim.x)
+            if ((size_t)r < slots) perm[r] = owner[r];
+    }
+    // gather: one warp per assignment, strided over all blocks.  Only rows that
+    // hold a token are written: the decode kernels read at most the first 64
+    // rows of a segment and discard the MMA columns of rows past the expert's
+    // token count, so padding rows are never used on this path.
+    const size_t nvec = row_bytes / 16;
+    const int gw = blockIdx.x * (blockDim.x >> 5) + warp;
+    const int nw = gridDim.x * (blockDim.x >> 5);
+    for (int a = gw; a < T * k; a += nw) {
+        const int r = row_of[a];
+        if (r < 0 || (size_t)r >= slots) continue;
+        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * row_bytes);
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(a / k) * row_bytes);
+        for (size_t v0 = lane; v0 < nvec; v0 += 32 * 8) {
+            uint4 buf[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const size_t v = v0 + (size_t)u * 32;
+                if (v < nvec) buf[u] = __ldg(src + v);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const size_t v = v0 + (size_t)u * 32;
+                if (v < nvec) dst[v] = buf[u];
+            }
+        }
+    }
+}
+
 // One warp per row of the padded buffer; rows past offsets[E] are left alone.
 __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ x, size_t row_bytes, int T, int k,
                                                      const Meta* __restrict__ meta, int E,
@@ -281,6 +395,19 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* bl
         e = launch_pdl(scatter_kernel, dim3(NB), dim3(kDispatchTokens), 0, s, idx, T, E, k, blk_counts, perm, inv, slots,
                        status);
     return e;
+}
+
+cudaError_t launch_dispatch_gather_small(const int32_t* idx, int T, int E, int k, const void* x, size_t elem_bytes,
+                                         int d, Meta* meta, int32_t* perm, int32_t* inv, void* xp, size_t slots,
+                                         int* status, cudaStream_t s) {
+    if (T > kSmallTokens) return cudaErrorInvalidValue;
+    const int rows = T * k;
+    int blocks = (rows + 7) / 8;   // about one row per warp
+    if (blocks < 1) blocks = 1;
+    if (blocks > 64) blocks = 64;
+    return launch_pdl(dispatch_gather_small_kernel, dim3(blocks), dim3(256), 0, s, idx, T, E, k,
+                      static_cast<const uint8_t*>(x), (size_t)d * elem_bytes, meta, perm, inv,
+                      static_cast<uint8_t*>(xp), slots, status);
 }
 
 cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,

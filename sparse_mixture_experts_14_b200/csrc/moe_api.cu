@@ -170,11 +170,20 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
     }
     n += 1;
     MOE_TRY(mark(MOE_STAGE_DISPATCH));
-    MOE_TRY(launch_dispatch(idx, T, E, k, blk, meta, perm, inv, dev.status, s));
-    n += dispatch_launches(T);
-    MOE_TRY(mark(MOE_STAGE_GATHER));
-    MOE_TRY(launch_gather(x, dtype == MOE_DTYPE_BF16 ? 2 : 4, T, d, E, k, meta, perm, xp, p.slots, s));
-    n += 1;
+    const size_t es = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+    if (dtype == MOE_DTYPE_BF16 && T <= kDecodeMaxTokens &&
+        (path == MOE_PATH_DECODE || path == MOE_PATH_AUTO)) {
+        // decode path: one launch sorts and gathers the token rows (the gather stage is empty)
+        MOE_TRY(launch_dispatch_gather_small(idx, T, E, k, x, es, d, meta, perm, inv, xp, p.slots, dev.status, s));
+        n += 1;
+        MOE_TRY(mark(MOE_STAGE_GATHER));
+    } else {
+        MOE_TRY(launch_dispatch(idx, T, E, k, blk, meta, perm, inv, dev.status, s));
+        n += dispatch_launches(T);
+        MOE_TRY(mark(MOE_STAGE_GATHER));
+        MOE_TRY(launch_gather(x, es, T, d, E, k, meta, perm, xp, p.slots, s));
+        n += 1;
+    }
     if (dtype == MOE_DTYPE_BF16) {
         TcGemmArgs a{xp, W1, W3, W2, h, y, meta, E, d, F, p.slots, dev.num_sms, dev.status, wait_limit_ns()};
         const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxTokens);

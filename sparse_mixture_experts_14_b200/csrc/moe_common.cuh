@@ -92,6 +92,10 @@ cudaError_t launch_router_f32(const float* x, const float* Wg, int T, int d, int
 inline int dispatch_launches(int T) { return T <= kDispatchTokens ? 1 : 3; }
 cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* blk_counts, Meta* meta,
                             int32_t* perm, int32_t* inv, int* status, cudaStream_t s);
+// T <= 64: dispatch and gather fused in one launch (same results as the two separately).
+cudaError_t launch_dispatch_gather_small(const int32_t* idx, int T, int E, int k, const void* x, size_t elem_bytes,
+                                         int d, Meta* meta, int32_t* perm, int32_t* inv, void* xp, size_t slots,
+                                         int* status, cudaStream_t s);
 cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
                           const int32_t* perm, void* xp, size_t slots, cudaStream_t s);
 
