@@ -42,9 +42,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// SiLU(a) * b with SiLU(a) = a / (1 + e^-a).
+// SiLU(a) * b with SiLU(a) = a / (1 + e^-a).  For a < -88 the denominator is
+// +inf and the fast division gives the correct limit 0.
 __device__ __forceinline__ float silu_mul(float a, float b) {
-    return a / (1.0f + __expf(-a)) * b;
+    return __fdividef(a, 1.0f + __expf(-a)) * b;
 }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

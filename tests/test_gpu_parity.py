@@ -248,3 +248,59 @@ def test_decode_path_rejects_large_batches(moe):
         moe.moe_forward_ws(*dev, 2, path=moe.MOE_PATH_DECODE)
     assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
     assert moe.moe_decode_max_tokens() == 64
+
+
+# ---------------------------------------------------------------- experts with no tokens, decode invariants
+
+
+@pytest.mark.parametrize("T,path", [(16, "decode"), (48, "decode"), (48, "prefill"), (900, "prefill")])
+def test_experts_without_tokens(moe, T, path):
+    """Experts 5..7 never win (feature 0 pinned to 1.0 and a -30 offset on their scores)."""
+    inp = moe_inputs.make_inputs(T, 256, 512, 8, 2, "bf16", seed=31 + T,
+                                 bias=[0.5, 0.25, 0.0, -0.25, -0.5, -30.0, -30.0, -30.0])
+    dev = upload(inp)
+    code = moe.MOE_PATH_DECODE if path == "decode" else moe.MOE_PATH_PREFILL
+    out = moe.moe_forward_ws(*dev, 2, path=code)
+    _status_clear(moe)
+    ref = oracle.moe(*inp.arrays(), k=2, dtype="bf16")
+    assert not np.isin(ref["idx"], [5, 6, 7]).any()
+    idx, w = moe.moe_route(dev[0], dev[1], 2)
+    keep = compare_routing(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    compare_outputs(out_to_f64(out), ref["out"], keep, "bf16")
+
+
+@pytest.fixture(scope="module")
+def small():
+    inp = moe_inputs.make_inputs(24, 512, 1024, 8, 2, "bf16", seed=55)
+    return inp, upload(inp)
+
+
+def test_decode_run_to_run_bitwise(moe, small):
+    _, dev = small
+    a = moe.moe_forward(*dev, 2)
+    b = moe.moe_forward(*dev, 2)
+    assert torch.equal(a, b)
+
+
+def test_decode_token_permutation_equivariance(moe, small):
+    _, dev = small
+    out = moe.moe_forward(*dev, 2)
+    p = torch.randperm(24, generator=torch.Generator().manual_seed(1)).cuda()
+    out_p = moe.moe_forward(dev[0][p].contiguous(), *dev[1:], 2)
+    assert torch.equal(out_p, out[p])
+
+
+def test_decode_host_entry_matches_device(moe, small):
+    _, dev = small
+    a = moe.moe_forward(*dev, 2)
+    b = moe.moe_forward_host(dev[0].cpu().pin_memory(), *dev[1:], 2)
+    assert torch.equal(a.cpu(), b)
+
+
+def test_paths_agree_closely(moe, small):
+    """Decode and grouped-GEMM paths compute the same function (different summation order)."""
+    _, dev = small
+    a = moe.moe_forward_ws(*dev, 2, path=moe.MOE_PATH_DECODE).float()
+    b = moe.moe_forward_ws(*dev, 2, path=moe.MOE_PATH_PREFILL).float()
+    rms = b.pow(2).mean().sqrt()
+    assert (a - b).abs().max() <= 1e-2 * rms
