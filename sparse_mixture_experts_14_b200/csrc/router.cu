@@ -343,6 +343,97 @@ __global__ void __launch_bounds__(256) router_smem_kernel(const __nv_bfloat16* _
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// bf16 scores on the tensor cores (mma.sync m16n8k16, bf16 x bf16 -> fp32).
+// The score matrix is the contraction x [T][d] . Wg^T [d][E]; with E <= 8 one
+// n8 tile holds all experts.  A block takes 16 tokens and its 8 warps split d
+// into 32-wide steps (warp w: steps w, w+8, ...).  Thread (g, q) of a warp
+// loads 16 bytes of rows g and g+8 of x and of row g of Wg at k0 + 8q and
+// feeds them to two MMAs: the MMA's k slots are a fixed permutation of the 32
+// physical k of the step, the same for A and B, so the dot product is
+// unchanged.  Each warp adds its MMA accumulator into fp32 registers every 16
+// MMAs (K = 256), bounding the accumulation inside the tensor core; the 8 warp
+// sums are added in warp order.  Products of bf16 values are exact in fp32.
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int NT>
+__global__ void __launch_bounds__(256) router_mma_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ Wg, int T, int d, int E,
+                                                         int k, int32_t* __restrict__ idx, float* __restrict__ w) {
+    pdl_trigger();
+    pdl_wait();
+    constexpr int EB = 8 * NT;
+    __shared__ float part[8][16][EB + 1];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, q = lane & 3;
+    const int nsteps = d / 32;
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    for (int t0 = blockIdx.x * 16; t0 < T; t0 += gridDim.x * 16) {
+        const int r0 = t0 + g, r1 = t0 + g + 8;
+        const uint4* xr0 = reinterpret_cast<const uint4*>(x + (size_t)(r0 < T ? r0 : 0) * d);
+        const uint4* xr1 = reinterpret_cast<const uint4*>(x + (size_t)(r1 < T ? r1 : 0) * d);
+        float tot[NT][4], acc[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tot[n][i] = acc[n][i] = 0.f;
+        int since_flush = 0;
+#pragma unroll 4
+        for (int st = warp; st < nsteps; st += 8) {
+            const int c = st * 4 + q;   // 16-byte chunk index of k0 + 8q
+            const uint4 xa = r0 < T ? __ldg(xr0 + c) : zero;
+            const uint4 xb = r1 < T ? __ldg(xr1 + c) : zero;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int e = n * 8 + g;
+                const uint4 wv = e < E ? __ldg(reinterpret_cast<const uint4*>(Wg + (size_t)e * d) + c) : zero;
+                mma_bf16_16816(acc[n], xa.x, xb.x, xa.y, xb.y, wv.x, wv.y);
+                mma_bf16_16816(acc[n], xa.z, xb.z, xa.w, xb.w, wv.z, wv.w);
+            }
+            if (++since_flush == 8) {
+                since_flush = 0;
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        tot[n][i] += acc[n][i];
+                        acc[n][i] = 0.f;
+                    }
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tot[n][i] += acc[n][i];
+            // c0, c1: token g, experts 2q, 2q+1; c2, c3: token g + 8
+            part[warp][g][n * 8 + 2 * q] = tot[n][0];
+            part[warp][g][n * 8 + 2 * q + 1] = tot[n][1];
+            part[warp][g + 8][n * 8 + 2 * q] = tot[n][2];
+            part[warp][g + 8][n * 8 + 2 * q + 1] = tot[n][3];
+        }
+        __syncthreads();
+        if (threadIdx.x < 16 && t0 + (int)threadIdx.x < T) {
+            const int t = threadIdx.x;
+            float sc[EB];
+#pragma unroll
+            for (int e = 0; e < EB; ++e) {
+                float v = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < 8; ++ww) v += part[ww][t][e];
+                sc[e] = v;
+            }
+            select_and_gate<EB>(sc, E, k, idx + (size_t)(t0 + t) * k, w + (size_t)(t0 + t) * k);
+        }
+        __syncthreads();
+    }
+}
+
 constexpr int kSmemRouterTB = 4;
 constexpr size_t kSmemRouterMax = 200 * 1024;
 
@@ -391,6 +482,16 @@ cudaError_t launch_router_any(const In* x, const In* Wg, int T, int d, int E, in
 
 cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
                                int num_sms, cudaStream_t s) {
+    if (d % 32 == 0) {
+        const int tiles = (T + 15) / 16;
+        int grid = tiles < num_sms * 16 ? tiles : num_sms * 16;
+        if (grid < 1) grid = 1;
+        const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+        const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(Wg);
+        if (E <= 8) return launch_pdl(router_mma_kernel<1>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
+        if (E <= 16) return launch_pdl(router_mma_kernel<2>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
+        return launch_pdl(router_mma_kernel<4>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
+    }
     const size_t smem = router_smem_bytes(d, E);
     if (E <= 8 && smem > 0 && T > 4 * num_sms) {
         static bool attr = false;
