@@ -244,6 +244,19 @@ def run_reference(args, rank):
 # ------------------------------------------------------------------ our arm
 
 
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank number over all ranks (the job's time is its slowest rank's)."""
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Tokens per second of the whole job: every rank processes its own batch each step."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1000.0)
+
+
 def to_dev(a, dtype, device):
     if dtype == "bf16":
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
@@ -308,11 +321,8 @@ def run_ours(args, rank, world, local):
     else:
         total_ms = start.elapsed_time(end)
     stage_ms = [statistics.mean(events[i][s].elapsed_time(events[i][s + 1]) for i in range(K)) for s in range(ns)]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
-    value = world * T * K / (total_ms / 1000.0)
+    total_ms = reduce_max(total_ms, world, device)
+    value = weak_scaling_value(T, K, world, total_ms)
 
     # e2e: host buffers, copies inside every step
     e2e = None
@@ -327,10 +337,8 @@ def run_ours(args, rank, world, local):
             t0 = time.perf_counter()
             for _ in range(K):
                 moe.moe_forward_host(x_host, *dev[1:], k, out_host)
-            wall = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=device)
-            if world > 1:
-                torch.distributed.all_reduce(wall, op=torch.distributed.ReduceOp.MAX)
-            e2e = {"value": world * T * K / float(wall.item()), "unit": "tokens/s",
+            wall = reduce_max(time.perf_counter() - t0, world, device)
+            e2e = {"value": weak_scaling_value(T, K, world, wall * 1000.0), "unit": "tokens/s",
                    "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
                    "timing": "host wall clock around moe_forward_host (synchronises every step)"}
 

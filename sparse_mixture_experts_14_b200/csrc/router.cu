@@ -482,7 +482,8 @@ cudaError_t launch_router_any(const In* x, const In* Wg, int T, int d, int E, in
 
 cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
                                int num_sms, cudaStream_t s) {
-    if (d % 32 == 0) {
+    // tensor-core scores for large batches; small batches spread one token per block instead
+    if (d % 32 == 0 && T > 4 * num_sms) {
         const int tiles = (T + 15) / 16;
         int grid = tiles < num_sms * 16 ? tiles : num_sms * 16;
         if (grid < 1) grid = 1;

@@ -1,0 +1,77 @@
+"""The multi-rank plumbing of bench.py on CPU: gloo, world size 2, no GPU.
+
+The layer shards by tokens with no exchange (replicas), so the only
+cross-rank steps are the barrier and the max-over-ranks of the timings.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import bench
+    from datetime import timedelta
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        ms = 10.0 + 5.0 * rank                       # rank 1 is the slow one
+        m = bench.reduce_max(ms, world)
+        v = bench.weak_scaling_value(16, 100, world, m)
+        torch.distributed.barrier()
+        q.put((rank, m, v))
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+def test_max_over_ranks_and_weak_scaling_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, m, v in res:
+        assert m == 15.0                             # every rank sees the slowest rank's time
+        assert v == pytest.approx(2 * 16 * 100 / 0.015)
+
+
+def test_single_rank_helpers():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.reduce_max(3.5, 1) == 3.5
+    assert bench.weak_scaling_value(16, 10, 1, 100.0) == pytest.approx(1600.0)
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """Rank 0 prints one JSON line for the reference arm; rank 1 exits 0 without work."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "1", "--gpus", "2",
+           "--steps", "2", "--warmup", "1"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["n_gpus"] == 2
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"

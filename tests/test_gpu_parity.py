@@ -39,6 +39,19 @@ def test_route_small(moe, dtype, d, E, k):
     _status_clear(moe)
 
 
+@pytest.mark.parametrize("d", [192, 320, 1024])
+@pytest.mark.parametrize("E,k", [(3, 2), (8, 2), (16, 4), (32, 2)])
+def test_route_large_batches(moe, d, E, k):
+    """Batches above 4 x SMs take the tensor-core score path (16-token tiles, warps split d)."""
+    inp = moe_inputs.make_inputs(1000, d, 128, E, k, "bf16", seed=500 + d + E, weights=False)
+    x, Wg = upload(inp)[:2]
+    idx, w = moe.moe_route(x, Wg, k)
+    ref = oracle.route(inp.x, inp.Wg, k, "bf16")
+    keep = compare_routing(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    assert keep.mean() > 0.98
+    _status_clear(moe)
+
+
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
 def test_route_configs(moe, cfg):
     inp = moe_inputs.make_config(cfg, weights=False)
