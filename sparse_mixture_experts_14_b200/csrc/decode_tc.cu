@@ -328,13 +328,12 @@ bool map_x(CUtensorMap* m, const void* base, size_t rows, int K) {
 template <bool GATE>
 cudaError_t launch_stage(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& x, const TcGemmArgs& g, int K,
                          int R, void* out, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e =
-            cudaFuncSetAttribute(decode_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsmem_bytes<GATE>());
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static PerDeviceOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(decode_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    dsmem_bytes<GATE>());
+    });
+    if (e != cudaSuccess) return e;
     int grid = g.num_sms > 0 ? g.num_sms : 148;
     const int upper = g.E * ((R + DM - 1) / DM);
     if (grid > upper) grid = upper;

@@ -384,21 +384,17 @@ bool map_weights(CUtensorMap* m, const void* base, int E, int R, int K, int box_
 
 template <bool SWIGLU>
 cudaError_t ensure_smem_attr() {
-    static bool done = false;
-    if (!done) {
-        cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        done = true;
-    }
-    return cudaSuccess;
+    static PerDeviceOnce once;
+    return once.run([] {
+        return cudaFuncSetAttribute(tc_gemm_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    });
 }
 
 // Persistent grid: as many CTA pairs as fit at once, no more than there are pair tiles.
 template <bool SWIGLU>
 int grid_for(size_t slots, int n_tiles_per_m, int num_sms) {
-    static int max_clusters = -1;
-    if (max_clusters < 0) {
+    static PerDeviceInt clusters_per_device;
+    const int max_clusters = clusters_per_device.get([num_sms] {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * 74, 1, 1);
         cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -415,8 +411,8 @@ int grid_for(size_t slots, int n_tiles_per_m, int num_sms) {
             cudaGetLastError();
             n = (num_sms > 0 ? num_sms : 148) / 2;
         }
-        max_clusters = n;
-    }
+        return n;
+    });
     const size_t pair_rows = (slots / BM + 1) / 2;
     const size_t upper = pair_rows * (size_t)n_tiles_per_m;
     size_t clusters = (size_t)max_clusters;

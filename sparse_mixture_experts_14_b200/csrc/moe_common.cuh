@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -49,6 +51,49 @@ __device__ __forceinline__ float silu_mul(float a, float b) {
 }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Set-up that CUDA keeps per device (function attributes, occupancy facts):
+// run f once on each device that is current when it is needed.  Concurrent
+// first calls may both run f, which must therefore be idempotent.
+class PerDeviceOnce {
+   public:
+    template <typename F>
+    cudaError_t run(F&& f) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSlots) return f();
+        if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        const cudaError_t e = f();
+        if (e == cudaSuccess) done_[dev].store(1, std::memory_order_release);
+        return e;
+    }
+
+   private:
+    static constexpr int kSlots = 64;
+    std::atomic<int> done_[kSlots] = {};
+};
+
+// A per-device integer computed once (e.g. an occupancy limit).
+class PerDeviceInt {
+   public:
+    template <typename F>
+    int get(F&& f) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSlots) return f();
+        int v = val_[dev].load(std::memory_order_acquire);
+        if (v < 0) {
+            v = f();
+            val_[dev].store(v, std::memory_order_release);
+        }
+        return v;
+    }
+    PerDeviceInt() {
+        for (auto& x : val_) x.store(-1);
+    }
+
+   private:
+    static constexpr int kSlots = 64;
+    std::atomic<int> val_[kSlots];
+};
 
 // Programmatic dependent launch.  Every kernel of the layer is launched with
 // programmatic stream serialisation: it lets the next kernel in the stream be

@@ -495,13 +495,12 @@ cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int 
     }
     const size_t smem = router_smem_bytes(d, E);
     if (E <= 8 && smem > 0 && T > 4 * num_sms) {
-        static bool attr = false;
-        if (!attr) {
-            cudaError_t e = cudaFuncSetAttribute(router_smem_kernel<8, kSmemRouterTB>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemRouterMax);
-            if (e != cudaSuccess) return e;
-            attr = true;
-        }
+        static PerDeviceOnce attr;
+        cudaError_t e = attr.run([] {
+            return cudaFuncSetAttribute(router_smem_kernel<8, kSmemRouterTB>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemRouterMax);
+        });
+        if (e != cudaSuccess) return e;
         const int groups = (T + kSmemRouterTB - 1) / kSmemRouterTB;
         const int per_sm = smem <= 110 * 1024 ? 2 : 1;
         int grid = num_sms * per_sm;
