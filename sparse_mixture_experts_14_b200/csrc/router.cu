@@ -3,12 +3,14 @@
 // "Mistral/Mixtral architecture" page (score, Top-2 and gate equations) and its
 // MoERouter.forward in "簡易MoEルーターの実装", fused into one pass over x.
 //
-// One block (8 warps) owns a few consecutive tokens (one per block for small
-// batches); its threads split each row into 16-byte chunks, and every chunk a
-// thread needs is in flight before the arithmetic starts.  Partial sums are
-// reduced in a fixed order (xor-butterfly, then warp order), so the fp32
-// scores are identical run to run for a given batch size; they are never
-// rounded to bf16.  The pass is bound by reading x once from HBM.
+// Large bf16 batches: scores on the tensor cores (router_mma_kernel, 16
+// tokens per block, warps split d).  Small batches and fp32 inputs: CUDA-core
+// dot products (router_kernel, one block per token or per few tokens, every
+// 16-byte chunk a thread needs in flight before the arithmetic; rows longer
+// than 1024 chunks loop, router_loop_kernel).  Partial sums are reduced in a
+// fixed order (xor-butterfly or MMA accumulation, then warp order), so the
+// fp32 scores are identical run to run for a given batch size; they are
+// never rounded to bf16.  The pass is bound by reading x once from HBM.
 #include "moe_common.cuh"
 
 namespace moe {
@@ -205,144 +207,6 @@ __global__ void __launch_bounds__(256) router_kernel(const In* __restrict__ x, c
     }
 }
 
-// (bf16 pair) -> (f32, f32) in one 64-bit register: element 0 low, element 1 high
-__device__ __forceinline__ unsigned long long bf16x2_to_f32x2(uint32_t w) {
-    unsigned long long r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xffff0000u));
-    return r;
-}
-// acc.lo += a.lo * b.lo, acc.hi += a.hi * b.hi (one instruction, round to nearest)
-__device__ __forceinline__ void ffma2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
-}
-__device__ __forceinline__ float sum_f32x2(unsigned long long v) {
-    uint32_t lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
-    return __uint_as_float(lo) + __uint_as_float(hi);
-}
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
-                 "l"(gmem_src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-
-// Large batches: persistent blocks that keep Wg in shared memory and walk
-// groups of TB tokens, the next group's rows streaming into the other half of
-// a double buffer (cp.async) while the current group is reduced.  HBM sees x
-// once and Wg once per SM.  The arithmetic is packed: each f32x2 FMA handles
-// an (even k, odd k) pair, so every thread keeps two partial sums per (token,
-// expert), added at the end; a reduce-scatter butterfly then leaves one
-// (token, expert) sum per lane, and the 8 warp sums are added in warp order.
-// The order is fixed, so the scores are identical run to run.
-template <int EB, int TB>
-__global__ void __launch_bounds__(256) router_smem_kernel(const __nv_bfloat16* __restrict__ x,
-                                                          const __nv_bfloat16* __restrict__ Wg, int T, int d, int E,
-                                                          int k, int32_t* __restrict__ idx, float* __restrict__ w) {
-    pdl_trigger();
-    pdl_wait();
-    extern __shared__ uint4 sm[];
-    using Raw = uint4;
-    const int nchunks = d / 8;
-    uint4* sWg = sm;                                   // [E][nchunks]
-    uint4* sx = sm + (size_t)E * nchunks;              // [2][TB][nchunks]
-    static_assert(TB * EB == 32, "one reduced value per lane");
-    __shared__ float part_flat[8][32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int ngroups = (T + TB - 1) / TB;
-
-    const uint4* gW = reinterpret_cast<const uint4*>(Wg);
-    for (int i = threadIdx.x; i < E * nchunks; i += 256) cp_async16(sWg + i, gW + i);
-    auto issue = [&](int g, int buf) {
-        if (g < ngroups) {
-            for (int i = threadIdx.x; i < TB * nchunks; i += 256) {
-                const int t = g * TB + i / nchunks;
-                const int c = i - (i / nchunks) * nchunks;
-                if (t < T) cp_async16(sx + ((size_t)buf * TB * nchunks + i), reinterpret_cast<const uint4*>(x + (size_t)t * d) + c);
-            }
-        }
-        cp_async_commit();
-    };
-    int buf = 0;
-    issue(blockIdx.x, 0);
-    for (int g = blockIdx.x; g < ngroups; g += gridDim.x) {
-        issue(g + gridDim.x, buf ^ 1);
-        cp_async_wait1();
-        __syncthreads();
-        const int t0 = g * TB;
-        // acc[t][e] holds two partial sums (even and odd k) in one f32x2 register
-        unsigned long long acc[TB][EB];
-#pragma unroll
-        for (int t = 0; t < TB; ++t)
-#pragma unroll
-            for (int e = 0; e < EB; ++e) acc[t][e] = 0ull;
-        const uint4* xb = sx + (size_t)buf * TB * nchunks;
-        for (int c = threadIdx.x; c < nchunks; c += 256) {
-            unsigned long long xv[TB][4];
-#pragma unroll
-            for (int t = 0; t < TB; ++t) {
-                const uint4 r = (t0 + t < T) ? xb[t * nchunks + c] : make_uint4(0, 0, 0, 0);
-                xv[t][0] = bf16x2_to_f32x2(r.x);
-                xv[t][1] = bf16x2_to_f32x2(r.y);
-                xv[t][2] = bf16x2_to_f32x2(r.z);
-                xv[t][3] = bf16x2_to_f32x2(r.w);
-            }
-#pragma unroll
-            for (int e = 0; e < EB; ++e) {
-                const uint4 r = sWg[(size_t)(e < E ? e : E - 1) * nchunks + c];
-                const unsigned long long w0 = bf16x2_to_f32x2(r.x), w1 = bf16x2_to_f32x2(r.y);
-                const unsigned long long w2 = bf16x2_to_f32x2(r.z), w3 = bf16x2_to_f32x2(r.w);
-#pragma unroll
-                for (int t = 0; t < TB; ++t) {
-                    ffma2(acc[t][e], xv[t][0], w0);
-                    ffma2(acc[t][e], xv[t][1], w1);
-                    ffma2(acc[t][e], xv[t][2], w2);
-                    ffma2(acc[t][e], xv[t][3], w3);
-                }
-            }
-        }
-        // even + odd partials, then a reduce-scatter butterfly: lane L ends with
-        // the warp's sum of value L = t * EB + e
-        float v[TB * EB];
-#pragma unroll
-        for (int t = 0; t < TB; ++t)
-#pragma unroll
-            for (int e = 0; e < EB; ++e) v[t * EB + e] = sum_f32x2(acc[t][e]);
-#pragma unroll
-        for (int m = 16, n = 16; m >= 1; m >>= 1, n >>= 1) {
-            const bool upper = (lane & m) != 0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                if (i < n) {
-                    const float send = upper ? v[i] : v[i + n];
-                    const float keep = upper ? v[i + n] : v[i];
-                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                }
-            }
-        }
-        part_flat[warp][lane] = v[0];
-        __syncthreads();
-        if (threadIdx.x < TB && t0 + (int)threadIdx.x < T) {
-            const int t = threadIdx.x;
-            float sc[EB];
-#pragma unroll
-            for (int e = 0; e < EB; ++e) {
-                float acc_e = 0.f;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) acc_e += part_flat[q][t * EB + e];
-                sc[e] = acc_e;
-            }
-            select_and_gate<EB>(sc, E, k, idx + (size_t)(t0 + t) * k, w + (size_t)(t0 + t) * k);
-        }
-        buf ^= 1;
-        __syncthreads();
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
 // bf16 scores on the tensor cores (mma.sync m16n8k16, bf16 x bf16 -> fp32).
 // The score matrix is the contraction x [T][d] . Wg^T [d][E]; with E <= 8 one
 // n8 tile holds all experts.  A block takes 16 tokens and its 8 warps split d
@@ -434,15 +298,6 @@ __global__ void __launch_bounds__(256) router_mma_kernel(const __nv_bfloat16* __
     }
 }
 
-constexpr int kSmemRouterTB = 4;
-constexpr size_t kSmemRouterMax = 200 * 1024;
-
-// Shared memory the persistent bf16 router needs, or 0 when it does not fit.
-size_t router_smem_bytes(int d, int E) {
-    const size_t b = ((size_t)E + 2 * kSmemRouterTB) * (size_t)d * 2;
-    return b <= kSmemRouterMax ? b : 0;
-}
-
 // Chunks per thread the kernels are compiled for: 16-byte chunks x 256 threads x RMAX
 // cover d <= 8192 (bf16) / 4096 (fp32) with RMAX = 4; longer rows take the looping form.
 template <typename In, int EB, int TB>
@@ -492,22 +347,6 @@ cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int 
         if (E <= 8) return launch_pdl(router_mma_kernel<1>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
         if (E <= 16) return launch_pdl(router_mma_kernel<2>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
         return launch_pdl(router_mma_kernel<4>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
-    }
-    const size_t smem = router_smem_bytes(d, E);
-    if (E <= 8 && smem > 0 && T > 4 * num_sms) {
-        static PerDeviceOnce attr;
-        cudaError_t e = attr.run([] {
-            return cudaFuncSetAttribute(router_smem_kernel<8, kSmemRouterTB>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemRouterMax);
-        });
-        if (e != cudaSuccess) return e;
-        const int groups = (T + kSmemRouterTB - 1) / kSmemRouterTB;
-        const int per_sm = smem <= 110 * 1024 ? 2 : 1;
-        int grid = num_sms * per_sm;
-        if (grid > groups) grid = groups;
-        return launch_pdl(router_smem_kernel<8, kSmemRouterTB>, dim3(grid), dim3(256), smem, s,
-                          static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wg), T, d, E, k,
-                          idx, w);
     }
     return launch_router_any<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x),
                                             static_cast<const __nv_bfloat16*>(Wg), T, d, E, k, idx, w, num_sms,

@@ -52,6 +52,17 @@ def test_route_large_batches(moe, d, E, k):
     _status_clear(moe)
 
 
+@pytest.mark.parametrize("dtype,d", [("bf16", 8256), ("f32", 4200)])
+def test_route_long_rows(moe, dtype, d):
+    """Rows longer than 1024 16-byte chunks take the looping router."""
+    inp = moe_inputs.make_inputs(40, d, 64, 8, 2, dtype, seed=d, weights=False)
+    x, Wg = upload(inp)[:2]
+    idx, w = moe.moe_route(x, Wg, 2)
+    ref = oracle.route(inp.x, inp.Wg, 2, dtype)
+    compare_routing(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    _status_clear(moe)
+
+
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
 def test_route_configs(moe, cfg):
     inp = moe_inputs.make_config(cfg, weights=False)
