@@ -25,6 +25,7 @@
 
 #include "moe_common.cuh"
 #include "ptx_sm100.cuh"
+#include "tma_map.cuh"
 
 namespace moe {
 namespace {
@@ -288,42 +289,13 @@ __global__ void __launch_bounds__(DTHREADS, 1)
     }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-            const cuuint32_t* box) {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return false;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // E x R x K weights, K contiguous, box 64 x 128 x 1
 bool map_w(CUtensorMap* m, const void* base, int E, int R, int K) {
-    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)R, (cuuint64_t)E};
-    cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)R * K * 2};
-    cuuint32_t box[3] = {(cuuint32_t)DK, (cuuint32_t)DM, 1};
-    return encode(m, base, 3, dims, strides, box);
+    return map_expert_weights(m, base, E, R, K, DK, DM);
 }
 
 // rows x K token matrix, box 64 x 64
-bool map_x(CUtensorMap* m, const void* base, size_t rows, int K) {
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)DK, (cuuint32_t)DNMAX};
-    return encode(m, base, 2, dims, strides, box);
-}
+bool map_x(CUtensorMap* m, const void* base, size_t rows, int K) { return map_matrix(m, base, rows, K, DK, DNMAX); }
 
 template <bool GATE>
 cudaError_t launch_stage(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& x, const TcGemmArgs& g, int K,
