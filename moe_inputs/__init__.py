@@ -14,6 +14,11 @@ Operand layouts (row-major, the ``nn.Linear`` weight convention of the
 Initialisation: x ~ N(0, 1), Wg, W1, W3 ~ N(0, 1/d), W2 ~ N(0, 1/F).  bf16
 operands are returned as uint16 bit patterns, fp32 operands as float32.
 
+Block operands (the MoE sub-layer with its pre-norm and residual): the
+residual stream h is x with row t scaled by 2^((t mod 5) - 2), an exact
+power-of-two scale in bf16 and fp32, so rows span a 16x range of norms; the
+norm gain is gamma_j = 1 + 0.2 N(0, 1), rounded to the operand dtype.
+
 The skewed workload sets feature 0 of every token to exactly 1.0 and
 Wg[e][0] to a stored per-expert constant b_e, which adds b_e to the logit of
 expert e (the router has no bias term, so the bias rides on a constant input
@@ -37,7 +42,8 @@ _LIB_PATH = os.path.join(_HERE, "libmoe_inputs.so")
 _lock = threading.Lock()
 _lib = None
 
-TENSOR_IDS = {"x": 0, "Wg": 1, "W1": 2, "W3": 3, "W2": 4}
+TENSOR_IDS = {"x": 0, "Wg": 1, "W1": 2, "W3": 3, "W2": 4, "gamma": 5}
+BLOCK_EPS = 1e-5      # eps of the block's RMSNorm in every test and workload
 BF16_ONE = 0x3F80
 
 
@@ -125,6 +131,7 @@ class MoEInputs:
     W1: np.ndarray = field(default=None, repr=False)
     W3: np.ndarray = field(default=None, repr=False)
     W2: np.ndarray = field(default=None, repr=False)
+    gamma: np.ndarray = field(default=None, repr=False)   # block operands only
 
     def arrays(self):
         return self.x, self.Wg, self.W1, self.W3, self.W2
@@ -156,6 +163,24 @@ def make_inputs(T: int, d: int, F: int, E: int, k: int, dtype: str = "bf16", see
         inp.W1 = normal((E, F, d), seed, TENSOR_IDS["W1"], 1.0 / np.sqrt(d), dtype)
         inp.W3 = normal((E, F, d), seed, TENSOR_IDS["W3"], 1.0 / np.sqrt(d), dtype)
         inp.W2 = normal((E, d, F), seed, TENSOR_IDS["W2"], 1.0 / np.sqrt(F), dtype)
+    return inp
+
+
+def row_scales(T: int) -> np.ndarray:
+    """The block recipe's per-row power-of-two scales of the residual stream."""
+    return np.ldexp(np.float32(1.0), (np.arange(T) % 5) - 2).astype(np.float32)
+
+
+def make_block(inp: MoEInputs) -> MoEInputs:
+    """Turn one layer's operands into block operands: x becomes the residual h, gamma is added."""
+    sc = row_scales(inp.T)[:, None]
+    if inp.dtype == "bf16":
+        inp.x = f32_to_bf16_bits(bf16_bits_to_f32(inp.x) * sc)          # exact: power-of-two scales
+        g = normal((inp.d,), inp.seed, TENSOR_IDS["gamma"], 0.2, "f32")
+        inp.gamma = f32_to_bf16_bits(np.float32(1.0) + g)
+    else:
+        inp.x = np.ascontiguousarray(inp.x * sc, dtype=np.float32)
+        inp.gamma = (np.float32(1.0) + normal((inp.d,), inp.seed, TENSOR_IDS["gamma"], 0.2, "f32")).astype(np.float32)
     return inp
 
 

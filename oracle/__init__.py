@@ -17,6 +17,18 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   moe                      pinned: k=E uniform average, E=1 dense FFN, hand
                            example, permutation/relabelling invariances
   counts                   pinned: sums to k*T, brute-force histogram
+  rmsnorm                  pinned: torch's rms_norm in fp64, hand example,
+                           power-of-two homogeneity, unit RMS at eps = 0
+  block / block_scores     pinned: E=1 dense block and k=E uniform block
+                           against torch fp64, scale invariance of the
+                           routing, zero row
+  balance                  pinned: uniform scores (loss = alpha*k), cyclic
+                           balanced batch, brute force against torch,
+                           sums of f and p
+
+The block and balance steps follow the same page, section "Mixtral 8x7B —
+Sparse MoEの導入" (subsection "Mixtralのアーキテクチャ": RMSNorm, MoE layer,
+residual) and subsection "ロードバランス損失" (f, p and loss equations).
 """
 from __future__ import annotations
 
@@ -58,6 +70,12 @@ def _load():
             lib.oracle_moe.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, ci, vp, vp, vp, vp,
                                        vp, ci]
             lib.oracle_counts.argtypes = [ci, ci, ci, vp, vp]
+            cd = ctypes.c_double
+            lib.oracle_rmsnorm.argtypes = [ci, ci, vp, vp, cd, ci, vp]
+            lib.oracle_block_scores.argtypes = [ci, ci, ci, vp, vp, cd, vp, ci, vp, ci]
+            lib.oracle_block.argtypes = [ci, ci, ci, ci, ci, vp, vp, cd, vp, vp, vp, vp, ci, vp, ci, vp, vp, vp,
+                                         vp, vp, ci]
+            lib.oracle_balance.argtypes = [ci, ci, ci, vp, cd, vp, vp, vp]
             lib.oracle_max_threads.restype = ci
             _lib = lib
     return _lib
@@ -161,3 +179,62 @@ def counts(idx, E: int) -> np.ndarray:
     c = np.empty(E, dtype=np.int64)
     _check(_load().oracle_counts(T, k, E, idx.ctypes.data, c.ctypes.data), "counts")
     return c
+
+
+def rmsnorm(h, gamma, eps: float, dtype: str) -> np.ndarray:
+    """RMSNorm of every row, in double: gamma_j h_j / sqrt(mean(h^2) + eps)."""
+    h, gamma = _arr(h, dtype), _arr(gamma, dtype)
+    T, d = h.shape
+    if gamma.shape != (d,):
+        raise ValueError("gamma must have shape [d]")
+    u = np.empty((T, d), dtype=np.float64)
+    _check(_load().oracle_rmsnorm(T, d, h.ctypes.data, gamma.ctypes.data, float(eps), DTYPE_CODE[dtype],
+                                  u.ctypes.data), "rmsnorm")
+    return u
+
+
+def block_scores(h, gamma, eps: float, Wg, dtype: str, nthreads: int = 0) -> np.ndarray:
+    """Router scores of the normalised rows: [T][E] = Wg RMSNorm(h_t)."""
+    h, gamma, Wg = _arr(h, dtype), _arr(gamma, dtype), _arr(Wg, dtype)
+    T, d = h.shape
+    E = Wg.shape[0]
+    out = np.empty((T, E), dtype=np.float64)
+    _check(_load().oracle_block_scores(T, d, E, h.ctypes.data, gamma.ctypes.data, float(eps), Wg.ctypes.data,
+                                       DTYPE_CODE[dtype], out.ctypes.data, nthreads), "block_scores")
+    return out
+
+
+def block(h, gamma, eps: float, Wg, W1, W3, W2, k: int, dtype: str, tokens=None, nthreads: int = 0) -> dict:
+    """out = h + MoE(RMSNorm(h)) for all tokens or the listed ones; same dict as moe()."""
+    h, gamma, Wg, W1, W3, W2 = (_arr(a, dtype) for a in (h, gamma, Wg, W1, W3, W2))
+    T, d = h.shape
+    E, F = W1.shape[0], W1.shape[1]
+    if tokens is None:
+        tok = None
+        n = T
+    else:
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = tok.size
+    out = np.empty((n, d), dtype=np.float64)
+    idx = np.empty((n, k), dtype=np.int32)
+    g = np.empty((n, k), dtype=np.float64)
+    margin = np.empty(n, dtype=np.float64)
+    mingap = np.empty(n, dtype=np.float64)
+    _check(_load().oracle_block(T, d, F, E, k, h.ctypes.data, gamma.ctypes.data, float(eps), Wg.ctypes.data,
+                                W1.ctypes.data, W3.ctypes.data, W2.ctypes.data, DTYPE_CODE[dtype],
+                                None if tok is None else tok.ctypes.data, n, out.ctypes.data, idx.ctypes.data,
+                                g.ctypes.data, margin.ctypes.data, mingap.ctypes.data, nthreads), "block")
+    return dict(out=out, idx=idx, g=g, margin=margin, mingap=mingap,
+                tokens=np.arange(T, dtype=np.int32) if tok is None else tok)
+
+
+def balance(logits, k: int, alpha: float):
+    """Load-balance statistics from fp64 scores [T][E]: (f [E], p [E], loss)."""
+    s = np.ascontiguousarray(logits, dtype=np.float64)
+    T, E = s.shape
+    f = np.empty(E, dtype=np.float64)
+    p = np.empty(E, dtype=np.float64)
+    loss = np.empty(1, dtype=np.float64)
+    _check(_load().oracle_balance(T, E, k, s.ctypes.data, float(alpha), f.ctypes.data, p.ctypes.data,
+                                  loss.ctypes.data), "balance")
+    return f, p, float(loss[0])

@@ -35,6 +35,21 @@
  * Only selected experts are evaluated: an unselected expert has gate weight
  * exactly zero, so it adds nothing.
  *
+ * Two steps around the layer, from the same page:
+ *
+ *   6. the block       out = h + MoE(RMSNorm(h)): section "Mixtral 8x7B — Sparse
+ *                      MoEの導入", subsection "Mixtralのアーキテクチャ" (the second
+ *                      sub-layer of every Transformer block: RMSNorm, then the MoE
+ *                      layer, then the residual connection).  The page names
+ *                      RMSNorm without printing it; this file uses the usual
+ *                      definition RMSNorm(h)_j = gamma_j h_j / sqrt(mean_i(h_i^2) + eps)
+ *                      with a per-channel gain gamma and the caller's eps.
+ *   7. load balance    f_i = (1/T) #{t : i among the top-k of s_t},
+ *                      p_i = (1/T) sum_t softmax(s_t)_i over all E experts,
+ *                      L = alpha * E * sum_i f_i p_i: subsection "ロードバランス損失"
+ *                      (f, p and loss equations), with f counting all k
+ *                      selections as the page's load_balance_loss code does.
+ *
  * Operands are row-major: x[T][d], Wg[E][d], W1[E][F][d], W3[E][F][d],
  * W2[E][d][F].  dtype 0 = float32 storage, 1 = bfloat16 bit patterns; every
  * element is widened exactly to double before use.
@@ -225,6 +240,145 @@ int oracle_moe(int T, int d, int F, int E, int k, const void* x, const void* Wg,
         free(y);
     }
     return fail ? 2 : 0;
+}
+
+/* ------------------------------------------------------------------ block */
+
+/* step 6, the norm, for one row: u_j = gamma_j * h_j / sqrt((1/d) sum_i h_i^2 + eps) */
+static void row_rmsnorm(int d, const void* h, const void* gamma, double eps, int dtype, size_t t, double* u) {
+    double ss = 0.0;
+    for (int j = 0; j < d; ++j) {
+        double v = elem(h, dtype, t * (size_t)d + j);
+        ss += v * v;
+    }
+    double r = 1.0 / sqrt(ss / (double)d + eps);
+    for (int j = 0; j < d; ++j) u[j] = elem(gamma, dtype, (size_t)j) * (elem(h, dtype, t * (size_t)d + j) * r);
+}
+
+/* step 1 on a vector already in double: s[e] = sum_j v[j] * Wg[e][j], j ascending */
+static void vector_scores(int d, int E, const double* v, const void* Wg, int dtype, double* s) {
+    for (int e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int j = 0; j < d; ++j) acc += v[j] * elem(Wg, dtype, (size_t)e * d + j);
+        s[e] = acc;
+    }
+}
+
+/* the norm alone for every row: u[T][d] */
+int oracle_rmsnorm(int T, int d, const void* h, const void* gamma, double eps, int dtype, double* u) {
+    if (T < 0 || d <= 0 || !(eps >= 0.0)) return 1;
+    for (int t = 0; t < T; ++t) row_rmsnorm(d, h, gamma, eps, dtype, (size_t)t, u + (size_t)t * d);
+    return 0;
+}
+
+/* router scores of the normalised rows: logits[T][E] = Wg RMSNorm(h_t) */
+int oracle_block_scores(int T, int d, int E, const void* h, const void* gamma, double eps, const void* Wg,
+                        int dtype, double* logits, int nthreads) {
+    if (T < 0 || d <= 0 || E <= 0 || E > 64 || !(eps >= 0.0)) return 1;
+    int fail = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        double* u = (double*)malloc(sizeof(double) * d);
+        if (!u) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int t = 0; t < T; ++t) {
+                row_rmsnorm(d, h, gamma, eps, dtype, (size_t)t, u);
+                vector_scores(d, E, u, Wg, dtype, logits + (size_t)t * E);
+            }
+        }
+        free(u);
+    }
+    return fail ? 2 : 0;
+}
+
+/*
+ * The block out = h + MoE(RMSNorm(h)) for the tokens listed in tokens[0..n)
+ * (all tokens when tokens == NULL, n == T).  Steps 1-5 run on u = RMSNorm(h_t)
+ * exactly as in oracle_moe, then the row h_t is added.  out[n][d] in double.
+ */
+int oracle_block(int T, int d, int F, int E, int k, const void* h, const void* gamma, double eps, const void* Wg,
+                 const void* W1, const void* W3, const void* W2, int dtype, const int32_t* tokens, int n,
+                 double* out, int32_t* idx, double* g, double* margin, double* mingap, int nthreads) {
+    if (T < 0 || d <= 0 || F <= 0 || E <= 0 || E > 64 || k <= 0 || k > E || n < 0 || !(eps >= 0.0)) return 1;
+    if (!tokens && n != T) return 1;
+    for (int r = 0; r < n; ++r)
+        if (tokens && (tokens[r] < 0 || tokens[r] >= T)) return 1;
+    int fail = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        double* u = (double*)malloc(sizeof(double) * d);
+        double* hh = (double*)malloc(sizeof(double) * F);
+        double* y = (double*)malloc(sizeof(double) * d);
+        double* m = (double*)malloc(sizeof(double) * d);
+        if (!u || !hh || !y || !m) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int r = 0; r < n; ++r) {
+                size_t t = tokens ? (size_t)tokens[r] : (size_t)r;
+                row_rmsnorm(d, h, gamma, eps, dtype, t, u);
+                double s[64];
+                vector_scores(d, E, u, Wg, dtype, s);
+                int32_t* ir = idx + (size_t)r * k;
+                double* gr = g + (size_t)r * k;
+                token_select(E, k, s, ir, gr, margin + r, mingap + r);
+                for (int i = 0; i < d; ++i) m[i] = 0.0;
+                for (int j = 0; j < k; ++j) {
+                    expert_apply(d, F, u, W1, W3, W2, dtype, ir[j], hh, y);
+                    for (int i = 0; i < d; ++i) m[i] += gr[j] * y[i];
+                }
+                double* o = out + (size_t)r * d;
+                for (int i = 0; i < d; ++i) o[i] = elem(h, dtype, t * (size_t)d + i) + m[i];
+            }
+        }
+        free(u);
+        free(hh);
+        free(y);
+        free(m);
+    }
+    return fail ? 2 : 0;
+}
+
+/* ------------------------------------------------------------ load balance */
+
+/*
+ * step 7 from given scores logits[T][E]: f[E], p[E] and the loss.
+ * softmax over all E is evaluated as exp(s_e - max) / sum, the same number.
+ */
+int oracle_balance(int T, int E, int k, const double* logits, double alpha, double* f, double* p, double* loss) {
+    if (T <= 0 || E <= 0 || E > 64 || k <= 0 || k > E) return 1;
+    for (int e = 0; e < E; ++e) f[e] = p[e] = 0.0;
+    for (int t = 0; t < T; ++t) {
+        const double* s = logits + (size_t)t * E;
+        int32_t idx[64];
+        double g[64];
+        token_select(E, k, s, idx, g, NULL, NULL);
+        for (int j = 0; j < k; ++j) f[idx[j]] += 1.0;
+        double mx = s[0];
+        for (int e = 1; e < E; ++e)
+            if (s[e] > mx) mx = s[e];
+        double denom = 0.0;
+        for (int e = 0; e < E; ++e) denom += exp(s[e] - mx);
+        for (int e = 0; e < E; ++e) p[e] += exp(s[e] - mx) / denom;
+    }
+    double acc = 0.0;
+    for (int e = 0; e < E; ++e) {
+        f[e] /= (double)T;
+        p[e] /= (double)T;
+        acc += f[e] * p[e];
+    }
+    *loss = alpha * (double)E * acc;
+    return 0;
 }
 
 /* per-expert assignment counts: counts[e] = #{(t, j) : idx[t][j] == e} */
