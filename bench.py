@@ -45,6 +45,9 @@ sys.path.insert(0, ROOT)
 import moe_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/sec at 1 B200; achieved % of roofline (tensor TFLOPS or HBM GB/s)"
+BLOCK_METRIC = ("MoE sub-layer (RMSNorm + MoE + residual, load-balance statistics) tokens/sec at 1 B200; "
+                "achieved % of roofline")
+BLOCK_ALPHA = 0.01
 L2_BYTES = 126 * 1000 * 1000
 DEFAULT_CONFIG = 2   # the Mixtral-shape decode layer (T=16, d=4096, ffn=14336, E=8, k=2)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -60,6 +63,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--block", action="store_true",
+                    help="time the block form out = h + MoE(RMSNorm(h)) with load-balance statistics")
     ap.add_argument("--stage-every", type=int, default=8,
                     help="record per-stage events on every n-th timed step (events between launches "
                          "break the overlap of dependent launches, so most steps run without them)")
@@ -145,16 +150,22 @@ class ClockSampler:
 # ------------------------------------------------------------------ work accounting
 
 
-def accounting(inp, counts):
-    """Algorithmic FLOPs and bytes of the layer and of each expert GEMM (padding rows excluded)."""
+def accounting(inp, counts, block=False):
+    """Algorithmic FLOPs and bytes of the layer and of each expert GEMM (padding rows excluded).
+
+    The block form adds the norm (square, sum, two products per element), the
+    residual add and the gain vector; h is read once and out written once, as x is.
+    """
     T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
     es = 2 if inp.dtype == "bf16" else 4
     touched = int((np.asarray(counts) > 0).sum())
     kT = k * T
+    extra_flops = 5.0 * T * d if block else 0.0
+    extra_bytes = d * es if block else 0.0
     return {
         "touched": touched,
-        "layer_flops": 2.0 * T * d * E + 6.0 * kT * d * F,
-        "layer_bytes": touched * 3.0 * d * F * es + 2.0 * T * d * es + E * d * es,
+        "layer_flops": 2.0 * T * d * E + 6.0 * kT * d * F + extra_flops,
+        "layer_bytes": touched * 3.0 * d * F * es + 2.0 * T * d * es + E * d * es + extra_bytes,
         "expert1_flops": 4.0 * kT * d * F,
         "expert1_bytes": touched * 2.0 * F * d * es + kT * d * es + kT * F * es,
         "expert2_flops": 2.0 * kT * d * F,
@@ -188,11 +199,25 @@ def recorded_traffic(kernel, workload):
 # ------------------------------------------------------------------ CPU oracle
 
 
-def cpu_oracle_run(inp, target_s, threads):
-    """Time the fp64 oracle on a token sample sized for about target_s seconds; returns (tokens/s, sample text)."""
+def oracle_fn(inp, block):
+    """The oracle call the CPU legs time: fn(tokens, nthreads) for the layer or the block form."""
     import oracle
+    if block:
+        return lambda toks, nt: oracle.block(inp.x, inp.gamma, moe_inputs.BLOCK_EPS, inp.Wg, inp.W1, inp.W3, inp.W2,
+                                             k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=nt)
+    return lambda toks, nt: oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=nt)
+
+
+def make_workload(cfg, block):
+    inp = moe_inputs.make_config(cfg)
+    return moe_inputs.make_block(inp) if block else inp
+
+
+def cpu_oracle_run(inp, target_s, threads, block=False):
+    """Time the fp64 oracle on a token sample sized for about target_s seconds; returns (tokens/s, sample text)."""
+    run = oracle_fn(inp, block)
     t0 = time.perf_counter()
-    oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=[0], nthreads=1)
+    run([0], 1)
     per_tok = max(time.perf_counter() - t0, 1e-5)
     n = int(max(1, min(inp.T, round(target_s * threads / per_tok))))
     toks = np.unique(np.linspace(0, inp.T - 1, n).astype(np.int32))
@@ -200,10 +225,12 @@ def cpu_oracle_run(inp, target_s, threads):
     reps = min(reps, 50)
     t0 = time.perf_counter()
     for _ in range(reps):
-        oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=threads)
+        run(toks, threads)
     dt = time.perf_counter() - t0
-    sample = (f"{len(toks)} of {inp.T} tokens (evenly spaced), x{reps}, full layer per token "
-              f"(routing over all E, k SwiGLU experts, weighted sum) in fp64")
+    what = "RMSNorm, routing over all E, k SwiGLU experts, weighted sum, residual" if block else \
+        "routing over all E, k SwiGLU experts, weighted sum"
+    sample = f"{len(toks)} of {inp.T} tokens (evenly spaced), x{reps}, full {'block' if block else 'layer'} " \
+             f"per token ({what}) in fp64"
     return reps * len(toks) / dt, sample, dt
 
 
@@ -214,30 +241,31 @@ def run_reference(args, rank):
     if rank != 0:
         return
     c = moe_inputs.CONFIGS[args.config]
-    inp = moe_inputs.make_config(args.config)
+    inp = make_workload(args.config, args.block)
+    run = oracle_fn(inp, args.block)
     threads = len(os.sched_getaffinity(0))
     total_steps = args.steps + args.warmup
     per_step = max(0.5, min(30.0, 150.0 / max(total_steps, 1)))
-    import oracle
     t0 = time.perf_counter()
-    oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=[0], nthreads=1)
+    run([0], 1)
     per_tok = max(time.perf_counter() - t0, 1e-5)
     n = int(max(1, min(inp.T, round(per_step * threads / per_tok))))
     toks = np.unique(np.linspace(0, inp.T - 1, n).astype(np.int32))
     for _ in range(args.warmup):
-        oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=threads)
+        run(toks, threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=threads)
+        run(toks, threads)
     dt = time.perf_counter() - t0
     value = args.steps * len(toks) / dt
     sample = f"{len(toks)} of {inp.T} tokens per step (evenly spaced), fp64 oracle, {threads} threads"
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": BLOCK_METRIC if args.block else METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt / max(args.steps, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": c["name"], "T": inp.T, "d": inp.d, "ffn": inp.F, "E": inp.E, "k": inp.k,
-                   "seed": c["seed"], "sample_tokens_per_step": int(len(toks))},
+        "config": {"workload": c["name"] + ("+block" if args.block else ""), "T": inp.T, "d": inp.d,
+                   "ffn": inp.F, "E": inp.E, "k": inp.k, "seed": c["seed"],
+                   "sample_tokens_per_step": int(len(toks))},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -271,17 +299,33 @@ def run_ours(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     c = moe_inputs.CONFIGS[args.config]
-    inp = moe_inputs.make_config(args.config)
+    block = args.block
+    inp = make_workload(args.config, block)
     dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
     tdt = dev[0].dtype
     T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
     code = moe.MOE_DTYPE_BF16 if inp.dtype == "bf16" else moe.MOE_DTYPE_F32
-    ws = torch.empty(moe.moe_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
+    wsize = moe.moe_block_workspace_size if block else moe.moe_workspace_size
+    ws = torch.empty(wsize(T, d, F, E, k, code), dtype=torch.uint8, device=device)
     out = torch.empty((T, d), dtype=tdt, device=device)
+    if block:
+        gamma = to_dev(inp.gamma, inp.dtype, device)
+        stats = torch.empty(2 * E + 1, dtype=torch.float32, device=device)
 
-    idx, _ = moe.moe_route(dev[0], dev[1], k)
-    counts = moe.moe_dispatch(idx, E)[0].cpu().numpy()
-    acc = accounting(inp, counts)
+    def step(events=None):
+        if block:
+            return moe.moe_block_forward_ws(dev[0], gamma, moe_inputs.BLOCK_EPS, *dev[1:], k, ws, out,
+                                            alpha=BLOCK_ALPHA, stats=stats, events=events)
+        return moe.moe_forward_profiled(*dev, k, ws, out, events=events)
+
+    if block:
+        # the block routes the normalised rows: take its counts from its own statistics (f = count / T)
+        step()
+        counts = np.rint(stats[:E].double().cpu().numpy() * T).astype(np.int64)
+    else:
+        idx, _ = moe.moe_route(dev[0], dev[1], k)
+        counts = moe.moe_dispatch(idx, E)[0].cpu().numpy()
+    acc = accounting(inp, counts, block)
     flush = acc["layer_bytes"] < 3 * L2_BYTES
     flush_buf = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if flush else None
 
@@ -296,7 +340,7 @@ def run_ours(args, rank, world, local):
         for e in row:
             e.record(stream)
     for _ in range(W):
-        moe.moe_forward_profiled(*dev, k, ws, out)
+        step()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -311,7 +355,7 @@ def run_ours(args, rank, world, local):
         if flush:
             flush_buf.zero_()
             events[i][0].record(stream)
-        launches += moe.moe_forward_profiled(*dev, k, ws, out, events=events[i] if i % every == 0 else None)
+        launches += step(events=events[i] if i % every == 0 else None)
     end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -332,7 +376,7 @@ def run_ours(args, rank, world, local):
 
     # e2e: host buffers, copies inside every step
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not block:
         x_host = dev[0].cpu().pin_memory() if inp.dtype == "bf16" else None
         if x_host is not None:
             out_host = torch.empty((T, d), dtype=tdt, pin_memory=True)
@@ -385,14 +429,16 @@ def run_ours(args, rank, world, local):
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         threads = len(os.sched_getaffinity(0))
-        v, sample, _ = cpu_oracle_run(inp, args.cpu_seconds, threads)
+        v, sample, _ = cpu_oracle_run(inp, args.cpu_seconds, threads, block)
         cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
 
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "metric": BLOCK_METRIC if block else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp.dtype, "data": "synthetic",
-        "config": {"workload": c["name"], "T": T, "d": d, "ffn": F, "E": E, "k": k, "seed": c["seed"],
+        "config": {"workload": c["name"] + ("+block" if block else ""), "T": T, "d": d, "ffn": F, "E": E, "k": k,
+                   "seed": c["seed"],
                    "routing": "zipf1.2-skewed" if c["skew"] else "near-uniform",
                    "l2": "L2 flushed between steps" if flush else "touched weights larger than L2 (no flush)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},

@@ -243,6 +243,75 @@ MOE_API const char* moe_status_string(moe_status status);
 /* Token count at or below which MOE_PATH_AUTO takes the decode path. */
 MOE_API int moe_decode_max_tokens(void);
 
+/* ------------------------------------------------------------------------
+ * Block form: the MoE sub-layer of a Mixtral Transformer block, section
+ * "Mixtral 8x7B — Sparse MoEの導入", subsection "Mixtralのアーキテクチャ" of the
+ * same page (RMSNorm, then the MoE layer, then the residual connection):
+ *
+ *   u   = RMSNorm(h),  u_j = gamma_j h_j / sqrt((1/d) sum_i h_i^2 + eps)
+ *   out = h + MoE(u)                    MoE as defined at the top of this file
+ *
+ * The page names RMSNorm without printing it; this is its usual definition,
+ * with a per-channel gain gamma [d] and the caller's eps (>= 0; Mixtral-style
+ * models use 1e-5).  Precision: each row's factor 1/sqrt(mean(h^2) + eps) is
+ * computed in fp32; the router scores see the unrounded normalised row (they
+ * are r * (Wg (gamma * h)) with exact fp32 products); the experts see u
+ * rounded once to the operand type; the residual is added to the fp32
+ * gate-weighted sum before the output is rounded once.  eps == 0 with an
+ * all-zero row gives NaN, as the definition does.
+ *
+ * Load-balance statistics (optional, `stats`; subsection "ロードバランス損失"):
+ *   f_e = (1/T) #{(t, j): topk_idx[t][j] == e}   (every one of the k selections)
+ *   p_e = (1/T) sum_t softmax(s_t)_e             (softmax over all E scores)
+ *   L   = alpha * E * sum_e f_e p_e
+ * written as stats[0..E) = f, stats[E..2E) = p, stats[2E] = L (device, float,
+ * 2E + 1 values).  The page's formula carries alpha and its code does not;
+ * alpha = 1 gives the code's value.  Sums run in a fixed order: the same
+ * inputs give the same bits on every run.
+ *
+ * h, out: [T][d] (device); gamma: [d] (device), same element type as h.
+ * out may be h itself (the update is then in place); it must not overlap h in
+ * any other way.  stats may be NULL (nothing is computed for it).
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes moe_block_forward_ws needs (0 for invalid sizes or dtype). */
+MOE_API size_t moe_block_workspace_size(int T, int d, int ffn, int E, int k, int dtype);
+
+/* bfloat16 block; the workspace comes from a stream-ordered pool as in moe_forward. */
+MOE_API moe_status moe_block_forward(const void* h, const void* gamma, float eps, const void* Wg,
+                                     const void* W1, const void* W3, const void* W2, void* out, int T,
+                                     int d, int ffn, int E, int k, float alpha, float* stats,
+                                     cudaStream_t stream);
+
+/* fp32 block (fp32 throughout). */
+MOE_API moe_status moe_block_forward_f32(const float* h, const float* gamma, float eps, const float* Wg,
+                                         const float* W1, const float* W3, const float* W2, float* out,
+                                         int T, int d, int ffn, int E, int k, float alpha, float* stats,
+                                         cudaStream_t stream);
+
+/*
+ * Block with a caller-provided workspace of at least moe_block_workspace_size()
+ * bytes (device, 256-byte aligned, not in use by another call in flight), an
+ * explicit path and dtype, and the optional stage events and launch count of
+ * moe_forward_profiled (the statistics, when asked for, run in the route stage).
+ */
+MOE_API moe_status moe_block_forward_ws(const void* h, const void* gamma, float eps, const void* Wg,
+                                        const void* W1, const void* W3, const void* W2, void* out, int T,
+                                        int d, int ffn, int E, int k, float alpha, float* stats, int dtype,
+                                        int path, void* workspace, size_t workspace_bytes,
+                                        cudaEvent_t* stage_events, int* launches, cudaStream_t stream);
+
+/*
+ * moe_route (bfloat16) / moe_route_f32 plus the load-balance statistics of
+ * that routing into stats (device, 2E + 1 floats, required).  Scratch comes
+ * from the stream-ordered pool.
+ */
+MOE_API moe_status moe_route_stats(const void* x, const void* Wg, int T, int d, int E, int k, float alpha,
+                                   int32_t* topk_idx, float* topk_w, float* stats, cudaStream_t stream);
+MOE_API moe_status moe_route_stats_f32(const float* x, const float* Wg, int T, int d, int E, int k,
+                                       float alpha, int32_t* topk_idx, float* topk_w, float* stats,
+                                       cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

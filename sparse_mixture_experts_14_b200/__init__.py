@@ -9,6 +9,9 @@ importing this package raises.
 
 bf16 tensors are torch.bfloat16; the layer's operand layouts are
     x [T][d], Wg [E][d], W1 [E][F][d], W3 [E][F][d], W2 [E][d][F], out [T][d].
+The block form adds h [T][d] (the residual stream, in place of x) and
+gamma [d]; load-balance statistics come back as a float32 [2E+1] tensor
+(f, p, loss).
 """
 from __future__ import annotations
 
@@ -34,7 +37,7 @@ MOE_NUM_STAGES = 6
 STAGE_NAMES = ("route", "dispatch", "gather", "expert1", "expert2", "combine")
 
 # every symbol include/moe.h declares, with its ctypes signature
-_vp, _ci, _sz, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
+_vp, _ci, _sz, _ll, _cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong, ctypes.c_float
 SIGNATURES = {
     "moe_route": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _vp, _vp, _vp]),
     "moe_route_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _vp, _vp, _vp]),
@@ -52,6 +55,14 @@ SIGNATURES = {
     "moe_selftest_wait_timeout": (_ci, [_ll, _vp]),
     "moe_status_string": (ctypes.c_char_p, [_ci]),
     "moe_decode_max_tokens": (_ci, []),
+    "moe_block_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
+    "moe_block_forward": (_ci, [_vp, _vp, _cf, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp]),
+    "moe_block_forward_f32": (_ci, [_vp, _vp, _cf, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp,
+                                    _vp]),
+    "moe_block_forward_ws": (_ci, [_vp, _vp, _cf, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _ci,
+                                   _ci, _vp, _sz, _vp, _vp, _vp]),
+    "moe_route_stats": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
+    "moe_route_stats_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -204,11 +215,7 @@ def moe_forward_profiled(x, Wg, W1, W3, W2, k, workspace, out, events=None, path
     at the stage boundaries; returns the number of kernels launched."""
     code = _dtype_code(x)
     T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
-    ev_arr = None
-    if events is not None:
-        if len(events) != MOE_NUM_STAGES + 1:
-            raise ValueError(f"need {MOE_NUM_STAGES + 1} events")
-        ev_arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    ev_arr = _events(events)
     n = ctypes.c_int(0)
     _check(_lib.moe_forward_profiled(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, code,
                                      path, _ptr(workspace), workspace.numel(), ev_arr, ctypes.byref(n),
@@ -229,6 +236,79 @@ def moe_forward_host(x_host, Wg, W1, W3, W2, k, out_host=None, stream=None):
     _check(_lib.moe_forward_host(_ptr(x_host), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out_host), T, d, F, E,
                                  k, _stream(stream)), "moe_forward_host")
     return out_host
+
+
+def _events(events):
+    if events is None:
+        return None
+    if len(events) != MOE_NUM_STAGES + 1:
+        raise ValueError(f"need {MOE_NUM_STAGES + 1} events")
+    return (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+
+
+def _block_args(h, gamma, Wg, W1, W3, W2, stats):
+    for t, n in ((h, "h"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2"), (gamma, "gamma")):
+        _dev(t, h.dtype, n)
+    T, d, F, E = _layer_shapes(h, Wg, W1, W3, W2)
+    if gamma.shape != (d,):
+        raise ValueError(f"gamma must have shape ({d},), got {tuple(gamma.shape)}")
+    if stats is not None:
+        _dev(stats, torch.float32, "stats")
+        if stats.numel() < 2 * E + 1:
+            raise ValueError(f"stats needs {2 * E + 1} floats")
+    return T, d, F, E
+
+
+def moe_block_workspace_size(T, d, ffn, E, k, dtype=MOE_DTYPE_BF16) -> int:
+    return int(_lib.moe_block_workspace_size(T, d, ffn, E, k, dtype))
+
+
+def moe_block_forward(h, gamma, eps, Wg, W1, W3, W2, k, alpha=1.0, stats=None, out=None, stream=None):
+    """out = h + MoE(RMSNorm(h)); bf16 tensors use moe_block_forward, float32 moe_block_forward_f32.
+    stats (float32 [2E+1] CUDA tensor or None) receives f, p and the load-balance loss.  out may be h."""
+    code = _dtype_code(h)
+    T, d, F, E = _block_args(h, gamma, Wg, W1, W3, W2, stats)
+    if out is None:
+        out = torch.empty((T, d), dtype=h.dtype, device=h.device)
+    _dev(out, h.dtype, "out")
+    fn = _lib.moe_block_forward if code == MOE_DTYPE_BF16 else _lib.moe_block_forward_f32
+    _check(fn(_ptr(h), _ptr(gamma), float(eps), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k,
+              float(alpha), _ptr(stats), _stream(stream)), "moe_block_forward")
+    return out
+
+
+moe_block_forward_f32 = moe_block_forward
+
+
+def moe_block_forward_ws(h, gamma, eps, Wg, W1, W3, W2, k, workspace, out, alpha=1.0, stats=None,
+                         path=MOE_PATH_AUTO, events=None, stream=None):
+    """moe_block_forward with an explicit workspace, path and optional stage events; returns the launch count."""
+    code = _dtype_code(h)
+    T, d, F, E = _block_args(h, gamma, Wg, W1, W3, W2, stats)
+    _dev(workspace, torch.uint8, "workspace")
+    _dev(out, h.dtype, "out")
+    n = ctypes.c_int(0)
+    _check(_lib.moe_block_forward_ws(_ptr(h), _ptr(gamma), float(eps), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2),
+                                     _ptr(out), T, d, F, E, k, float(alpha), _ptr(stats), code, path,
+                                     _ptr(workspace), workspace.numel(), _events(events), ctypes.byref(n),
+                                     _stream(stream)), "moe_block_forward_ws")
+    return n.value
+
+
+def moe_route_stats(x, Wg, k, alpha=1.0, stream=None):
+    """moe_route plus load-balance statistics: (topk_idx, topk_w, stats [2E+1] = f, p, loss)."""
+    code = _dtype_code(x)
+    _dev(x, x.dtype, "x")
+    _dev(Wg, x.dtype, "Wg")
+    T, d = x.shape
+    E = Wg.shape[0]
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    stats = torch.empty(2 * E + 1, dtype=torch.float32, device=x.device)
+    fn = _lib.moe_route_stats if code == MOE_DTYPE_BF16 else _lib.moe_route_stats_f32
+    _check(fn(_ptr(x), _ptr(Wg), T, d, E, k, float(alpha), _ptr(idx), _ptr(w), _ptr(stats), _stream(stream)),
+           "moe_route_stats")
+    return idx, w, stats
 
 
 def moe_get_device_status(stream=None) -> int:

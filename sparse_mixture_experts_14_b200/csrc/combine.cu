@@ -4,15 +4,19 @@
 // in the page code's order (slot 0 first, then slot 1, ...).  No atomics:
 // each output element is owned by one thread, so the result is the same on
 // every run.  Bound by HBM (k fp32 rows in, one row out per token).
+//
+// Block form: the residual row of the MoE sub-layer (section "Mixtral 8x7B —
+// Sparse MoEの導入", subsection "Mixtralのアーキテクチャ") is added to the fp32
+// sum before the single rounding: out[t] = h[t] + sum_j g[t][j] * Y[...].
 #include "moe_common.cuh"
 
 namespace moe {
 namespace {
 
-template <bool BF16_OUT>
+template <bool BF16_OUT, bool RESID>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ Y, const float* __restrict__ w,
                                                       const int32_t* __restrict__ inv, int T, int d, int k,
-                                                      void* __restrict__ out) {
+                                                      void* __restrict__ out, const void* __restrict__ resid) {
     pdl_trigger();
     pdl_wait();
     const int q = d / 4;   // float4 columns per row
@@ -31,6 +35,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
             acc.z = fmaf(g, y.z, acc.z);
             acc.w = fmaf(g, y.w, acc.w);
         }
+        if (RESID) {
+            if (BF16_OUT) {
+                const uint2 h = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(resid) +
+                                                                     (size_t)t * d * 2) + c);
+                acc.x += bf16_lo(h.x);
+                acc.y += bf16_hi(h.x);
+                acc.z += bf16_lo(h.y);
+                acc.w += bf16_hi(h.y);
+            } else {
+                const float4 h = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(resid) +
+                                                                       (size_t)t * d) + c);
+                acc.x += h.x;
+                acc.y += h.y;
+                acc.z += h.z;
+                acc.w += h.w;
+            }
+        }
         if (BF16_OUT) {
             uint2 o;
             o.x = pack_bf16x2(acc.x, acc.y);
@@ -44,24 +65,25 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 template <bool BF16_OUT>
 cudaError_t launch_combine_t(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, void* out,
-                             cudaStream_t s) {
+                             cudaStream_t s, const void* resid) {
     const size_t n = (size_t)T * (d / 4);
     size_t blocks = (n + 255) / 256;
     if (blocks > 148 * 32) blocks = 148 * 32;
     if (blocks < 1) blocks = 1;
-    return launch_pdl(combine_kernel<BF16_OUT>, dim3((unsigned)blocks), dim3(256), 0, s, Y, w, inv, T, d, k, out);
+    auto kern = resid ? combine_kernel<BF16_OUT, true> : combine_kernel<BF16_OUT, false>;
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(256), 0, s, Y, w, inv, T, d, k, out, resid);
 }
 
 }  // namespace
 
 cudaError_t launch_combine_bf16(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, void* out,
-                                cudaStream_t s) {
-    return launch_combine_t<true>(Y, w, inv, T, d, k, out, s);
+                                cudaStream_t s, const void* resid) {
+    return launch_combine_t<true>(Y, w, inv, T, d, k, out, s, resid);
 }
 
 cudaError_t launch_combine_f32(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, float* out,
-                               cudaStream_t s) {
-    return launch_combine_t<false>(Y, w, inv, T, d, k, out, s);
+                               cudaStream_t s, const float* resid) {
+    return launch_combine_t<false>(Y, w, inv, T, d, k, out, s, resid);
 }
 
 }  // namespace moe

@@ -13,10 +13,61 @@
 // (per 1024-token block), scan (one block: totals, padded offsets, per-block
 // bases) and scatter (per-block stable ranks by warp ballots).  Then gather
 // (one warp per row, 16-byte copies).
+//
+// Block form: the gather also applies the pre-norm of the MoE sub-layer
+// (section "Mixtral 8x7B — Sparse MoEの導入", subsection "Mixtralのアーキテクチャ"),
+// writing (gamma * x) * r, r = the row's 1/sqrt(mean(x^2) + eps) from the
+// router pass, rounded once to the row type.  NORM selects the row type:
+// 0 = plain copy, 1 = bf16, 2 = fp32.
 #include "moe_common.cuh"
 
 namespace moe {
 namespace {
+
+// One 16-byte vector of a row after the optional normalisation.
+template <int NORM>
+__device__ __forceinline__ uint4 norm_vec(uint4 v, uint4 g, float r) {
+    if (NORM == 1) {
+        uint4 o;
+        o.x = pack_bf16x2(bf16_lo(v.x) * bf16_lo(g.x) * r, bf16_hi(v.x) * bf16_hi(g.x) * r);
+        o.y = pack_bf16x2(bf16_lo(v.y) * bf16_lo(g.y) * r, bf16_hi(v.y) * bf16_hi(g.y) * r);
+        o.z = pack_bf16x2(bf16_lo(v.z) * bf16_lo(g.z) * r, bf16_hi(v.z) * bf16_hi(g.z) * r);
+        o.w = pack_bf16x2(bf16_lo(v.w) * bf16_lo(g.w) * r, bf16_hi(v.w) * bf16_hi(g.w) * r);
+        return o;
+    }
+    if (NORM == 2) {
+        uint4 o;
+        o.x = __float_as_uint(__uint_as_float(v.x) * __uint_as_float(g.x) * r);
+        o.y = __float_as_uint(__uint_as_float(v.y) * __uint_as_float(g.y) * r);
+        o.z = __float_as_uint(__uint_as_float(v.z) * __uint_as_float(g.z) * r);
+        o.w = __float_as_uint(__uint_as_float(v.w) * __uint_as_float(g.w) * r);
+        return o;
+    }
+    return v;
+}
+
+// Copy one row of nvec 16-byte vectors with this warp, 8 loads in flight per
+// lane before their stores; NORM != 0 normalises with gamma and r.
+template <int NORM>
+__device__ __forceinline__ void copy_row(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t nvec,
+                                         int lane, const uint4* __restrict__ gam, float r) {
+    for (size_t v0 = lane; v0 < nvec; v0 += 32 * 8) {
+        uint4 buf[8], gb[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const size_t v = v0 + (size_t)u * 32;
+            if (v < nvec) {
+                buf[u] = __ldg(src + v);
+                if (NORM) gb[u] = __ldg(gam + v);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const size_t v = v0 + (size_t)u * 32;
+            if (v < nvec) dst[v] = NORM ? norm_vec<NORM>(buf[u], gb[u], r) : buf[u];
+        }
+    }
+}
 
 __global__ void __launch_bounds__(kDispatchTokens) hist_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
                                                                int32_t* __restrict__ blk_counts, int* status) {
@@ -233,13 +284,15 @@ __global__ void __launch_bounds__(kDispatchTokens) dispatch_single_kernel(const 
 constexpr int kSmallTokens = 64;
 constexpr int kSmallMaxRows = kSmallTokens * kMaxExperts + kMaxExperts * kSegRows;
 
+template <int NORM>
 __global__ void __launch_bounds__(256) dispatch_gather_small_kernel(const int32_t* __restrict__ idx, int T, int E,
                                                                     int k, const uint8_t* __restrict__ x,
                                                                     size_t row_bytes, Meta* __restrict__ meta,
                                                                     int32_t* __restrict__ perm,
                                                                     int32_t* __restrict__ inv,
                                                                     uint8_t* __restrict__ xp, size_t slots,
-                                                                    int* status) {
+                                                                    int* status, const uint4* __restrict__ gam,
+                                                                    const float* __restrict__ rstd) {
     pdl_trigger();
     pdl_wait();
     __shared__ int offs[kMaxExperts + 1];
@@ -322,29 +375,20 @@ __global__ void __launch_bounds__(256) dispatch_gather_small_kernel(const int32_
     for (int a = gw; a < T * k; a += nw) {
         const int r = row_of[a];
         if (r < 0 || (size_t)r >= slots) continue;
-        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * row_bytes);
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(a / k) * row_bytes);
-        for (size_t v0 = lane; v0 < nvec; v0 += 32 * 8) {
-            uint4 buf[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const size_t v = v0 + (size_t)u * 32;
-                if (v < nvec) buf[u] = __ldg(src + v);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const size_t v = v0 + (size_t)u * 32;
-                if (v < nvec) dst[v] = buf[u];
-            }
-        }
+        const int t = a / k;
+        copy_row<NORM>(reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes),
+                       reinterpret_cast<uint4*>(xp + (size_t)r * row_bytes), nvec, lane, gam,
+                       NORM ? rstd[t] : 0.f);
     }
 }
 
 // One warp per row of the padded buffer; rows past offsets[E] are left alone.
+template <int NORM>
 __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ x, size_t row_bytes, int T, int k,
                                                      const Meta* __restrict__ meta, int E,
                                                      const int32_t* __restrict__ perm, uint8_t* __restrict__ xp,
-                                                     size_t slots) {
+                                                     size_t slots, const uint4* __restrict__ gam,
+                                                     const float* __restrict__ rstd) {
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -357,21 +401,9 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__
         const int a = perm[r];
         uint4* dst = reinterpret_cast<uint4*>(xp + r * row_bytes);
         if (a >= 0 && a < TK) {
-            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(a / k) * row_bytes);
-            // 8 loads in flight per lane before their stores
-            for (size_t v0 = lane; v0 < nvec; v0 += 32 * 8) {
-                uint4 buf[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const size_t v = v0 + (size_t)u * 32;
-                    if (v < nvec) buf[u] = __ldg(src + v);
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const size_t v = v0 + (size_t)u * 32;
-                    if (v < nvec) dst[v] = buf[u];
-                }
-            }
+            const int t = a / k;
+            copy_row<NORM>(reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes), dst, nvec, lane, gam,
+                           NORM ? rstd[t] : 0.f);
         } else {
             const uint4 z = make_uint4(0, 0, 0, 0);
             for (size_t v = lane; v < nvec; v += 32) dst[v] = z;
@@ -399,24 +431,31 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* bl
 
 cudaError_t launch_dispatch_gather_small(const int32_t* idx, int T, int E, int k, const void* x, size_t elem_bytes,
                                          int d, Meta* meta, int32_t* perm, int32_t* inv, void* xp, size_t slots,
-                                         int* status, cudaStream_t s) {
+                                         int* status, cudaStream_t s, const GatherNorm& nm) {
     if (T > kSmallTokens) return cudaErrorInvalidValue;
     const int rows = T * k;
     int blocks = (rows + 7) / 8;   // about one row per warp
     if (blocks < 1) blocks = 1;
     if (blocks > 64) blocks = 64;
-    return launch_pdl(dispatch_gather_small_kernel, dim3(blocks), dim3(256), 0, s, idx, T, E, k,
-                      static_cast<const uint8_t*>(x), (size_t)d * elem_bytes, meta, perm, inv,
-                      static_cast<uint8_t*>(xp), slots, status);
+    const uint8_t* xb = static_cast<const uint8_t*>(x);
+    uint8_t* xpb = static_cast<uint8_t*>(xp);
+    const uint4* gam = static_cast<const uint4*>(nm.gamma);
+    const size_t rb = (size_t)d * elem_bytes;
+    auto kern = !nm.gamma ? dispatch_gather_small_kernel<0>
+                          : (elem_bytes == 2 ? dispatch_gather_small_kernel<1> : dispatch_gather_small_kernel<2>);
+    return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, idx, T, E, k, xb, rb, meta, perm, inv, xpb, slots, status,
+                      gam, nm.rstd);
 }
 
 cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
-                          const int32_t* perm, void* xp, size_t slots, cudaStream_t s) {
+                          const int32_t* perm, void* xp, size_t slots, cudaStream_t s, const GatherNorm& nm) {
     const size_t rows_per_block = 8;
     size_t blocks = (slots + rows_per_block - 1) / rows_per_block;
     if (blocks > 65535 * 4) blocks = 65535 * 4;
-    return launch_pdl(gather_kernel, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const uint8_t*>(x),
-                      (size_t)d * elem_bytes, T, k, meta, E, perm, static_cast<uint8_t*>(xp), slots);
+    const uint4* gam = static_cast<const uint4*>(nm.gamma);
+    auto kern = !nm.gamma ? gather_kernel<0> : (elem_bytes == 2 ? gather_kernel<1> : gather_kernel<2>);
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const uint8_t*>(x),
+                      (size_t)d * elem_bytes, T, k, meta, E, perm, static_cast<uint8_t*>(xp), slots, gam, nm.rstd);
 }
 
 }  // namespace moe

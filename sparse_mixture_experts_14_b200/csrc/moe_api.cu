@@ -109,11 +109,15 @@ moe_status check_layer(const void* x, const void* Wg, const void* W1, const void
 }
 
 struct Plan {
-    size_t idx, w, blk, meta, perm, inv, xp, h, y, total;
+    size_t idx, w, blk, meta, perm, inv, xp, h, y;
+    size_t rstd, logits, bal;   // block form only (see make_plan's `block`)
+    size_t total;
     size_t slots;
 };
 
-Plan make_plan(int T, int d, int F, int E, int k, int dtype) {
+// Workspace layout.  The block form adds each row's norm factor [T], the fp32
+// scores [T][E] and the load-balance partial sums.
+Plan make_plan(int T, int d, int F, int E, int k, int dtype, bool block = false) {
     Plan p{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -133,9 +137,22 @@ Plan make_plan(int T, int d, int F, int E, int k, int dtype) {
     p.xp = take(p.slots * (size_t)d * es);
     p.h = take(p.slots * (size_t)F * es);
     p.y = take(p.slots * (size_t)d * 4);
+    if (block) {
+        p.rstd = take((size_t)T * 4);
+        p.logits = take((size_t)T * E * 4);
+        p.bal = take(balance_part_bytes(T, E));
+    }
     p.total = off;
     return p;
 }
+
+// The block form's extra operands and outputs (null for the plain layer).
+struct BlockArgs {
+    const void* gamma;
+    float eps;
+    float alpha;
+    float* stats;   // [2E + 1] or null
+};
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -147,8 +164,20 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 
 moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2, void* out, int T,
                      int d, int F, int E, int k, int dtype, int path, uint8_t* ws, const DeviceState& dev,
-                     cudaStream_t s, cudaEvent_t* ev = nullptr, int* launches = nullptr) {
-    const Plan p = make_plan(T, d, F, E, k, dtype);
+                     cudaStream_t s, cudaEvent_t* ev = nullptr, int* launches = nullptr,
+                     const BlockArgs* bo = nullptr) {
+    const Plan p = make_plan(T, d, F, E, k, dtype, bo != nullptr);
+    RouteExtras ex;
+    GatherNorm nm;
+    if (bo) {
+        ex.gamma = bo->gamma;
+        ex.eps = bo->eps;
+        ex.rstd = reinterpret_cast<float*>(ws + p.rstd);
+        if (bo->stats) ex.logits = reinterpret_cast<float*>(ws + p.logits);
+        nm.gamma = bo->gamma;
+        nm.rstd = ex.rstd;
+    }
+    const void* resid = bo ? x : nullptr;
     int32_t* idx = reinterpret_cast<int32_t*>(ws + p.idx);
     float* w = reinterpret_cast<float*>(ws + p.w);
     int32_t* blk = reinterpret_cast<int32_t*>(ws + p.blk);
@@ -163,25 +192,29 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
     int n = 0;
     MOE_TRY(mark(MOE_STAGE_ROUTE));
     if (dtype == MOE_DTYPE_BF16) {
-        MOE_TRY(launch_router_bf16(x, Wg, T, d, E, k, idx, w, dev.num_sms, s));
+        MOE_TRY(launch_router_bf16(x, Wg, T, d, E, k, idx, w, dev.num_sms, s, ex));
     } else {
         MOE_TRY(launch_router_f32(static_cast<const float*>(x), static_cast<const float*>(Wg), T, d, E, k, idx, w,
-                                  dev.num_sms, s));
+                                  dev.num_sms, s, ex));
     }
     n += 1;
+    if (bo && bo->stats) {
+        MOE_TRY(launch_balance(ex.logits, idx, T, E, k, bo->alpha, ws + p.bal, bo->stats, s));
+        n += 2;
+    }
     MOE_TRY(mark(MOE_STAGE_DISPATCH));
     const size_t es = dtype == MOE_DTYPE_BF16 ? 2 : 4;
     if (dtype == MOE_DTYPE_BF16 && T <= kDecodeMaxTokens &&
         (path == MOE_PATH_DECODE || path == MOE_PATH_AUTO)) {
         // decode path: one launch sorts and gathers the token rows (the gather stage is empty)
-        MOE_TRY(launch_dispatch_gather_small(idx, T, E, k, x, es, d, meta, perm, inv, xp, p.slots, dev.status, s));
+        MOE_TRY(launch_dispatch_gather_small(idx, T, E, k, x, es, d, meta, perm, inv, xp, p.slots, dev.status, s, nm));
         n += 1;
         MOE_TRY(mark(MOE_STAGE_GATHER));
     } else {
         MOE_TRY(launch_dispatch(idx, T, E, k, blk, meta, perm, inv, dev.status, s));
         n += dispatch_launches(T);
         MOE_TRY(mark(MOE_STAGE_GATHER));
-        MOE_TRY(launch_gather(x, es, T, d, E, k, meta, perm, xp, p.slots, s));
+        MOE_TRY(launch_gather(x, es, T, d, E, k, meta, perm, xp, p.slots, s, nm));
         n += 1;
     }
     if (dtype == MOE_DTYPE_BF16) {
@@ -192,7 +225,7 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
         MOE_TRY(mark(MOE_STAGE_EXPERT2));
         MOE_TRY(decode ? launch_decode(a, 2, s) : launch_tc_gemm2(a, s));
         MOE_TRY(mark(MOE_STAGE_COMBINE));
-        MOE_TRY(launch_combine_bf16(y, w, inv, T, d, k, out, s));
+        MOE_TRY(launch_combine_bf16(y, w, inv, T, d, k, out, s, resid));
     } else {
         MOE_TRY(mark(MOE_STAGE_EXPERT1));
         MOE_TRY(launch_simt_gemm1_f32(static_cast<const float*>(xp), static_cast<const float*>(W1),
@@ -202,7 +235,8 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
         MOE_TRY(launch_simt_gemm2_f32(static_cast<const float*>(h), static_cast<const float*>(W2), meta, E, d, F, y,
                                       p.slots, s));
         MOE_TRY(mark(MOE_STAGE_COMBINE));
-        MOE_TRY(launch_combine_f32(y, w, inv, T, d, k, static_cast<float*>(out), s));
+        MOE_TRY(launch_combine_f32(y, w, inv, T, d, k, static_cast<float*>(out), s,
+                                   static_cast<const float*>(resid)));
     }
     n += 3;
     MOE_TRY(mark(MOE_NUM_STAGES));
@@ -222,6 +256,65 @@ moe_status forward_pooled(const void* x, const void* Wg, const void* W1, const v
     st = run_layer(x, Wg, W1, W3, W2, out, T, d, F, E, k, dtype, MOE_PATH_AUTO, static_cast<uint8_t*>(ws), dev, s);
     if (cudaFreeAsync(ws, s) != cudaSuccess && st == MOE_OK) st = MOE_ERR_CUDA;
     return st;
+}
+
+// Checks of the block form's extra arguments (after check_layer).
+moe_status check_block(const void* h, const void* gamma, float eps, float alpha, const float* stats, const void* out,
+                       int T, int d, int dtype) {
+    if (!(eps >= 0.f) || !(eps <= 3.4e38f) || !(alpha == alpha) || !(alpha - alpha == 0.f)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!gamma || !aligned16(gamma)) return MOE_ERR_INVALID_ARG;
+    if (stats && (reinterpret_cast<uintptr_t>(stats) & 3u) != 0) return MOE_ERR_INVALID_ARG;
+    // out may be h itself (each element reads its h before writing it), no other overlap
+    const size_t row = (size_t)d * (dtype == MOE_DTYPE_BF16 ? 2 : 4);
+    const uintptr_t hb = reinterpret_cast<uintptr_t>(h), ob = reinterpret_cast<uintptr_t>(out);
+    const uintptr_t he = hb + row * (size_t)T, oe = ob + row * (size_t)T;
+    if (ob != hb && ob < he && hb < oe) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+moe_status block_pooled(const void* h, const void* gamma, float eps, const void* Wg, const void* W1, const void* W3,
+                        const void* W2, void* out, int T, int d, int F, int E, int k, float alpha, float* stats,
+                        int dtype, cudaStream_t s) {
+    moe_status st = check_layer(h, Wg, W1, W3, W2, out, T, d, F, E, k, dtype);
+    if (st == MOE_OK) st = check_block(h, gamma, eps, alpha, stats, out, T, d, dtype);
+    if (st != MOE_OK || T == 0) return st;
+    DeviceState dev;
+    if (!device_state(select_device(h), &dev)) return MOE_ERR_CUDA;
+    const Plan p = make_plan(T, d, F, E, k, dtype, true);
+    void* ws = nullptr;
+    if (cudaMallocFromPoolAsync(&ws, p.total, dev.pool, s) != cudaSuccess) return MOE_ERR_WORKSPACE;
+    const BlockArgs bo{gamma, eps, alpha, stats};
+    st = run_layer(h, Wg, W1, W3, W2, out, T, d, F, E, k, dtype, MOE_PATH_AUTO, static_cast<uint8_t*>(ws), dev, s,
+                   nullptr, nullptr, &bo);
+    if (cudaFreeAsync(ws, s) != cudaSuccess && st == MOE_OK) st = MOE_ERR_CUDA;
+    return st;
+}
+
+moe_status route_stats(const void* x, const void* Wg, int T, int d, int E, int k, float alpha, int32_t* idx,
+                       float* w, float* stats, int dtype, cudaStream_t s) {
+    moe_status st = check_sizes(T, d, E, k);
+    if (st != MOE_OK) return st;
+    if (d % (dtype == MOE_DTYPE_BF16 ? 8 : 4) != 0) return MOE_ERR_UNSUPPORTED;
+    if (!(alpha == alpha) || !(alpha - alpha == 0.f)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !Wg || !idx || !w || !stats || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
+    DeviceState dev;
+    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const size_t lbytes = align_up((size_t)T * E * 4, 256);
+    void* scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, lbytes + balance_part_bytes(T, E), dev.pool, s) != cudaSuccess)
+        return MOE_ERR_WORKSPACE;
+    RouteExtras ex;
+    ex.logits = static_cast<float*>(scratch);
+    cudaError_t e = dtype == MOE_DTYPE_BF16
+                        ? launch_router_bf16(x, Wg, T, d, E, k, idx, w, dev.num_sms, s, ex)
+                        : launch_router_f32(static_cast<const float*>(x), static_cast<const float*>(Wg), T, d, E, k,
+                                            idx, w, dev.num_sms, s, ex);
+    if (e == cudaSuccess)
+        e = launch_balance(ex.logits, idx, T, E, k, alpha, static_cast<uint8_t*>(scratch) + lbytes, stats, s);
+    cudaError_t f = cudaFreeAsync(scratch, s);
+    return (e == cudaSuccess && f == cudaSuccess) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 __global__ void wait_selftest_kernel(int* status, long long limit_ns) {
@@ -430,5 +523,54 @@ const char* moe_status_string(moe_status status) {
 }
 
 int moe_decode_max_tokens(void) { return kDecodeMaxTokens; }
+
+size_t moe_block_workspace_size(int T, int d, int ffn, int E, int k, int dtype) {
+    if (check_sizes(T, d, E, k) != MOE_OK || ffn <= 0) return 0;
+    if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_F32) return 0;
+    return make_plan(T, d, ffn, E, k, dtype, true).total;
+}
+
+moe_status moe_block_forward(const void* h, const void* gamma, float eps, const void* Wg, const void* W1,
+                             const void* W3, const void* W2, void* out, int T, int d, int ffn, int E, int k,
+                             float alpha, float* stats, cudaStream_t stream) {
+    return block_pooled(h, gamma, eps, Wg, W1, W3, W2, out, T, d, ffn, E, k, alpha, stats, MOE_DTYPE_BF16, stream);
+}
+
+moe_status moe_block_forward_f32(const float* h, const float* gamma, float eps, const float* Wg, const float* W1,
+                                 const float* W3, const float* W2, float* out, int T, int d, int ffn, int E, int k,
+                                 float alpha, float* stats, cudaStream_t stream) {
+    return block_pooled(h, gamma, eps, Wg, W1, W3, W2, out, T, d, ffn, E, k, alpha, stats, MOE_DTYPE_F32, stream);
+}
+
+moe_status moe_block_forward_ws(const void* h, const void* gamma, float eps, const void* Wg, const void* W1,
+                                const void* W3, const void* W2, void* out, int T, int d, int ffn, int E, int k,
+                                float alpha, float* stats, int dtype, int path, void* workspace,
+                                size_t workspace_bytes, cudaEvent_t* stage_events, int* launches,
+                                cudaStream_t stream) {
+    if (launches) *launches = 0;
+    moe_status st = check_layer(h, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype);
+    if (st == MOE_OK) st = check_block(h, gamma, eps, alpha, stats, out, T, d, dtype);
+    if (st != MOE_OK) return st;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE) return MOE_ERR_INVALID_ARG;
+    if (path == MOE_PATH_DECODE && (dtype != MOE_DTYPE_BF16 || T > kDecodeMaxTokens)) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype, true).total) return MOE_ERR_WORKSPACE;
+    DeviceState dev;
+    if (!device_state(select_device(h), &dev)) return MOE_ERR_CUDA;
+    const BlockArgs bo{gamma, eps, alpha, stats};
+    return run_layer(h, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
+                     stream, stage_events, launches, &bo);
+}
+
+moe_status moe_route_stats(const void* x, const void* Wg, int T, int d, int E, int k, float alpha,
+                           int32_t* topk_idx, float* topk_w, float* stats, cudaStream_t stream) {
+    return route_stats(x, Wg, T, d, E, k, alpha, topk_idx, topk_w, stats, MOE_DTYPE_BF16, stream);
+}
+
+moe_status moe_route_stats_f32(const float* x, const float* Wg, int T, int d, int E, int k, float alpha,
+                               int32_t* topk_idx, float* topk_w, float* stats, cudaStream_t stream) {
+    return route_stats(x, Wg, T, d, E, k, alpha, topk_idx, topk_w, stats, MOE_DTYPE_F32, stream);
+}
 
 }  // extern "C"

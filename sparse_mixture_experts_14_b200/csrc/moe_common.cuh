@@ -129,26 +129,53 @@ inline size_t slots_capacity(int T, int E, int k) {
 inline int dispatch_blocks(int T) { return (T + kDispatchTokens - 1) / kDispatchTokens; }
 
 // ---- kernel launchers (one per translation unit) ----
+// Extra work of the router pass, all optional.  With gamma set, the pass
+// routes RMSNorm(x) = gamma * x / sqrt(mean(x^2) + eps) instead of x and
+// writes each row's 1/sqrt(mean(x^2) + eps) to rstd[T].  With logits set it
+// also writes every fp32 score, [T][E], for the load-balance statistics.
+struct RouteExtras {
+    const void* gamma = nullptr;   // [d], same element type as x
+    float eps = 0.f;
+    float* rstd = nullptr;
+    float* logits = nullptr;
+};
+
 cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx,
-                               float* w, int num_sms, cudaStream_t s);
+                               float* w, int num_sms, cudaStream_t s, const RouteExtras& ex = RouteExtras());
 cudaError_t launch_router_f32(const float* x, const float* Wg, int T, int d, int E, int k, int32_t* idx,
-                              float* w, int num_sms, cudaStream_t s);
+                              float* w, int num_sms, cudaStream_t s, const RouteExtras& ex = RouteExtras());
+
+// Load-balance statistics from the router's scores and selections:
+// stats[0..E) = f, stats[E..2E) = p, stats[2E] = alpha * E * sum f p.
+// part holds balance_part_bytes(T, E) bytes of scratch.  Launches 2 kernels.
+size_t balance_part_bytes(int T, int E);
+cudaError_t launch_balance(const float* logits, const int32_t* idx, int T, int E, int k, float alpha, void* part,
+                           float* stats, cudaStream_t s);
 
 // Launches 1 kernel when T <= kDispatchTokens, else 3.
 inline int dispatch_launches(int T) { return T <= kDispatchTokens ? 1 : 3; }
 cudaError_t launch_dispatch(const int32_t* idx, int T, int E, int k, int32_t* blk_counts, Meta* meta,
                             int32_t* perm, int32_t* inv, int* status, cudaStream_t s);
 // T <= 64: dispatch and gather fused in one launch (same results as the two separately).
+// Row normalisation applied while gathering: row t becomes
+// gamma * x_t * rstd[t], rounded to the row type.  gamma == nullptr copies rows unchanged.
+struct GatherNorm {
+    const void* gamma = nullptr;
+    const float* rstd = nullptr;
+};
+
 cudaError_t launch_dispatch_gather_small(const int32_t* idx, int T, int E, int k, const void* x, size_t elem_bytes,
                                          int d, Meta* meta, int32_t* perm, int32_t* inv, void* xp, size_t slots,
-                                         int* status, cudaStream_t s);
+                                         int* status, cudaStream_t s, const GatherNorm& nm = GatherNorm());
 cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
-                          const int32_t* perm, void* xp, size_t slots, cudaStream_t s);
+                          const int32_t* perm, void* xp, size_t slots, cudaStream_t s,
+                          const GatherNorm& nm = GatherNorm());
 
+// resid (nullable, [T][d] in the output type) is added after the gate-weighted sum.
 cudaError_t launch_combine_bf16(const float* Y, const float* w, const int32_t* inv, int T, int d, int k,
-                                void* out, cudaStream_t s);
+                                void* out, cudaStream_t s, const void* resid = nullptr);
 cudaError_t launch_combine_f32(const float* Y, const float* w, const int32_t* inv, int T, int d, int k,
-                               float* out, cudaStream_t s);
+                               float* out, cudaStream_t s, const float* resid = nullptr);
 
 cudaError_t launch_simt_gemm1_f32(const float* xp, const float* W1, const float* W3, const Meta* meta, int E,
                                   int d, int F, float* H, size_t slots, cudaStream_t s);

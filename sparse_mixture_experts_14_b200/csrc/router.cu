@@ -11,6 +11,15 @@
 // fixed order (xor-butterfly or MMA accumulation, then warp order), so the
 // fp32 scores are identical run to run for a given batch size; they are
 // never rounded to bf16.  The pass is bound by reading x once from HBM.
+//
+// Block form (the MoE sub-layer's pre-norm, section "Mixtral 8x7B — Sparse
+// MoEの導入", subsection "Mixtralのアーキテクチャ"): the same pass routes
+// u = RMSNorm(x) = gamma * x * r with r = 1/sqrt(mean(x^2) + eps).  Since r is
+// one positive number per row, s = r * (Wg (gamma * x)): the pass sums the
+// squares of x beside the dot products and scales the scores by r at the end.
+// gamma * x is exact in fp32 for bf16 operands; on the tensor cores it enters
+// as two bf16 operands, hi = bf16(gamma x) and lo = gamma x - hi, which are
+// exact too, so the scores see the unrounded normalised row.
 #include "moe_common.cuh"
 
 namespace moe {
@@ -73,12 +82,42 @@ __device__ __forceinline__ void select_and_gate(const float (&s)[EB], int E, int
     for (int j = 0; j < k; ++j) w[j] = expf(sel[j] - sel[0]) / denom;
 }
 
+// Where a router pass writes its results (see RouteExtras for the optional ones).
+template <typename In>
+struct RouterIO {
+    int32_t* idx;
+    float* w;
+    const In* gamma;   // non-null exactly when the kernel is instantiated with NORM
+    float eps;
+    float* rstd;
+    float* logits;
+};
+
+// Per-token end of the pass: apply the row's norm factor, dump the scores if
+// asked, select and gate.  ss = sum of x^2 over the row (NORM only).
+template <typename In, int EB, bool NORM>
+__device__ __forceinline__ void finish_token(float (&sc)[EB], float ss, int t, int d, int E, int k,
+                                             const RouterIO<In>& io) {
+    if (NORM) {
+        const float r = 1.0f / sqrtf(ss / (float)d + io.eps);
+#pragma unroll
+        for (int e = 0; e < EB; ++e) sc[e] *= r;
+        io.rstd[t] = r;
+    }
+    if (io.logits) {
+        for (int e = 0; e < E; ++e) io.logits[(size_t)t * E + e] = sc[e];
+    }
+    select_and_gate<EB>(sc, E, k, io.idx + (size_t)t * k, io.w + (size_t)t * k);
+}
+
 // acc[t][e] += x_t[chunk] . Wg_e[chunk] for one 16-byte chunk; rows of Wg
 // past E alias row E-1 (their sums are never read), so every load is
-// unconditional and issues before the arithmetic.
-template <typename In, int EB, int TPW>
-__device__ __forceinline__ void chunk_dot(const typename Chunk<In>::Raw (&xr)[TPW], const In* __restrict__ Wg, int d,
-                                          int E, int c, float (&acc)[TPW][EB]) {
+// unconditional and issues before the arithmetic.  NORM: x is multiplied by
+// gamma first and ss[t] collects the squares of x.
+template <typename In, int EB, int TPW, bool NORM>
+__device__ __forceinline__ void chunk_dot(const typename Chunk<In>::Raw (&xr)[TPW], const In* __restrict__ Wg,
+                                          const In* __restrict__ gamma, int d, int E, int c, float (&acc)[TPW][EB],
+                                          float (&ss)[TPW]) {
     constexpr int CN = Chunk<In>::N;
     typename Chunk<In>::Raw wr[EB];
 #pragma unroll
@@ -86,6 +125,17 @@ __device__ __forceinline__ void chunk_dot(const typename Chunk<In>::Raw (&xr)[TP
     float xv[TPW][CN];
 #pragma unroll
     for (int t = 0; t < TPW; ++t) Chunk<In>::widen(xr[t], xv[t]);
+    if (NORM) {
+        float gv[CN];
+        Chunk<In>::widen(Chunk<In>::load(gamma + (size_t)c * CN), gv);
+#pragma unroll
+        for (int t = 0; t < TPW; ++t)
+#pragma unroll
+            for (int i = 0; i < CN; ++i) {
+                ss[t] = fmaf(xv[t][i], xv[t][i], ss[t]);
+                xv[t][i] *= gv[i];
+            }
+    }
 #pragma unroll
     for (int e = 0; e < EB; ++e) {
         float wv[CN];
@@ -99,36 +149,42 @@ __device__ __forceinline__ void chunk_dot(const typename Chunk<In>::Raw (&xr)[TP
 
 // Rows longer than 1024 chunks: one block per token, its threads loop over
 // the row; warp sums meet in shared memory and are added in warp order.
-template <typename In, int EB>
+template <typename In, int EB, bool NORM>
 __global__ void __launch_bounds__(256) router_loop_kernel(const In* __restrict__ x, const In* __restrict__ Wg, int T,
-                                                           int d, int E, int k, int32_t* __restrict__ idx,
-                                                           float* __restrict__ w) {
+                                                           int d, int E, int k, RouterIO<In> io) {
     pdl_trigger();
     pdl_wait();
     using Raw = typename Chunk<In>::Raw;
     constexpr int CN = Chunk<In>::N;
-    __shared__ float part[8][EB];
+    __shared__ float part[8][EB + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nchunks = d / CN;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         float acc[1][EB];
+        float ss[1] = {0.f};
 #pragma unroll
         for (int e = 0; e < EB; ++e) acc[0][e] = 0.f;
         for (int c = threadIdx.x; c < nchunks; c += 256) {
             Raw xr[1] = {Chunk<In>::load(x + (size_t)t * d + (size_t)c * CN)};
-            chunk_dot<In, EB, 1>(xr, Wg, d, E, c, acc);
+            chunk_dot<In, EB, 1, NORM>(xr, Wg, io.gamma, d, E, c, acc, ss);
         }
 #pragma unroll
         for (int e = 0; e < EB; ++e)
 #pragma unroll
             for (int m = 16; m >= 1; m >>= 1) acc[0][e] += __shfl_xor_sync(0xffffffffu, acc[0][e], m);
+        if (NORM) {
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], m);
+        }
         if (lane == 0) {
 #pragma unroll
             for (int e = 0; e < EB; ++e) part[warp][e] = acc[0][e];
+            part[warp][EB] = ss[0];
         }
         __syncthreads();
         if (threadIdx.x == 0) {
             float s[EB];
+            float sq = 0.f;
 #pragma unroll
             for (int e = 0; e < EB; ++e) {
                 float v = 0.f;
@@ -136,7 +192,9 @@ __global__ void __launch_bounds__(256) router_loop_kernel(const In* __restrict__
                 for (int q = 0; q < 8; ++q) v += part[q][e];
                 s[e] = v;
             }
-            select_and_gate<EB>(s, E, k, idx + (size_t)t * k, w + (size_t)t * k);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) sq += part[q][EB];
+            finish_token<In, EB, NORM>(s, sq, t, d, E, k, io);
         }
         __syncthreads();
     }
@@ -147,15 +205,14 @@ __global__ void __launch_bounds__(256) router_loop_kernel(const In* __restrict__
 // needs is requested before any arithmetic, so a block has TB rows in flight
 // at once; each Wg chunk it loads serves all TB tokens.  Lane partial sums
 // are reduced by a fixed xor-butterfly, the 8 warp sums in warp order.
-template <typename In, int EB, int TB, int RMAX>
+template <typename In, int EB, int TB, int RMAX, bool NORM>
 __global__ void __launch_bounds__(256) router_kernel(const In* __restrict__ x, const In* __restrict__ Wg, int T, int d,
-                                                     int E, int k, int32_t* __restrict__ idx,
-                                                     float* __restrict__ w) {
+                                                     int E, int k, RouterIO<In> io) {
     pdl_trigger();
     pdl_wait();
     using Raw = typename Chunk<In>::Raw;
     constexpr int CN = Chunk<In>::N;
-    __shared__ float part[8][TB][EB];
+    __shared__ float part[8][TB][EB + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nchunks = d / CN;
     for (int t0 = blockIdx.x * TB; t0 < T; t0 += gridDim.x * TB) {
@@ -169,31 +226,42 @@ __global__ void __launch_bounds__(256) router_kernel(const In* __restrict__ x, c
                                                        : Chunk<In>::zero();
         }
         float acc[TB][EB];
+        float ss[TB];
 #pragma unroll
-        for (int t = 0; t < TB; ++t)
+        for (int t = 0; t < TB; ++t) {
+            ss[t] = 0.f;
 #pragma unroll
             for (int e = 0; e < EB; ++e) acc[t][e] = 0.f;
+        }
 #pragma unroll
         for (int r = 0; r < RMAX; ++r) {
             const int c = threadIdx.x + r * 256;
-            if (c < nchunks) chunk_dot<In, EB, TB>(xr[r], Wg, d, E, c, acc);
+            if (c < nchunks) chunk_dot<In, EB, TB, NORM>(xr[r], Wg, io.gamma, d, E, c, acc, ss);
         }
 #pragma unroll
-        for (int t = 0; t < TB; ++t)
+        for (int t = 0; t < TB; ++t) {
 #pragma unroll
             for (int e = 0; e < EB; ++e)
 #pragma unroll
                 for (int m = 16; m >= 1; m >>= 1) acc[t][e] += __shfl_xor_sync(0xffffffffu, acc[t][e], m);
+            if (NORM) {
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) ss[t] += __shfl_xor_sync(0xffffffffu, ss[t], m);
+            }
+        }
         if (lane == 0) {
 #pragma unroll
-            for (int t = 0; t < TB; ++t)
+            for (int t = 0; t < TB; ++t) {
 #pragma unroll
                 for (int e = 0; e < EB; ++e) part[warp][t][e] = acc[t][e];
+                part[warp][t][EB] = ss[t];
+            }
         }
         __syncthreads();
         if (threadIdx.x < TB && t0 + (int)threadIdx.x < T) {
             const int t = threadIdx.x;
             float sc[EB];
+            float sq = 0.f;
 #pragma unroll
             for (int e = 0; e < EB; ++e) {
                 float v = 0.f;
@@ -201,7 +269,9 @@ __global__ void __launch_bounds__(256) router_kernel(const In* __restrict__ x, c
                 for (int q = 0; q < 8; ++q) v += part[q][t][e];
                 sc[e] = v;
             }
-            select_and_gate<EB>(sc, E, k, idx + (size_t)(t0 + t) * k, w + (size_t)(t0 + t) * k);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) sq += part[q][t][EB];
+            finish_token<In, EB, NORM>(sc, sq, t0 + t, d, E, k, io);
         }
         __syncthreads();
     }
@@ -226,23 +296,40 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int NT>
+// gamma * x for the bf16 pair xv (x) and gv (gamma), split into bf16 parts
+// hi + lo that sum to the fp32 product exactly; ss collects x^2.
+__device__ __forceinline__ void scaled_pair(uint32_t xv, uint32_t gv, uint32_t& hi, uint32_t& lo, float& ss) {
+    const float x0 = bf16_lo(xv), x1 = bf16_hi(xv);
+    ss = fmaf(x0, x0, ss);
+    ss = fmaf(x1, x1, ss);
+    const float p0 = x0 * bf16_lo(gv), p1 = x1 * bf16_hi(gv);
+    hi = pack_bf16x2(p0, p1);
+    lo = pack_bf16x2(p0 - bf16_lo(hi), p1 - bf16_hi(hi));
+}
+
+// NORM: the A operand is gamma * x as hi + lo (four MMAs per step instead of
+// two, so the accumulator is flushed every 4 steps to keep 16 MMAs per flush).
+template <int NT, bool NORM>
 __global__ void __launch_bounds__(256) router_mma_kernel(const __nv_bfloat16* __restrict__ x,
                                                          const __nv_bfloat16* __restrict__ Wg, int T, int d, int E,
-                                                         int k, int32_t* __restrict__ idx, float* __restrict__ w) {
+                                                         int k, RouterIO<__nv_bfloat16> io) {
     pdl_trigger();
     pdl_wait();
     constexpr int EB = 8 * NT;
+    constexpr int FLUSH = NORM ? 4 : 8;
     __shared__ float part[8][16][EB + 1];
+    __shared__ float sqp[8][16];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, q = lane & 3;
     const int nsteps = d / 32;
     const uint4 zero = make_uint4(0, 0, 0, 0);
+    const uint4* gam = reinterpret_cast<const uint4*>(io.gamma);
     for (int t0 = blockIdx.x * 16; t0 < T; t0 += gridDim.x * 16) {
         const int r0 = t0 + g, r1 = t0 + g + 8;
         const uint4* xr0 = reinterpret_cast<const uint4*>(x + (size_t)(r0 < T ? r0 : 0) * d);
         const uint4* xr1 = reinterpret_cast<const uint4*>(x + (size_t)(r1 < T ? r1 : 0) * d);
         float tot[NT][4], acc[NT][4];
+        float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll
         for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -253,14 +340,36 @@ __global__ void __launch_bounds__(256) router_mma_kernel(const __nv_bfloat16* __
             const int c = st * 4 + q;   // 16-byte chunk index of k0 + 8q
             const uint4 xa = r0 < T ? __ldg(xr0 + c) : zero;
             const uint4 xb = r1 < T ? __ldg(xr1 + c) : zero;
+            if (NORM) {
+                const uint4 gv = __ldg(gam + c);
+                uint4 ah, al, bh, bl;
+                scaled_pair(xa.x, gv.x, ah.x, al.x, ss0);
+                scaled_pair(xa.y, gv.y, ah.y, al.y, ss0);
+                scaled_pair(xa.z, gv.z, ah.z, al.z, ss0);
+                scaled_pair(xa.w, gv.w, ah.w, al.w, ss0);
+                scaled_pair(xb.x, gv.x, bh.x, bl.x, ss1);
+                scaled_pair(xb.y, gv.y, bh.y, bl.y, ss1);
+                scaled_pair(xb.z, gv.z, bh.z, bl.z, ss1);
+                scaled_pair(xb.w, gv.w, bh.w, bl.w, ss1);
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const int e = n * 8 + g;
-                const uint4 wv = e < E ? __ldg(reinterpret_cast<const uint4*>(Wg + (size_t)e * d) + c) : zero;
-                mma_bf16_16816(acc[n], xa.x, xb.x, xa.y, xb.y, wv.x, wv.y);
-                mma_bf16_16816(acc[n], xa.z, xb.z, xa.w, xb.w, wv.z, wv.w);
+                for (int n = 0; n < NT; ++n) {
+                    const int e = n * 8 + g;
+                    const uint4 wv = e < E ? __ldg(reinterpret_cast<const uint4*>(Wg + (size_t)e * d) + c) : zero;
+                    mma_bf16_16816(acc[n], ah.x, bh.x, ah.y, bh.y, wv.x, wv.y);
+                    mma_bf16_16816(acc[n], ah.z, bh.z, ah.w, bh.w, wv.z, wv.w);
+                    mma_bf16_16816(acc[n], al.x, bl.x, al.y, bl.y, wv.x, wv.y);
+                    mma_bf16_16816(acc[n], al.z, bl.z, al.w, bl.w, wv.z, wv.w);
+                }
+            } else {
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const int e = n * 8 + g;
+                    const uint4 wv = e < E ? __ldg(reinterpret_cast<const uint4*>(Wg + (size_t)e * d) + c) : zero;
+                    mma_bf16_16816(acc[n], xa.x, xb.x, xa.y, xb.y, wv.x, wv.y);
+                    mma_bf16_16816(acc[n], xa.z, xb.z, xa.w, xb.w, wv.z, wv.w);
+                }
             }
-            if (++since_flush == 8) {
+            if (++since_flush == FLUSH) {
                 since_flush = 0;
 #pragma unroll
                 for (int n = 0; n < NT; ++n)
@@ -281,10 +390,23 @@ __global__ void __launch_bounds__(256) router_mma_kernel(const __nv_bfloat16* __
             part[warp][g + 8][n * 8 + 2 * q] = tot[n][2];
             part[warp][g + 8][n * 8 + 2 * q + 1] = tot[n][3];
         }
+        if (NORM) {
+            // the 4 lanes of a group hold the row's chunks q = 0..3
+#pragma unroll
+            for (int m = 1; m <= 2; m <<= 1) {
+                ss0 += __shfl_xor_sync(0xffffffffu, ss0, m);
+                ss1 += __shfl_xor_sync(0xffffffffu, ss1, m);
+            }
+            if (q == 0) {
+                sqp[warp][g] = ss0;
+                sqp[warp][g + 8] = ss1;
+            }
+        }
         __syncthreads();
         if (threadIdx.x < 16 && t0 + (int)threadIdx.x < T) {
             const int t = threadIdx.x;
             float sc[EB];
+            float sq = 0.f;
 #pragma unroll
             for (int e = 0; e < EB; ++e) {
                 float v = 0.f;
@@ -292,7 +414,11 @@ __global__ void __launch_bounds__(256) router_mma_kernel(const __nv_bfloat16* __
                 for (int ww = 0; ww < 8; ++ww) v += part[ww][t][e];
                 sc[e] = v;
             }
-            select_and_gate<EB>(sc, E, k, idx + (size_t)(t0 + t) * k, w + (size_t)(t0 + t) * k);
+            if (NORM) {
+#pragma unroll
+                for (int ww = 0; ww < 8; ++ww) sq += sqp[ww][t];
+            }
+            finish_token<__nv_bfloat16, EB, NORM>(sc, sq, t0 + t, d, E, k, io);
         }
         __syncthreads();
     }
@@ -300,8 +426,8 @@ __global__ void __launch_bounds__(256) router_mma_kernel(const __nv_bfloat16* __
 
 // Chunks per thread the kernels are compiled for: 16-byte chunks x 256 threads x RMAX
 // cover d <= 8192 (bf16) / 4096 (fp32) with RMAX = 4; longer rows take the looping form.
-template <typename In, int EB, int TB>
-cudaError_t launch_router_t(const In* x, const In* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
+template <typename In, int EB, int TB, bool NORM>
+cudaError_t launch_router_t(const In* x, const In* Wg, int T, int d, int E, int k, const RouterIO<In>& io,
                             int num_sms, cudaStream_t s) {
     const int nchunks = d / Chunk<In>::N;
     // small batches: one token per block, so every SM gets work
@@ -309,53 +435,66 @@ cudaError_t launch_router_t(const In* x, const In* Wg, int T, int d, int E, int 
     const int tb = small ? 1 : TB;
     int blocks = (T + tb - 1) / tb;
     if (blocks < 1) blocks = 1;
+    const dim3 grid(blocks), block(256);
     if (nchunks <= 256) {
-        if (small) return launch_pdl(router_kernel<In, EB, 1, 1>, dim3(blocks), dim3(256), 0, s, x, Wg, T, d, E, k, idx, w);
-        else return launch_pdl(router_kernel<In, EB, TB, 1>, dim3(blocks), dim3(256), 0, s, x, Wg, T, d, E, k, idx, w);
+        if (small) return launch_pdl(router_kernel<In, EB, 1, 1, NORM>, grid, block, 0, s, x, Wg, T, d, E, k, io);
+        return launch_pdl(router_kernel<In, EB, TB, 1, NORM>, grid, block, 0, s, x, Wg, T, d, E, k, io);
     } else if (nchunks <= 512) {
-        if (small) return launch_pdl(router_kernel<In, EB, 1, 2>, dim3(blocks), dim3(256), 0, s, x, Wg, T, d, E, k, idx, w);
-        else return launch_pdl(router_kernel<In, EB, TB, 2>, dim3(blocks), dim3(256), 0, s, x, Wg, T, d, E, k, idx, w);
+        if (small) return launch_pdl(router_kernel<In, EB, 1, 2, NORM>, grid, block, 0, s, x, Wg, T, d, E, k, io);
+        return launch_pdl(router_kernel<In, EB, TB, 2, NORM>, grid, block, 0, s, x, Wg, T, d, E, k, io);
     } else if (nchunks <= 1024) {
-        if (small) return launch_pdl(router_kernel<In, EB, 1, 4>, dim3(blocks), dim3(256), 0, s, x, Wg, T, d, E, k, idx, w);
-        else return launch_pdl(router_kernel<In, EB, TB, 4>, dim3(blocks), dim3(256), 0, s, x, Wg, T, d, E, k, idx, w);
-    } else {
-        const int g = T < 65535 ? T : 65535;
-        return launch_pdl(router_loop_kernel<In, EB>, dim3(g), dim3(256), 0, s, x, Wg, T, d, E, k, idx, w);
+        if (small) return launch_pdl(router_kernel<In, EB, 1, 4, NORM>, grid, block, 0, s, x, Wg, T, d, E, k, io);
+        return launch_pdl(router_kernel<In, EB, TB, 4, NORM>, grid, block, 0, s, x, Wg, T, d, E, k, io);
     }
-    return cudaGetLastError();
+    const int g = T < 65535 ? T : 65535;
+    return launch_pdl(router_loop_kernel<In, EB, NORM>, dim3(g), block, 0, s, x, Wg, T, d, E, k, io);
+}
+
+template <typename In, bool NORM>
+cudaError_t launch_router_any(const In* x, const In* Wg, int T, int d, int E, int k, const RouterIO<In>& io,
+                              int num_sms, cudaStream_t s) {
+    if (E <= 8) return launch_router_t<In, 8, 4, NORM>(x, Wg, T, d, E, k, io, num_sms, s);
+    if (E <= 16) return launch_router_t<In, 16, 2, NORM>(x, Wg, T, d, E, k, io, num_sms, s);
+    return launch_router_t<In, 32, 1, NORM>(x, Wg, T, d, E, k, io, num_sms, s);
+}
+
+template <bool NORM>
+cudaError_t launch_router_mma(const __nv_bfloat16* x, const __nv_bfloat16* Wg, int T, int d, int E, int k,
+                              const RouterIO<__nv_bfloat16>& io, int num_sms, cudaStream_t s) {
+    const int tiles = (T + 15) / 16;
+    int grid = tiles < num_sms * 16 ? tiles : num_sms * 16;
+    if (grid < 1) grid = 1;
+    if (E <= 8) return launch_pdl(router_mma_kernel<1, NORM>, dim3(grid), dim3(256), 0, s, x, Wg, T, d, E, k, io);
+    if (E <= 16) return launch_pdl(router_mma_kernel<2, NORM>, dim3(grid), dim3(256), 0, s, x, Wg, T, d, E, k, io);
+    return launch_pdl(router_mma_kernel<4, NORM>, dim3(grid), dim3(256), 0, s, x, Wg, T, d, E, k, io);
 }
 
 template <typename In>
-cudaError_t launch_router_any(const In* x, const In* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
-                              int num_sms, cudaStream_t s) {
-    if (E <= 8) return launch_router_t<In, 8, 4>(x, Wg, T, d, E, k, idx, w, num_sms, s);
-    if (E <= 16) return launch_router_t<In, 16, 2>(x, Wg, T, d, E, k, idx, w, num_sms, s);
-    return launch_router_t<In, 32, 1>(x, Wg, T, d, E, k, idx, w, num_sms, s);
+RouterIO<In> make_io(int32_t* idx, float* w, const RouteExtras& ex) {
+    return RouterIO<In>{idx, w, static_cast<const In*>(ex.gamma), ex.eps, ex.rstd, ex.logits};
 }
 
 }  // namespace
 
 cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
-                               int num_sms, cudaStream_t s) {
+                               int num_sms, cudaStream_t s, const RouteExtras& ex) {
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(Wg);
+    const RouterIO<__nv_bfloat16> io = make_io<__nv_bfloat16>(idx, w, ex);
     // tensor-core scores for large batches; small batches spread one token per block instead
     if (d % 32 == 0 && T > 4 * num_sms) {
-        const int tiles = (T + 15) / 16;
-        int grid = tiles < num_sms * 16 ? tiles : num_sms * 16;
-        if (grid < 1) grid = 1;
-        const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-        const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(Wg);
-        if (E <= 8) return launch_pdl(router_mma_kernel<1>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
-        if (E <= 16) return launch_pdl(router_mma_kernel<2>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
-        return launch_pdl(router_mma_kernel<4>, dim3(grid), dim3(256), 0, s, xb, wb, T, d, E, k, idx, w);
+        return ex.gamma ? launch_router_mma<true>(xb, wb, T, d, E, k, io, num_sms, s)
+                        : launch_router_mma<false>(xb, wb, T, d, E, k, io, num_sms, s);
     }
-    return launch_router_any<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x),
-                                            static_cast<const __nv_bfloat16*>(Wg), T, d, E, k, idx, w, num_sms,
-                                            s);
+    return ex.gamma ? launch_router_any<__nv_bfloat16, true>(xb, wb, T, d, E, k, io, num_sms, s)
+                    : launch_router_any<__nv_bfloat16, false>(xb, wb, T, d, E, k, io, num_sms, s);
 }
 
 cudaError_t launch_router_f32(const float* x, const float* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
-                              int num_sms, cudaStream_t s) {
-    return launch_router_any<float>(x, Wg, T, d, E, k, idx, w, num_sms, s);
+                              int num_sms, cudaStream_t s, const RouteExtras& ex) {
+    const RouterIO<float> io = make_io<float>(idx, w, ex);
+    return ex.gamma ? launch_router_any<float, true>(x, Wg, T, d, E, k, io, num_sms, s)
+                    : launch_router_any<float, false>(x, Wg, T, d, E, k, io, num_sms, s);
 }
 
 }  // namespace moe

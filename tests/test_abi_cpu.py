@@ -106,3 +106,49 @@ def test_selftest_rejects_bad_limit(lib):
     f.argtypes = [ctypes.c_longlong, ctypes.c_void_p]
     assert f(10, None) == 1
     assert f(10 ** 12, None) == 1
+
+
+def _block(lib, T=8, d=128, F=256, E=8, k=2, h=0x1000, gamma=0x3000, out=0x100000, eps=1e-5, alpha=1.0,
+           stats=0x5000, f32=False):
+    fn = lib.moe_block_forward_f32 if f32 else lib.moe_block_forward
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float] + [ctypes.c_void_p] * 5 + \
+        [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
+    return fn(_vp(h), _vp(gamma) if gamma else None, eps, _vp(), _vp(), _vp(), _vp(), _vp(out), T, d, F, E, k,
+              alpha, _vp(stats) if stats else None, None)
+
+
+def test_block_argument_checks(lib):
+    assert _block(lib, k=9) == 1                      # k > E
+    assert _block(lib, d=100) == 2                    # bf16 needs d % 64 == 0
+    assert _block(lib, gamma=0) == 1                  # no gain
+    assert _block(lib, gamma=0x3004) == 1             # misaligned gain
+    assert _block(lib, eps=-1e-5) == 1                # negative eps
+    assert _block(lib, eps=float("inf")) == 1
+    assert _block(lib, eps=float("nan")) == 1
+    assert _block(lib, alpha=float("nan")) == 1
+    assert _block(lib, alpha=float("inf")) == 1
+    assert _block(lib, stats=0x5002) == 1             # misaligned stats
+    assert _block(lib, out=0x1000 + 256) == 1         # out overlaps h partly (rows are 256 bytes)
+    assert _block(lib, T=0, h=0, gamma=0, out=0) == 0  # empty batch: no-op
+    assert _block(lib, d=102, f32=True) == 2          # fp32 needs d % 4 == 0
+
+
+def test_block_workspace_size(lib):
+    lib.moe_block_workspace_size.restype = ctypes.c_size_t
+    lib.moe_workspace_size.restype = ctypes.c_size_t
+    plain = lib.moe_workspace_size(4096, 4096, 14336, 8, 2, 1)
+    blk = lib.moe_block_workspace_size(4096, 4096, 14336, 8, 2, 1)
+    assert blk >= plain + 4096 * 4 + 4096 * 8 * 4     # row factors and fp32 scores on top
+    assert lib.moe_block_workspace_size(4096, 4096, 14336, 8, 2, 7) == 0
+
+
+def test_route_stats_argument_checks(lib):
+    f = lib.moe_route_stats
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 4 + [ctypes.c_float] + \
+        [ctypes.c_void_p] * 4
+    assert f(_vp(), _vp(), 4, 128, 8, 9, 1.0, _vp(), _vp(), _vp(), None) == 1
+    assert f(_vp(), _vp(), 4, 128, 8, 2, 1.0, _vp(), _vp(), None, None) == 1   # stats required
+    assert f(_vp(), _vp(), 4, 128, 8, 2, float("nan"), _vp(), _vp(), _vp(), None) == 1
+    assert f(_vp(), _vp(), 0, 128, 8, 2, 1.0, None, None, None, None) == 0
