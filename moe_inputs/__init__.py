@@ -14,6 +14,8 @@ Operand layouts (row-major, the ``nn.Linear`` weight convention of the
 Initialisation: x ~ N(0, 1), Wg, W1, W3 ~ N(0, 1/d), W2 ~ N(0, 1/F).  bf16
 operands are returned as uint16 bit patterns, fp32 operands as float32.
 
+Backward workloads add dout = dL/dout [T][d] (id 6): N(0, 1).
+
 Block operands (the MoE sub-layer with its pre-norm and residual): the
 residual stream h is x with row t scaled by 2^((t mod 5) - 2), an exact
 power-of-two scale in bf16 and fp32, so rows span a 16x range of norms; the
@@ -42,7 +44,7 @@ _LIB_PATH = os.path.join(_HERE, "libmoe_inputs.so")
 _lock = threading.Lock()
 _lib = None
 
-TENSOR_IDS = {"x": 0, "Wg": 1, "W1": 2, "W3": 3, "W2": 4, "gamma": 5}
+TENSOR_IDS = {"x": 0, "Wg": 1, "W1": 2, "W3": 3, "W2": 4, "gamma": 5, "dout": 6}
 BLOCK_EPS = 1e-5      # eps of the block's RMSNorm in every test and workload
 BF16_ONE = 0x3F80
 
@@ -164,6 +166,11 @@ def make_inputs(T: int, d: int, F: int, E: int, k: int, dtype: str = "bf16", see
         inp.W3 = normal((E, F, d), seed, TENSOR_IDS["W3"], 1.0 / np.sqrt(d), dtype)
         inp.W2 = normal((E, d, F), seed, TENSOR_IDS["W2"], 1.0 / np.sqrt(F), dtype)
     return inp
+
+
+def make_dout(T: int, d: int, dtype: str, seed: int) -> np.ndarray:
+    """The upstream gradient dL/dout [T][d] of the backward workloads: N(0, 1)."""
+    return normal((T, d), seed, TENSOR_IDS["dout"], 1.0, dtype)
 
 
 def row_scales(T: int) -> np.ndarray:

@@ -25,6 +25,11 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   balance                  pinned: uniform scores (loss = alpha*k), cyclic
                            balanced batch, brute force against torch,
                            sums of f and p
+  backward / backward_tokens / weight_grad_slices
+                           pinned: central finite differences of moe();
+                           torch autograd of the E=1 dense FFN and of the
+                           k=E softmax mixture; slices and token rows equal
+                           the full backward
 
 The block and balance steps follow the same page, section "Mixtral 8x7B —
 Sparse MoEの導入" (subsection "Mixtralのアーキテクチャ": RMSNorm, MoE layer,
@@ -76,6 +81,11 @@ def _load():
             lib.oracle_block.argtypes = [ci, ci, ci, ci, ci, vp, vp, cd, vp, vp, vp, vp, ci, vp, ci, vp, vp, vp,
                                          vp, vp, ci]
             lib.oracle_balance.argtypes = [ci, ci, ci, vp, cd, vp, vp, vp]
+            lib.oracle_backward.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp] + [vp] * 10
+            lib.oracle_backward_tokens.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, vp, ci] + \
+                [vp] * 6 + [ci]
+            lib.oracle_weight_grad_slices.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, ci, vp, ci,
+                                                      vp, vp, vp, ci]
             lib.oracle_max_threads.restype = ci
             _lib = lib
     return _lib
@@ -238,3 +248,52 @@ def balance(logits, k: int, alpha: float):
     _check(_load().oracle_balance(T, E, k, s.ctypes.data, float(alpha), f.ctypes.data, p.ctypes.data,
                                   loss.ctypes.data), "balance")
     return f, p, float(loss[0])
+
+
+def backward(x, Wg, W1, W3, W2, dout, k: int, dtype: str) -> dict:
+    """Every gradient of L = sum <dout, out> (small shapes): dict(dx, dlogits, dWg, dW1, dW3, dW2, idx, g,
+    margin, mingap), all float64."""
+    x, Wg, W1, W3, W2, dout = (_arr(a, dtype) for a in (x, Wg, W1, W3, W2, dout))
+    T, d = x.shape
+    E, F = W1.shape[0], W1.shape[1]
+    r = dict(dx=np.empty((T, d)), dlogits=np.empty((T, E)), dWg=np.empty((E, d)), dW1=np.empty((E, F, d)),
+             dW3=np.empty((E, F, d)), dW2=np.empty((E, d, F)), idx=np.empty((T, k), dtype=np.int32),
+             g=np.empty((T, k)), margin=np.empty(T), mingap=np.empty(T))
+    _check(_load().oracle_backward(T, d, F, E, k, x.ctypes.data, Wg.ctypes.data, W1.ctypes.data, W3.ctypes.data,
+                                   W2.ctypes.data, DTYPE_CODE[dtype], dout.ctypes.data,
+                                   *[r[n].ctypes.data for n in ("dx", "dlogits", "dWg", "dW1", "dW3", "dW2", "idx",
+                                                                "g", "margin", "mingap")]), "backward")
+    return r
+
+
+def backward_tokens(x, Wg, W1, W3, W2, dout, k: int, dtype: str, tokens, nthreads: int = 0) -> dict:
+    """dx and the router-score gradient of the listed tokens only: dict(dx, dlogits, idx, g, margin, mingap, tokens)."""
+    x, Wg, W1, W3, W2, dout = (_arr(a, dtype) for a in (x, Wg, W1, W3, W2, dout))
+    T, d = x.shape
+    E, F = W1.shape[0], W1.shape[1]
+    tok = np.ascontiguousarray(tokens, dtype=np.int32)
+    n = tok.size
+    r = dict(dx=np.empty((n, d)), dlogits=np.empty((n, E)), idx=np.empty((n, k), dtype=np.int32),
+             g=np.empty((n, k)), margin=np.empty(n), mingap=np.empty(n))
+    _check(_load().oracle_backward_tokens(T, d, F, E, k, x.ctypes.data, Wg.ctypes.data, W1.ctypes.data,
+                                          W3.ctypes.data, W2.ctypes.data, DTYPE_CODE[dtype], dout.ctypes.data,
+                                          tok.ctypes.data, n,
+                                          *[r[m].ctypes.data for m in ("dx", "dlogits", "idx", "g", "margin",
+                                                                       "mingap")], nthreads), "backward_tokens")
+    r["tokens"] = tok
+    return r
+
+
+def weight_grad_slices(x, Wg, W1, W3, W2, dout, k: int, dtype: str, e: int, fs, nthreads: int = 0):
+    """Rows fs of dW1_e and dW3_e ([n][d] each) and columns fs of dW2_e ([d][n]) over all tokens."""
+    x, Wg, W1, W3, W2, dout = (_arr(a, dtype) for a in (x, Wg, W1, W3, W2, dout))
+    T, d = x.shape
+    E, F = W1.shape[0], W1.shape[1]
+    f = np.ascontiguousarray(fs, dtype=np.int32)
+    n = f.size
+    r1, r3, c2 = np.empty((n, d)), np.empty((n, d)), np.empty((d, n))
+    _check(_load().oracle_weight_grad_slices(T, d, F, E, k, x.ctypes.data, Wg.ctypes.data, W1.ctypes.data,
+                                             W3.ctypes.data, W2.ctypes.data, DTYPE_CODE[dtype], dout.ctypes.data,
+                                             int(e), f.ctypes.data, n, r1.ctypes.data, r3.ctypes.data,
+                                             c2.ctypes.data, nthreads), "weight_grad_slices")
+    return r1, r3, c2

@@ -49,6 +49,20 @@
  *                      L = alpha * E * sum_i f_i p_i: subsection "ロードバランス損失"
  *                      (f, p and loss equations), with f counting all k
  *                      selections as the page's load_balance_loss code does.
+ *   8. backward        gradients of a scalar loss L through the layer, given
+ *                      dout = dL/dout (the training step the page's subsection
+ *                      "ロードバランス損失" closes with: the layer is trained
+ *                      by gradient descent on L_LM + L_balance).  The top-k
+ *                      choice is piecewise constant, so no gradient flows
+ *                      through it; for each selected slot j with expert e:
+ *                        dy_j  = g_j dout                      dg_j = <dout, y_j>
+ *                        ds_e  = g_j (dg_j - sum_m g_m dg_m)   (softmax over the k)
+ *                        dh    = W2_e^T dy_j
+ *                        da    = dh * b * SiLU'(a),  db = dh * SiLU(a)
+ *                        dx   += W1_e^T da + W3_e^T db,  plus Wg^T ds from the router
+ *                        dW2_e += dy_j h^T, dW1_e += da x^T, dW3_e += db x^T,
+ *                        dWg   += ds x^T
+ *                      with SiLU'(a) = sigmoid(a) (1 + a (1 - sigmoid(a))).
  *
  * Operands are row-major: x[T][d], Wg[E][d], W1[E][F][d], W3[E][F][d],
  * W2[E][d][F].  dtype 0 = float32 storage, 1 = bfloat16 bit patterns; every
@@ -378,6 +392,245 @@ int oracle_balance(int T, int E, int k, const double* logits, double alpha, doub
         acc += f[e] * p[e];
     }
     *loss = alpha * (double)E * acc;
+    return 0;
+}
+
+/* ------------------------------------------------------------------ backward */
+
+static double sigmoid(double a) { return 1.0 / (1.0 + exp(-a)); }
+
+/* the forward of one expert on xv, keeping a, b and h (step 4 with its intermediates) */
+static void expert_forward_keep(int d, int F, const double* xv, const void* W1, const void* W3, const void* W2,
+                                int dtype, int e, double* a, double* b, double* h, double* y) {
+    size_t w13 = (size_t)e * F * d;
+    for (int f = 0; f < F; ++f) {
+        double sa = 0.0, sb = 0.0;
+        for (int j = 0; j < d; ++j) {
+            sa += elem(W1, dtype, w13 + (size_t)f * d + j) * xv[j];
+            sb += elem(W3, dtype, w13 + (size_t)f * d + j) * xv[j];
+        }
+        a[f] = sa;
+        b[f] = sb;
+        h[f] = sa / (1.0 + exp(-sa)) * sb;
+    }
+    size_t w2 = (size_t)e * d * F;
+    for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int f = 0; f < F; ++f) acc += elem(W2, dtype, w2 + (size_t)i * F + f) * h[f];
+        y[i] = acc;
+    }
+}
+
+struct bwd_scratch {
+    double *xv, *go, *a, *b, *h, *y, *dy, *dh, *da, *db;   /* a, b, h: [k][F]; y: [k][d] */
+};
+
+static int scratch_alloc(struct bwd_scratch* w, int d, int F, int k) {
+    w->xv = (double*)malloc(sizeof(double) * d);
+    w->go = (double*)malloc(sizeof(double) * d);
+    w->a = (double*)malloc(sizeof(double) * (size_t)k * F);
+    w->b = (double*)malloc(sizeof(double) * (size_t)k * F);
+    w->h = (double*)malloc(sizeof(double) * (size_t)k * F);
+    w->y = (double*)malloc(sizeof(double) * (size_t)k * d);
+    w->dy = (double*)malloc(sizeof(double) * d);
+    w->dh = (double*)malloc(sizeof(double) * F);
+    w->da = (double*)malloc(sizeof(double) * F);
+    w->db = (double*)malloc(sizeof(double) * F);
+    return w->xv && w->go && w->a && w->b && w->h && w->y && w->dy && w->dh && w->da && w->db;
+}
+
+static void scratch_free(struct bwd_scratch* w) {
+    free(w->xv); free(w->go); free(w->a); free(w->b); free(w->h);
+    free(w->y); free(w->dy); free(w->dh); free(w->da); free(w->db);
+}
+
+/*
+ * step 8 for one token t: dx_t [d] and the router-score gradient ds [E]
+ * (zero for unselected experts).  When dWg/dW1/dW3/dW2 are non-null the
+ * token's contributions are added to them (the caller runs tokens in order).
+ */
+static void token_backward(int d, int F, int E, int k, const void* x, const void* Wg, const void* W1, const void* W3,
+                           const void* W2, int dtype, const void* dout, size_t t, struct bwd_scratch* w, double* dx,
+                           double* ds, int32_t* idx, double* g, double* margin, double* mingap, double* dWg,
+                           double* dW1, double* dW3, double* dW2) {
+    for (int j = 0; j < d; ++j) {
+        w->xv[j] = elem(x, dtype, t * (size_t)d + j);
+        w->go[j] = elem(dout, dtype, t * (size_t)d + j);
+    }
+    double s[64], dg[64];
+    token_scores(d, E, x, Wg, dtype, t, s);
+    token_select(E, k, s, idx, g, margin, mingap);
+    for (int j = 0; j < k; ++j) {
+        expert_forward_keep(d, F, w->xv, W1, W3, W2, dtype, idx[j], w->a + (size_t)j * F, w->b + (size_t)j * F,
+                            w->h + (size_t)j * F, w->y + (size_t)j * d);
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += w->go[i] * w->y[(size_t)j * d + i];
+        dg[j] = acc;
+    }
+    double gdg = 0.0;
+    for (int j = 0; j < k; ++j) gdg += g[j] * dg[j];
+    for (int e = 0; e < E; ++e) ds[e] = 0.0;
+    for (int j = 0; j < k; ++j) ds[idx[j]] = g[j] * (dg[j] - gdg);
+    /* router path: dx = Wg^T ds */
+    for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int e = 0; e < E; ++e) acc += elem(Wg, dtype, (size_t)e * d + i) * ds[e];
+        dx[i] = acc;
+    }
+    if (dWg)
+        for (int e = 0; e < E; ++e)
+            for (int i = 0; i < d; ++i) dWg[(size_t)e * d + i] += ds[e] * w->xv[i];
+    for (int j = 0; j < k; ++j) {
+        const int e = idx[j];
+        const double* a = w->a + (size_t)j * F;
+        const double* b = w->b + (size_t)j * F;
+        const double* h = w->h + (size_t)j * F;
+        for (int i = 0; i < d; ++i) w->dy[i] = g[j] * w->go[i];
+        const size_t w2 = (size_t)e * d * F, w13 = (size_t)e * F * d;
+        for (int f = 0; f < F; ++f) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i) acc += elem(W2, dtype, w2 + (size_t)i * F + f) * w->dy[i];
+            w->dh[f] = acc;
+            const double sg = sigmoid(a[f]);
+            w->da[f] = acc * b[f] * sg * (1.0 + a[f] * (1.0 - sg));
+            w->db[f] = acc * a[f] * sg;
+        }
+        for (int i = 0; i < d; ++i) {
+            double acc = 0.0;
+            for (int f = 0; f < F; ++f)
+                acc += elem(W1, dtype, w13 + (size_t)f * d + i) * w->da[f] +
+                       elem(W3, dtype, w13 + (size_t)f * d + i) * w->db[f];
+            dx[i] += acc;
+        }
+        if (dW2)
+            for (int i = 0; i < d; ++i)
+                for (int f = 0; f < F; ++f) dW2[w2 + (size_t)i * F + f] += w->dy[i] * h[f];
+        if (dW1)
+            for (int f = 0; f < F; ++f)
+                for (int i = 0; i < d; ++i) {
+                    dW1[w13 + (size_t)f * d + i] += w->da[f] * w->xv[i];
+                    dW3[w13 + (size_t)f * d + i] += w->db[f] * w->xv[i];
+                }
+    }
+}
+
+/*
+ * Every gradient of L = sum_t <dout_t, out_t> (step 8), tokens in order.
+ * dx [T][d], dlogits [T][E] (the router-score gradient ds), dWg [E][d],
+ * dW1/dW3 [E][F][d], dW2 [E][d][F]; idx/g [T][k], margin/mingap [T] as in
+ * oracle_route.  Slow by design: for small shapes.
+ */
+int oracle_backward(int T, int d, int F, int E, int k, const void* x, const void* Wg, const void* W1, const void* W3,
+                    const void* W2, int dtype, const void* dout, double* dx, double* dlogits, double* dWg, double* dW1,
+                    double* dW3, double* dW2, int32_t* idx, double* g, double* margin, double* mingap) {
+    if (T < 0 || d <= 0 || F <= 0 || E <= 0 || E > 64 || k <= 0 || k > E) return 1;
+    struct bwd_scratch w;
+    if (!scratch_alloc(&w, d, F, k)) {
+        scratch_free(&w);
+        return 2;
+    }
+    memset(dWg, 0, sizeof(double) * (size_t)E * d);
+    memset(dW1, 0, sizeof(double) * (size_t)E * F * d);
+    memset(dW3, 0, sizeof(double) * (size_t)E * F * d);
+    memset(dW2, 0, sizeof(double) * (size_t)E * d * F);
+    for (int t = 0; t < T; ++t)
+        token_backward(d, F, E, k, x, Wg, W1, W3, W2, dtype, dout, (size_t)t, &w, dx + (size_t)t * d,
+                       dlogits + (size_t)t * E, idx + (size_t)t * k, g + (size_t)t * k, margin + t, mingap + t, dWg,
+                       dW1, dW3, dW2);
+    scratch_free(&w);
+    return 0;
+}
+
+/* dx and ds of the listed tokens only (no weight gradients); rows in list order */
+int oracle_backward_tokens(int T, int d, int F, int E, int k, const void* x, const void* Wg, const void* W1,
+                           const void* W3, const void* W2, int dtype, const void* dout, const int32_t* tokens, int n,
+                           double* dx, double* dlogits, int32_t* idx, double* g, double* margin, double* mingap,
+                           int nthreads) {
+    if (T < 0 || d <= 0 || F <= 0 || E <= 0 || E > 64 || k <= 0 || k > E || n < 0) return 1;
+    for (int r = 0; r < n; ++r)
+        if (tokens[r] < 0 || tokens[r] >= T) return 1;
+    int fail = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        struct bwd_scratch w;
+        if (!scratch_alloc(&w, d, F, k)) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int r = 0; r < n; ++r)
+                token_backward(d, F, E, k, x, Wg, W1, W3, W2, dtype, dout, (size_t)tokens[r], &w,
+                               dx + (size_t)r * d, dlogits + (size_t)r * E, idx + (size_t)r * k, g + (size_t)r * k,
+                               margin + r, mingap + r, NULL, NULL, NULL, NULL);
+        }
+        scratch_free(&w);
+    }
+    return fail ? 2 : 0;
+}
+
+/*
+ * Selected slices of expert e's weight gradients over all tokens (step 8):
+ * rows f of dW1_e and dW3_e ([nf][d] each) and columns f of dW2_e ([d][nf]),
+ * for f in fs[0..nf).  Each needs only row f of W1_e/W3_e and column f of
+ * W2_e per routed token, so full-size batches stay cheap.
+ */
+int oracle_weight_grad_slices(int T, int d, int F, int E, int k, const void* x, const void* Wg, const void* W1,
+                              const void* W3, const void* W2, int dtype, const void* dout, int e, const int32_t* fs,
+                              int nf, double* dW1_rows, double* dW3_rows, double* dW2_cols, int nthreads) {
+    if (T < 0 || d <= 0 || F <= 0 || E <= 0 || E > 64 || k <= 0 || k > E || e < 0 || e >= E || nf < 0) return 1;
+    for (int r = 0; r < nf; ++r)
+        if (fs[r] < 0 || fs[r] >= F) return 1;
+    /* routing of every token: slot of e and its gate (0 when e is not selected) */
+    double* ge = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!ge) return 2;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int t = 0; t < T; ++t) {
+        double s[64], g[64];
+        int32_t idx[64];
+        token_scores(d, E, x, Wg, dtype, (size_t)t, s);
+        token_select(E, k, s, idx, g, NULL, NULL);
+        ge[t] = 0.0;
+        for (int j = 0; j < k; ++j)
+            if (idx[j] == e) ge[t] = g[j];
+    }
+    const size_t w13 = (size_t)e * F * d, w2 = (size_t)e * d * F;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nf; ++r) {
+        const int f = fs[r];
+        double* r1 = dW1_rows + (size_t)r * d;
+        double* r3 = dW3_rows + (size_t)r * d;
+        for (int i = 0; i < d; ++i) {
+            r1[i] = r3[i] = 0.0;
+            dW2_cols[(size_t)i * nf + r] = 0.0;
+        }
+        for (int t = 0; t < T; ++t) {
+            if (ge[t] == 0.0) continue;
+            double a = 0.0, b = 0.0, dh = 0.0;
+            for (int j = 0; j < d; ++j) {
+                const double xj = elem(x, dtype, (size_t)t * d + j);
+                a += elem(W1, dtype, w13 + (size_t)f * d + j) * xj;
+                b += elem(W3, dtype, w13 + (size_t)f * d + j) * xj;
+            }
+            const double sg = sigmoid(a);
+            const double h = a * sg * b;
+            for (int i = 0; i < d; ++i) dh += elem(W2, dtype, w2 + (size_t)i * F + f) * ge[t] * elem(dout, dtype, (size_t)t * d + i);
+            const double da = dh * b * sg * (1.0 + a * (1.0 - sg));
+            const double db = dh * a * sg;
+            for (int i = 0; i < d; ++i) {
+                const double xi = elem(x, dtype, (size_t)t * d + i);
+                r1[i] += da * xi;
+                r3[i] += db * xi;
+                dW2_cols[(size_t)i * nf + r] += ge[t] * elem(dout, dtype, (size_t)t * d + i) * h;
+            }
+        }
+    }
+    free(ge);
     return 0;
 }
 
