@@ -48,6 +48,7 @@ METRIC = "MoE-layer tokens/sec at 1 B200; achieved % of roofline (tensor TFLOPS 
 BLOCK_METRIC = ("MoE sub-layer (RMSNorm + MoE + residual, load-balance statistics) tokens/sec at 1 B200; "
                 "achieved % of roofline")
 BLOCK_ALPHA = 0.01
+TRAIN_METRIC = "MoE-layer training step (forward + backward) tokens/sec at 1 B200; achieved % of roofline"
 L2_BYTES = 126 * 1000 * 1000
 DEFAULT_CONFIG = 2   # the Mixtral-shape decode layer (T=16, d=4096, ffn=14336, E=8, k=2)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -65,6 +66,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--block", action="store_true",
                     help="time the block form out = h + MoE(RMSNorm(h)) with load-balance statistics")
+    ap.add_argument("--train", action="store_true",
+                    help="time a training step: forward (grouped-GEMM path) + backward with all gradients")
     ap.add_argument("--stage-every", type=int, default=8,
                     help="record per-stage events on every n-th timed step (events between launches "
                          "break the overlap of dependent launches, so most steps run without them)")
@@ -208,6 +211,25 @@ def oracle_fn(inp, block):
     return lambda toks, nt: oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=nt)
 
 
+def oracle_train_run(inp, dout, target_s):
+    """Time the oracle's forward + backward (all gradients) on an evenly spaced token sample of about
+    target_s seconds (the oracle's backward runs on one thread); returns (tokens/s, sample text, seconds)."""
+    import oracle
+    sub = lambda toks: [np.ascontiguousarray(inp.x[toks]), inp.Wg, inp.W1, inp.W3, inp.W2,
+                        np.ascontiguousarray(dout[toks])]
+    t0 = time.perf_counter()
+    oracle.backward(*sub([0]), inp.k, inp.dtype)
+    per_tok = max(time.perf_counter() - t0, 1e-5)
+    n = int(max(1, min(inp.T, round(target_s / per_tok))))
+    toks = np.unique(np.linspace(0, inp.T - 1, n).astype(np.int64))
+    t0 = time.perf_counter()
+    oracle.backward(*sub(toks), inp.k, inp.dtype)
+    dt = time.perf_counter() - t0
+    sample = (f"{len(toks)} of {inp.T} tokens (evenly spaced): forward and every gradient (dx, dWg, dW1, dW3, dW2) "
+              f"of those tokens in fp64, one thread")
+    return len(toks) / dt, sample, dt
+
+
 def make_workload(cfg, block):
     inp = moe_inputs.make_config(cfg)
     return moe_inputs.make_block(inp) if block else inp
@@ -242,6 +264,28 @@ def run_reference(args, rank):
         return
     c = moe_inputs.CONFIGS[args.config]
     inp = make_workload(args.config, args.block)
+    if args.train:
+        dout = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
+        per_step = max(0.5, min(30.0, 150.0 / max(args.steps + args.warmup, 1)))
+        for _ in range(args.warmup):
+            oracle_train_run(inp, dout, per_step)
+        total_tok, total_t = 0.0, 0.0
+        for _ in range(args.steps):
+            v, sample, dt = oracle_train_run(inp, dout, per_step)
+            total_tok += v * dt
+            total_t += dt
+        value = total_tok / total_t
+        line = {
+            "impl": "reference", "metric": TRAIN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_t / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": c["name"] + "+train", "T": inp.T, "d": inp.d, "ffn": inp.F, "E": inp.E,
+                       "k": inp.k, "seed": c["seed"]},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     run = oracle_fn(inp, args.block)
     threads = len(os.sched_getaffinity(0))
     total_steps = args.steps + args.warmup
@@ -455,6 +499,119 @@ def run_ours(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+def run_train(args, rank, world, local):
+    """One step = moe_forward_ws (grouped-GEMM path) + moe_backward_ws over one batch, inputs resident."""
+    import sparse_mixture_experts_14_b200 as moe
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    c = moe_inputs.CONFIGS[args.config]
+    inp = moe_inputs.make_config(args.config)
+    dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
+    dout_np = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
+    dout = to_dev(dout_np, inp.dtype, device)
+    T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
+    code = moe.MOE_DTYPE_BF16 if inp.dtype == "bf16" else moe.MOE_DTYPE_F32
+    fws = torch.empty(moe.moe_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
+    bws = torch.empty(moe.moe_backward_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
+    out = torch.empty((T, d), dtype=dev[0].dtype, device=device)
+    f32 = torch.float32
+    grads = dict(dx=torch.empty((T, d), dtype=dev[0].dtype, device=device),
+                 dWg=torch.empty((E, d), dtype=f32, device=device), dW1=torch.empty((E, F, d), dtype=f32, device=device),
+                 dW3=torch.empty((E, F, d), dtype=f32, device=device),
+                 dW2=torch.empty((E, d, F), dtype=f32, device=device))
+    idx, _ = moe.moe_route(dev[0], dev[1], k)
+    counts = moe.moe_dispatch(idx, E)[0].cpu().numpy()
+    acc = accounting(inp, counts)
+    kT = k * T
+    bwd_flops = {"dgrad_h": 2.0 * kT * d * F, "swiglu_bwd": 4.0 * kT * d * F, "dgrad_x": 4.0 * kT * d * F,
+                 "wgrad2": 2.0 * kT * d * F, "wgrad13": 4.0 * kT * d * F}
+    # algorithmic work of a training step: the forward, then 12 kT d F of expert gradients (the SwiGLU
+    # recompute is this implementation's choice, not counted) and 4 T d E for the router's two gradients
+    step_flops = acc["layer_flops"] + 12.0 * kT * d * F + 4.0 * T * d * E
+
+    ns, nb = moe.MOE_NUM_STAGES, moe.MOE_BWD_NUM_STAGES
+    K, W = args.steps, args.warmup
+    every = max(1, args.stage_every)
+    staged = [i for i in range(K) if i % every == 0]
+    fev = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(K)]
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(nb + 1)] for _ in range(K)]
+    stream = torch.cuda.current_stream()
+    for row in fev + bev:
+        for e in row:
+            e.record(stream)
+
+    def step(i=None):
+        on = i is not None and i % every == 0
+        n = moe.moe_forward_profiled(*dev, k, fws, out, events=fev[i] if on else None, path=moe.MOE_PATH_PREFILL)
+        _, m = moe.moe_backward_ws(*dev, dout, k, fws, workspace=bws, grads=grads, events=bev[i] if on else None)
+        return n + m
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    launches = 0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(K):
+        launches += step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    status = moe.moe_get_device_status()
+    if status != moe.MOE_OK:
+        raise RuntimeError(f"device fault during the timed region: {moe.moe_status_string(status)}")
+    total_ms = reduce_max(start.elapsed_time(end), world, device)
+    value = weak_scaling_value(T, K, world, total_ms)
+    if rank != 0:
+        return
+    fst = {n: statistics.mean(fev[i][s].elapsed_time(fev[i][s + 1]) for i in staged)
+           for s, n in enumerate(moe.STAGE_NAMES)}
+    bst = {n: statistics.mean(bev[i][s].elapsed_time(bev[i][s + 1]) for i in staged)
+           for s, n in enumerate(moe.BWD_STAGE_NAMES)}
+    peaks, peak_src = load_peaks()
+    long_run = total_ms > 1000.0
+    tflops_peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
+    dom = max(bwd_flops, key=lambda n: bst[n])
+    sec = bst[dom] / 1000.0
+    roof = {"bound": "tensor", "achieved": bwd_flops[dom] / sec / 1e12, "peak": tflops_peak, "unit": "TFLOP/s",
+            "traffic": recorded_traffic(f"tc_gemm_kernel<{dom}>", c["name"]), "kernel": f"tc_gemm_kernel ({dom})",
+            "per_launch": {"flops": bwd_flops[dom], "ms": bst[dom]},
+            "peak_source": f"{peak_src} ({'sustained' if long_run else 'burst'})"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof_tps = T / (step_flops / (tflops_peak * 1e12))
+    step_roof = {"bound": "tensor", "roofline_tokens_per_s": roof_tps, "frac": (value / world) / roof_tps,
+                 "flops": step_flops}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, sample, _ = oracle_train_run(inp, dout_np, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
+    line = {
+        "metric": TRAIN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": inp.dtype, "data": "synthetic",
+        "config": {"workload": c["name"] + "+train", "T": T, "d": d, "ffn": F, "E": E, "k": k, "seed": c["seed"],
+                   "l2": "touched weights larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "step_roofline": step_roof,
+        "stages_ms": {"forward": fst, "backward": bst},
+        "stage_events": f"recorded on {len(staged)} of {K} timed steps (every {every})",
+        "cpu_baseline": cpu,
+        "e2e": None,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -468,7 +625,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
                                              device_id=torch.device("cuda", local))
     try:
-        run_ours(args, rank, world, local)
+        (run_train if args.train else run_ours)(args, rank, world, local)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

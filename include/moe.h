@@ -312,6 +312,53 @@ MOE_API moe_status moe_route_stats_f32(const float* x, const float* Wg, int T, i
                                        float alpha, int32_t* topk_idx, float* topk_w, float* stats,
                                        cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Backward pass: gradients of a scalar loss L through the layer, given
+ * dout = dL/dout [T][d].  The page trains the layer by gradient descent on
+ * the language-model loss plus the load-balance loss (subsection
+ * "ロードバランス損失"); these are the gradients of the equations at the top of
+ * this file, with the top-k choice held fixed (it is piecewise constant):
+ *
+ *   dy_j = g_j dout,  dg_j = <dout, E_ij(x)>,  ds = g_j (dg_j - sum_m g_m dg_m)
+ *   dh = W2^T dy,  da = dh * b * SiLU'(a),  db = dh * SiLU(a)   (a = W1 x, b = W3 x)
+ *   dx = sum_j (W1^T da + W3^T db) + Wg^T ds
+ *   dW2 += dy h^T,  dW1 += da x^T,  dW3 += db x^T,  dWg += ds x^T
+ *
+ * The gradient of the load-balance loss is not included (its p term depends
+ * on the scores; add it through dlogits if needed).
+ *
+ * Use: run moe_forward_ws with MOE_PATH_PREFILL (MOE_PATH_AUTO takes it when
+ * T > moe_decode_max_tokens(); the fp32 forward always does) on the same
+ * operands, then pass its workspace here unchanged as fwd_workspace (device,
+ * read only).  workspace: at least moe_backward_workspace_size() bytes
+ * (device, 256-byte aligned).  Outputs (device, overwritten): dx [T][d] in
+ * the layer's element type; dWg [E][d], dW1 [E][F][d], dW3 [E][F][d] and
+ * dW2 [E][d][F] in float; dlogits [T][E] float (optional, NULL allowed): the
+ * gradient of the router scores, zero for unselected experts.  Every sum runs
+ * in a fixed order (no float atomics), so results are bitwise repeatable.
+ * stage_events (optional) receives MOE_BWD_NUM_STAGES + 1 events as in
+ * moe_forward_profiled; launches (optional) the number of kernels launched.
+ * ------------------------------------------------------------------------ */
+enum {
+    MOE_BWD_STAGE_SCATTER = 0,  /* dy = g dout into the expert segments, dg, ds */
+    MOE_BWD_STAGE_DGRAD_H = 1,  /* dH = dY W2 */
+    MOE_BWD_STAGE_SWIGLU = 2,   /* GEMM1 recomputed, dA and dB */
+    MOE_BWD_STAGE_DGRAD_X = 3,  /* dXp = dA W1 + dB W3 */
+    MOE_BWD_STAGE_WGRAD2 = 4,   /* dW2 */
+    MOE_BWD_STAGE_WGRAD13 = 5,  /* dW1, dW3 */
+    MOE_BWD_STAGE_ROUTER = 6,   /* dWg and the dx combine */
+    MOE_BWD_NUM_STAGES = 7
+};
+
+MOE_API size_t moe_backward_workspace_size(int T, int d, int ffn, int E, int k, int dtype);
+
+MOE_API moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const void* W3,
+                                   const void* W2, const void* dout, void* dx, float* dWg, float* dW1,
+                                   float* dW3, float* dW2, float* dlogits, int T, int d, int ffn, int E,
+                                   int k, int dtype, const void* fwd_workspace, size_t fwd_workspace_bytes,
+                                   void* workspace, size_t workspace_bytes, cudaEvent_t* stage_events,
+                                   int* launches, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

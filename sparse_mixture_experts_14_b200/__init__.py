@@ -35,6 +35,8 @@ MOE_PATH_AUTO, MOE_PATH_PREFILL, MOE_PATH_DECODE = 0, 1, 2
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_NUM_STAGES = 6
 STAGE_NAMES = ("route", "dispatch", "gather", "expert1", "expert2", "combine")
+MOE_BWD_NUM_STAGES = 7
+BWD_STAGE_NAMES = ("scatter", "dgrad_h", "swiglu_bwd", "dgrad_x", "wgrad2", "wgrad13", "router")
 
 # every symbol include/moe.h declares, with its ctypes signature
 _vp, _ci, _sz, _ll, _cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong, ctypes.c_float
@@ -62,6 +64,8 @@ SIGNATURES = {
     "moe_block_forward_ws": (_ci, [_vp, _vp, _cf, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _ci,
                                    _ci, _vp, _sz, _vp, _vp, _vp]),
     "moe_route_stats": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
+    "moe_backward_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
+    "moe_backward_ws": (_ci, [_vp] * 12 + [_ci] * 6 + [_vp, _sz, _vp, _sz, _vp, _vp, _vp]),
     "moe_route_stats_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
@@ -238,11 +242,11 @@ def moe_forward_host(x_host, Wg, W1, W3, W2, k, out_host=None, stream=None):
     return out_host
 
 
-def _events(events):
+def _events(events, n=MOE_NUM_STAGES):
     if events is None:
         return None
-    if len(events) != MOE_NUM_STAGES + 1:
-        raise ValueError(f"need {MOE_NUM_STAGES + 1} events")
+    if len(events) != n + 1:
+        raise ValueError(f"need {n + 1} events")
     return (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
 
 
@@ -309,6 +313,47 @@ def moe_route_stats(x, Wg, k, alpha=1.0, stream=None):
     _check(fn(_ptr(x), _ptr(Wg), T, d, E, k, float(alpha), _ptr(idx), _ptr(w), _ptr(stats), _stream(stream)),
            "moe_route_stats")
     return idx, w, stats
+
+
+def moe_backward_workspace_size(T, d, ffn, E, k, dtype=MOE_DTYPE_BF16) -> int:
+    return int(_lib.moe_backward_workspace_size(T, d, ffn, E, k, dtype))
+
+
+def moe_backward_ws(x, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, grads=None, dlogits=None,
+                    events=None, stream=None):
+    """Gradients of the layer given dout = dL/dout, after moe_forward_ws(..., path=MOE_PATH_PREFILL,
+    workspace=fwd_workspace) on the same operands.  Returns (grads, launches) with grads a dict of
+    dx (layer dtype), dWg, dW1, dW3, dW2 (float32); pass `grads` to reuse buffers, `dlogits` (float32
+    [T][E]) to also get the router-score gradient."""
+    code = _dtype_code(x)
+    for t, n in ((x, "x"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2"), (dout, "dout")):
+        _dev(t, x.dtype, n)
+    T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
+    if dout.shape != (T, d):
+        raise ValueError("dout must have the shape of x")
+    dev = x.device
+    if grads is None:
+        f32 = torch.float32
+        grads = dict(dx=torch.empty((T, d), dtype=x.dtype, device=dev), dWg=torch.empty((E, d), dtype=f32, device=dev),
+                     dW1=torch.empty((E, F, d), dtype=f32, device=dev), dW3=torch.empty((E, F, d), dtype=f32, device=dev),
+                     dW2=torch.empty((E, d, F), dtype=f32, device=dev))
+    _dev(grads["dx"], x.dtype, "dx")
+    for n in ("dWg", "dW1", "dW3", "dW2"):
+        _dev(grads[n], torch.float32, n)
+    if dlogits is not None:
+        _dev(dlogits, torch.float32, "dlogits")
+    _dev(fwd_workspace, torch.uint8, "fwd_workspace")
+    if workspace is None:
+        workspace = torch.empty(max(moe_backward_workspace_size(T, d, F, E, k, code), 1), dtype=torch.uint8,
+                                device=dev)
+    _dev(workspace, torch.uint8, "workspace")
+    n = ctypes.c_int(0)
+    _check(_lib.moe_backward_ws(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dout), _ptr(grads["dx"]),
+                                _ptr(grads["dWg"]), _ptr(grads["dW1"]), _ptr(grads["dW3"]), _ptr(grads["dW2"]),
+                                _ptr(dlogits), T, d, F, E, k, code, _ptr(fwd_workspace), fwd_workspace.numel(),
+                                _ptr(workspace), workspace.numel(), _events(events, MOE_BWD_NUM_STAGES),
+                                ctypes.byref(n), _stream(stream)), "moe_backward_ws")
+    return grads, n.value
 
 
 def moe_get_device_status(stream=None) -> int:

@@ -1,0 +1,407 @@
+// Backward pass of the layer: gradients of a loss L given dout = dL/dout.
+//
+// The layer is trained by gradient descent on the language-model loss plus
+// the load-balance loss (subsection "ロードバランス損失" of the
+// "Mistral/Mixtral architecture" page); this file holds everything of the
+// backward except the tensor-core GEMMs (gemm_tc.cu).  Differentiating the
+// output equation of subsection "Top-2ゲーティングの定式化" and the expert
+// equation of subsection "各エキスパートの構造", with the top-k choice fixed
+// (it is piecewise constant), per assignment (t, j) of expert e in slot r:
+//     dY[r]  = g_tj dout_t                 dg_tj = <dout_t, Y[r]>
+//     ds_te  = g_tj (dg_tj - sum_m g_tm dg_tm)       (softmax over the k)
+//     dH     = dY W2_e,  dA, dB = SwiGLU backward,  dXp = dA W1_e + dB W3_e
+//     dW2_e  = dY_e^T H_e,  dW1_e = dA_e^T Xp_e,  dW3_e = dB_e^T Xp_e
+//     dWg    = ds^T x,      dx_t = sum_j dXp[slot(t, j)] + ds_t Wg
+// Every sum runs in a fixed order (no float atomics), so the gradients are
+// the same bits on every run.
+//
+// Kernels here: the gate-scaled scatter of dout into the expert segments
+// (with dg), the router-score gradient ds, dWg (per-chunk partial sums, then
+// one ordered pass), the dx combine, and the fp32 entry points' grouped GEMMs
+// on the CUDA cores (operands read through strides, so none is transposed).
+#include "moe_common.cuh"
+
+namespace moe {
+namespace {
+
+template <typename T>
+struct Elt;
+template <>
+struct Elt<float> {
+    __device__ __forceinline__ static float get(const float* p, size_t i) { return __ldg(p + i); }
+    __device__ __forceinline__ static void put(float* p, size_t i, float v) { p[i] = v; }
+};
+template <>
+struct Elt<__nv_bfloat16> {
+    __device__ __forceinline__ static float get(const __nv_bfloat16* p, size_t i) { return __bfloat162float(p[i]); }
+    __device__ __forceinline__ static void put(__nv_bfloat16* p, size_t i, float v) { p[i] = __float2bfloat16_rn(v); }
+};
+
+// One warp per padded row r < offsets[E]: dY[r] = g dout_t rounded to the
+// operand type (zero on padding rows) and dg[t][j] = <dout_t, Y[r]> (lane
+// partial sums in column order, then a fixed butterfly).  Block 0 also
+// zeroes the backward GEMMs' wave counters.
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_scatter_kernel(const T* __restrict__ dout, const float* __restrict__ w,
+                                                          const float* __restrict__ Y, Meta* __restrict__ meta,
+                                                          const int32_t* __restrict__ perm, int E, int T_, int k,
+                                                          int d, size_t slots, T* __restrict__ dY,
+                                                          float* __restrict__ dg) {
+    pdl_trigger();
+    pdl_wait();
+    if (blockIdx.x == 0 && threadIdx.x >= kWaveDgradH && threadIdx.x < kWaveSlots) meta->waves[threadIdx.x] = 0;
+    const int lane = threadIdx.x & 31;
+    const size_t total = (size_t)meta->offsets[E];
+    const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
+    const long long TK = (long long)T_ * k;
+    for (size_t r = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < total && r < slots; r += warps) {
+        const int a = perm[r];
+        T* dst = dY + r * (size_t)d;
+        if (a >= 0 && a < TK) {
+            const int t = a / k;
+            const float g = w[a];
+            const T* src = dout + (size_t)t * d;
+            const float* y = Y + r * (size_t)d;
+            float acc = 0.f;
+            if (sizeof(T) == 2) {
+                // 8 elements per lane and step (d % 64 == 0 on the bf16 path)
+                for (int v = lane; v < d / 8; v += 32) {
+                    const uint4 u = __ldg(reinterpret_cast<const uint4*>(src) + v);
+                    const float4 y0 = __ldg(reinterpret_cast<const float4*>(y) + 2 * v);
+                    const float4 y1 = __ldg(reinterpret_cast<const float4*>(y) + 2 * v + 1);
+                    const float go[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                                         bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+                    const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc = fmaf(go[i], yv[i], acc);
+                    uint4 o;
+                    o.x = pack_bf16x2(g * go[0], g * go[1]);
+                    o.y = pack_bf16x2(g * go[2], g * go[3]);
+                    o.z = pack_bf16x2(g * go[4], g * go[5]);
+                    o.w = pack_bf16x2(g * go[6], g * go[7]);
+                    reinterpret_cast<uint4*>(dst)[v] = o;
+                }
+            } else {
+                for (int i = lane; i < d; i += 32) {
+                    const float go = Elt<T>::get(src, i);
+                    Elt<T>::put(dst, i, g * go);
+                    acc = fmaf(go, y[i], acc);
+                }
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+            if (lane == 0) dg[a] = acc;
+        } else {
+            for (int i = lane; i < d; i += 32) Elt<T>::put(dst, i, 0.f);
+        }
+    }
+}
+
+// ds[t][e]: the gradient of the router scores (zero for unselected experts).
+__global__ void __launch_bounds__(256) router_bwd_kernel(const int32_t* __restrict__ idx, const float* __restrict__ w,
+                                                         const float* __restrict__ dg, int T_, int E, int k,
+                                                         float* __restrict__ ds) {
+    pdl_trigger();
+    pdl_wait();
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T_) return;
+    float gdg = 0.f;
+    for (int j = 0; j < k; ++j) gdg = fmaf(w[(size_t)t * k + j], dg[(size_t)t * k + j], gdg);
+    float* row = ds + (size_t)t * E;
+    for (int e = 0; e < E; ++e) row[e] = 0.f;
+    for (int j = 0; j < k; ++j) {
+        const int e = idx[(size_t)t * k + j];
+        if (e >= 0 && e < E) row[e] = w[(size_t)t * k + j] * (dg[(size_t)t * k + j] - gdg);
+    }
+}
+
+constexpr int kWgChunk = 256;   // tokens per dWg partial sum
+
+// part[c][e][j] = sum over tokens t of chunk c (ascending) of ds[t][e] x[t][j]
+template <typename T, int EB>
+__global__ void __launch_bounds__(256) dwg_part_kernel(const T* __restrict__ x, const float* __restrict__ ds, int T_,
+                                                       int d, int E, float* __restrict__ part) {
+    pdl_trigger();
+    pdl_wait();
+    __shared__ float sds[kWgChunk][EB];
+    const int c = blockIdx.y;
+    const int t0 = c * kWgChunk;
+    const int nt = min(kWgChunk, T_ - t0);
+    for (int i = threadIdx.x; i < nt * EB; i += blockDim.x) {
+        const int t = i / EB, e = i - t * EB;
+        sds[t][e] = e < E ? ds[(size_t)(t0 + t) * E + e] : 0.f;
+    }
+    __syncthreads();
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= d) return;
+    float acc[EB];
+#pragma unroll
+    for (int e = 0; e < EB; ++e) acc[e] = 0.f;
+    for (int t = 0; t < nt; ++t) {
+        const float xv = Elt<T>::get(x, (size_t)(t0 + t) * d + j);
+#pragma unroll
+        for (int e = 0; e < EB; ++e) acc[e] = fmaf(sds[t][e], xv, acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < EB; ++e)
+        if (e < E) part[((size_t)c * E + e) * d + j] = acc[e];
+}
+
+__global__ void __launch_bounds__(256) dwg_final_kernel(const float* __restrict__ part, int chunks, int E, int d,
+                                                        float* __restrict__ dWg) {
+    pdl_trigger();
+    pdl_wait();
+    const size_t n = (size_t)E * d;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        float v = 0.f;
+        for (int c = 0; c < chunks; ++c) v += part[(size_t)c * n + i];
+        dWg[i] = v;
+    }
+}
+
+// dx[t] = sum_j dXp[inv[t][j]] (j ascending) + sum_e ds[t][e] Wg[e] (e ascending), one rounding.
+template <typename T>
+__global__ void __launch_bounds__(256) dx_combine_kernel(const float* __restrict__ dXp, const int32_t* __restrict__ inv,
+                                                         const float* __restrict__ ds, const T* __restrict__ Wg,
+                                                         int T_, int d, int E, int k, T* __restrict__ dx) {
+    pdl_trigger();
+    pdl_wait();
+    const size_t n = (size_t)T_ * d;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const int t = (int)(i / d);
+        const int c = (int)(i - (size_t)t * d);
+        float acc = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const int slot = inv[(size_t)t * k + j];
+            if (slot >= 0) acc += dXp[(size_t)slot * d + c];
+        }
+        for (int e = 0; e < E; ++e) {
+            const float s = ds[(size_t)t * E + e];
+            if (s != 0.f) acc = fmaf(s, Elt<T>::get(Wg, (size_t)e * d + c), acc);
+        }
+        Elt<T>::put(dx, i, acc);
+    }
+}
+
+// ---------------------------------------------------------------- fp32 grouped GEMMs (CUDA cores)
+
+// Strided view of one operand: element (row, k) of expert e is
+// base[e * es + row * sr + k * sk]; a second base takes over for k >= ksplit.
+struct View {
+    const float* base;
+    const float* base2;
+    size_t es, sr, sk;
+    int ksplit;
+    __device__ __forceinline__ float at(int e, int row, int k) const {
+        const float* b = base;
+        if (k >= ksplit) {
+            b = base2;
+            k -= ksplit;
+        }
+        return __ldg(b + (size_t)e * es + (size_t)row * sr + (size_t)k * sk);
+    }
+};
+
+constexpr int GT = 64, GK = 16;
+
+// Row-grouped (ROWS): C[r][n] = sum_k A(r, k) B_e(n, k) over the rows r of
+// expert e's segment, K = K.  Grouped by K (!ROWS): C_e[m][n] = sum over the
+// expert's rows r of A(r, m) B(r, n).  SWIGLU_BWD: B and B3 give a and b of
+// the row; the output row is dA | dB from dh.  Sums run over k ascending.
+template <bool ROWS, bool SWIGLU_BWD>
+__global__ void __launch_bounds__(256) simt_gemm_bwd_kernel(View A, View B, View B3, const Meta* __restrict__ meta,
+                                                            int E, int M, int N, int K, const float* __restrict__ dh,
+                                                            float* __restrict__ C, float* __restrict__ C_hi,
+                                                            int split) {
+    pdl_trigger();
+    pdl_wait();
+    __shared__ float As[GK][GT + 4];
+    __shared__ float Bs[GK][GT + 4];
+    __shared__ float B3s[SWIGLU_BWD ? GK : 1][GT + 4];
+    int e, m0, k0, k1;
+    if (ROWS) {
+        m0 = blockIdx.x * GT;
+        const int total = meta->offsets[E];
+        if (m0 >= total) return;
+        e = 0;
+        while (e + 1 < E && m0 >= meta->offsets[e + 1]) ++e;
+        k0 = 0;
+        k1 = K;
+    } else {
+        e = blockIdx.z;
+        m0 = blockIdx.x * GT;
+        if (m0 >= M) return;
+        k0 = meta->offsets[e];
+        k1 = meta->offsets[e + 1];
+    }
+    const int n0 = blockIdx.y * GT;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float acc[4][4], acc3[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = acc3[i][j] = 0.f;
+    for (int kk = k0; kk < k1; kk += GK) {
+        for (int l = threadIdx.x; l < GT * GK; l += 256) {
+            const int r = l / GK, c = l % GK;
+            const int k = kk + c;
+            const bool kin = k < k1;
+            const int m = m0 + r, n = n0 + r;
+            if (ROWS) {
+                As[c][r] = kin ? A.at(0, m, k) : 0.f;
+                Bs[c][r] = (kin && n < N) ? B.at(e, n, k) : 0.f;
+                if (SWIGLU_BWD) B3s[c][r] = (kin && n < N) ? B3.at(e, n, k) : 0.f;
+            } else {
+                As[c][r] = (kin && m < M) ? A.at(0, k, m) : 0.f;
+                Bs[c][r] = (kin && n < N) ? B.at(0, k, n) : 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < GK; ++c) {
+            float a[4], b[4], b3[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = As[c][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                b[j] = Bs[c][tx * 4 + j];
+                if (SWIGLU_BWD) b3[j] = B3s[c][tx * 4 + j];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+                    if (SWIGLU_BWD) acc3[i][j] = fmaf(a[i], b3[j], acc3[i][j]);
+                }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int m = m0 + ty * 4 + i;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + tx * 4 + j;
+            if (n >= N) continue;
+            if (SWIGLU_BWD) {
+                const float av = acc[i][j], bv = acc3[i][j], g = dh[(size_t)m * N + n];
+                const float s = 1.0f / (1.0f + expf(-av));
+                C[(size_t)m * (2 * N) + n] = g * bv * s * (1.0f + av * (1.0f - s));
+                C[(size_t)m * (2 * N) + N + n] = g * av * s;
+            } else if (ROWS) {
+                C[(size_t)m * N + n] = acc[i][j];
+            } else if (m < M) {
+                float* dst = m < split ? C + ((size_t)e * split + m) * N
+                                       : C_hi + ((size_t)e * (M - split) + (m - split)) * N;
+                dst[n] = acc[i][j];
+            }
+        }
+    }
+}
+
+View view(const float* base, size_t es, size_t sr, size_t sk, const float* base2 = nullptr, int ksplit = INT32_MAX) {
+    return View{base, base2 ? base2 : base, es, sr, sk, ksplit};
+}
+
+template <typename T>
+cudaError_t launch_scatter(const BwdArgs& a, cudaStream_t s) {
+    size_t blocks = (a.slots + 7) / 8;
+    if (blocks > 65535 * 4) blocks = 65535 * 4;
+    if (blocks < 1) blocks = 1;
+    return launch_pdl(bwd_scatter_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, s,
+                      static_cast<const T*>(a.dout), a.w, a.Y, a.meta, a.perm, a.E, a.T, a.k, a.d, a.slots,
+                      static_cast<T*>(a.dy), a.dg);
+}
+
+template <typename T>
+cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s) {
+    const int chunks = (a.T + kWgChunk - 1) / kWgChunk;
+    const dim3 grid((a.d + 255) / 256, chunks);
+    const T* x = static_cast<const T*>(a.x);
+    cudaError_t e;
+    if (a.E <= 8) e = launch_pdl(dwg_part_kernel<T, 8>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part);
+    else if (a.E <= 16) e = launch_pdl(dwg_part_kernel<T, 16>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part);
+    else e = launch_pdl(dwg_part_kernel<T, 32>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part);
+    if (e != cudaSuccess) return e;
+    size_t blocks = ((size_t)a.E * a.d + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    return launch_pdl(dwg_final_kernel, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const float*>(a.dwg_part),
+                      chunks, a.E, a.d, a.dWg);
+}
+
+template <typename T>
+cudaError_t launch_dx(const BwdArgs& a, cudaStream_t s) {
+    size_t blocks = ((size_t)a.T * a.d + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    if (blocks < 1) blocks = 1;
+    return launch_pdl(dx_combine_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const float*>(a.dxp),
+                      a.inv, static_cast<const float*>(a.ds), static_cast<const T*>(a.Wg), a.T, a.d, a.E, a.k,
+                      static_cast<T*>(a.dx));
+}
+
+}  // namespace
+
+size_t dwg_part_bytes(int T, int E, int d) {
+    const size_t chunks = (size_t)(T > 0 ? (T + kWgChunk - 1) / kWgChunk : 1);
+    return chunks * (size_t)E * d * 4;
+}
+
+cudaError_t launch_bwd_scatter(const BwdArgs& a, cudaStream_t s) {
+    return a.bf16 ? launch_scatter<__nv_bfloat16>(a, s) : launch_scatter<float>(a, s);
+}
+
+cudaError_t launch_router_bwd(const BwdArgs& a, cudaStream_t s) {
+    return launch_pdl(router_bwd_kernel, dim3((a.T + 255) / 256), dim3(256), 0, s, a.idx, a.w,
+                      static_cast<const float*>(a.dg), a.T, a.E, a.k, a.ds);
+}
+
+cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s) {
+    return a.bf16 ? launch_dwg<__nv_bfloat16>(a, s) : launch_dwg<float>(a, s);
+}
+
+cudaError_t launch_dx_combine(const BwdArgs& a, cudaStream_t s) {
+    return a.bf16 ? launch_dx<__nv_bfloat16>(a, s) : launch_dx<float>(a, s);
+}
+
+cudaError_t launch_simt_bwd_gemms(const BwdArgs& a, cudaStream_t s) {
+    const int E = a.E, d = a.d, F = a.F;
+    const size_t S = a.slots;
+    const float* xp = static_cast<const float*>(a.xp);
+    const float* W1 = static_cast<const float*>(a.W1);
+    const float* W3 = static_cast<const float*>(a.W3);
+    const float* W2 = static_cast<const float*>(a.W2);
+    const float* H = static_cast<const float*>(a.H);
+    const float* dy = static_cast<const float*>(a.dy);
+    float* dab = static_cast<float*>(a.dab);
+    const View none = view(nullptr, 0, 0, 0);
+    const dim3 blk(256);
+    // dH [S][F] = dY . W2_e : B(n = f, k = i) = W2[e][i][f]
+    cudaError_t e = launch_pdl(simt_gemm_bwd_kernel<true, false>, dim3((unsigned)(S / GT), (F + GT - 1) / GT), blk, 0, s,
+                               view(dy, 0, d, 1), view(W2, (size_t)d * F, 1, F), none, a.meta, E, 0, F, d,
+                               static_cast<const float*>(nullptr), a.dh, static_cast<float*>(nullptr), 0);
+    // dA | dB [S][2F] from a = Xp W1_e^T, b = Xp W3_e^T and dH
+    if (e == cudaSuccess)
+        e = launch_pdl(simt_gemm_bwd_kernel<true, true>, dim3((unsigned)(S / GT), (F + GT - 1) / GT), blk, 0, s,
+                       view(xp, 0, d, 1), view(W1, (size_t)F * d, d, 1), view(W3, (size_t)F * d, d, 1), a.meta, E, 0,
+                       F, d, static_cast<const float*>(a.dh), dab, static_cast<float*>(nullptr), 0);
+    // dXp [S][d] = [dA dB] . [W1_e ; W3_e] : B(n = j, k = f) = W1[e][f][j], then W3 for k >= F
+    if (e == cudaSuccess)
+        e = launch_pdl(simt_gemm_bwd_kernel<true, false>, dim3((unsigned)(S / GT), (d + GT - 1) / GT), blk, 0, s,
+                       view(dab, 0, 2 * F, 1), view(W1, (size_t)F * d, 1, d, W3, F), none, a.meta, E, 0, d, 2 * F,
+                       static_cast<const float*>(nullptr), static_cast<float*>(a.dxp), static_cast<float*>(nullptr),
+                       0);
+    // dW2_e [d][F] = dY_e^T H_e
+    if (e == cudaSuccess)
+        e = launch_pdl(simt_gemm_bwd_kernel<false, false>, dim3((d + GT - 1) / GT, (F + GT - 1) / GT, E), blk, 0, s,
+                       view(dy, 0, d, 1), view(H, 0, F, 1), none, a.meta, E, d, F, 0,
+                       static_cast<const float*>(nullptr), a.dW2, a.dW2, d);
+    // [dW1_e ; dW3_e] [2F][d] = [dA dB]_e^T Xp_e
+    if (e == cudaSuccess)
+        e = launch_pdl(simt_gemm_bwd_kernel<false, false>, dim3((2 * F + GT - 1) / GT, (d + GT - 1) / GT, E), blk, 0, s,
+                       view(dab, 0, 2 * F, 1), view(xp, 0, d, 1), none, a.meta, E, 2 * F, d, 0,
+                       static_cast<const float*>(nullptr), a.dW1, a.dW3, F);
+    return e;
+}
+
+}  // namespace moe

@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ blk, i
         if ((size_t)offs[E] > slots) record_status(status, MOE_ERR_DEVICE);
         for (int e = 0; e < E; ++e) meta->counts[e] = tot[e];
         for (int e = 0; e <= E; ++e) meta->offsets[e] = offs[e];
-        meta->waves[0] = meta->waves[1] = 0;
+        for (int i = 0; i < kWaveSlots; ++i) meta->waves[i] = 0;
     }
     __syncthreads();
     if (warp < E) {
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kDispatchTokens) dispatch_single_kernel(const 
         if ((size_t)offs[E] > slots) record_status(status, MOE_ERR_DEVICE);
         for (int e = 0; e < E; ++e) meta->counts[e] = tot[e];
         for (int e = 0; e <= E; ++e) meta->offsets[e] = offs[e];
-        meta->waves[0] = meta->waves[1] = 0;
+        for (int i = 0; i < kWaveSlots; ++i) meta->waves[i] = 0;
     }
     __syncthreads();
     if (t < T) {
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(256) dispatch_gather_small_kernel(const int32_
             if ((size_t)total > slots) record_status(status, MOE_ERR_DEVICE);
             for (int e = 0; e < E; ++e) meta->counts[e] = cnt[e];
             for (int e = 0; e <= E; ++e) meta->offsets[e] = offs[e];
-            meta->waves[0] = meta->waves[1] = 0;
+            for (int i = 0; i < kWaveSlots; ++i) meta->waves[i] = 0;
         }
         for (int a = tid; a < T * k; a += blockDim.x) inv[a] = row_of[a];
         for (int r = tid; r < total; r += blockDim.x)

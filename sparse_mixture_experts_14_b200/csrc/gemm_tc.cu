@@ -32,6 +32,16 @@
 // has an odd number of m-tiles, the peer of its last pair computes rows past
 // the expert's segment and stores nothing.  The tile list is derived on the
 // device from the dispatch offsets: no host synchronisation.
+//
+// The same kernel runs the layer's backward GEMMs (gradients of the expert
+// equations, the training the page's "ロードバランス損失" subsection closes with):
+//     dH    = dY_e W2_e                  W2 read MN-major (no transpose)
+//     dA,dB = SwiGLU backward of GEMM1 recomputed in TMEM, with dH from HBM
+//     dXp   = dA_e W1_e + dB_e W3_e      W1 / W3 read MN-major, K = 2F
+//     dW2_e = dY_e^T H_e                 both operands MN-major, K = the
+//     dW1_e|dW3_e = [dA dB]_e^T Xp_e     expert's rows (grouped by K)
+// MN-major tiles come in as two 64-wide TMA boxes (128-byte swizzle) and are
+// described to tcgen05.mma as MN-major, so no operand is ever transposed in HBM.
 #include <cuda.h>
 
 #include "moe_common.cuh"
@@ -53,7 +63,47 @@ constexpr uint32_t PAIR_TX_BYTES = 2 * STAGE_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int NUM_THREADS = 192;
 constexpr int NUM_EPI_WARPS = 4;
-constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BM, BN);
+constexpr int MN_BOX = 64;                     // MN-major operands: two 64-wide boxes per 128 rows
+constexpr uint32_t MN_LBO = MN_BOX * BK * 2;   // bytes between the two boxes (atoms along M/N)
+constexpr uint32_t MN_SBO = 1024;              // bytes between 8-row groups along K
+
+// What one instantiation computes.
+enum : int {
+    kFwd1 = 0,       // H = SiLU(Xp W1^T) * (Xp W3^T)            -> bf16 [slots][N]
+    kFwd2 = 1,       // C = A B_e^T, B K-major                   -> fp32 [slots][N]
+    kDgradH = 2,     // dH = dY W2_e (W2 MN-major)                -> fp32 [slots][N]
+    kSwigluBwd = 3,  // dA | dB from recomputed a, b and dH        -> bf16 [slots][2N]
+    kDgradX = 4,     // dXp = dA W1_e + dB W3_e (MN-major, K = 2F) -> fp32 [slots][N]
+    kWgrad = 5,      // dW_e = A_e^T B_e over the expert's rows     -> fp32 [E][M][N]
+};
+
+template <int MODE>
+struct ModeT {
+    static constexpr bool GATED = MODE == kFwd1 || MODE == kSwigluBwd;   // B halves = W1 / W3 blocks
+    static constexpr bool A_MN = MODE == kWgrad;
+    static constexpr bool B_MN = MODE == kDgradH || MODE == kDgradX || MODE == kWgrad;
+    static constexpr bool KGROUP = MODE == kWgrad;                        // tiles grouped by K, not by rows
+    static constexpr int N_PER_TILE = GATED ? BNH : BN;
+    static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
+};
+
+// Scalar arguments of one launch.
+struct GemmParams {
+    Meta* meta;
+    int E;
+    int M;           // kWgrad: output rows per expert
+    int N;           // output columns (kSwigluBwd: F; its output rows hold 2N)
+    int K;           // reduction length of the row-grouped modes
+    int split;       // kWgrad: output rows m >= split go to out_hi, row m - split
+    int kb_split;    // kDgradX: K blocks from mapB3 start here
+    int wave_slot;
+    size_t slots;
+    void* out;
+    void* out_hi;
+    const float* aux;   // kSwigluBwd: dH [slots][N] fp32
+    int* status;
+    long long wait_ns;
+};
 
 struct Ctrl {
     uint64_t full[STAGES];      // leader: both CTAs' bytes of a stage landed
@@ -67,7 +117,8 @@ struct Ctrl {
     int tile_base[kMaxExperts + 1];
     int mt[kMaxExperts];        // 128-row m-tiles of expert e
     int pt[kMaxExperts];        // pairs of m-tiles of expert e
-    int row0[kMaxExperts];
+    int row0[kMaxExperts];      // first row of expert e's segment
+    int nkb[kMaxExperts];       // K blocks of expert e (grouped-by-K tiles)
 };
 
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + (int)sizeof(Ctrl) + 1024;
@@ -97,13 +148,11 @@ __device__ __forceinline__ void wave_sync(int* counter, int target) {
     }
 }
 
-// SWIGLU: GEMM1 (B halves = 128-row blocks of W1 and W3, out = H bf16 [slots][N]).
-// !SWIGLU: GEMM2 (B halves = the two 128-row halves of a 256-row W2 block, out = Y fp32 [slots][N]).
-template <bool SWIGLU>
+template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB1,
-                   const __grid_constant__ CUtensorMap mapB3, Meta* __restrict__ meta, int E, int K, int N,
-                   size_t slots, void* __restrict__ out, int* status, long long wait_ns) {
+                   const __grid_constant__ CUtensorMap mapB3, const GemmParams p) {
+    using MT = ModeT<MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES);
@@ -113,7 +162,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool leader = rank == 0;
     const int cluster = blockIdx.x >> 1;
     const int nclusters = gridDim.x >> 1;
-    constexpr int N_PER_TILE = SWIGLU ? BNH : BN;   // output columns per tile
+    constexpr int N_PER_TILE = MT::N_PER_TILE;   // output columns per tile
+    Meta* meta = p.meta;
+    const int E = p.E, N = p.N;
 
     pdl_trigger();
     if (threadIdx.x == 0) {
@@ -132,7 +183,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == 0 && lane == 0) {
         ptx::tma_prefetch_desc(&mapA);
         ptx::tma_prefetch_desc(&mapB1);
-        if (SWIGLU) ptx::tma_prefetch_desc(&mapB3);
+        if (MT::GATED || MODE == kDgradX) ptx::tma_prefetch_desc(&mapB3);
     }
     if (warp == 1) {
         ptx::tmem_alloc_pair(&ctrl->tmem_base, TMEM_COLS);
@@ -146,15 +197,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bool ok = true;
         for (int e = 0; e < E; ++e) {
             const int r0 = meta->offsets[e], r1 = meta->offsets[e + 1];
-            if (r1 < r0 || (r1 - r0) % BM != 0 || (size_t)r1 > slots) ok = false;
-            const int mt = ok ? (r1 - r0) / BM : 0;
-            ctrl->mt[e] = mt;
-            ctrl->pt[e] = (mt + 1) / 2;
+            if (r1 < r0 || (r1 - r0) % BM != 0 || (size_t)r1 > p.slots) ok = false;
+            const int rows = ok ? r1 - r0 : 0;
+            if (MT::KGROUP) {
+                // every expert has the same output tiles; K = its rows (zero rows: zero gradient)
+                const int mt = (p.M + BM - 1) / BM;
+                ctrl->mt[e] = mt;
+                ctrl->pt[e] = (mt + 1) / 2;
+                ctrl->nkb[e] = rows / BK;
+            } else {
+                const int mt = rows / BM;
+                ctrl->mt[e] = mt;
+                ctrl->pt[e] = (mt + 1) / 2;
+                ctrl->nkb[e] = (p.K + BK - 1) / BK;
+            }
             ctrl->row0[e] = r0;
             ctrl->tile_base[e + 1] = ctrl->tile_base[e] + ctrl->pt[e] * ntn;
         }
         ctrl->total = ok ? ctrl->tile_base[E] : 0;
-        if (!ok) record_status(status, MOE_ERR_DEVICE);
+        if (!ok) record_status(p.status, MOE_ERR_DEVICE);
     }
     ptx::tc_fence_before_sync();
     ptx::cluster_sync();
@@ -162,8 +223,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     const uint32_t tmem_base = ctrl->tmem_base;
     const int total = ctrl->total;
-    const int nk = (K + BK - 1) / BK;
-    const ptx::WaitCtl wc{&ctrl->abort, status, (uint64_t)wait_ns};
+    const ptx::WaitCtl wc{&ctrl->abort, p.status, (uint64_t)p.wait_ns};
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer (both CTAs)
@@ -183,11 +243,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int tile = cluster; tile < total && !aborted; tile += nclusters, ++wave) {
                 int e, pair, n_blk;
                 decode_tile(ctrl, tile, e, pair, n_blk);
-                const int rowA = ctrl->row0[e] + (2 * pair + (int)rank) * BM;
-                if (leader) wave_sync(&meta->waves[SWIGLU ? 0 : 1], min(total, (wave + 1) * nclusters));
-                const CUtensorMap* mapB = (SWIGLU && !leader) ? &mapB3 : &mapB1;
-                const int rowB = SWIGLU ? n_blk * BNH : n_blk * BN + (int)rank * BNH;
-                for (int kb = 0; kb < nk; ++kb) {
+                const int m_tile = 2 * pair + (int)rank;
+                const int rowA = ctrl->row0[e] + m_tile * BM;            // row-grouped: A rows
+                const int n0 = n_blk * BN + (int)rank * BNH;             // this CTA's B rows (non-gated)
+                const int nkb = ctrl->nkb[e];
+                if (leader) wave_sync(&meta->waves[p.wave_slot], min(total, (wave + 1) * nclusters));
+                for (int kb = 0; kb < nkb; ++kb) {
                     if (!ptx::mbar_wait(&ctrl->empty[stage], phase ^ 1u, wc)) {
                         aborted = true;
                         break;
@@ -196,8 +257,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     uint8_t* sb = sa + A_BYTES;
                     const uint32_t full_leader = ptx::map_to_rank(ptx::smem_addr(&ctrl->full[stage]), 0);
                     if (leader) ptx::mbar_arrive_expect_tx(&ctrl->full[stage], PAIR_TX_BYTES);
-                    ptx::tma_load_2d_pair(sa, &mapA, full_leader, kb * BK, rowA, pol);
-                    ptx::tma_load_3d_pair(sb, mapB, full_leader, kb * BK, rowB, e, pol);
+                    if (MT::KGROUP) {
+                        // A^T and B^T tiles of the expert's rows: [64 k][64 m] boxes, m / n contiguous
+                        const int krow = ctrl->row0[e] + kb * BK;
+                        const int m0 = m_tile * BM;
+                        ptx::tma_load_2d_pair(sa, &mapA, full_leader, m0, krow, pol);
+                        ptx::tma_load_2d_pair(sa + MN_LBO, &mapA, full_leader, m0 + MN_BOX, krow, pol);
+                        ptx::tma_load_2d_pair(sb, &mapB1, full_leader, n0, krow, pol);
+                        ptx::tma_load_2d_pair(sb + MN_LBO, &mapB1, full_leader, n0 + MN_BOX, krow, pol);
+                    } else {
+                        ptx::tma_load_2d_pair(sa, &mapA, full_leader, kb * BK, rowA, pol);
+                        if (MT::B_MN) {
+                            // weights [E][K][N], N contiguous: [64 k][64 n] boxes
+                            const bool hi = MODE == kDgradX && kb >= p.kb_split;
+                            const CUtensorMap* mapB = hi ? &mapB3 : &mapB1;
+                            const int kk = (hi ? kb - p.kb_split : kb) * BK;
+                            ptx::tma_load_3d_pair(sb, mapB, full_leader, n0, kk, e, pol);
+                            ptx::tma_load_3d_pair(sb + MN_LBO, mapB, full_leader, n0 + MN_BOX, kk, e, pol);
+                        } else {
+                            const CUtensorMap* mapB = (MT::GATED && !leader) ? &mapB3 : &mapB1;
+                            const int rowB = MT::GATED ? n_blk * BNH : n0;
+                            ptx::tma_load_3d_pair(sb, mapB, full_leader, kb * BK, rowB, e, pol);
+                        }
+                    }
 #pragma unroll
                     for (int s = 0; s < STAGES; ++s)
                         if (s == stage) {
@@ -226,13 +308,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t acc_phase = 0;
             bool issued = false, aborted = false;
             for (int tile = cluster; tile < total && !aborted; tile += nclusters) {
+                int e, pair, n_blk;
+                decode_tile(ctrl, tile, e, pair, n_blk);
+                const int nkb = ctrl->nkb[e];
                 if (!ptx::mbar_wait(&ctrl->tempty[acc], acc_phase ^ 1u, wc)) {
                     aborted = true;
                     break;
                 }
                 ptx::tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int kb = 0; kb < nkb; ++kb) {
                     if (!ptx::mbar_wait(&ctrl->full[stage], phase, wc)) {
                         aborted = true;
                         break;
@@ -242,8 +327,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        ptx::tc_mma_bf16_pair(d_tmem, ptx::desc_kmajor_sw128(a0 + kk * 32),
-                                              ptx::desc_kmajor_sw128(b0 + kk * 32), IDESC, (kb | kk) != 0);
+                        // one K = 16 slice: 32 bytes into each K-major row, or 16 rows of an MN-major tile
+                        const uint64_t da = MT::A_MN ? ptx::desc_mnmajor_sw128(a0 + kk * 2048, MN_LBO, MN_SBO)
+                                                     : ptx::desc_kmajor_sw128(a0 + kk * 32);
+                        const uint64_t db = MT::B_MN ? ptx::desc_mnmajor_sw128(b0 + kk * 2048, MN_LBO, MN_SBO)
+                                                     : ptx::desc_kmajor_sw128(b0 + kk * 32);
+                        ptx::tc_mma_bf16_pair(d_tmem, da, db, MT::IDESC, (kb | kk) != 0);
                     }
                     ptx::tc_commit_pair_multicast(&ctrl->empty[stage], 0x3);
                     issued = true;
@@ -276,11 +365,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             ptx::tc_fence_after_sync();
-            if (m_tile < ctrl->mt[e]) {
-                const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
+            const bool live = MT::KGROUP ? m_tile * BM < p.M : m_tile < ctrl->mt[e];
+            if (live) {
                 const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-                if (SWIGLU) {
-                    __nv_bfloat16* H = static_cast<__nv_bfloat16*>(out);
+                if (MODE == kFwd1) {
+                    const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
+                    __nv_bfloat16* H = static_cast<__nv_bfloat16*>(p.out);
 #pragma unroll 1
                     for (int c = 0; c < BNH; c += 32) {
                         uint32_t ra[32], rb[32];
@@ -300,16 +390,79 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             ptx::st_global_v4_hint(dst + 16 * v, hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3],
                                                    pol_out);
                     }
+                } else if (MODE == kSwigluBwd) {
+                    // h = SiLU(a) b:  dA = dH b SiLU'(a),  dB = dH SiLU(a)
+                    const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
+                    __nv_bfloat16* dAB = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll 1
+                    for (int c = 0; c < BNH; c += 32) {
+                        uint32_t ra[32], rb[32];
+                        ptx::tmem_ld_32x32b_x32(taddr + c, ra);
+                        ptx::tmem_ld_32x32b_x32(taddr + BNH + c, rb);
+                        const float4* dhp = reinterpret_cast<const float4*>(p.aux + row * (size_t)N + n_blk * BNH + c);
+                        float dh[32];
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const float4 t = __ldg(dhp + v);
+                            dh[4 * v] = t.x;
+                            dh[4 * v + 1] = t.y;
+                            dh[4 * v + 2] = t.z;
+                            dh[4 * v + 3] = t.w;
+                        }
+                        ptx::tmem_ld_wait();
+                        uint32_t pa[16], pb[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float da[2], dbv[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const float av = __uint_as_float(ra[2 * i + u]);
+                                const float bv = __uint_as_float(rb[2 * i + u]);
+                                silu_bwd(av, bv, dh[2 * i + u], da[u], dbv[u]);
+                            }
+                            pa[i] = pack_bf16x2(da[0], da[1]);
+                            pb[i] = pack_bf16x2(dbv[0], dbv[1]);
+                        }
+                        uint8_t* dst_a = reinterpret_cast<uint8_t*>(dAB + row * (size_t)(2 * N) + n_blk * BNH + c);
+                        uint8_t* dst_b = dst_a + (size_t)N * 2;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            ptx::st_global_v4_hint(dst_a + 16 * v, pa[4 * v], pa[4 * v + 1], pa[4 * v + 2],
+                                                   pa[4 * v + 3], pol_out);
+                            ptx::st_global_v4_hint(dst_b + 16 * v, pb[4 * v], pb[4 * v + 1], pb[4 * v + 2],
+                                                   pb[4 * v + 3], pol_out);
+                        }
+                    }
                 } else {
-                    float* Y = static_cast<float*>(out);
+                    // fp32 tile: row-grouped modes write row r of [slots][N]; grouped-by-K writes
+                    // row m of expert e's [M][N] gradient (rows >= split to out_hi)
+                    float* dst_row = nullptr;
+                    bool zero = false;
+                    if (MT::KGROUP) {
+                        const int m = m_tile * BM + q * 32 + lane;
+                        if (m < p.M) {
+                            dst_row = m < p.split
+                                          ? static_cast<float*>(p.out) + ((size_t)e * p.split + m) * (size_t)N
+                                          : static_cast<float*>(p.out_hi) +
+                                                ((size_t)e * (p.M - p.split) + (m - p.split)) * (size_t)N;
+                        }
+                        zero = ctrl->nkb[e] == 0;   // no rows: the accumulator was never written
+                    } else {
+                        const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
+                        dst_row = static_cast<float*>(p.out) + row * (size_t)N;
+                    }
 #pragma unroll 1
                     for (int c = 0; c < BN; c += 32) {
                         uint32_t r[32];
                         ptx::tmem_ld_32x32b_x32(taddr + c, r);
                         ptx::tmem_ld_wait();
                         const int col = n_blk * BN + c;
-                        if (col < N) {
-                            uint8_t* dst = reinterpret_cast<uint8_t*>(Y + row * (size_t)N + col);
+                        if (dst_row && col < N) {
+                            if (zero) {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) r[i] = 0u;
+                            }
+                            uint8_t* dst = reinterpret_cast<uint8_t*>(dst_row + col);
 #pragma unroll
                             for (int v = 0; v < 8; ++v)
                                 ptx::st_global_v4_hint(dst + 16 * v, r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3],
@@ -347,17 +500,27 @@ bool map_weights(CUtensorMap* m, const void* base, int E, int R, int K, int box_
     return map_expert_weights(m, base, E, R, K, BK, box_rows);
 }
 
-template <bool SWIGLU>
+// [rows][inner] bf16 matrix read as MN-major 64 x 64 boxes (inner contiguous)
+bool map_mn_rows(CUtensorMap* m, const void* base, size_t rows, int inner) {
+    return map_matrix(m, base, rows, inner, MN_BOX, BK);
+}
+
+// [E][K][N] bf16 weights read as MN-major 64 (n) x 64 (k) x 1 boxes
+bool map_mn_weights(CUtensorMap* m, const void* base, int E, int K, int N) {
+    return map_expert_weights(m, base, E, K, N, MN_BOX, BK);
+}
+
+template <int MODE>
 cudaError_t ensure_smem_attr() {
     static PerDeviceOnce once;
     return once.run([] {
-        return cudaFuncSetAttribute(tc_gemm_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        return cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     });
 }
 
 // Persistent grid: as many CTA pairs as fit at once, no more than there are pair tiles.
-template <bool SWIGLU>
-int grid_for(size_t slots, int n_tiles_per_m, int num_sms) {
+template <int MODE>
+int grid_for(size_t pair_tiles, int num_sms) {
     static PerDeviceInt clusters_per_device;
     const int max_clusters = clusters_per_device.get([num_sms] {
         cudaLaunchConfig_t cfg = {};
@@ -372,25 +535,30 @@ int grid_for(size_t slots, int n_tiles_per_m, int num_sms) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_kernel<SWIGLU>, &cfg) != cudaSuccess || n <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_kernel<MODE>, &cfg) != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = (num_sms > 0 ? num_sms : 148) / 2;
         }
         return n;
     });
-    const size_t pair_rows = (slots / BM + 1) / 2;
-    const size_t upper = pair_rows * (size_t)n_tiles_per_m;
     size_t clusters = (size_t)max_clusters;
-    if (clusters > upper) clusters = upper;
+    if (clusters > pair_tiles) clusters = pair_tiles;
     if (clusters < 1) clusters = 1;
     return (int)(2 * clusters);
 }
 
-template <bool SWIGLU>
-cudaError_t launch_pair(int grid, const CUtensorMap& mA, const CUtensorMap& mB1, const CUtensorMap& mB3,
-                        const TcGemmArgs& a, int K, int N, void* out, cudaStream_t s) {
+// Upper bound of the row-grouped pair tiles: every expert may add one half-empty pair.
+size_t row_pair_tiles(size_t slots, int E, int n_tiles) {
+    return ((slots / BM + (size_t)E) / 2 + 1) * (size_t)n_tiles;
+}
+
+template <int MODE>
+cudaError_t launch_pair(size_t pair_tiles, int num_sms, const CUtensorMap& mA, const CUtensorMap& mB1,
+                        const CUtensorMap& mB3, const GemmParams& gp, cudaStream_t s) {
+    cudaError_t e = ensure_smem_attr<MODE>();
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.gridDim = dim3(grid_for<MODE>(pair_tiles, num_sms), 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = s;
@@ -403,8 +571,23 @@ cudaError_t launch_pair(int grid, const CUtensorMap& mA, const CUtensorMap& mB1,
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<SWIGLU>, mA, mB1, mB3, const_cast<Meta*>(a.meta), a.E, K, N,
-                              a.slots, out, a.status, a.wait_ns);
+    e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<MODE>, mA, mB1, mB3, gp);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+GemmParams params(Meta* meta, int E, int N, int K, int wave_slot, size_t slots, void* out, int* status,
+                  long long wait_ns) {
+    GemmParams gp = {};
+    gp.meta = meta;
+    gp.E = E;
+    gp.N = N;
+    gp.K = K;
+    gp.wave_slot = wave_slot;
+    gp.slots = slots;
+    gp.out = out;
+    gp.status = status;
+    gp.wait_ns = wait_ns;
+    return gp;
 }
 
 }  // namespace
@@ -414,22 +597,75 @@ cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s) {
     if (!map_rows(&mA, a.xp, a.slots, a.d, BM) || !map_weights(&mB1, a.W1, a.E, a.F, a.d, BNH) ||
         !map_weights(&mB3, a.W3, a.E, a.F, a.d, BNH))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_attr<true>();
-    if (e != cudaSuccess) return e;
-    const int grid = grid_for<true>(a.slots, (a.F + BNH - 1) / BNH, a.num_sms);
-    e = launch_pair<true>(grid, mA, mB1, mB3, a, a.d, a.F, a.H, s);
-    return e != cudaSuccess ? e : cudaGetLastError();
+    const GemmParams gp = params(const_cast<Meta*>(a.meta), a.E, a.F, a.d, kWaveFwd1, a.slots, a.H, a.status,
+                                 a.wait_ns);
+    return launch_pair<kFwd1>(row_pair_tiles(a.slots, a.E, (a.F + BNH - 1) / BNH), a.num_sms, mA, mB1, mB3, gp, s);
 }
 
 cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s) {
     CUtensorMap mA, mB;
     if (!map_rows(&mA, a.H, a.slots, a.F, BM) || !map_weights(&mB, a.W2, a.E, a.d, a.F, BNH))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_attr<false>();
-    if (e != cudaSuccess) return e;
-    const int grid = grid_for<false>(a.slots, (a.d + BN - 1) / BN, a.num_sms);
-    e = launch_pair<false>(grid, mA, mB, mB, a, a.F, a.d, a.Y, s);
-    return e != cudaSuccess ? e : cudaGetLastError();
+    const GemmParams gp = params(const_cast<Meta*>(a.meta), a.E, a.d, a.F, kWaveFwd2, a.slots, a.Y, a.status,
+                                 a.wait_ns);
+    return launch_pair<kFwd2>(row_pair_tiles(a.slots, a.E, (a.d + BN - 1) / BN), a.num_sms, mA, mB, mB, gp, s);
+}
+
+cudaError_t launch_tc_dgrad_h(const TcBwdArgs& a, cudaStream_t s) {
+    // dH [slots][F] = dY [slots][d] . W2_e [d][F]: B[n = f][k = i] is W2 read MN-major
+    CUtensorMap mA, mB;
+    if (!map_rows(&mA, a.dy, a.slots, a.d, BM) || !map_mn_weights(&mB, a.W2, a.E, a.d, a.F))
+        return cudaErrorInvalidValue;
+    const GemmParams gp = params(a.meta, a.E, a.F, a.d, kWaveDgradH, a.slots, a.dh, a.status, a.wait_ns);
+    return launch_pair<kDgradH>(row_pair_tiles(a.slots, a.E, (a.F + BN - 1) / BN), a.num_sms, mA, mB, mB, gp, s);
+}
+
+cudaError_t launch_tc_swiglu_bwd(const TcBwdArgs& a, cudaStream_t s) {
+    CUtensorMap mA, mB1, mB3;
+    if (!map_rows(&mA, a.xp, a.slots, a.d, BM) || !map_weights(&mB1, a.W1, a.E, a.F, a.d, BNH) ||
+        !map_weights(&mB3, a.W3, a.E, a.F, a.d, BNH))
+        return cudaErrorInvalidValue;
+    GemmParams gp = params(a.meta, a.E, a.F, a.d, kWaveSwigluBwd, a.slots, a.dab, a.status, a.wait_ns);
+    gp.aux = a.dh;
+    return launch_pair<kSwigluBwd>(row_pair_tiles(a.slots, a.E, (a.F + BNH - 1) / BNH), a.num_sms, mA, mB1, mB3,
+                                   gp, s);
+}
+
+cudaError_t launch_tc_dgrad_x(const TcBwdArgs& a, cudaStream_t s) {
+    // dXp [slots][d] = [dA dB] [slots][2F] . [W1_e ; W3_e] [2F][d]: W1 / W3 read MN-major
+    CUtensorMap mA, mB1, mB3;
+    if (!map_rows(&mA, a.dab, a.slots, 2 * a.F, BM) || !map_mn_weights(&mB1, a.W1, a.E, a.F, a.d) ||
+        !map_mn_weights(&mB3, a.W3, a.E, a.F, a.d))
+        return cudaErrorInvalidValue;
+    GemmParams gp = params(a.meta, a.E, a.d, 2 * a.F, kWaveDgradX, a.slots, a.dxp, a.status, a.wait_ns);
+    gp.kb_split = a.F / BK;
+    return launch_pair<kDgradX>(row_pair_tiles(a.slots, a.E, (a.d + BN - 1) / BN), a.num_sms, mA, mB1, mB3, gp,
+                                s);
+}
+
+cudaError_t launch_tc_wgrad2(const TcBwdArgs& a, cudaStream_t s) {
+    // dW2_e [d][F] = dY_e^T . H_e over the expert's rows: both read MN-major
+    CUtensorMap mA, mB;
+    if (!map_mn_rows(&mA, a.dy, a.slots, a.d) || !map_mn_rows(&mB, a.H, a.slots, a.F)) return cudaErrorInvalidValue;
+    GemmParams gp = params(a.meta, a.E, a.F, 0, kWaveWgrad2, a.slots, a.dW2, a.status, a.wait_ns);
+    gp.M = a.d;
+    gp.split = a.d;
+    gp.out_hi = a.dW2;
+    const size_t tiles = (size_t)a.E * (((a.d + BM - 1) / BM + 1) / 2) * ((a.F + BN - 1) / BN);
+    return launch_pair<kWgrad>(tiles, a.num_sms, mA, mB, mB, gp, s);
+}
+
+cudaError_t launch_tc_wgrad13(const TcBwdArgs& a, cudaStream_t s) {
+    // [dW1_e ; dW3_e] [2F][d] = [dA dB]_e^T . Xp_e over the expert's rows: both read MN-major
+    CUtensorMap mA, mB;
+    if (!map_mn_rows(&mA, a.dab, a.slots, 2 * a.F) || !map_mn_rows(&mB, a.xp, a.slots, a.d))
+        return cudaErrorInvalidValue;
+    GemmParams gp = params(a.meta, a.E, a.d, 0, kWaveWgrad13, a.slots, a.dW1, a.status, a.wait_ns);
+    gp.M = 2 * a.F;
+    gp.split = a.F;
+    gp.out_hi = a.dW3;
+    const size_t tiles = (size_t)a.E * (((2 * a.F + BM - 1) / BM + 1) / 2) * ((a.d + BN - 1) / BN);
+    return launch_pair<kWgrad>(tiles, a.num_sms, mA, mB, mB, gp, s);
 }
 
 }  // namespace moe

@@ -317,6 +317,130 @@ moe_status route_stats(const void* x, const void* Wg, int T, int d, int E, int k
     return (e == cudaSuccess && f == cudaSuccess) ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Backward workspace layout (on top of the forward's workspace, which it reads).
+struct BwdPlan {
+    size_t dy, dg, ds, dh, dab, dxp, dwg, total;
+};
+
+BwdPlan make_bwd_plan(int T, int d, int F, int E, int k, int dtype) {
+    BwdPlan b{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + (bytes ? bytes : 1), 256);
+        return o;
+    };
+    const size_t es = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+    const size_t S = slots_capacity(T, E, k);
+    b.dy = take(S * d * es);
+    b.dg = take((size_t)T * k * 4);
+    b.ds = take((size_t)T * E * 4);
+    b.dh = take(S * F * 4);
+    b.dab = take(S * 2 * (size_t)F * es);
+    b.dxp = take(S * d * 4);
+    b.dwg = take(dwg_part_bytes(T, E, d));
+    b.total = off;
+    return b;
+}
+
+moe_status run_backward(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2,
+                        const void* dout, void* dx, float* dWg, float* dW1, float* dW3, float* dW2, float* dlogits,
+                        int T, int d, int F, int E, int k, int dtype, const uint8_t* fws, uint8_t* bws,
+                        const DeviceState& dev, cudaStream_t s, cudaEvent_t* ev, int* launches) {
+    const Plan p = make_plan(T, d, F, E, k, dtype);
+    const BwdPlan b = make_bwd_plan(T, d, F, E, k, dtype);
+    uint8_t* fw = const_cast<uint8_t*>(fws);
+    BwdArgs a{};
+    a.bf16 = dtype == MOE_DTYPE_BF16;
+    a.x = x;
+    a.Wg = Wg;
+    a.W1 = W1;
+    a.W3 = W3;
+    a.W2 = W2;
+    a.dout = dout;
+    a.idx = reinterpret_cast<const int32_t*>(fw + p.idx);
+    a.w = reinterpret_cast<const float*>(fw + p.w);
+    a.meta = reinterpret_cast<Meta*>(fw + p.meta);
+    a.perm = reinterpret_cast<const int32_t*>(fw + p.perm);
+    a.inv = reinterpret_cast<const int32_t*>(fw + p.inv);
+    a.xp = fw + p.xp;
+    a.H = fw + p.h;
+    a.Y = reinterpret_cast<const float*>(fw + p.y);
+    a.dy = bws + b.dy;
+    a.dg = reinterpret_cast<float*>(bws + b.dg);
+    a.ds = dlogits ? dlogits : reinterpret_cast<float*>(bws + b.ds);
+    a.dh = reinterpret_cast<float*>(bws + b.dh);
+    a.dab = bws + b.dab;
+    a.dxp = reinterpret_cast<float*>(bws + b.dxp);
+    a.dwg_part = reinterpret_cast<float*>(bws + b.dwg);
+    a.dx = dx;
+    a.dWg = dWg;
+    a.dW1 = dW1;
+    a.dW3 = dW3;
+    a.dW2 = dW2;
+    a.T = T;
+    a.d = d;
+    a.F = F;
+    a.E = E;
+    a.k = k;
+    a.slots = p.slots;
+
+    auto mark = [&](int stage) -> cudaError_t { return ev ? cudaEventRecord(ev[stage], s) : cudaSuccess; };
+    int n = 0;
+    MOE_TRY(mark(MOE_BWD_STAGE_SCATTER));
+    MOE_TRY(launch_bwd_scatter(a, s));
+    MOE_TRY(launch_router_bwd(a, s));
+    n += 2;
+    if (a.bf16) {
+        TcBwdArgs t{};
+        t.xp = a.xp;
+        t.W1 = W1;
+        t.W3 = W3;
+        t.W2 = W2;
+        t.H = a.H;
+        t.dy = a.dy;
+        t.dh = a.dh;
+        t.dab = a.dab;
+        t.dxp = a.dxp;
+        t.dW1 = dW1;
+        t.dW3 = dW3;
+        t.dW2 = dW2;
+        t.meta = a.meta;
+        t.E = E;
+        t.d = d;
+        t.F = F;
+        t.slots = p.slots;
+        t.num_sms = dev.num_sms;
+        t.status = dev.status;
+        t.wait_ns = wait_limit_ns();
+        MOE_TRY(mark(MOE_BWD_STAGE_DGRAD_H));
+        MOE_TRY(launch_tc_dgrad_h(t, s));
+        MOE_TRY(mark(MOE_BWD_STAGE_SWIGLU));
+        MOE_TRY(launch_tc_swiglu_bwd(t, s));
+        MOE_TRY(mark(MOE_BWD_STAGE_DGRAD_X));
+        MOE_TRY(launch_tc_dgrad_x(t, s));
+        MOE_TRY(mark(MOE_BWD_STAGE_WGRAD2));
+        MOE_TRY(launch_tc_wgrad2(t, s));
+        MOE_TRY(mark(MOE_BWD_STAGE_WGRAD13));
+        MOE_TRY(launch_tc_wgrad13(t, s));
+    } else {
+        MOE_TRY(mark(MOE_BWD_STAGE_DGRAD_H));
+        MOE_TRY(mark(MOE_BWD_STAGE_SWIGLU));
+        MOE_TRY(mark(MOE_BWD_STAGE_DGRAD_X));
+        MOE_TRY(mark(MOE_BWD_STAGE_WGRAD2));
+        MOE_TRY(launch_simt_bwd_gemms(a, s));
+        MOE_TRY(mark(MOE_BWD_STAGE_WGRAD13));
+    }
+    n += 5;
+    MOE_TRY(mark(MOE_BWD_STAGE_ROUTER));
+    MOE_TRY(launch_dwg(a, s));
+    MOE_TRY(launch_dx_combine(a, s));
+    n += 3;
+    MOE_TRY(mark(MOE_BWD_NUM_STAGES));
+    if (launches) *launches = n;
+    return MOE_OK;
+}
+
 __global__ void wait_selftest_kernel(int* status, long long limit_ns) {
     __shared__ uint64_t bar;
     __shared__ int abort_flag;
@@ -561,6 +685,36 @@ moe_status moe_block_forward_ws(const void* h, const void* gamma, float eps, con
     const BlockArgs bo{gamma, eps, alpha, stats};
     return run_layer(h, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
                      stream, stage_events, launches, &bo);
+}
+
+size_t moe_backward_workspace_size(int T, int d, int ffn, int E, int k, int dtype) {
+    if (check_sizes(T, d, E, k) != MOE_OK || ffn <= 0) return 0;
+    if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_F32) return 0;
+    return make_bwd_plan(T, d, ffn, E, k, dtype).total;
+}
+
+moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2,
+                           const void* dout, void* dx, float* dWg, float* dW1, float* dW3, float* dW2, float* dlogits,
+                           int T, int d, int ffn, int E, int k, int dtype, const void* fwd_workspace,
+                           size_t fwd_workspace_bytes, void* workspace, size_t workspace_bytes,
+                           cudaEvent_t* stage_events, int* launches, cudaStream_t stream) {
+    if (launches) *launches = 0;
+    moe_status st = check_layer(x, Wg, W1, W3, W2, dx, T, d, ffn, E, k, dtype);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    const void* ptrs[5] = {dout, dWg, dW1, dW3, dW2};
+    for (const void* q : ptrs)
+        if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (dlogits && (reinterpret_cast<uintptr_t>(dlogits) & 3u) != 0) return MOE_ERR_INVALID_ARG;
+    if (!fwd_workspace || (reinterpret_cast<uintptr_t>(fwd_workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (fwd_workspace_bytes < make_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (workspace_bytes < make_bwd_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
+    DeviceState dev;
+    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    return run_backward(x, Wg, W1, W3, W2, dout, dx, dWg, dW1, dW3, dW2, dlogits, T, d, ffn, E, k, dtype,
+                        static_cast<const uint8_t*>(fwd_workspace), static_cast<uint8_t*>(workspace), dev, stream,
+                        stage_events, launches);
 }
 
 moe_status moe_route_stats(const void* x, const void* Wg, int T, int d, int E, int k, float alpha,

@@ -15,6 +15,11 @@ namespace moe {
 // a 128-row tensor-core tile never straddles two experts.
 constexpr int kSegRows = 128;
 constexpr int kMaxExperts = 32;
+// wave counters in Meta: forward GEMM1, GEMM2, then the backward GEMMs (dH,
+// SwiGLU backward, dX, dW2, dW1/dW3)
+constexpr int kWaveSlots = 8;
+enum WaveSlot : int { kWaveFwd1 = 0, kWaveFwd2 = 1, kWaveDgradH = 2, kWaveSwigluBwd = 3, kWaveDgradX = 4,
+                      kWaveWgrad2 = 5, kWaveWgrad13 = 6 };
 // Tokens handled by one dispatch block (histogram / scatter).
 constexpr int kDispatchTokens = 1024;
 
@@ -22,7 +27,7 @@ constexpr int kDispatchTokens = 1024;
 struct Meta {
     int32_t counts[kMaxExperts];        // assignments per expert
     int32_t offsets[kMaxExperts + 1];   // padded segment start rows; offsets[E] = padded total
-    int32_t waves[2];                   // wave counters of the two expert GEMMs (zeroed by dispatch)
+    int32_t waves[kWaveSlots];          // wave counters of the expert GEMMs (zeroed by dispatch / backward)
 };
 
 // Per-device sticky status word (first fault wins).
@@ -48,6 +53,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // +inf and the fast division gives the correct limit 0.
 __device__ __forceinline__ float silu_mul(float a, float b) {
     return __fdividef(a, 1.0f + __expf(-a)) * b;
+}
+
+// Backward of h = SiLU(a) b for the upstream gradient dh:
+//     da = dh b SiLU'(a),  db = dh SiLU(a),  SiLU'(a) = s (1 + a (1 - s)),  s = 1 / (1 + e^-a).
+// For a < -88, e^-a is +inf, s is 0 and both gradients are 0.
+__device__ __forceinline__ void silu_bwd(float a, float b, float dh, float& da, float& db) {
+    const float s = __fdividef(1.0f, 1.0f + __expf(-a));
+    db = dh * a * s;
+    da = dh * b * s * (1.0f + a * (1.0f - s));
 }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -198,6 +212,76 @@ struct TcGemmArgs {
 };
 cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s);
 cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s);
+
+// Backward GEMMs on the same CTA-pair kernel (bf16 operands, fp32 accumulate).
+struct TcBwdArgs {
+    const void* xp;     // forward: [slots][d] bf16 gathered rows (padding rows zero)
+    const void* W1;     // [E][F][d]
+    const void* W3;
+    const void* W2;     // [E][d][F]
+    const void* H;      // forward: [slots][F] bf16
+    const void* dy;     // [slots][d] bf16: g * dout scattered to the slots (padding rows zero)
+    float* dh;          // [slots][F] fp32
+    void* dab;          // [slots][2F] bf16: dA | dB
+    float* dxp;         // [slots][d] fp32
+    float* dW1;         // [E][F][d] fp32
+    float* dW3;
+    float* dW2;         // [E][d][F] fp32
+    Meta* meta;
+    int E, d, F;
+    size_t slots;
+    int num_sms;
+    int* status;
+    long long wait_ns;
+};
+// Operands and buffers of one backward call (backward.cu); pointers are device
+// memory, the *_f32 path uses float where bf16 is noted.
+struct BwdArgs {
+    bool bf16;
+    const void* x;          // [T][d]
+    const void* Wg;         // [E][d]
+    const void* W1;
+    const void* W3;
+    const void* W2;
+    const void* dout;       // [T][d]
+    // forward state
+    const int32_t* idx;     // [T][k]
+    const float* w;         // [T][k] gates
+    Meta* meta;
+    const int32_t* perm;    // [slots]
+    const int32_t* inv;     // [T][k]
+    const void* xp;         // [slots][d]
+    const void* H;          // [slots][F]
+    const float* Y;         // [slots][d]
+    // backward buffers
+    void* dy;               // [slots][d]
+    float* dg;              // [T][k]
+    float* ds;              // [T][E]
+    float* dh;              // [slots][F]
+    void* dab;              // [slots][2F]
+    float* dxp;             // [slots][d]
+    float* dwg_part;        // dwg_part_bytes(T, E, d)
+    // outputs
+    void* dx;               // [T][d]
+    float* dWg;             // [E][d]
+    float* dW1;             // [E][F][d]
+    float* dW3;
+    float* dW2;             // [E][d][F]
+    int T, d, F, E, k;
+    size_t slots;
+};
+size_t dwg_part_bytes(int T, int E, int d);
+cudaError_t launch_bwd_scatter(const BwdArgs& a, cudaStream_t s);      // dY and dg (1 launch)
+cudaError_t launch_router_bwd(const BwdArgs& a, cudaStream_t s);       // ds (1 launch)
+cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s);              // dWg (2 launches)
+cudaError_t launch_dx_combine(const BwdArgs& a, cudaStream_t s);       // dx (1 launch)
+cudaError_t launch_simt_bwd_gemms(const BwdArgs& a, cudaStream_t s);   // fp32 expert GEMMs (5 launches)
+
+cudaError_t launch_tc_dgrad_h(const TcBwdArgs& a, cudaStream_t s);      // dH = dY W2_e
+cudaError_t launch_tc_swiglu_bwd(const TcBwdArgs& a, cudaStream_t s);   // dA, dB from Xp, W1, W3 and dH
+cudaError_t launch_tc_dgrad_x(const TcBwdArgs& a, cudaStream_t s);      // dXp = dA W1_e + dB W3_e
+cudaError_t launch_tc_wgrad2(const TcBwdArgs& a, cudaStream_t s);       // dW2_e = dY_e^T H_e
+cudaError_t launch_tc_wgrad13(const TcBwdArgs& a, cudaStream_t s);      // [dW1_e; dW3_e] = [dA dB]_e^T Xp_e
 // Decode path: stage 1 (W1/W3 -> H) or stage 2 (W2 -> Y); at most 64 tokens per expert.
 constexpr int kDecodeMaxTokens = 64;
 cudaError_t launch_decode(const TcGemmArgs& a, int stage, cudaStream_t s);

@@ -1,0 +1,158 @@
+"""Backward pass against the fp64 oracle, through the C ABI on a B200.
+
+The forward runs with the grouped-GEMM (prefill) path into a caller
+workspace; the backward reads that workspace.  Tokens within the routing
+margin are excluded from the token-wise checks.
+
+Tolerances, derived from the arithmetic.  On the bf16 path dy = g dout, dA
+and dB are rounded to bf16 before their GEMMs, so each product term carries
+up to three bf16 roundings (2^-9 each) in series where the forward output
+carries one (H); independent rounding errors add in quadrature, so the
+forward's 2e-2 becomes 2e-2 sqrt(3) = 3.5e-2.  An entry's error also scales
+with the entry itself (weight-gradient entries are heavy-tailed: a few
+tokens with large |dout| and |h| dominate them).  Two checks per gradient G
+against the oracle's G*:
+  * every entry:  |G - G*| <= tol (RMS(G*) + |G*|),  tol = 3.5e-2 (bf16) or
+    1e-5 (fp32);
+  * the bulk:     RMS(G - G*) <= bulk RMS(G*),  bulk = 1e-2 (bf16, about 4x the
+    3 x 2^-9 / sqrt(3) expected) or 2e-6 (fp32).
+fp32 bounds are scaled by sqrt(K / 256) for reductions longer than 256
+(K = the longest of d, ffn and T).
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+from moe_testlib import MARGIN, out_to_f64, sample_tokens, to_dev, upload
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": 2e-2 * np.sqrt(3.0), "f32": 1e-5}
+BULK = {"bf16": 1e-2, "f32": 2e-6}
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import sparse_mixture_experts_14_b200 as m
+    return m
+
+
+def _status_clear(moe):
+    assert moe.moe_get_device_status() == moe.MOE_OK
+
+
+def _run(moe, inp, dev, dout_d, dlogits=False):
+    x, Wg, W1, W3, W2 = dev
+    code = moe.MOE_DTYPE_BF16 if inp.dtype == "bf16" else moe.MOE_DTYPE_F32
+    fws = torch.empty(moe.moe_workspace_size(inp.T, inp.d, inp.F, inp.E, inp.k, code), dtype=torch.uint8,
+                      device="cuda")
+    out = moe.moe_forward_ws(x, Wg, W1, W3, W2, inp.k, path=moe.MOE_PATH_PREFILL, workspace=fws)
+    dl = torch.empty((inp.T, inp.E), dtype=torch.float32, device="cuda") if dlogits else None
+    grads, n = moe.moe_backward_ws(x, Wg, W1, W3, W2, dout_d, inp.k, fws, dlogits=dl)
+    _status_clear(moe)
+    if dl is not None:
+        grads["dlogits"] = dl
+    return out, grads, n
+
+
+def _f64(t):
+    return t.double().cpu().numpy() if t.dtype == torch.float32 else out_to_f64(t)
+
+
+def _check(name, got, want, dtype, K=256):
+    scale = max(1.0, np.sqrt(K / 256.0)) if dtype == "f32" else 1.0
+    tol, bulk = TOL[dtype] * scale, BULK[dtype] * scale
+    rms = np.sqrt((want ** 2).mean())
+    err = np.abs(got - want)
+    excess = (err - tol * np.abs(want)).max()
+    l2 = np.sqrt((err ** 2).mean()) / rms
+    print(f"  {name}: max|err|/RMS {err.max() / rms:.3e}  excess/RMS {excess / rms:.3e}  rms err/RMS {l2:.3e}")
+    assert excess <= tol * rms, f"{name}: max excess {excess:.3e} > {tol:.2e} x RMS {rms:.3e}"
+    assert l2 <= bulk, f"{name}: RMS error {l2:.3e} x RMS > {bulk:.2e}"
+    return l2
+
+
+@pytest.mark.parametrize("dtype,T,d,F,E,k", [("bf16", 200, 256, 512, 8, 2), ("bf16", 700, 192, 384, 4, 2),
+                                             ("bf16", 90, 128, 256, 16, 4), ("bf16", 40, 256, 128, 8, 8),
+                                             ("f32", 64, 128, 256, 8, 2), ("f32", 150, 96, 160, 5, 3)])
+def test_backward_small(moe, dtype, T, d, F, E, k):
+    inp = moe_inputs.make_inputs(T, d, F, E, k, dtype, seed=T + d + E + k)
+    dout = moe_inputs.make_dout(T, d, dtype, seed=T)
+    dev = upload(inp)
+    _, g, n = _run(moe, inp, dev, to_dev(dout, dtype), dlogits=True)
+    assert n >= 10
+    ref = oracle.backward(*inp.arrays(), dout, k, dtype)
+    keep = ref["margin"] >= MARGIN
+    if not keep.all():
+        pytest.skip("a token sits within the routing margin; the weight gradients would include its choice")
+    K = max(d, F, T)
+    rel = {}
+    rel["dx"] = _check("dx", _f64(g["dx"]), ref["dx"], dtype, K)
+    rel["dlogits"] = _check("dlogits", _f64(g["dlogits"]), ref["dlogits"], dtype, K)
+    for n_ in ("dWg", "dW1", "dW3", "dW2"):
+        rel[n_] = _check(n_, _f64(g[n_]), ref[n_], dtype, K)
+    print(dtype, T, d, F, E, k, {a: f"{b:.2e}" for a, b in rel.items()})
+
+
+def test_backward_run_to_run_bitwise(moe):
+    inp = moe_inputs.make_inputs(300, 256, 256, 8, 2, "bf16", seed=41)
+    dev = upload(inp)
+    dout = to_dev(moe_inputs.make_dout(300, 256, "bf16", seed=41), "bf16")
+    _, a, _ = _run(moe, inp, dev, dout, dlogits=True)
+    _, b, _ = _run(moe, inp, dev, dout, dlogits=True)
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
+
+
+def test_backward_experts_without_tokens(moe):
+    """Experts no token chose get exactly zero weight gradients."""
+    inp = moe_inputs.make_inputs(100, 128, 256, 8, 2, "bf16", seed=42)
+    inp.Wg[:] = 0
+    inp.Wg[0, :] = moe_inputs.f32_to_bf16_bits(np.full(128, 0.5, dtype=np.float32))
+    inp.Wg[1, :] = moe_inputs.f32_to_bf16_bits(np.full(128, 0.25, dtype=np.float32))
+    inp.x[:] = moe_inputs.f32_to_bf16_bits(np.abs(moe_inputs.bf16_bits_to_f32(inp.x)) + 0.01)
+    dev = upload(inp)
+    dout = moe_inputs.make_dout(100, 128, "bf16", seed=42)
+    _, g, _ = _run(moe, inp, dev, to_dev(dout, "bf16"))
+    for n in ("dW1", "dW3", "dW2"):
+        assert torch.all(g[n][2:] == 0), n
+        assert torch.any(g[n][:2] != 0), n
+    ref = oracle.backward(*inp.arrays(), dout, 2, "bf16")
+    for n in ("dW1", "dW3", "dW2"):   # the two experts with tokens (the zero blocks would halve the RMS)
+        _check(n, _f64(g[n][:2]), ref[n][:2], "bf16")
+    _check("dx", _f64(g["dx"]), ref["dx"], "bf16")
+
+
+@pytest.mark.parametrize("cfg,n_tok", [(1, 0), (3, 12)])
+def test_backward_configs(moe, cfg, n_tok):
+    """Full-size workloads: dx and dlogits on sampled tokens, slices of every expert's weight
+    gradients, and dWg against the GPU's own dlogits reduced on the host."""
+    inp = moe_inputs.make_config(cfg)
+    dtype = inp.dtype
+    dout = moe_inputs.make_dout(inp.T, inp.d, dtype, seed=inp.seed)
+    dev = upload(inp)
+    _, g, _ = _run(moe, inp, dev, to_dev(dout, dtype), dlogits=True)
+    K = max(inp.d, inp.F, inp.T)
+    if n_tok == 0:
+        ref = oracle.backward(*inp.arrays(), dout, inp.k, dtype)
+        for n in ("dx", "dlogits", "dWg", "dW1", "dW3", "dW2"):
+            _check(n, _f64(g[n]), ref[n], dtype, K)
+        return
+    toks = sample_tokens(inp.T, n_tok, seed=cfg)
+    ref = oracle.backward_tokens(*inp.arrays(), dout, inp.k, dtype, toks)
+    keep = ref["margin"] >= MARGIN
+    _check("dx", _f64(g["dx"])[toks][keep], ref["dx"][keep], dtype)
+    _check("dlogits", _f64(g["dlogits"])[toks][keep], ref["dlogits"][keep], dtype)
+    fs = [0, 777, inp.F - 1]
+    for e in (0, inp.E - 1):
+        r1, r3, c2 = oracle.weight_grad_slices(*inp.arrays(), dout, inp.k, dtype, e, fs)
+        _check(f"dW1[{e}]", _f64(g["dW1"][e][fs]), r1, dtype)
+        _check(f"dW3[{e}]", _f64(g["dW3"][e][fs]), r3, dtype)
+        _check(f"dW2[{e}]", _f64(g["dW2"][e][:, fs]), c2, dtype)
+    # dWg = dlogits^T x: the GPU's reduction of its own router-score gradient
+    want = g["dlogits"].double().T @ dev[0].double()
+    _check("dWg", _f64(g["dWg"]), want.cpu().numpy(), "f32", inp.T)
+    del dev, g
+    torch.cuda.empty_cache()
