@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const int32_t* __restri
     }
 }
 
-constexpr int kWgChunk = 256;   // tokens per dWg partial sum
+constexpr int kWgChunk = 64;    // tokens per dWg partial sum
 
 // part[c][e][j] = sum over tokens t of chunk c (ascending) of ds[t][e] x[t][j]
 template <typename T, int EB>
@@ -137,7 +137,17 @@ __global__ void __launch_bounds__(256) dwg_part_kernel(const T* __restrict__ x, 
     float acc[EB];
 #pragma unroll
     for (int e = 0; e < EB; ++e) acc[e] = 0.f;
-    for (int t = 0; t < nt; ++t) {
+    int t = 0;
+    for (; t + 8 <= nt; t += 8) {
+        float xv[8];   // eight rows in flight before the arithmetic
+#pragma unroll
+        for (int u = 0; u < 8; ++u) xv[u] = Elt<T>::get(x, (size_t)(t0 + t + u) * d + j);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int e = 0; e < EB; ++e) acc[e] = fmaf(sds[t + u][e], xv[u], acc[e]);
+    }
+    for (; t < nt; ++t) {
         const float xv = Elt<T>::get(x, (size_t)(t0 + t) * d + j);
 #pragma unroll
         for (int e = 0; e < EB; ++e) acc[e] = fmaf(sds[t][e], xv, acc[e]);
@@ -159,27 +169,62 @@ __global__ void __launch_bounds__(256) dwg_final_kernel(const float* __restrict_
     }
 }
 
-// dx[t] = sum_j dXp[inv[t][j]] (j ascending) + sum_e ds[t][e] Wg[e] (e ascending), one rounding.
+// dx[t] = sum_j dXp[inv[t][j]] + sum_j ds[t][idx[t][j]] Wg[idx[t][j]], both j ascending, in fp32,
+// rounded once; four columns per thread (d % 4 == 0 on both paths).
 template <typename T>
 __global__ void __launch_bounds__(256) dx_combine_kernel(const float* __restrict__ dXp, const int32_t* __restrict__ inv,
-                                                         const float* __restrict__ ds, const T* __restrict__ Wg,
-                                                         int T_, int d, int E, int k, T* __restrict__ dx) {
+                                                         const int32_t* __restrict__ idx, const float* __restrict__ ds,
+                                                         const T* __restrict__ Wg, int T_, int d, int E, int k,
+                                                         T* __restrict__ dx) {
     pdl_trigger();
     pdl_wait();
-    const size_t n = (size_t)T_ * d;
+    const unsigned q = (unsigned)d / 4;
+    const size_t n = (size_t)T_ * q;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-        const int t = (int)(i / d);
-        const int c = (int)(i - (size_t)t * d);
-        float acc = 0.f;
+        const unsigned t = (unsigned)(i / q);
+        const unsigned c = (unsigned)(i - (size_t)t * q);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
             const int slot = inv[(size_t)t * k + j];
-            if (slot >= 0) acc += dXp[(size_t)slot * d + c];
+            if (slot < 0) continue;
+            const float4 v = __ldg(reinterpret_cast<const float4*>(dXp + (size_t)slot * d) + c);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
         }
-        for (int e = 0; e < E; ++e) {
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[(size_t)t * k + j];
+            if (e < 0 || e >= E) continue;
             const float s = ds[(size_t)t * E + e];
-            if (s != 0.f) acc = fmaf(s, Elt<T>::get(Wg, (size_t)e * d + c), acc);
+            float w[4];
+            if (sizeof(T) == 2) {
+                const uint2 u = __ldg(reinterpret_cast<const uint2*>(Wg + (size_t)e * d) + c);
+                w[0] = bf16_lo(u.x);
+                w[1] = bf16_hi(u.x);
+                w[2] = bf16_lo(u.y);
+                w[3] = bf16_hi(u.y);
+            } else {
+                const float4 u = __ldg(reinterpret_cast<const float4*>(Wg + (size_t)e * d) + c);
+                w[0] = u.x;
+                w[1] = u.y;
+                w[2] = u.z;
+                w[3] = u.w;
+            }
+            acc.x = fmaf(s, w[0], acc.x);
+            acc.y = fmaf(s, w[1], acc.y);
+            acc.z = fmaf(s, w[2], acc.z);
+            acc.w = fmaf(s, w[3], acc.w);
         }
-        Elt<T>::put(dx, i, acc);
+        T* out = dx + (size_t)t * d + 4 * c;
+        if (sizeof(T) == 2) {
+            uint2 o;
+            o.x = pack_bf16x2(acc.x, acc.y);
+            o.y = pack_bf16x2(acc.z, acc.w);
+            *reinterpret_cast<uint2*>(out) = o;
+        } else {
+            *reinterpret_cast<float4*>(out) = acc;
+        }
     }
 }
 
@@ -332,11 +377,11 @@ cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s) {
 
 template <typename T>
 cudaError_t launch_dx(const BwdArgs& a, cudaStream_t s) {
-    size_t blocks = ((size_t)a.T * a.d + 255) / 256;
+    size_t blocks = ((size_t)a.T * (a.d / 4) + 255) / 256;
     if (blocks > 148 * 32) blocks = 148 * 32;
     if (blocks < 1) blocks = 1;
     return launch_pdl(dx_combine_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const float*>(a.dxp),
-                      a.inv, static_cast<const float*>(a.ds), static_cast<const T*>(a.Wg), a.T, a.d, a.E, a.k,
+                      a.inv, a.idx, static_cast<const float*>(a.ds), static_cast<const T*>(a.Wg), a.T, a.d, a.E, a.k,
                       static_cast<T*>(a.dx));
 }
 

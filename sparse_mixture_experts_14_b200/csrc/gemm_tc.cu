@@ -66,6 +66,7 @@ constexpr int NUM_EPI_WARPS = 4;
 constexpr int MN_BOX = 64;                     // MN-major operands: two 64-wide boxes per 128 rows
 constexpr uint32_t MN_LBO = MN_BOX * BK * 2;   // bytes between the two boxes (atoms along M/N)
 constexpr uint32_t MN_SBO = 1024;              // bytes between 8-row groups along K
+constexpr int OUT_PITCH = 36;                  // floats per staged output row (16-byte aligned, no bank conflicts)
 
 // What one instantiation computes.
 enum : int {
@@ -77,15 +78,7 @@ enum : int {
     kWgrad = 5,      // dW_e = A_e^T B_e over the expert's rows     -> fp32 [E][M][N]
 };
 
-template <int MODE>
-struct ModeT {
-    static constexpr bool GATED = MODE == kFwd1 || MODE == kSwigluBwd;   // B halves = W1 / W3 blocks
-    static constexpr bool A_MN = MODE == kWgrad;
-    static constexpr bool B_MN = MODE == kDgradH || MODE == kDgradX || MODE == kWgrad;
-    static constexpr bool KGROUP = MODE == kWgrad;                        // tiles grouped by K, not by rows
-    static constexpr int N_PER_TILE = GATED ? BNH : BN;
-    static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
-};
+
 
 // Scalar arguments of one launch.
 struct GemmParams {
@@ -119,16 +112,41 @@ struct Ctrl {
     int pt[kMaxExperts];        // pairs of m-tiles of expert e
     int row0[kMaxExperts];      // first row of expert e's segment
     int nkb[kMaxExperts];       // K blocks of expert e (grouped-by-K tiles)
+    int ntn;                    // n-blocks per expert
+    int n_fast;                 // tile order (decode_tile)
 };
 
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + (int)sizeof(Ctrl) + 1024;
+template <int MODE>
+struct ModeT {
+    static constexpr bool GATED = MODE == kFwd1 || MODE == kSwigluBwd;   // B halves = W1 / W3 blocks
+    static constexpr bool A_MN = MODE == kWgrad;
+    static constexpr bool B_MN = MODE == kDgradH || MODE == kDgradX || MODE == kWgrad;
+    static constexpr bool KGROUP = MODE == kWgrad;                        // tiles grouped by K, not by rows
+    static constexpr int N_PER_TILE = GATED ? BNH : BN;
+    static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
+    // Grouped-by-K tiles are short (K = one expert's rows), so their fp32 epilogue is staged
+    // through shared memory for row-contiguous stores; that space comes from one ring stage.
+    static constexpr bool STAGED_OUT = KGROUP;
+    static constexpr int STAGES_M = STAGED_OUT ? STAGES - 1 : STAGES;
+    static constexpr int STAGE_OUT_BYTES = STAGED_OUT ? NUM_EPI_WARPS * 32 * OUT_PITCH * 4 : 0;
+    static constexpr int SMEM = STAGES_M * STAGE_BYTES + STAGE_OUT_BYTES + (int)sizeof(Ctrl) + 1024;
+};
 
+
+// Tile order inside an expert: m-tile pairs fastest (the CTAs at work share one
+// block of B), or with n_fast the n-blocks fastest (they share one block of A;
+// for gradients whose A operand is the large one).
 __device__ __forceinline__ void decode_tile(const Ctrl* c, int tile, int& e, int& pair, int& n_blk) {
     e = 0;
     while (tile >= c->tile_base[e + 1]) ++e;
     const int local = tile - c->tile_base[e];
-    n_blk = local / c->pt[e];
-    pair = local - n_blk * c->pt[e];
+    if (c->n_fast) {
+        pair = local / c->ntn;
+        n_blk = local - pair * c->ntn;
+    } else {
+        n_blk = local / c->pt[e];
+        pair = local - n_blk * c->pt[e];
+    }
 }
 
 // Soft per-wave alignment of the clusters.  CTA pairs that share a block of
@@ -153,9 +171,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB1,
                    const __grid_constant__ CUtensorMap mapB3, const GemmParams p) {
     using MT = ModeT<MODE>;
+    constexpr int NST = MT::STAGES_M;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES);
+    float* stage_out = reinterpret_cast<float*>(smem + NST * STAGE_BYTES);
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + NST * STAGE_BYTES + MT::STAGE_OUT_BYTES);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = ptx::cluster_ctarank();
@@ -168,7 +188,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     pdl_trigger();
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             ptx::mbar_init(&ctrl->full[s], 1);
             ptx::mbar_init(&ctrl->empty[s], 1);
         }
@@ -193,6 +213,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     pdl_wait();
     if (threadIdx.x == 0) {
         const int ntn = (N + N_PER_TILE - 1) / N_PER_TILE;
+        ctrl->ntn = ntn;
+        ctrl->n_fast = MT::KGROUP && p.M > N;
         ctrl->tile_base[0] = 0;
         bool ok = true;
         for (int e = 0; e < E; ++e) {
@@ -231,10 +253,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint64_t pol = ptx::policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
-            bool armed[STAGES];
-            uint32_t armed_phase[STAGES];
+            bool armed[NST];
+            uint32_t armed_phase[NST];
 #pragma unroll
-            for (int s = 0; s < STAGES; ++s) {
+            for (int s = 0; s < NST; ++s) {
                 armed[s] = false;
                 armed_phase[s] = 0;
             }
@@ -281,12 +303,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         }
                     }
 #pragma unroll
-                    for (int s = 0; s < STAGES; ++s)
+                    for (int s = 0; s < NST; ++s)
                         if (s == stage) {
                             armed[s] = true;
                             armed_phase[s] = phase;
                         }
-                    if (++stage == STAGES) {
+                    if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -295,7 +317,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (leader && (aborted || ctrl->abort)) {
                 // let copies still in flight land before shared memory is released
 #pragma unroll
-                for (int s = 0; s < STAGES; ++s)
+                for (int s = 0; s < NST; ++s)
                     if (armed[s]) ptx::mbar_wait_drain(&ctrl->full[s], armed_phase[s], 100000000ull);
             }
         }
@@ -336,7 +358,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     ptx::tc_commit_pair_multicast(&ctrl->empty[stage], 0x3);
                     issued = true;
-                    if (++stage == STAGES) {
+                    if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -433,6 +455,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                                    pb[4 * v + 3], pol_out);
                         }
                     }
+                } else if (MT::STAGED_OUT) {
+                    // fp32 gradient tile of expert e, rows m of [M][N] (rows >= split to out_hi):
+                    // each 32 x 32 chunk goes through shared memory so that the stores run along
+                    // rows (8 lanes per 128-byte row segment) instead of one row per lane
+                    float* stg = stage_out + q * 32 * OUT_PITCH;
+                    const bool zero = ctrl->nkb[e] == 0;   // no rows: the accumulator was never written
+                    const int mbase = m_tile * BM + q * 32;
+#pragma unroll 1
+                    for (int c = 0; c < BN; c += 32) {
+                        uint32_t r[32];
+                        ptx::tmem_ld_32x32b_x32(taddr + c, r);
+                        ptx::tmem_ld_wait();
+                        const int col = n_blk * BN + c;
+                        if (col >= N) continue;
+                        float4* srow = reinterpret_cast<float4*>(stg + lane * OUT_PITCH);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            srow[v] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                           : make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                        __syncwarp();
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int rr = it * 4 + (lane >> 3);
+                            const int cc = (lane & 7) * 4;
+                            const int m = mbase + rr;
+                            if (m < p.M) {
+                                const float4 v = *reinterpret_cast<const float4*>(stg + rr * OUT_PITCH + cc);
+                                float* dst = m < p.split
+                                                 ? static_cast<float*>(p.out) + ((size_t)e * p.split + m) * (size_t)N
+                                                 : static_cast<float*>(p.out_hi) +
+                                                       ((size_t)e * (p.M - p.split) + (m - p.split)) * (size_t)N;
+                                ptx::st_global_v4_hint(dst + col + cc, __float_as_uint(v.x), __float_as_uint(v.y),
+                                                       __float_as_uint(v.z), __float_as_uint(v.w), pol_out);
+                            }
+                        }
+                        __syncwarp();
+                    }
                 } else {
                     // fp32 tile: row-grouped modes write row r of [slots][N]; grouped-by-K writes
                     // row m of expert e's [M][N] gradient (rows >= split to out_hi)
@@ -514,7 +574,8 @@ template <int MODE>
 cudaError_t ensure_smem_attr() {
     static PerDeviceOnce once;
     return once.run([] {
-        return cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        return cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ModeT<MODE>::SMEM);
     });
 }
 
@@ -526,7 +587,7 @@ int grid_for(size_t pair_tiles, int num_sms) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * 74, 1, 1);
         cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.dynamicSmemBytes = ModeT<MODE>::SMEM;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -560,7 +621,7 @@ cudaError_t launch_pair(size_t pair_tiles, int num_sms, const CUtensorMap& mA, c
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid_for<MODE>(pair_tiles, num_sms), 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = ModeT<MODE>::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
