@@ -511,7 +511,7 @@ def run_train(args, rank, world, local):
     dout = to_dev(dout_np, inp.dtype, device)
     T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
     code = moe.MOE_DTYPE_BF16 if inp.dtype == "bf16" else moe.MOE_DTYPE_F32
-    fws = torch.empty(moe.moe_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
+    fws = torch.empty(moe.moe_train_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
     bws = torch.empty(moe.moe_backward_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
     out = torch.empty((T, d), dtype=dev[0].dtype, device=device)
     f32 = torch.float32
@@ -523,10 +523,14 @@ def run_train(args, rank, world, local):
     counts = moe.moe_dispatch(idx, E)[0].cpu().numpy()
     acc = accounting(inp, counts)
     kT = k * T
-    bwd_flops = {"dgrad_h": 2.0 * kT * d * F, "swiglu_bwd": 4.0 * kT * d * F, "dgrad_x": 4.0 * kT * d * F,
-                 "wgrad2": 2.0 * kT * d * F, "wgrad13": 4.0 * kT * d * F}
-    # algorithmic work of a training step: the forward, then 12 kT d F of expert gradients (the SwiGLU
-    # recompute is this implementation's choice, not counted) and 4 T d E for the router's two gradients
+    # executed FLOPs of each backward GEMM stage (bf16: the SwiGLU backward is fused into dgrad_h and
+    # reads GEMM1's kept pre-activations; fp32 recomputes GEMM1 in the swiglu_bwd stage)
+    bwd_flops = {"dgrad_h": 2.0 * kT * d * F, "dgrad_x": 4.0 * kT * d * F, "wgrad2": 2.0 * kT * d * F,
+                 "wgrad13": 4.0 * kT * d * F}
+    if inp.dtype != "bf16":
+        bwd_flops["swiglu_bwd"] = 4.0 * kT * d * F
+    # algorithmic work of a training step: the forward, then 12 kT d F of expert gradients and
+    # 4 T d E for the router's two gradients
     step_flops = acc["layer_flops"] + 12.0 * kT * d * F + 4.0 * T * d * E
 
     ns, nb = moe.MOE_NUM_STAGES, moe.MOE_BWD_NUM_STAGES
@@ -542,7 +546,7 @@ def run_train(args, rank, world, local):
 
     def step(i=None):
         on = i is not None and i % every == 0
-        n = moe.moe_forward_profiled(*dev, k, fws, out, events=fev[i] if on else None, path=moe.MOE_PATH_PREFILL)
+        n = moe.moe_forward_profiled(*dev, k, fws, out, events=fev[i] if on else None, path=moe.MOE_PATH_TRAIN)
         _, m = moe.moe_backward_ws(*dev, dout, k, fws, workspace=bws, grads=grads, events=bev[i] if on else None)
         return n + m
 

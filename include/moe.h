@@ -86,8 +86,11 @@ typedef enum {
 enum {
     MOE_PATH_AUTO = 0,    /* decode path when T <= moe_decode_max_tokens(), else grouped GEMMs */
     MOE_PATH_PREFILL = 1, /* gather + tensor-core grouped GEMMs (CTA pairs, 256-row tiles) */
-    MOE_PATH_DECODE = 2   /* expert-weight streaming, weights as the MMA's M side
+    MOE_PATH_DECODE = 2,  /* expert-weight streaming, weights as the MMA's M side
                              (bfloat16 only, T <= moe_decode_max_tokens()) */
+    MOE_PATH_TRAIN = 3    /* the grouped-GEMM path, and the workspace keeps what
+                             moe_backward_ws needs (bfloat16: GEMM1's a = W1 x and
+                             b = W3 x in fp32); workspace of moe_train_workspace_size() */
 };
 
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
@@ -186,6 +189,9 @@ MOE_API moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1,
                           const void* W2, void* out, int T, int d, int ffn, int E, int k,
                           int dtype, int path, void* workspace, size_t workspace_bytes,
                           cudaStream_t stream);
+
+/* Workspace bytes of moe_forward_ws / moe_forward_profiled with MOE_PATH_TRAIN. */
+MOE_API size_t moe_train_workspace_size(int T, int d, int ffn, int E, int k, int dtype);
 
 /* Stages of one layer call, in launch order (moe_forward_profiled). */
 enum {
@@ -327,10 +333,11 @@ MOE_API moe_status moe_route_stats_f32(const float* x, const float* Wg, int T, i
  * The gradient of the load-balance loss is not included (its p term depends
  * on the scores; add it through dlogits if needed).
  *
- * Use: run moe_forward_ws with MOE_PATH_PREFILL (MOE_PATH_AUTO takes it when
- * T > moe_decode_max_tokens(); the fp32 forward always does) on the same
- * operands, then pass its workspace here unchanged as fwd_workspace (device,
- * read only).  workspace: at least moe_backward_workspace_size() bytes
+ * Use: run moe_forward_ws (or moe_forward_profiled) with MOE_PATH_TRAIN and
+ * a workspace of moe_train_workspace_size() bytes on the same operands, then
+ * pass that workspace here unchanged as fwd_workspace (device, read only).
+ * The bfloat16 backward reads GEMM1's kept a and b instead of recomputing
+ * them; the fp32 backward recomputes them.  workspace: at least moe_backward_workspace_size() bytes
  * (device, 256-byte aligned).  Outputs (device, overwritten): dx [T][d] in
  * the layer's element type; dWg [E][d], dW1 [E][F][d], dW3 [E][F][d] and
  * dW2 [E][d][F] in float; dlogits [T][E] float (optional, NULL allowed): the
@@ -341,8 +348,8 @@ MOE_API moe_status moe_route_stats_f32(const float* x, const float* Wg, int T, i
  * ------------------------------------------------------------------------ */
 enum {
     MOE_BWD_STAGE_SCATTER = 0,  /* dy = g dout into the expert segments, dg, ds */
-    MOE_BWD_STAGE_DGRAD_H = 1,  /* dH = dY W2 */
-    MOE_BWD_STAGE_SWIGLU = 2,   /* GEMM1 recomputed, dA and dB */
+    MOE_BWD_STAGE_DGRAD_H = 1,  /* dH = dY W2 (bfloat16: with the SwiGLU backward fused) */
+    MOE_BWD_STAGE_SWIGLU = 2,   /* dA and dB (fp32 path: GEMM1 recomputed; bfloat16: empty) */
     MOE_BWD_STAGE_DGRAD_X = 3,  /* dXp = dA W1 + dB W3 */
     MOE_BWD_STAGE_WGRAD2 = 4,   /* dW2 */
     MOE_BWD_STAGE_WGRAD13 = 5,  /* dW1, dW3 */

@@ -31,7 +31,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_WORKSPACE, \
     MOE_ERR_DEVICE = range(7)
-MOE_PATH_AUTO, MOE_PATH_PREFILL, MOE_PATH_DECODE = 0, 1, 2
+MOE_PATH_AUTO, MOE_PATH_PREFILL, MOE_PATH_DECODE, MOE_PATH_TRAIN = 0, 1, 2, 3
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_NUM_STAGES = 6
 STAGE_NAMES = ("route", "dispatch", "gather", "expert1", "expert2", "combine")
@@ -65,6 +65,7 @@ SIGNATURES = {
                                    _ci, _vp, _sz, _vp, _vp, _vp]),
     "moe_route_stats": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
     "moe_backward_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
+    "moe_train_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
     "moe_backward_ws": (_ci, [_vp] * 12 + [_ci] * 6 + [_vp, _sz, _vp, _sz, _vp, _vp, _vp]),
     "moe_route_stats_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
 }
@@ -202,7 +203,7 @@ def moe_forward_ws(x, Wg, W1, W3, W2, k, path=MOE_PATH_AUTO, workspace=None, out
     for t, n in ((x, "x"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2")):
         _dev(t, x.dtype, n)
     T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
-    need = moe_workspace_size(T, d, F, E, k, code)
+    need = (moe_train_workspace_size if path == MOE_PATH_TRAIN else moe_workspace_size)(T, d, F, E, k, code)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
     _dev(workspace, torch.uint8, "workspace")
@@ -315,14 +316,18 @@ def moe_route_stats(x, Wg, k, alpha=1.0, stream=None):
     return idx, w, stats
 
 
+def moe_train_workspace_size(T, d, ffn, E, k, dtype=MOE_DTYPE_BF16) -> int:
+    return int(_lib.moe_train_workspace_size(T, d, ffn, E, k, dtype))
+
+
 def moe_backward_workspace_size(T, d, ffn, E, k, dtype=MOE_DTYPE_BF16) -> int:
     return int(_lib.moe_backward_workspace_size(T, d, ffn, E, k, dtype))
 
 
 def moe_backward_ws(x, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, grads=None, dlogits=None,
                     events=None, stream=None):
-    """Gradients of the layer given dout = dL/dout, after moe_forward_ws(..., path=MOE_PATH_PREFILL,
-    workspace=fwd_workspace) on the same operands.  Returns (grads, launches) with grads a dict of
+    """Gradients of the layer given dout = dL/dout, after moe_forward_ws(..., path=MOE_PATH_TRAIN,
+    workspace=fwd_workspace) on the same operands (fwd_workspace: moe_train_workspace_size bytes).  Returns (grads, launches) with grads a dict of
     dx (layer dtype), dWg, dW1, dW3, dW2 (float32); pass `grads` to reuse buffers, `dlogits` (float32
     [T][E]) to also get the router-score gradient."""
     code = _dtype_code(x)

@@ -35,8 +35,10 @@
 //
 // The same kernel runs the layer's backward GEMMs (gradients of the expert
 // equations, the training the page's "ロードバランス損失" subsection closes with):
-//     dH    = dY_e W2_e                  W2 read MN-major (no transpose)
-//     dA,dB = SwiGLU backward of GEMM1 recomputed in TMEM, with dH from HBM
+//     dH    = dY_e W2_e                  W2 read MN-major (no transpose); the
+//                                        epilogue turns dH into dA, dB with the
+//                                        a = Xp W1^T, b = Xp W3^T that the training
+//                                        forward's GEMM1 epilogue kept (fp32)
 //     dXp   = dA_e W1_e + dB_e W3_e      W1 / W3 read MN-major, K = 2F
 //     dW2_e = dY_e^T H_e                 both operands MN-major, K = the
 //     dW1_e|dW3_e = [dA dB]_e^T Xp_e     expert's rows (grouped by K)
@@ -70,12 +72,12 @@ constexpr int OUT_PITCH = 36;                  // floats per staged output row (
 
 // What one instantiation computes.
 enum : int {
-    kFwd1 = 0,       // H = SiLU(Xp W1^T) * (Xp W3^T)            -> bf16 [slots][N]
-    kFwd2 = 1,       // C = A B_e^T, B K-major                   -> fp32 [slots][N]
-    kDgradH = 2,     // dH = dY W2_e (W2 MN-major)                -> fp32 [slots][N]
-    kSwigluBwd = 3,  // dA | dB from recomputed a, b and dH        -> bf16 [slots][2N]
-    kDgradX = 4,     // dXp = dA W1_e + dB W3_e (MN-major, K = 2F) -> fp32 [slots][N]
-    kWgrad = 5,      // dW_e = A_e^T B_e over the expert's rows     -> fp32 [E][M][N]
+    kFwd1 = 0,       // H = SiLU(Xp W1^T) * (Xp W3^T)              -> bf16 [slots][N]
+    kFwd2 = 1,       // C = A B_e^T, B K-major                     -> fp32 [slots][N]
+    kFwd1Train = 2,  // kFwd1, and a = Xp W1^T, b = Xp W3^T kept    -> + fp32 [slots][N] x 2
+    kDgradH = 3,     // dH = dY W2_e (W2 MN-major), SwiGLU backward -> dA | dB bf16 [slots][2N]
+    kDgradX = 4,     // dXp = dA W1_e + dB W3_e (MN-major, K = 2F)   -> fp32 [slots][N]
+    kWgrad = 5,      // dW_e = A_e^T B_e over the expert's rows       -> fp32 [E][M][N]
 };
 
 
@@ -85,7 +87,7 @@ struct GemmParams {
     Meta* meta;
     int E;
     int M;           // kWgrad: output rows per expert
-    int N;           // output columns (kSwigluBwd: F; its output rows hold 2N)
+    int N;           // output columns (kDgradH: F; its output rows hold dA | dB, 2N)
     int K;           // reduction length of the row-grouped modes
     int split;       // kWgrad: output rows m >= split go to out_hi, row m - split
     int kb_split;    // kDgradX: K blocks from mapB3 start here
@@ -93,7 +95,10 @@ struct GemmParams {
     size_t slots;
     void* out;
     void* out_hi;
-    const float* aux;   // kSwigluBwd: dH [slots][N] fp32
+    float* keep_a;      // kFwd1Train: a and b [slots][N] fp32
+    float* keep_b;
+    const float* aux_a; // kDgradH: the kept a and b [slots][N] fp32
+    const float* aux_b;
     int* status;
     long long wait_ns;
 };
@@ -118,7 +123,7 @@ struct Ctrl {
 
 template <int MODE>
 struct ModeT {
-    static constexpr bool GATED = MODE == kFwd1 || MODE == kSwigluBwd;   // B halves = W1 / W3 blocks
+    static constexpr bool GATED = MODE == kFwd1 || MODE == kFwd1Train;   // B halves = W1 / W3 blocks
     static constexpr bool A_MN = MODE == kWgrad;
     static constexpr bool B_MN = MODE == kDgradH || MODE == kDgradX || MODE == kWgrad;
     static constexpr bool KGROUP = MODE == kWgrad;                        // tiles grouped by K, not by rows
@@ -390,7 +395,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const bool live = MT::KGROUP ? m_tile * BM < p.M : m_tile < ctrl->mt[e];
             if (live) {
                 const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-                if (MODE == kFwd1) {
+                if (MODE == kFwd1 || MODE == kFwd1Train) {
                     const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
                     __nv_bfloat16* H = static_cast<__nv_bfloat16*>(p.out);
 #pragma unroll 1
@@ -411,41 +416,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         for (int v = 0; v < 4; ++v)
                             ptx::st_global_v4_hint(dst + 16 * v, hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3],
                                                    pol_out);
+                        if (MODE == kFwd1Train) {
+                            // keep the pre-activations for the backward
+                            uint8_t* ka = reinterpret_cast<uint8_t*>(p.keep_a + row * (size_t)N + n_blk * BNH + c);
+                            uint8_t* kb = reinterpret_cast<uint8_t*>(p.keep_b + row * (size_t)N + n_blk * BNH + c);
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) {
+                                ptx::st_global_v4_hint(ka + 16 * v, ra[4 * v], ra[4 * v + 1], ra[4 * v + 2],
+                                                       ra[4 * v + 3], pol_out);
+                                ptx::st_global_v4_hint(kb + 16 * v, rb[4 * v], rb[4 * v + 1], rb[4 * v + 2],
+                                                       rb[4 * v + 3], pol_out);
+                            }
+                        }
                     }
-                } else if (MODE == kSwigluBwd) {
-                    // h = SiLU(a) b:  dA = dH b SiLU'(a),  dB = dH SiLU(a)
+                } else if (MODE == kDgradH) {
+                    // dH tile (TMEM) -> SwiGLU backward with the kept a, b:
+                    //     dA = dH b SiLU'(a),  dB = dH SiLU(a)   -> bf16 [slots][2N], dA | dB
                     const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
                     __nv_bfloat16* dAB = static_cast<__nv_bfloat16*>(p.out);
 #pragma unroll 1
-                    for (int c = 0; c < BNH; c += 32) {
-                        uint32_t ra[32], rb[32];
-                        ptx::tmem_ld_32x32b_x32(taddr + c, ra);
-                        ptx::tmem_ld_32x32b_x32(taddr + BNH + c, rb);
-                        const float4* dhp = reinterpret_cast<const float4*>(p.aux + row * (size_t)N + n_blk * BNH + c);
-                        float dh[32];
+                    for (int c = 0; c < BN; c += 32) {
+                        const int col = n_blk * BN + c;
+                        if (col >= N) break;
+                        const float4* ap = reinterpret_cast<const float4*>(p.aux_a + row * (size_t)N + col);
+                        const float4* bp = reinterpret_cast<const float4*>(p.aux_b + row * (size_t)N + col);
+                        float av[32], bv[32];
 #pragma unroll
                         for (int v = 0; v < 8; ++v) {
-                            const float4 t = __ldg(dhp + v);
-                            dh[4 * v] = t.x;
-                            dh[4 * v + 1] = t.y;
-                            dh[4 * v + 2] = t.z;
-                            dh[4 * v + 3] = t.w;
+                            const float4 ta = __ldg(ap + v), tb = __ldg(bp + v);
+                            av[4 * v] = ta.x;
+                            av[4 * v + 1] = ta.y;
+                            av[4 * v + 2] = ta.z;
+                            av[4 * v + 3] = ta.w;
+                            bv[4 * v] = tb.x;
+                            bv[4 * v + 1] = tb.y;
+                            bv[4 * v + 2] = tb.z;
+                            bv[4 * v + 3] = tb.w;
                         }
+                        uint32_t r[32];
+                        ptx::tmem_ld_32x32b_x32(taddr + c, r);
                         ptx::tmem_ld_wait();
                         uint32_t pa[16], pb[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             float da[2], dbv[2];
 #pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const float av = __uint_as_float(ra[2 * i + u]);
-                                const float bv = __uint_as_float(rb[2 * i + u]);
-                                silu_bwd(av, bv, dh[2 * i + u], da[u], dbv[u]);
-                            }
+                            for (int u = 0; u < 2; ++u)
+                                silu_bwd(av[2 * i + u], bv[2 * i + u], __uint_as_float(r[2 * i + u]), da[u], dbv[u]);
                             pa[i] = pack_bf16x2(da[0], da[1]);
                             pb[i] = pack_bf16x2(dbv[0], dbv[1]);
                         }
-                        uint8_t* dst_a = reinterpret_cast<uint8_t*>(dAB + row * (size_t)(2 * N) + n_blk * BNH + c);
+                        uint8_t* dst_a = reinterpret_cast<uint8_t*>(dAB + row * (size_t)(2 * N) + col);
                         uint8_t* dst_b = dst_a + (size_t)N * 2;
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
@@ -663,6 +684,18 @@ cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s) {
     return launch_pair<kFwd1>(row_pair_tiles(a.slots, a.E, (a.F + BNH - 1) / BNH), a.num_sms, mA, mB1, mB3, gp, s);
 }
 
+cudaError_t launch_tc_gemm1_train(const TcGemmArgs& a, float* keep_a, float* keep_b, cudaStream_t s) {
+    CUtensorMap mA, mB1, mB3;
+    if (!map_rows(&mA, a.xp, a.slots, a.d, BM) || !map_weights(&mB1, a.W1, a.E, a.F, a.d, BNH) ||
+        !map_weights(&mB3, a.W3, a.E, a.F, a.d, BNH))
+        return cudaErrorInvalidValue;
+    GemmParams gp = params(const_cast<Meta*>(a.meta), a.E, a.F, a.d, kWaveFwd1, a.slots, a.H, a.status, a.wait_ns);
+    gp.keep_a = keep_a;
+    gp.keep_b = keep_b;
+    return launch_pair<kFwd1Train>(row_pair_tiles(a.slots, a.E, (a.F + BNH - 1) / BNH), a.num_sms, mA, mB1, mB3, gp,
+                                   s);
+}
+
 cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s) {
     CUtensorMap mA, mB;
     if (!map_rows(&mA, a.H, a.slots, a.F, BM) || !map_weights(&mB, a.W2, a.E, a.d, a.F, BNH))
@@ -673,23 +706,15 @@ cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_tc_dgrad_h(const TcBwdArgs& a, cudaStream_t s) {
-    // dH [slots][F] = dY [slots][d] . W2_e [d][F]: B[n = f][k = i] is W2 read MN-major
+    // dH [slots][F] = dY [slots][d] . W2_e [d][F] (B[n = f][k = i] is W2 read MN-major), turned into
+    // dA | dB [slots][2F] in the epilogue with the kept a, b
     CUtensorMap mA, mB;
     if (!map_rows(&mA, a.dy, a.slots, a.d, BM) || !map_mn_weights(&mB, a.W2, a.E, a.d, a.F))
         return cudaErrorInvalidValue;
-    const GemmParams gp = params(a.meta, a.E, a.F, a.d, kWaveDgradH, a.slots, a.dh, a.status, a.wait_ns);
+    GemmParams gp = params(a.meta, a.E, a.F, a.d, kWaveDgradH, a.slots, a.dab, a.status, a.wait_ns);
+    gp.aux_a = a.keep_a;
+    gp.aux_b = a.keep_b;
     return launch_pair<kDgradH>(row_pair_tiles(a.slots, a.E, (a.F + BN - 1) / BN), a.num_sms, mA, mB, mB, gp, s);
-}
-
-cudaError_t launch_tc_swiglu_bwd(const TcBwdArgs& a, cudaStream_t s) {
-    CUtensorMap mA, mB1, mB3;
-    if (!map_rows(&mA, a.xp, a.slots, a.d, BM) || !map_weights(&mB1, a.W1, a.E, a.F, a.d, BNH) ||
-        !map_weights(&mB3, a.W3, a.E, a.F, a.d, BNH))
-        return cudaErrorInvalidValue;
-    GemmParams gp = params(a.meta, a.E, a.F, a.d, kWaveSwigluBwd, a.slots, a.dab, a.status, a.wait_ns);
-    gp.aux = a.dh;
-    return launch_pair<kSwigluBwd>(row_pair_tiles(a.slots, a.E, (a.F + BNH - 1) / BNH), a.num_sms, mA, mB1, mB3,
-                                   gp, s);
 }
 
 cudaError_t launch_tc_dgrad_x(const TcBwdArgs& a, cudaStream_t s) {

@@ -111,13 +111,14 @@ moe_status check_layer(const void* x, const void* Wg, const void* W1, const void
 struct Plan {
     size_t idx, w, blk, meta, perm, inv, xp, h, y;
     size_t rstd, logits, bal;   // block form only (see make_plan's `block`)
+    size_t keep_a, keep_b;      // training path, bf16: GEMM1's a and b, fp32 [slots][F]
     size_t total;
     size_t slots;
 };
 
 // Workspace layout.  The block form adds each row's norm factor [T], the fp32
 // scores [T][E] and the load-balance partial sums.
-Plan make_plan(int T, int d, int F, int E, int k, int dtype, bool block = false) {
+Plan make_plan(int T, int d, int F, int E, int k, int dtype, bool block = false, bool train = false) {
     Plan p{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -137,6 +138,10 @@ Plan make_plan(int T, int d, int F, int E, int k, int dtype, bool block = false)
     p.xp = take(p.slots * (size_t)d * es);
     p.h = take(p.slots * (size_t)F * es);
     p.y = take(p.slots * (size_t)d * 4);
+    if (train && dtype == MOE_DTYPE_BF16) {
+        p.keep_a = take(p.slots * (size_t)F * 4);
+        p.keep_b = take(p.slots * (size_t)F * 4);
+    }
     if (block) {
         p.rstd = take((size_t)T * 4);
         p.logits = take((size_t)T * E * 4);
@@ -166,7 +171,8 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
                      int d, int F, int E, int k, int dtype, int path, uint8_t* ws, const DeviceState& dev,
                      cudaStream_t s, cudaEvent_t* ev = nullptr, int* launches = nullptr,
                      const BlockArgs* bo = nullptr) {
-    const Plan p = make_plan(T, d, F, E, k, dtype, bo != nullptr);
+    const bool train = path == MOE_PATH_TRAIN;
+    const Plan p = make_plan(T, d, F, E, k, dtype, bo != nullptr, train);
     RouteExtras ex;
     GatherNorm nm;
     if (bo) {
@@ -221,7 +227,12 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
         TcGemmArgs a{xp, W1, W3, W2, h, y, meta, E, d, F, p.slots, dev.num_sms, dev.status, wait_limit_ns()};
         const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxTokens);
         MOE_TRY(mark(MOE_STAGE_EXPERT1));
-        MOE_TRY(decode ? launch_decode(a, 1, s) : launch_tc_gemm1(a, s));
+        if (train) {
+            MOE_TRY(launch_tc_gemm1_train(a, reinterpret_cast<float*>(ws + p.keep_a),
+                                          reinterpret_cast<float*>(ws + p.keep_b), s));
+        } else {
+            MOE_TRY(decode ? launch_decode(a, 1, s) : launch_tc_gemm1(a, s));
+        }
         MOE_TRY(mark(MOE_STAGE_EXPERT2));
         MOE_TRY(decode ? launch_decode(a, 2, s) : launch_tc_gemm2(a, s));
         MOE_TRY(mark(MOE_STAGE_COMBINE));
@@ -335,7 +346,7 @@ BwdPlan make_bwd_plan(int T, int d, int F, int E, int k, int dtype) {
     b.dy = take(S * d * es);
     b.dg = take((size_t)T * k * 4);
     b.ds = take((size_t)T * E * 4);
-    b.dh = take(S * F * 4);
+    b.dh = take(dtype == MOE_DTYPE_BF16 ? 0 : S * F * 4);   // the bf16 path never stores dH
     b.dab = take(S * 2 * (size_t)F * es);
     b.dxp = take(S * d * 4);
     b.dwg = take(dwg_part_bytes(T, E, d));
@@ -347,7 +358,7 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
                         const void* dout, void* dx, float* dWg, float* dW1, float* dW3, float* dW2, float* dlogits,
                         int T, int d, int F, int E, int k, int dtype, const uint8_t* fws, uint8_t* bws,
                         const DeviceState& dev, cudaStream_t s, cudaEvent_t* ev, int* launches) {
-    const Plan p = make_plan(T, d, F, E, k, dtype);
+    const Plan p = make_plan(T, d, F, E, k, dtype, false, true);
     const BwdPlan b = make_bwd_plan(T, d, F, E, k, dtype);
     uint8_t* fw = const_cast<uint8_t*>(fws);
     BwdArgs a{};
@@ -366,6 +377,10 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
     a.xp = fw + p.xp;
     a.H = fw + p.h;
     a.Y = reinterpret_cast<const float*>(fw + p.y);
+    if (dtype == MOE_DTYPE_BF16) {
+        a.keep_a = reinterpret_cast<const float*>(fw + p.keep_a);
+        a.keep_b = reinterpret_cast<const float*>(fw + p.keep_b);
+    }
     a.dy = bws + b.dy;
     a.dg = reinterpret_cast<float*>(bws + b.dg);
     a.ds = dlogits ? dlogits : reinterpret_cast<float*>(bws + b.ds);
@@ -398,8 +413,9 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
         t.W3 = W3;
         t.W2 = W2;
         t.H = a.H;
+        t.keep_a = a.keep_a;
+        t.keep_b = a.keep_b;
         t.dy = a.dy;
-        t.dh = a.dh;
         t.dab = a.dab;
         t.dxp = a.dxp;
         t.dW1 = dW1;
@@ -414,15 +430,15 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
         t.status = dev.status;
         t.wait_ns = wait_limit_ns();
         MOE_TRY(mark(MOE_BWD_STAGE_DGRAD_H));
-        MOE_TRY(launch_tc_dgrad_h(t, s));
+        MOE_TRY(launch_tc_dgrad_h(t, s));   // SwiGLU backward fused into its epilogue
         MOE_TRY(mark(MOE_BWD_STAGE_SWIGLU));
-        MOE_TRY(launch_tc_swiglu_bwd(t, s));
         MOE_TRY(mark(MOE_BWD_STAGE_DGRAD_X));
         MOE_TRY(launch_tc_dgrad_x(t, s));
         MOE_TRY(mark(MOE_BWD_STAGE_WGRAD2));
         MOE_TRY(launch_tc_wgrad2(t, s));
         MOE_TRY(mark(MOE_BWD_STAGE_WGRAD13));
         MOE_TRY(launch_tc_wgrad13(t, s));
+        n += 4;
     } else {
         MOE_TRY(mark(MOE_BWD_STAGE_DGRAD_H));
         MOE_TRY(mark(MOE_BWD_STAGE_SWIGLU));
@@ -430,8 +446,8 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
         MOE_TRY(mark(MOE_BWD_STAGE_WGRAD2));
         MOE_TRY(launch_simt_bwd_gemms(a, s));
         MOE_TRY(mark(MOE_BWD_STAGE_WGRAD13));
+        n += 5;
     }
-    n += 5;
     MOE_TRY(mark(MOE_BWD_STAGE_ROUTER));
     MOE_TRY(launch_dwg(a, s));
     MOE_TRY(launch_dx_combine(a, s));
@@ -555,11 +571,13 @@ moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1, const v
                           size_t workspace_bytes, cudaStream_t stream) {
     moe_status st = check_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype);
     if (st != MOE_OK) return st;
-    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE) return MOE_ERR_INVALID_ARG;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE && path != MOE_PATH_TRAIN)
+        return MOE_ERR_INVALID_ARG;
     if (path == MOE_PATH_DECODE && (dtype != MOE_DTYPE_BF16 || T > kDecodeMaxTokens)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
-    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
+    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype, false, path == MOE_PATH_TRAIN).total)
+        return MOE_ERR_WORKSPACE;
     DeviceState dev;
     if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
     return run_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
@@ -573,11 +591,13 @@ moe_status moe_forward_profiled(const void* x, const void* Wg, const void* W1, c
     if (launches) *launches = 0;
     moe_status st = check_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype);
     if (st != MOE_OK) return st;
-    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE) return MOE_ERR_INVALID_ARG;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE && path != MOE_PATH_TRAIN)
+        return MOE_ERR_INVALID_ARG;
     if (path == MOE_PATH_DECODE && (dtype != MOE_DTYPE_BF16 || T > kDecodeMaxTokens)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
-    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
+    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype, false, path == MOE_PATH_TRAIN).total)
+        return MOE_ERR_WORKSPACE;
     DeviceState dev;
     if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
     return run_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
@@ -687,6 +707,12 @@ moe_status moe_block_forward_ws(const void* h, const void* gamma, float eps, con
                      stream, stage_events, launches, &bo);
 }
 
+size_t moe_train_workspace_size(int T, int d, int ffn, int E, int k, int dtype) {
+    if (check_sizes(T, d, E, k) != MOE_OK || ffn <= 0) return 0;
+    if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_F32) return 0;
+    return make_plan(T, d, ffn, E, k, dtype, false, true).total;
+}
+
 size_t moe_backward_workspace_size(int T, int d, int ffn, int E, int k, int dtype) {
     if (check_sizes(T, d, E, k) != MOE_OK || ffn <= 0) return 0;
     if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_F32) return 0;
@@ -707,7 +733,7 @@ moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const 
         if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
     if (dlogits && (reinterpret_cast<uintptr_t>(dlogits) & 3u) != 0) return MOE_ERR_INVALID_ARG;
     if (!fwd_workspace || (reinterpret_cast<uintptr_t>(fwd_workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
-    if (fwd_workspace_bytes < make_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
+    if (fwd_workspace_bytes < make_plan(T, d, ffn, E, k, dtype, false, true).total) return MOE_ERR_WORKSPACE;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (workspace_bytes < make_bwd_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
     DeviceState dev;

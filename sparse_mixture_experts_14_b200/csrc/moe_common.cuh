@@ -211,6 +211,8 @@ struct TcGemmArgs {
     long long wait_ns;
 };
 cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s);
+// GEMM1 of the training forward: also keeps a = Xp W1^T and b = Xp W3^T, fp32 [slots][F] each.
+cudaError_t launch_tc_gemm1_train(const TcGemmArgs& a, float* keep_a, float* keep_b, cudaStream_t s);
 cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s);
 
 // Backward GEMMs on the same CTA-pair kernel (bf16 operands, fp32 accumulate).
@@ -220,8 +222,9 @@ struct TcBwdArgs {
     const void* W3;
     const void* W2;     // [E][d][F]
     const void* H;      // forward: [slots][F] bf16
+    const float* keep_a;  // forward (training path): a, b [slots][F] fp32
+    const float* keep_b;
     const void* dy;     // [slots][d] bf16: g * dout scattered to the slots (padding rows zero)
-    float* dh;          // [slots][F] fp32
     void* dab;          // [slots][2F] bf16: dA | dB
     float* dxp;         // [slots][d] fp32
     float* dW1;         // [E][F][d] fp32
@@ -253,6 +256,8 @@ struct BwdArgs {
     const void* xp;         // [slots][d]
     const void* H;          // [slots][F]
     const float* Y;         // [slots][d]
+    const float* keep_a;    // [slots][F] fp32 (bf16 training path), else null
+    const float* keep_b;
     // backward buffers
     void* dy;               // [slots][d]
     float* dg;              // [T][k]
@@ -277,8 +282,7 @@ cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s);              // dWg (2
 cudaError_t launch_dx_combine(const BwdArgs& a, cudaStream_t s);       // dx (1 launch)
 cudaError_t launch_simt_bwd_gemms(const BwdArgs& a, cudaStream_t s);   // fp32 expert GEMMs (5 launches)
 
-cudaError_t launch_tc_dgrad_h(const TcBwdArgs& a, cudaStream_t s);      // dH = dY W2_e
-cudaError_t launch_tc_swiglu_bwd(const TcBwdArgs& a, cudaStream_t s);   // dA, dB from Xp, W1, W3 and dH
+cudaError_t launch_tc_dgrad_h(const TcBwdArgs& a, cudaStream_t s);      // dH = dY W2_e -> dA, dB
 cudaError_t launch_tc_dgrad_x(const TcBwdArgs& a, cudaStream_t s);      // dXp = dA W1_e + dB W3_e
 cudaError_t launch_tc_wgrad2(const TcBwdArgs& a, cudaStream_t s);       // dW2_e = dY_e^T H_e
 cudaError_t launch_tc_wgrad13(const TcBwdArgs& a, cudaStream_t s);      // [dW1_e; dW3_e] = [dA dB]_e^T Xp_e
