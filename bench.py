@@ -66,6 +66,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--block", action="store_true",
                     help="time the block form out = h + MoE(RMSNorm(h)) with load-balance statistics")
+    ap.add_argument("--shape", default=None,
+                    help="T,d,ffn: run the workload's recipe (E, k, dtype, seed, routing) at other sizes, "
+                         "for profiler captures small enough to stay within a few GB")
     ap.add_argument("--train", action="store_true",
                     help="time a training step: forward (grouped-GEMM path) + backward with all gradients")
     ap.add_argument("--stage-every", type=int, default=8,
@@ -230,9 +233,19 @@ def oracle_train_run(inp, dout, target_s):
     return len(toks) / dt, sample, dt
 
 
-def make_workload(cfg, block):
-    inp = moe_inputs.make_config(cfg)
+def make_workload(cfg, block, shape=None):
+    if shape:
+        c = moe_inputs.CONFIGS[cfg]
+        T, d, F = (int(v) for v in shape.split(","))
+        inp = moe_inputs.make_inputs(T, d, F, c["E"], c["k"], c["dtype"], c["seed"], c["skew"])
+    else:
+        inp = moe_inputs.make_config(cfg)
     return moe_inputs.make_block(inp) if block else inp
+
+
+def workload_name(cfg, shape=None):
+    c = moe_inputs.CONFIGS[cfg]
+    return c["name"] + (f"@shape={shape}" if shape else "")
 
 
 def cpu_oracle_run(inp, target_s, threads, block=False):
@@ -263,7 +276,7 @@ def run_reference(args, rank):
     if rank != 0:
         return
     c = moe_inputs.CONFIGS[args.config]
-    inp = make_workload(args.config, args.block)
+    inp = make_workload(args.config, args.block, args.shape)
     if args.train:
         dout = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
         per_step = max(0.5, min(30.0, 150.0 / max(args.steps + args.warmup, 1)))
@@ -279,7 +292,8 @@ def run_reference(args, rank):
             "impl": "reference", "metric": TRAIN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_t / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": c["name"] + "+train", "T": inp.T, "d": inp.d, "ffn": inp.F, "E": inp.E,
+            "config": {"workload": workload_name(args.config, args.shape) + "+train", "T": inp.T, "d": inp.d,
+                       "ffn": inp.F, "E": inp.E,
                        "k": inp.k, "seed": c["seed"]},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -307,7 +321,8 @@ def run_reference(args, rank):
         "impl": "reference", "metric": BLOCK_METRIC if args.block else METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt / max(args.steps, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": c["name"] + ("+block" if args.block else ""), "T": inp.T, "d": inp.d,
+        "config": {"workload": workload_name(args.config, args.shape) + ("+block" if args.block else ""),
+                   "T": inp.T, "d": inp.d,
                    "ffn": inp.F, "E": inp.E, "k": inp.k, "seed": c["seed"],
                    "sample_tokens_per_step": int(len(toks))},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
@@ -344,7 +359,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.set_device(device)
     c = moe_inputs.CONFIGS[args.config]
     block = args.block
-    inp = make_workload(args.config, block)
+    inp = make_workload(args.config, block, args.shape)
     dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
     tdt = dev[0].dtype
     T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
@@ -465,7 +480,7 @@ def run_ours(args, rank, world, local):
         kname = {"expert1": "decode_kernel<true>", "expert2": "decode_kernel<false>"}[dom]
     else:
         kname = {"expert1": "tc_gemm_kernel<true>", "expert2": "tc_gemm_kernel<false>"}[dom]
-    roof["traffic"] = recorded_traffic(kname, c["name"])
+    roof["traffic"] = recorded_traffic(kname, workload_name(args.config, args.shape))
     roof["kernel"] = kname
     roof["per_launch"] = {"flops": fl, "bytes": by, "ms": stages[dom]}
     roof["peak_source"] = f"{peak_src} ({'sustained' if long_run and roof['unit'] == 'TFLOP/s' else 'burst'})"
@@ -481,7 +496,8 @@ def run_ours(args, rank, world, local):
         "steps": K, "warmup": W,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp.dtype, "data": "synthetic",
-        "config": {"workload": c["name"] + ("+block" if block else ""), "T": T, "d": d, "ffn": F, "E": E, "k": k,
+        "config": {"workload": workload_name(args.config, args.shape) + ("+block" if block else ""), "T": T, "d": d,
+                   "ffn": F, "E": E, "k": k,
                    "seed": c["seed"],
                    "routing": "zipf1.2-skewed" if c["skew"] else "near-uniform",
                    "l2": "L2 flushed between steps" if flush else "touched weights larger than L2 (no flush)",
@@ -505,7 +521,7 @@ def run_train(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     c = moe_inputs.CONFIGS[args.config]
-    inp = moe_inputs.make_config(args.config)
+    inp = make_workload(args.config, False, args.shape)
     dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
     dout_np = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
     dout = to_dev(dout_np, inp.dtype, device)
@@ -586,7 +602,8 @@ def run_train(args, rank, world, local):
     dom = max(bwd_flops, key=lambda n: bst[n])
     sec = bst[dom] / 1000.0
     roof = {"bound": "tensor", "achieved": bwd_flops[dom] / sec / 1e12, "peak": tflops_peak, "unit": "TFLOP/s",
-            "traffic": recorded_traffic(f"tc_gemm_kernel<{dom}>", c["name"]), "kernel": f"tc_gemm_kernel ({dom})",
+            "traffic": recorded_traffic(f"tc_gemm_kernel ({dom})", workload_name(args.config, args.shape)),
+            "kernel": f"tc_gemm_kernel ({dom})",
             "per_launch": {"flops": bwd_flops[dom], "ms": bst[dom]},
             "peak_source": f"{peak_src} ({'sustained' if long_run else 'burst'})"}
     roof["frac"] = roof["achieved"] / roof["peak"]
@@ -601,7 +618,8 @@ def run_train(args, rank, world, local):
         "metric": TRAIN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp.dtype, "data": "synthetic",
-        "config": {"workload": c["name"] + "+train", "T": T, "d": d, "ffn": F, "E": E, "k": k, "seed": c["seed"],
+        "config": {"workload": workload_name(args.config, args.shape) + "+train", "T": T, "d": d, "ffn": F, "E": E,
+                   "k": k, "seed": c["seed"],
                    "l2": "touched weights larger than L2 (no flush)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof,

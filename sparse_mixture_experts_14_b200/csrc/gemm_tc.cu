@@ -63,8 +63,7 @@ constexpr int B_BYTES = BNH * BK * 2;          // 16 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t PAIR_TX_BYTES = 2 * STAGE_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int NUM_THREADS = 192;
-constexpr int NUM_EPI_WARPS = 4;
+constexpr int NUM_EPI_WARPS = 4;                 // epilogue warps of the row-grouped modes (one per lane quarter)
 constexpr int MN_BOX = 64;                     // MN-major operands: two 64-wide boxes per 128 rows
 constexpr uint32_t MN_LBO = MN_BOX * BK * 2;   // bytes between the two boxes (atoms along M/N)
 constexpr uint32_t MN_SBO = 1024;              // bytes between 8-row groups along K
@@ -131,9 +130,13 @@ struct ModeT {
     static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
     // Grouped-by-K tiles are short (K = one expert's rows), so their fp32 epilogue is staged
     // through shared memory for row-contiguous stores; that space comes from one ring stage.
+    // Its fp32 tiles also get two epilogue warps per TMEM lane quarter (each takes half of the
+    // columns), and the ring gives up two stages for both.
     static constexpr bool STAGED_OUT = KGROUP;
-    static constexpr int STAGES_M = STAGED_OUT ? STAGES - 1 : STAGES;
-    static constexpr int STAGE_OUT_BYTES = STAGED_OUT ? NUM_EPI_WARPS * 32 * OUT_PITCH * 4 : 0;
+    static constexpr int EPI_WARPS = STAGED_OUT ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS);
+    static constexpr int STAGES_M = STAGED_OUT ? STAGES - 2 : STAGES;
+    static constexpr int STAGE_OUT_BYTES = STAGED_OUT ? EPI_WARPS * 32 * OUT_PITCH * 4 : 0;
     static constexpr int SMEM = STAGES_M * STAGE_BYTES + STAGE_OUT_BYTES + (int)sizeof(Ctrl) + 1024;
 };
 
@@ -172,7 +175,7 @@ __device__ __forceinline__ void wave_sync(int* counter, int target) {
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB1,
                    const __grid_constant__ CUtensorMap mapB3, const GemmParams p) {
     using MT = ModeT<MODE>;
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&ctrl->tfull[b], 1);
-            ptx::mbar_init(&ctrl->tempty[b], 2 * NUM_EPI_WARPS);
+            ptx::mbar_init(&ctrl->tempty[b], 2 * MT::EPI_WARPS);
         }
         ptx::mbar_init(&ctrl->drain, 1);
         ctrl->abort = 0;
@@ -381,6 +384,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else {
         // ---------------------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;   // TMEM lane quarter this warp may access
+        const int ew = warp - 2;  // epilogue warp index; with 8 of them, ew / 4 picks a column half
         const uint64_t pol_out = ptx::policy_evict_first();
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -480,11 +484,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     // fp32 gradient tile of expert e, rows m of [M][N] (rows >= split to out_hi):
                     // each 32 x 32 chunk goes through shared memory so that the stores run along
                     // rows (8 lanes per 128-byte row segment) instead of one row per lane
-                    float* stg = stage_out + q * 32 * OUT_PITCH;
+                    float* stg = stage_out + ew * 32 * OUT_PITCH;
                     const bool zero = ctrl->nkb[e] == 0;   // no rows: the accumulator was never written
                     const int mbase = m_tile * BM + q * 32;
+                    constexpr int CW = BN / (MT::EPI_WARPS / NUM_EPI_WARPS);   // columns per warp
+                    const int c0 = (ew / NUM_EPI_WARPS) * CW;
 #pragma unroll 1
-                    for (int c = 0; c < BN; c += 32) {
+                    for (int c = c0; c < c0 + CW; c += 32) {
                         uint32_t r[32];
                         ptx::tmem_ld_32x32b_x32(taddr + c, r);
                         ptx::tmem_ld_wait();
@@ -552,9 +558,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             }
+            // accumulator b is free once every lane's tcgen05.ld has completed (tmem_ld_wait above);
+            // the epilogue's global stores need not be visible to the MMA thread, so the arrive
+            // is relaxed and does not wait for them to drain
             ptx::tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&ctrl->tempty[acc]), 0));
+            if (lane == 0) ptx::mbar_arrive_cluster_relaxed(ptx::map_to_rank(ptx::smem_addr(&ctrl->tempty[acc]), 0));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
@@ -607,7 +616,7 @@ int grid_for(size_t pair_tiles, int num_sms) {
     const int max_clusters = clusters_per_device.get([num_sms] {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * 74, 1, 1);
-        cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+        cfg.blockDim = dim3(ModeT<MODE>::THREADS, 1, 1);
         cfg.dynamicSmemBytes = ModeT<MODE>::SMEM;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -641,7 +650,7 @@ cudaError_t launch_pair(size_t pair_tiles, int num_sms, const CUtensorMap& mA, c
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid_for<MODE>(pair_tiles, num_sms), 1, 1);
-    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.blockDim = dim3(ModeT<MODE>::THREADS, 1, 1);
     cfg.dynamicSmemBytes = ModeT<MODE>::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];

@@ -276,6 +276,14 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// The same arrive without release semantics: it orders nothing before it, so it
+// does not wait for the thread's outstanding global stores.  For signals that
+// only need the thread's own earlier waits to have finished (an accumulator
+// whose tcgen05.ld results are already in registers).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // Pair TMA loads: the box lands in this CTA's shared memory, completion bytes
 // are counted on the mbarrier at bar_cluster (the pair leader's barrier).
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0, int c1,

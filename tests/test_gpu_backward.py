@@ -156,3 +156,30 @@ def test_backward_configs(moe, cfg, n_tok):
     _check("dWg", _f64(g["dWg"]), want.cpu().numpy(), "f32", inp.T)
     del dev, g
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_training_forward_output_equals_prefill(moe, dtype):
+    """The training path only keeps more state: its output is the grouped-GEMM path's, bit for bit."""
+    inp = moe_inputs.make_inputs(333, 256, 384, 8, 2, dtype, seed=43) if dtype == "bf16" else \
+        moe_inputs.make_inputs(100, 96, 160, 8, 2, dtype, seed=43)
+    dev = upload(inp)
+    code = moe.MOE_DTYPE_BF16 if dtype == "bf16" else moe.MOE_DTYPE_F32
+    ws = torch.empty(moe.moe_train_workspace_size(inp.T, inp.d, inp.F, inp.E, inp.k, code), dtype=torch.uint8,
+                     device="cuda")
+    a = moe.moe_forward_ws(*dev, inp.k, path=moe.MOE_PATH_TRAIN, workspace=ws)
+    b = moe.moe_forward_ws(*dev, inp.k, path=moe.MOE_PATH_PREFILL)
+    _status_clear(moe)
+    assert torch.equal(a, b)
+
+
+def test_backward_rejects_inference_workspace(moe):
+    """A workspace sized for inference cannot hold the training state: the backward refuses it."""
+    inp = moe_inputs.make_inputs(200, 256, 512, 8, 2, "bf16", seed=44)
+    dev = upload(inp)
+    ws = torch.empty(moe.moe_workspace_size(inp.T, inp.d, inp.F, inp.E, inp.k), dtype=torch.uint8, device="cuda")
+    moe.moe_forward_ws(*dev, inp.k, path=moe.MOE_PATH_PREFILL, workspace=ws)
+    dout = to_dev(moe_inputs.make_dout(inp.T, inp.d, "bf16", seed=44), "bf16")
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_backward_ws(*dev, dout, inp.k, ws)
+    assert ei.value.status == moe.MOE_ERR_WORKSPACE
