@@ -321,6 +321,17 @@ def test_decode_host_entry_matches_device(moe, small):
     assert torch.equal(a.cpu(), b)
 
 
+def test_decode_host_entry_pageable_buffers(moe, small):
+    """Pageable host buffers go through the same copies, with the same result."""
+    _, dev = small
+    a = moe.moe_forward(*dev, 2)
+    x_host = dev[0].cpu()
+    out_host = torch.empty_like(x_host)
+    assert not x_host.is_pinned() and not out_host.is_pinned()
+    b = moe.moe_forward_host(x_host, *dev[1:], 2, out_host=out_host)
+    assert torch.equal(a.cpu(), b)
+
+
 def test_paths_agree_closely(moe, small):
     """Decode and grouped-GEMM paths compute the same function (different summation order)."""
     _, dev = small
