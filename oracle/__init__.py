@@ -25,8 +25,9 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   balance                  pinned: uniform scores (loss = alpha*k), cyclic
                            balanced batch, brute force against torch,
                            sums of f and p
-  backward / backward_tokens / weight_grad_slices
-                           pinned: central finite differences of moe();
+  backward / backward_tokens / weight_grad_slices / balance_grad
+                           pinned: central finite differences of moe() (and
+                           of moe() + balance() for the load-balance part);
                            torch autograd of the E=1 dense FFN and of the
                            k=E softmax mixture; slices and token rows equal
                            the full backward
@@ -81,9 +82,10 @@ def _load():
             lib.oracle_block.argtypes = [ci, ci, ci, ci, ci, vp, vp, cd, vp, vp, vp, vp, ci, vp, ci, vp, vp, vp,
                                          vp, vp, ci]
             lib.oracle_balance.argtypes = [ci, ci, ci, vp, cd, vp, vp, vp]
-            lib.oracle_backward.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp] + [vp] * 10
-            lib.oracle_backward_tokens.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, vp, ci] + \
+            lib.oracle_backward.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, cd] + [vp] * 10
+            lib.oracle_backward_tokens.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, cd, vp, ci] + \
                 [vp] * 6 + [ci]
+            lib.oracle_balance_grad.argtypes = [ci, ci, ci, vp, cd, vp]
             lib.oracle_weight_grad_slices.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, ci, vp, ci,
                                                       vp, vp, vp, ci]
             lib.oracle_max_threads.restype = ci
@@ -250,9 +252,9 @@ def balance(logits, k: int, alpha: float):
     return f, p, float(loss[0])
 
 
-def backward(x, Wg, W1, W3, W2, dout, k: int, dtype: str) -> dict:
-    """Every gradient of L = sum <dout, out> (small shapes): dict(dx, dlogits, dWg, dW1, dW3, dW2, idx, g,
-    margin, mingap), all float64."""
+def backward(x, Wg, W1, W3, W2, dout, k: int, dtype: str, alpha: float = 0.0) -> dict:
+    """Every gradient of L = sum <dout, out> + alpha E sum f p (small shapes): dict(dx, dlogits, dWg, dW1, dW3,
+    dW2, idx, g, margin, mingap), all float64."""
     x, Wg, W1, W3, W2, dout = (_arr(a, dtype) for a in (x, Wg, W1, W3, W2, dout))
     T, d = x.shape
     E, F = W1.shape[0], W1.shape[1]
@@ -260,13 +262,14 @@ def backward(x, Wg, W1, W3, W2, dout, k: int, dtype: str) -> dict:
              dW3=np.empty((E, F, d)), dW2=np.empty((E, d, F)), idx=np.empty((T, k), dtype=np.int32),
              g=np.empty((T, k)), margin=np.empty(T), mingap=np.empty(T))
     _check(_load().oracle_backward(T, d, F, E, k, x.ctypes.data, Wg.ctypes.data, W1.ctypes.data, W3.ctypes.data,
-                                   W2.ctypes.data, DTYPE_CODE[dtype], dout.ctypes.data,
+                                   W2.ctypes.data, DTYPE_CODE[dtype], dout.ctypes.data, float(alpha),
                                    *[r[n].ctypes.data for n in ("dx", "dlogits", "dWg", "dW1", "dW3", "dW2", "idx",
                                                                 "g", "margin", "mingap")]), "backward")
     return r
 
 
-def backward_tokens(x, Wg, W1, W3, W2, dout, k: int, dtype: str, tokens, nthreads: int = 0) -> dict:
+def backward_tokens(x, Wg, W1, W3, W2, dout, k: int, dtype: str, tokens, nthreads: int = 0,
+                    alpha: float = 0.0) -> dict:
     """dx and the router-score gradient of the listed tokens only: dict(dx, dlogits, idx, g, margin, mingap, tokens)."""
     x, Wg, W1, W3, W2, dout = (_arr(a, dtype) for a in (x, Wg, W1, W3, W2, dout))
     T, d = x.shape
@@ -277,7 +280,7 @@ def backward_tokens(x, Wg, W1, W3, W2, dout, k: int, dtype: str, tokens, nthread
              g=np.empty((n, k)), margin=np.empty(n), mingap=np.empty(n))
     _check(_load().oracle_backward_tokens(T, d, F, E, k, x.ctypes.data, Wg.ctypes.data, W1.ctypes.data,
                                           W3.ctypes.data, W2.ctypes.data, DTYPE_CODE[dtype], dout.ctypes.data,
-                                          tok.ctypes.data, n,
+                                          float(alpha), tok.ctypes.data, n,
                                           *[r[m].ctypes.data for m in ("dx", "dlogits", "idx", "g", "margin",
                                                                        "mingap")], nthreads), "backward_tokens")
     r["tokens"] = tok
@@ -297,3 +300,12 @@ def weight_grad_slices(x, Wg, W1, W3, W2, dout, k: int, dtype: str, e: int, fs, 
                                              int(e), f.ctypes.data, n, r1.ctypes.data, r3.ctypes.data,
                                              c2.ctypes.data, nthreads), "weight_grad_slices")
     return r1, r3, c2
+
+
+def balance_grad(logits, k: int, alpha: float) -> np.ndarray:
+    """Gradient of alpha E sum f p with respect to every score [T][E] (f held fixed)."""
+    s = np.ascontiguousarray(logits, dtype=np.float64)
+    T, E = s.shape
+    out = np.empty((T, E), dtype=np.float64)
+    _check(_load().oracle_balance_grad(T, E, k, s.ctypes.data, float(alpha), out.ctypes.data), "balance_grad")
+    return out

@@ -63,6 +63,12 @@
  *                        dW2_e += dy_j h^T, dW1_e += da x^T, dW3_e += db x^T,
  *                        dWg   += ds x^T
  *                      with SiLU'(a) = sigmoid(a) (1 + a (1 - sigmoid(a))).
+ *                      With alpha != 0 the loss also holds step 7's L_balance
+ *                      (the page's total loss L_LM + L_balance): f is piecewise
+ *                      constant, p = mean softmax(s), so each token's scores get
+ *                        ds_e += (alpha E / T) p_te (f_e - sum_m p_tm f_m)
+ *                      on every expert e, and that reaches dx and dWg through
+ *                      the router like the rest of ds.
  *
  * Operands are row-major: x[T][d], Wg[E][d], W1[E][F][d], W3[E][F][d],
  * W2[E][d][F].  dtype 0 = float32 storage, 1 = bfloat16 bit patterns; every
@@ -452,7 +458,7 @@ static void scratch_free(struct bwd_scratch* w) {
 static void token_backward(int d, int F, int E, int k, const void* x, const void* Wg, const void* W1, const void* W3,
                            const void* W2, int dtype, const void* dout, size_t t, struct bwd_scratch* w, double* dx,
                            double* ds, int32_t* idx, double* g, double* margin, double* mingap, double* dWg,
-                           double* dW1, double* dW3, double* dW2) {
+                           double* dW1, double* dW3, double* dW2, const double* ds_extra) {
     for (int j = 0; j < d; ++j) {
         w->xv[j] = elem(x, dtype, t * (size_t)d + j);
         w->go[j] = elem(dout, dtype, t * (size_t)d + j);
@@ -471,6 +477,8 @@ static void token_backward(int d, int F, int E, int k, const void* x, const void
     for (int j = 0; j < k; ++j) gdg += g[j] * dg[j];
     for (int e = 0; e < E; ++e) ds[e] = 0.0;
     for (int j = 0; j < k; ++j) ds[idx[j]] = g[j] * (dg[j] - gdg);
+    if (ds_extra)
+        for (int e = 0; e < E; ++e) ds[e] += ds_extra[e];
     /* router path: dx = Wg^T ds */
     for (int i = 0; i < d; ++i) {
         double acc = 0.0;
@@ -515,18 +523,71 @@ static void token_backward(int d, int F, int E, int k, const void* x, const void
 }
 
 /*
- * Every gradient of L = sum_t <dout_t, out_t> (step 8), tokens in order.
+ * Step 8's load-balance part from given scores logits[T][E]: the gradient of
+ * alpha E sum_e f_e p_e with respect to every score, f held fixed (it is
+ * piecewise constant): dbal[t][e] = (alpha E / T) p_te (f_e - sum_m p_tm f_m),
+ * p_t = softmax(s_t) over all E.
+ */
+int oracle_balance_grad(int T, int E, int k, const double* logits, double alpha, double* dbal) {
+    if (T <= 0 || E <= 0 || E > 64 || k <= 0 || k > E) return 1;
+    double f[64], p[64], loss;
+    if (oracle_balance(T, E, k, logits, alpha, f, p, &loss)) return 1;
+    const double c = alpha * (double)E / (double)T;
+    for (int t = 0; t < T; ++t) {
+        const double* s = logits + (size_t)t * E;
+        double mx = s[0];
+        for (int e = 1; e < E; ++e)
+            if (s[e] > mx) mx = s[e];
+        double den = 0.0;
+        for (int e = 0; e < E; ++e) den += exp(s[e] - mx);
+        double pf = 0.0;
+        for (int e = 0; e < E; ++e) {
+            p[e] = exp(s[e] - mx) / den;
+            pf += p[e] * f[e];
+        }
+        for (int e = 0; e < E; ++e) dbal[(size_t)t * E + e] = c * p[e] * (f[e] - pf);
+    }
+    return 0;
+}
+
+/* router scores of every token (step 1) and, when alpha != 0, the load-balance part of ds; NULL when alpha == 0 */
+static double* balance_part(int T, int d, int E, int k, const void* x, const void* Wg, int dtype, double alpha,
+                            int* fail) {
+    *fail = 0;
+    if (alpha == 0.0 || T <= 0) return NULL;
+    double* s = (double*)malloc(sizeof(double) * (size_t)T * E);
+    double* b = (double*)malloc(sizeof(double) * (size_t)T * E);
+    if (!s || !b) {
+        free(s);
+        free(b);
+        *fail = 2;
+        return NULL;
+    }
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int t = 0; t < T; ++t) token_scores(d, E, x, Wg, dtype, (size_t)t, s + (size_t)t * E);
+    if (oracle_balance_grad(T, E, k, s, alpha, b)) *fail = 1;
+    free(s);
+    return b;
+}
+
+/*
+ * Every gradient of L = sum_t <dout_t, out_t> (+ alpha L_balance) (step 8), tokens in order.
  * dx [T][d], dlogits [T][E] (the router-score gradient ds), dWg [E][d],
  * dW1/dW3 [E][F][d], dW2 [E][d][F]; idx/g [T][k], margin/mingap [T] as in
  * oracle_route.  Slow by design: for small shapes.
  */
 int oracle_backward(int T, int d, int F, int E, int k, const void* x, const void* Wg, const void* W1, const void* W3,
-                    const void* W2, int dtype, const void* dout, double* dx, double* dlogits, double* dWg, double* dW1,
-                    double* dW3, double* dW2, int32_t* idx, double* g, double* margin, double* mingap) {
+                    const void* W2, int dtype, const void* dout, double alpha, double* dx, double* dlogits,
+                    double* dWg, double* dW1, double* dW3, double* dW2, int32_t* idx, double* g, double* margin,
+                    double* mingap) {
     if (T < 0 || d <= 0 || F <= 0 || E <= 0 || E > 64 || k <= 0 || k > E) return 1;
+    int bfail = 0;
+    double* bal = balance_part(T, d, E, k, x, Wg, dtype, alpha, &bfail);
+    if (bfail) return bfail;
     struct bwd_scratch w;
     if (!scratch_alloc(&w, d, F, k)) {
         scratch_free(&w);
+        free(bal);
         return 2;
     }
     memset(dWg, 0, sizeof(double) * (size_t)E * d);
@@ -536,16 +597,17 @@ int oracle_backward(int T, int d, int F, int E, int k, const void* x, const void
     for (int t = 0; t < T; ++t)
         token_backward(d, F, E, k, x, Wg, W1, W3, W2, dtype, dout, (size_t)t, &w, dx + (size_t)t * d,
                        dlogits + (size_t)t * E, idx + (size_t)t * k, g + (size_t)t * k, margin + t, mingap + t, dWg,
-                       dW1, dW3, dW2);
+                       dW1, dW3, dW2, bal ? bal + (size_t)t * E : NULL);
     scratch_free(&w);
+    free(bal);
     return 0;
 }
 
 /* dx and ds of the listed tokens only (no weight gradients); rows in list order */
 int oracle_backward_tokens(int T, int d, int F, int E, int k, const void* x, const void* Wg, const void* W1,
-                           const void* W3, const void* W2, int dtype, const void* dout, const int32_t* tokens, int n,
-                           double* dx, double* dlogits, int32_t* idx, double* g, double* margin, double* mingap,
-                           int nthreads) {
+                           const void* W3, const void* W2, int dtype, const void* dout, double alpha,
+                           const int32_t* tokens, int n, double* dx, double* dlogits, int32_t* idx, double* g,
+                           double* margin, double* mingap, int nthreads) {
     if (T < 0 || d <= 0 || F <= 0 || E <= 0 || E > 64 || k <= 0 || k > E || n < 0) return 1;
     for (int r = 0; r < n; ++r)
         if (tokens[r] < 0 || tokens[r] >= T) return 1;
@@ -553,6 +615,9 @@ int oracle_backward_tokens(int T, int d, int F, int E, int k, const void* x, con
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #endif
+    int bfail = 0;
+    double* bal = balance_part(T, d, E, k, x, Wg, dtype, alpha, &bfail);
+    if (bfail) return bfail;
 #pragma omp parallel
     {
         struct bwd_scratch w;
@@ -564,10 +629,12 @@ int oracle_backward_tokens(int T, int d, int F, int E, int k, const void* x, con
             for (int r = 0; r < n; ++r)
                 token_backward(d, F, E, k, x, Wg, W1, W3, W2, dtype, dout, (size_t)tokens[r], &w,
                                dx + (size_t)r * d, dlogits + (size_t)r * E, idx + (size_t)r * k, g + (size_t)r * k,
-                               margin + r, mingap + r, NULL, NULL, NULL, NULL);
+                               margin + r, mingap + r, NULL, NULL, NULL, NULL,
+                               bal ? bal + (size_t)tokens[r] * E : NULL);
         }
         scratch_free(&w);
     }
+    free(bal);
     return fail ? 2 : 0;
 }
 

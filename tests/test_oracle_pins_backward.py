@@ -11,6 +11,10 @@
     so the layer is the dense softmax mixture sum_e softmax(Wg x)_e E_e(x);
     torch autograd of that expression gives every gradient, dWg included
   * the token-subset and weight-slice forms equal the full backward
+  * load-balance part (alpha != 0): finite differences of L + alpha E sum f p
+    (f computed by oracle.balance on the perturbed scores, routing unchanged);
+    torch autograd of alpha E sum_e f_e mean_t softmax(s_t)_e with f fixed; with
+    k = E every f_e = 1, the loss is the constant alpha E and its gradient 0
 """
 import numpy as np
 import pytest
@@ -130,3 +134,57 @@ def test_router_gradient_sums_to_zero_over_selected():
     sel = np.zeros_like(g["dlogits"], dtype=bool)
     np.put_along_axis(sel, g["idx"], True, axis=1)
     assert np.all(g["dlogits"][~sel] == 0.0)
+
+
+def _loss_bal(inp, dout, k, alpha):
+    r = oracle.moe(*inp.arrays(), k=k, dtype="f32")
+    _, _, lb = oracle.balance(oracle.scores(inp.x, inp.Wg, "f32"), k, alpha)
+    return float((r["out"] * dout.astype(np.float64)).sum()) + lb, r["idx"]
+
+
+def test_finite_differences_with_balance_loss():
+    T, d, F, E, k, alpha = 5, 8, 16, 4, 2, 0.7
+    inp = moe_inputs.make_inputs(T, d, F, E, k, "f32", seed=36)
+    dout = _dout(T, d, "f32", 36)
+    g = oracle.backward(*inp.arrays(), dout, k, "f32", alpha=alpha)
+    _, idx0 = _loss_bal(inp, dout, k, alpha)
+    h = 2.0 ** -12
+    checked = 0
+    for name, grad in (("x", g["dx"]), ("Wg", g["dWg"])):
+        flat = getattr(inp, name).reshape(-1)
+        for i in range(flat.size):
+            v = flat[i]
+            flat[i] = np.float32(v + h)
+            hp = float(flat[i]) - float(v)
+            lp, ip = _loss_bal(inp, dout, k, alpha)
+            flat[i] = np.float32(v - h)
+            hm = float(v) - float(flat[i])
+            lm, im = _loss_bal(inp, dout, k, alpha)
+            flat[i] = v
+            if not (np.array_equal(ip, idx0) and np.array_equal(im, idx0)):
+                continue
+            fd = (lp - lm) / (hp + hm)
+            an = grad.reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * (1 + abs(an)), (name, i, fd, an)
+            checked += 1
+    assert checked > 60
+    # the expert weights do not see the balance loss
+    g0 = oracle.backward(*inp.arrays(), dout, k, "f32")
+    for n in ("dW1", "dW3", "dW2"):
+        assert np.array_equal(g[n], g0[n])
+
+
+def test_balance_grad_matches_torch():
+    rng = np.random.default_rng(37)
+    s = rng.standard_normal((40, 6))
+    k, alpha = 2, 0.3
+    f, _, _ = oracle.balance(s, k, alpha)
+    st = _t64(s).requires_grad_()
+    loss = alpha * 6 * (_t64(f) * torch.softmax(st, dim=1).mean(dim=0)).sum()
+    loss.backward()
+    assert np.allclose(oracle.balance_grad(s, k, alpha), st.grad.numpy(), rtol=1e-12, atol=1e-15)
+
+
+def test_balance_grad_vanishes_when_every_expert_is_selected():
+    s = np.random.default_rng(38).standard_normal((25, 5))
+    assert np.allclose(oracle.balance_grad(s, 5, 1.3), 0.0, atol=1e-16)
