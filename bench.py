@@ -221,15 +221,15 @@ def oracle_train_run(inp, dout, target_s):
     sub = lambda toks: [np.ascontiguousarray(inp.x[toks]), inp.Wg, inp.W1, inp.W3, inp.W2,
                         np.ascontiguousarray(dout[toks])]
     t0 = time.perf_counter()
-    oracle.backward(*sub([0]), inp.k, inp.dtype)
+    oracle.backward(*sub([0]), inp.k, inp.dtype, alpha=BLOCK_ALPHA)
     per_tok = max(time.perf_counter() - t0, 1e-5)
     n = int(max(1, min(inp.T, round(target_s / per_tok))))
     toks = np.unique(np.linspace(0, inp.T - 1, n).astype(np.int64))
     t0 = time.perf_counter()
-    oracle.backward(*sub(toks), inp.k, inp.dtype)
+    oracle.backward(*sub(toks), inp.k, inp.dtype, alpha=BLOCK_ALPHA)
     dt = time.perf_counter() - t0
-    sample = (f"{len(toks)} of {inp.T} tokens (evenly spaced): forward and every gradient (dx, dWg, dW1, dW3, dW2) "
-              f"of those tokens in fp64, one thread")
+    sample = (f"{len(toks)} of {inp.T} tokens (evenly spaced): forward and every gradient (dx, dWg, dW1, dW3, dW2, "
+              f"load-balance loss included) of those tokens in fp64, one thread")
     return len(toks) / dt, sample, dt
 
 
@@ -516,7 +516,8 @@ def run_ours(args, rank, world, local):
 
 
 def run_train(args, rank, world, local):
-    """One step = moe_forward_ws (grouped-GEMM path) + moe_backward_ws over one batch, inputs resident."""
+    """One step = moe_forward_profiled (training path) + moe_backward_ws with the load-balance loss
+    (alpha = 0.01) over one batch, inputs resident."""
     import sparse_mixture_experts_14_b200 as moe
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -563,7 +564,8 @@ def run_train(args, rank, world, local):
     def step(i=None):
         on = i is not None and i % every == 0
         n = moe.moe_forward_profiled(*dev, k, fws, out, events=fev[i] if on else None, path=moe.MOE_PATH_TRAIN)
-        _, m = moe.moe_backward_ws(*dev, dout, k, fws, workspace=bws, grads=grads, events=bev[i] if on else None)
+        _, m = moe.moe_backward_ws(*dev, dout, k, fws, workspace=bws, grads=grads, alpha=BLOCK_ALPHA,
+                                   events=bev[i] if on else None)
         return n + m
 
     for _ in range(W):

@@ -330,8 +330,11 @@ MOE_API moe_status moe_route_stats_f32(const float* x, const float* Wg, int T, i
  *   dx = sum_j (W1^T da + W3^T db) + Wg^T ds
  *   dW2 += dy h^T,  dW1 += da x^T,  dW3 += db x^T,  dWg += ds x^T
  *
- * The gradient of the load-balance loss is not included (its p term depends
- * on the scores; add it through dlogits if needed).
+ * With alpha != 0 the loss also holds the load-balance loss alpha E sum f p
+ * of the forward's routing (the page's total loss L_LM + L_balance): f is
+ * piecewise constant, so every score of token t gets
+ *   ds_te += (alpha E / T) softmax(s_t)_e (f_e - sum_m softmax(s_t)_m f_m)
+ * before ds reaches dx and dWg.  alpha = 0 gives the output path alone.
  *
  * Use: run moe_forward_ws (or moe_forward_profiled) with MOE_PATH_TRAIN and
  * a workspace of moe_train_workspace_size() bytes on the same operands, then
@@ -341,7 +344,7 @@ MOE_API moe_status moe_route_stats_f32(const float* x, const float* Wg, int T, i
  * (device, 256-byte aligned).  Outputs (device, overwritten): dx [T][d] in
  * the layer's element type; dWg [E][d], dW1 [E][F][d], dW3 [E][F][d] and
  * dW2 [E][d][F] in float; dlogits [T][E] float (optional, NULL allowed): the
- * gradient of the router scores, zero for unselected experts.  Every sum runs
+ * gradient of the router scores (zero for unselected experts when alpha = 0).  Every sum runs
  * in a fixed order (no float atomics), so results are bitwise repeatable.
  * stage_events (optional) receives MOE_BWD_NUM_STAGES + 1 events as in
  * moe_forward_profiled; launches (optional) the number of kernels launched.
@@ -361,8 +364,8 @@ MOE_API size_t moe_backward_workspace_size(int T, int d, int ffn, int E, int k, 
 
 MOE_API moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const void* W3,
                                    const void* W2, const void* dout, void* dx, float* dWg, float* dW1,
-                                   float* dW3, float* dW2, float* dlogits, int T, int d, int ffn, int E,
-                                   int k, int dtype, const void* fwd_workspace, size_t fwd_workspace_bytes,
+                                   float* dW3, float* dW2, float* dlogits, float alpha, int T, int d, int ffn,
+                                   int E, int k, int dtype, const void* fwd_workspace, size_t fwd_workspace_bytes,
                                    void* workspace, size_t workspace_bytes, cudaEvent_t* stage_events,
                                    int* launches, cudaStream_t stream);
 

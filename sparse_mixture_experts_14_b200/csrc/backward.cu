@@ -12,6 +12,9 @@
 //     dH     = dY W2_e,  dA, dB = SwiGLU backward,  dXp = dA W1_e + dB W3_e
 //     dW2_e  = dY_e^T H_e,  dW1_e = dA_e^T Xp_e,  dW3_e = dB_e^T Xp_e
 //     dWg    = ds^T x,      dx_t = sum_j dXp[slot(t, j)] + ds_t Wg
+// With alpha != 0 the loss also holds alpha L_balance (f = counts / T held
+// fixed, p_t = softmax(s_t) over all E): every score of token t gets
+//     ds_te += (alpha E / T) p_te (f_e - sum_m p_tm f_m)
 // Every sum runs in a fixed order (no float atomics), so the gradients are
 // the same bits on every run.
 //
@@ -97,10 +100,12 @@ __global__ void __launch_bounds__(256) bwd_scatter_kernel(const T* __restrict__ 
     }
 }
 
-// ds[t][e]: the gradient of the router scores (zero for unselected experts).
+// ds[t][e]: the gradient of the router scores (output path: zero for unselected
+// experts; with alpha != 0 plus the load-balance part on every expert).
 __global__ void __launch_bounds__(256) router_bwd_kernel(const int32_t* __restrict__ idx, const float* __restrict__ w,
-                                                         const float* __restrict__ dg, int T_, int E, int k,
-                                                         float* __restrict__ ds) {
+                                                         const float* __restrict__ dg, const float* __restrict__ logits,
+                                                         const Meta* __restrict__ meta, float alpha, int T_, int E,
+                                                         int k, float* __restrict__ ds) {
     pdl_trigger();
     pdl_wait();
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -112,6 +117,19 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const int32_t* __restri
     for (int j = 0; j < k; ++j) {
         const int e = idx[(size_t)t * k + j];
         if (e >= 0 && e < E) row[e] = w[(size_t)t * k + j] * (dg[(size_t)t * k + j] - gdg);
+    }
+    if (alpha != 0.f) {
+        const float* s = logits + (size_t)t * E;
+        float mx = -INFINITY, den = 0.f, pf = 0.f;
+        for (int e = 0; e < E; ++e) mx = fmaxf(mx, s[e]);
+        for (int e = 0; e < E; ++e) den += expf(s[e] - mx);
+        const float invT = 1.0f / (float)T_;
+        for (int e = 0; e < E; ++e) pf += expf(s[e] - mx) / den * ((float)meta->counts[e] * invT);
+        const float c = alpha * (float)E * invT;
+        for (int e = 0; e < E; ++e) {
+            const float p = expf(s[e] - mx) / den;
+            row[e] += c * p * ((float)meta->counts[e] * invT - pf);
+        }
     }
 }
 
@@ -169,13 +187,12 @@ __global__ void __launch_bounds__(256) dwg_final_kernel(const float* __restrict_
     }
 }
 
-// dx[t] = sum_j dXp[inv[t][j]] + sum_j ds[t][idx[t][j]] Wg[idx[t][j]], both j ascending, in fp32,
-// rounded once; four columns per thread (d % 4 == 0 on both paths).
+// dx[t] = sum_j dXp[inv[t][j]] (j ascending) + sum_e ds[t][e] Wg[e] (e ascending, nonzero ds only),
+// in fp32, rounded once; four columns per thread (d % 4 == 0 on both paths).
 template <typename T>
 __global__ void __launch_bounds__(256) dx_combine_kernel(const float* __restrict__ dXp, const int32_t* __restrict__ inv,
-                                                         const int32_t* __restrict__ idx, const float* __restrict__ ds,
-                                                         const T* __restrict__ Wg, int T_, int d, int E, int k,
-                                                         T* __restrict__ dx) {
+                                                         const float* __restrict__ ds, const T* __restrict__ Wg, int T_,
+                                                         int d, int E, int k, T* __restrict__ dx) {
     pdl_trigger();
     pdl_wait();
     const unsigned q = (unsigned)d / 4;
@@ -193,10 +210,9 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float* __restrict
             acc.z += v.z;
             acc.w += v.w;
         }
-        for (int j = 0; j < k; ++j) {
-            const int e = idx[(size_t)t * k + j];
-            if (e < 0 || e >= E) continue;
+        for (int e = 0; e < E; ++e) {
             const float s = ds[(size_t)t * E + e];
+            if (s == 0.f) continue;
             float w[4];
             if (sizeof(T) == 2) {
                 const uint2 u = __ldg(reinterpret_cast<const uint2*>(Wg + (size_t)e * d) + c);
@@ -381,7 +397,7 @@ cudaError_t launch_dx(const BwdArgs& a, cudaStream_t s) {
     if (blocks > 148 * 32) blocks = 148 * 32;
     if (blocks < 1) blocks = 1;
     return launch_pdl(dx_combine_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const float*>(a.dxp),
-                      a.inv, a.idx, static_cast<const float*>(a.ds), static_cast<const T*>(a.Wg), a.T, a.d, a.E, a.k,
+                      a.inv, static_cast<const float*>(a.ds), static_cast<const T*>(a.Wg), a.T, a.d, a.E, a.k,
                       static_cast<T*>(a.dx));
 }
 
@@ -398,7 +414,8 @@ cudaError_t launch_bwd_scatter(const BwdArgs& a, cudaStream_t s) {
 
 cudaError_t launch_router_bwd(const BwdArgs& a, cudaStream_t s) {
     return launch_pdl(router_bwd_kernel, dim3((a.T + 255) / 256), dim3(256), 0, s, a.idx, a.w,
-                      static_cast<const float*>(a.dg), a.T, a.E, a.k, a.ds);
+                      static_cast<const float*>(a.dg), a.logits, static_cast<const Meta*>(a.meta), a.alpha, a.T, a.E,
+                      a.k, a.ds);
 }
 
 cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s) {

@@ -112,6 +112,7 @@ struct Plan {
     size_t idx, w, blk, meta, perm, inv, xp, h, y;
     size_t rstd, logits, bal;   // block form only (see make_plan's `block`)
     size_t keep_a, keep_b;      // training path, bf16: GEMM1's a and b, fp32 [slots][F]
+    size_t tlogits;             // training path: the router scores, fp32 [T][E]
     size_t total;
     size_t slots;
 };
@@ -142,6 +143,7 @@ Plan make_plan(int T, int d, int F, int E, int k, int dtype, bool block = false,
         p.keep_a = take(p.slots * (size_t)F * 4);
         p.keep_b = take(p.slots * (size_t)F * 4);
     }
+    if (train) p.tlogits = take((size_t)T * E * 4);
     if (block) {
         p.rstd = take((size_t)T * 4);
         p.logits = take((size_t)T * E * 4);
@@ -184,6 +186,7 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
         nm.rstd = ex.rstd;
     }
     const void* resid = bo ? x : nullptr;
+    if (train) ex.logits = reinterpret_cast<float*>(ws + p.tlogits);   // kept for the load-balance gradient
     int32_t* idx = reinterpret_cast<int32_t*>(ws + p.idx);
     float* w = reinterpret_cast<float*>(ws + p.w);
     int32_t* blk = reinterpret_cast<int32_t*>(ws + p.blk);
@@ -356,7 +359,7 @@ BwdPlan make_bwd_plan(int T, int d, int F, int E, int k, int dtype) {
 
 moe_status run_backward(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2,
                         const void* dout, void* dx, float* dWg, float* dW1, float* dW3, float* dW2, float* dlogits,
-                        int T, int d, int F, int E, int k, int dtype, const uint8_t* fws, uint8_t* bws,
+                        float alpha, int T, int d, int F, int E, int k, int dtype, const uint8_t* fws, uint8_t* bws,
                         const DeviceState& dev, cudaStream_t s, cudaEvent_t* ev, int* launches) {
     const Plan p = make_plan(T, d, F, E, k, dtype, false, true);
     const BwdPlan b = make_bwd_plan(T, d, F, E, k, dtype);
@@ -377,6 +380,8 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
     a.xp = fw + p.xp;
     a.H = fw + p.h;
     a.Y = reinterpret_cast<const float*>(fw + p.y);
+    a.logits = reinterpret_cast<const float*>(fw + p.tlogits);
+    a.alpha = alpha;
     if (dtype == MOE_DTYPE_BF16) {
         a.keep_a = reinterpret_cast<const float*>(fw + p.keep_a);
         a.keep_b = reinterpret_cast<const float*>(fw + p.keep_b);
@@ -721,7 +726,7 @@ size_t moe_backward_workspace_size(int T, int d, int ffn, int E, int k, int dtyp
 
 moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2,
                            const void* dout, void* dx, float* dWg, float* dW1, float* dW3, float* dW2, float* dlogits,
-                           int T, int d, int ffn, int E, int k, int dtype, const void* fwd_workspace,
+                           float alpha, int T, int d, int ffn, int E, int k, int dtype, const void* fwd_workspace,
                            size_t fwd_workspace_bytes, void* workspace, size_t workspace_bytes,
                            cudaEvent_t* stage_events, int* launches, cudaStream_t stream) {
     if (launches) *launches = 0;
@@ -732,13 +737,14 @@ moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const 
     for (const void* q : ptrs)
         if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
     if (dlogits && (reinterpret_cast<uintptr_t>(dlogits) & 3u) != 0) return MOE_ERR_INVALID_ARG;
+    if (!(alpha == alpha) || !(alpha - alpha == 0.f)) return MOE_ERR_INVALID_ARG;
     if (!fwd_workspace || (reinterpret_cast<uintptr_t>(fwd_workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (fwd_workspace_bytes < make_plan(T, d, ffn, E, k, dtype, false, true).total) return MOE_ERR_WORKSPACE;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (workspace_bytes < make_bwd_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
     DeviceState dev;
     if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
-    return run_backward(x, Wg, W1, W3, W2, dout, dx, dWg, dW1, dW3, dW2, dlogits, T, d, ffn, E, k, dtype,
+    return run_backward(x, Wg, W1, W3, W2, dout, dx, dWg, dW1, dW3, dW2, dlogits, alpha, T, d, ffn, E, k, dtype,
                         static_cast<const uint8_t*>(fwd_workspace), static_cast<uint8_t*>(workspace), dev, stream,
                         stage_events, launches);
 }

@@ -258,6 +258,8 @@ struct BwdArgs {
     const float* Y;         // [slots][d]
     const float* keep_a;    // [slots][F] fp32 (bf16 training path), else null
     const float* keep_b;
+    const float* logits;    // [T][E] fp32 router scores kept by the training forward
+    float alpha;            // load-balance loss coefficient (0: output-path gradient only)
     // backward buffers
     void* dy;               // [slots][d]
     float* dg;              // [T][k]

@@ -43,14 +43,14 @@ def _status_clear(moe):
     assert moe.moe_get_device_status() == moe.MOE_OK
 
 
-def _run(moe, inp, dev, dout_d, dlogits=False):
+def _run(moe, inp, dev, dout_d, dlogits=False, alpha=0.0):
     x, Wg, W1, W3, W2 = dev
     code = moe.MOE_DTYPE_BF16 if inp.dtype == "bf16" else moe.MOE_DTYPE_F32
     fws = torch.empty(moe.moe_train_workspace_size(inp.T, inp.d, inp.F, inp.E, inp.k, code), dtype=torch.uint8,
                       device="cuda")
     out = moe.moe_forward_ws(x, Wg, W1, W3, W2, inp.k, path=moe.MOE_PATH_TRAIN, workspace=fws)
     dl = torch.empty((inp.T, inp.E), dtype=torch.float32, device="cuda") if dlogits else None
-    grads, n = moe.moe_backward_ws(x, Wg, W1, W3, W2, dout_d, inp.k, fws, dlogits=dl)
+    grads, n = moe.moe_backward_ws(x, Wg, W1, W3, W2, dout_d, inp.k, fws, dlogits=dl, alpha=alpha)
     _status_clear(moe)
     if dl is not None:
         grads["dlogits"] = dl
@@ -183,3 +183,25 @@ def test_backward_rejects_inference_workspace(moe):
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_backward_ws(*dev, dout, inp.k, ws)
     assert ei.value.status == moe.MOE_ERR_WORKSPACE
+
+
+
+@pytest.mark.parametrize("dtype,T,d,F,E,k", [("bf16", 300, 256, 384, 8, 2), ("f32", 96, 128, 160, 6, 2)])
+def test_backward_with_balance_loss(moe, dtype, T, d, F, E, k):
+    """alpha != 0 adds the load-balance loss: the router-score gradient gains its part on every
+    expert (dx and dWg follow), the expert weight gradients stay bit for bit the same."""
+    alpha = 0.5
+    inp = moe_inputs.make_inputs(T, d, F, E, k, dtype, seed=T + 7)
+    dout = moe_inputs.make_dout(T, d, dtype, seed=T + 7)
+    dev = upload(inp)
+    _, g0, _ = _run(moe, inp, dev, to_dev(dout, dtype), dlogits=True)
+    _, g, _ = _run(moe, inp, dev, to_dev(dout, dtype), dlogits=True, alpha=alpha)
+    for n in ("dW1", "dW3", "dW2"):
+        assert torch.equal(g[n], g0[n]), n
+    ref = oracle.backward(*inp.arrays(), dout, k, dtype, alpha=alpha)
+    if not (ref["margin"] >= MARGIN).all():
+        pytest.skip("a token sits within the routing margin")
+    K = max(d, F, T)
+    for n in ("dx", "dlogits", "dWg"):
+        _check(n, _f64(g[n]), ref[n], dtype, K)
+    assert torch.count_nonzero(g["dlogits"]) > torch.count_nonzero(g0["dlogits"])
