@@ -306,9 +306,15 @@ cudaError_t launch_stage(const CUtensorMap& a, const CUtensorMap& b, const CUten
                                     dsmem_bytes<GATE>());
     });
     if (e != cudaSuccess) return e;
-    int grid = g.num_sms > 0 ? g.num_sms : 148;
+    // As many waves as one CTA per SM needs, then as few CTAs as cover the tiles in that many
+    // waves: every CTA gets the same number of tiles, so no short last wave leaves most SMs idle
+    // while a few stream alone (896 tiles of stage 1 at E = 8: 7 waves on 128 CTAs, not 6 and a
+    // tail of 8 on 148).  The tile count assumes every expert has tokens, as at decode sizes.
+    const int sms = g.num_sms > 0 ? g.num_sms : 148;
     const int upper = g.E * ((R + DM - 1) / DM);
-    if (grid > upper) grid = upper;
+    const int waves = (upper + sms - 1) / sms;
+    int grid = (upper + waves - 1) / waves;
+    if (grid > sms) grid = sms;
     if (grid < 1) grid = 1;
     return launch_pdl(decode_kernel<GATE>, dim3(grid), dim3(DTHREADS), dsmem_bytes<GATE>(), s, a, b, x, g.meta, g.E, K, R, out,
                       g.status, g.wait_ns);
