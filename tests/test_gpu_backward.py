@@ -125,27 +125,32 @@ def test_backward_experts_without_tokens(moe):
     _check("dx", _f64(g["dx"]), ref["dx"], "bf16")
 
 
-@pytest.mark.parametrize("cfg,n_tok", [(1, 0), (3, 12)])
-def test_backward_configs(moe, cfg, n_tok):
-    """Full-size workloads: dx and dlogits on sampled tokens, slices of every expert's weight
-    gradients, and dWg against the GPU's own dlogits reduced on the host."""
+@pytest.mark.parametrize("cfg,n_tok,alpha", [(1, 0, 0.0), (1, 0, 0.5), (3, 12, 0.0), (3, 8, 0.01), (5, 6, 0.0)])
+def test_backward_configs(moe, cfg, n_tok, alpha):
+    """Full-size workloads (in the launch configuration bench.py --train times): dx and dlogits on
+    sampled tokens, slices of the weight gradients of two experts, and dWg against the GPU's own
+    dlogits reduced on the host; alpha != 0 includes the load-balance loss."""
     inp = moe_inputs.make_config(cfg)
     dtype = inp.dtype
     dout = moe_inputs.make_dout(inp.T, inp.d, dtype, seed=inp.seed)
     dev = upload(inp)
-    _, g, _ = _run(moe, inp, dev, to_dev(dout, dtype), dlogits=True)
+    _, g, _ = _run(moe, inp, dev, to_dev(dout, dtype), dlogits=True, alpha=alpha)
     K = max(inp.d, inp.F, inp.T)
     if n_tok == 0:
-        ref = oracle.backward(*inp.arrays(), dout, inp.k, dtype)
+        ref = oracle.backward(*inp.arrays(), dout, inp.k, dtype, alpha=alpha)
         for n in ("dx", "dlogits", "dWg", "dW1", "dW3", "dW2"):
             _check(n, _f64(g[n]), ref[n], dtype, K)
         return
     toks = sample_tokens(inp.T, n_tok, seed=cfg)
-    ref = oracle.backward_tokens(*inp.arrays(), dout, inp.k, dtype, toks)
+    ref = oracle.backward_tokens(*inp.arrays(), dout, inp.k, dtype, toks, alpha=alpha)
     keep = ref["margin"] >= MARGIN
     _check("dx", _f64(g["dx"])[toks][keep], ref["dx"][keep], dtype)
     _check("dlogits", _f64(g["dlogits"])[toks][keep], ref["dlogits"][keep], dtype)
     fs = [0, 777, inp.F - 1]
+    if alpha != 0.0:   # the expert weight gradients do not see the balance loss
+        del dev, g
+        torch.cuda.empty_cache()
+        return
     for e in (0, inp.E - 1):
         r1, r3, c2 = oracle.weight_grad_slices(*inp.arrays(), dout, inp.k, dtype, e, fs)
         _check(f"dW1[{e}]", _f64(g["dW1"][e][fs]), r1, dtype)
