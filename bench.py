@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(moe_inputs.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU-oracle sample")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="target length of the whole --impl reference run (warm-up + timed steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--block", action="store_true",
@@ -279,7 +281,7 @@ def run_reference(args, rank):
     inp = make_workload(args.config, args.block, args.shape)
     if args.train:
         dout = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
-        per_step = max(0.5, min(30.0, 150.0 / max(args.steps + args.warmup, 1)))
+        per_step = max(0.05, min(30.0, args.ref_seconds / max(args.steps + args.warmup, 1)))
         for _ in range(args.warmup):
             oracle_train_run(inp, dout, per_step)
         total_tok, total_t = 0.0, 0.0
@@ -303,7 +305,7 @@ def run_reference(args, rank):
     run = oracle_fn(inp, args.block)
     threads = len(os.sched_getaffinity(0))
     total_steps = args.steps + args.warmup
-    per_step = max(0.5, min(30.0, 150.0 / max(total_steps, 1)))
+    per_step = max(0.05, min(30.0, args.ref_seconds / max(total_steps, 1)))
     t0 = time.perf_counter()
     run([0], 1)
     per_tok = max(time.perf_counter() - t0, 1e-5)
