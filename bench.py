@@ -59,7 +59,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(moe_inputs.CONFIGS))
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(moe_inputs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU-oracle sample")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
@@ -237,7 +237,7 @@ def oracle_train_run(inp, dout, target_s):
 
 def make_workload(cfg, block, shape=None):
     if shape:
-        c = moe_inputs.CONFIGS[cfg]
+        c = moe_inputs.WORKLOADS[cfg]
         T, d, F = (int(v) for v in shape.split(","))
         inp = moe_inputs.make_inputs(T, d, F, c["E"], c["k"], c["dtype"], c["seed"], c["skew"])
     else:
@@ -246,7 +246,7 @@ def make_workload(cfg, block, shape=None):
 
 
 def workload_name(cfg, shape=None):
-    c = moe_inputs.CONFIGS[cfg]
+    c = moe_inputs.WORKLOADS[cfg]
     return c["name"] + (f"@shape={shape}" if shape else "")
 
 
@@ -277,7 +277,7 @@ def cpu_oracle_run(inp, target_s, threads, block=False):
 def run_reference(args, rank):
     if rank != 0:
         return
-    c = moe_inputs.CONFIGS[args.config]
+    c = moe_inputs.WORKLOADS[args.config]
     inp = make_workload(args.config, args.block, args.shape)
     if args.train:
         dout = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
@@ -359,7 +359,7 @@ def run_ours(args, rank, world, local):
     import sparse_mixture_experts_14_b200 as moe
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    c = moe_inputs.CONFIGS[args.config]
+    c = moe_inputs.WORKLOADS[args.config]
     block = args.block
     inp = make_workload(args.config, block, args.shape)
     dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
@@ -523,7 +523,7 @@ def run_train(args, rank, world, local):
     import sparse_mixture_experts_14_b200 as moe
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    c = moe_inputs.CONFIGS[args.config]
+    c = moe_inputs.WORKLOADS[args.config]
     inp = make_workload(args.config, False, args.shape)
     dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
     dout_np = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)

@@ -75,7 +75,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1,  /* null pointer, negative size, k > E, misaligned pointer */
-    MOE_ERR_UNSUPPORTED = 2,  /* valid layer, but a size this build does not handle */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid layer, but a size this library does not handle */
     MOE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
     MOE_ERR_TIMEOUT = 4,      /* device: a pipeline wait ran past its time limit */
     MOE_ERR_WORKSPACE = 5,    /* workspace missing or smaller than moe_workspace_size() */

@@ -192,7 +192,7 @@ def make_block(inp: MoEInputs) -> MoEInputs:
 
 
 # The five named workloads (sizes, dtype, seed, routing recipe).
-CONFIGS = {
+WORKLOADS = {
     1: dict(name="tiny-f32", T=64, d=128, F=256, E=8, k=2, dtype="f32", seed=0, skew=False),
     2: dict(name="mixtral-8x7b-decode", T=16, d=4096, F=14336, E=8, k=2, dtype="bf16", seed=1, skew=False),
     3: dict(name="mixtral-8x7b-prefill", T=4096, d=4096, F=14336, E=8, k=2, dtype="bf16", seed=2, skew=False),
@@ -202,6 +202,6 @@ CONFIGS = {
 
 
 def make_config(cfg: int, weights: bool = True, T: int | None = None) -> MoEInputs:
-    c = CONFIGS[cfg]
+    c = WORKLOADS[cfg]
     return make_inputs(T if T is not None else c["T"], c["d"], c["F"], c["E"], c["k"], c["dtype"],
                        c["seed"], c["skew"], weights=weights)

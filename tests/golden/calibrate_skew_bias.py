@@ -40,7 +40,7 @@ def shares(z, b, k):
 
 
 def main():
-    c = moe_inputs.CONFIGS[4]
+    c = moe_inputs.WORKLOADS[4]
     T, d, E, k = c["T"], c["d"], c["E"], c["k"]
     inp = moe_inputs.make_inputs(T, d, c["F"], E, k, c["dtype"], c["seed"], bias=[0.0] * E, weights=False)
     z = oracle.scores(inp.x, inp.Wg, c["dtype"])

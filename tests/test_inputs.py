@@ -105,6 +105,6 @@ def test_skew_bias_file_is_bf16_exact():
 
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
 def test_config_table(cfg):
-    c = moe_inputs.CONFIGS[cfg]
+    c = moe_inputs.WORKLOADS[cfg]
     assert c["k"] == 2 and c["E"] == 8
     assert c["dtype"] == ("f32" if cfg == 1 else "bf16")
