@@ -183,7 +183,9 @@ MOE_API size_t moe_workspace_size(int T, int d, int ffn, int E, int k, int dtype
  * moe_forward / moe_forward_f32 with a caller-provided device workspace of
  * at least moe_workspace_size() bytes (256-byte aligned), and an explicit
  * path (MOE_PATH_*; the decode path needs dtype == MOE_DTYPE_BF16).  The
- * workspace must not be in use by another call in flight.
+ * workspace must not be in use by another call in flight.  After one call on
+ * a device, calls can be captured into a CUDA graph (stream capture) and the
+ * graph replayed with the same operands and workspace.
  */
 MOE_API moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1, const void* W3,
                           const void* W2, void* out, int T, int d, int ffn, int E, int k,

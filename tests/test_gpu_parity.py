@@ -339,3 +339,26 @@ def test_paths_agree_closely(moe, small):
     b = moe.moe_forward_ws(*dev, 2, path=moe.MOE_PATH_PREFILL).float()
     rms = b.pow(2).mean().sqrt()
     assert (a - b).abs().max() <= 1e-2 * rms
+
+
+@pytest.mark.parametrize("T", [16, 700])
+def test_forward_ws_graph_capture(moe, T):
+    """moe_forward_ws with a caller workspace can be captured into a CUDA graph and replayed
+    (decode path at T=16, grouped GEMMs at T=700); the replay gives the eager result bit for bit."""
+    inp = moe_inputs.make_inputs(T, 256, 512, 8, 2, "bf16", seed=900 + T)
+    dev = upload(inp)
+    ws = torch.empty(moe.moe_workspace_size(T, 256, 512, 8, 2), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(dev[0])
+    moe.moe_forward_ws(*dev, 2, workspace=ws, out=out)   # first call: per-device set-up outside capture
+    torch.cuda.synchronize()
+    want = out.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_forward_ws(*dev, 2, workspace=ws, out=out)
+    out.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    _status_clear(moe)
+    assert torch.equal(out, want)
+    del g
