@@ -73,6 +73,8 @@ def parse_args():
                          "for profiler captures small enough to stay within a few GB")
     ap.add_argument("--train", action="store_true",
                     help="time a training step: forward (grouped-GEMM path) + backward with all gradients")
+    ap.add_argument("--bf16-wgrad", action="store_true",
+                    help="with --train: weight gradients rounded to bf16 in the GEMM epilogue (fp32 otherwise)")
     ap.add_argument("--stage-every", type=int, default=8,
                     help="record per-stage events on every n-th timed step (events between launches "
                          "break the overlap of dependent launches, so most steps run without them)")
@@ -534,10 +536,11 @@ def run_train(args, rank, world, local):
     bws = torch.empty(moe.moe_backward_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
     out = torch.empty((T, d), dtype=dev[0].dtype, device=device)
     f32 = torch.float32
+    wd = torch.bfloat16 if (args.bf16_wgrad and inp.dtype == "bf16") else f32
     grads = dict(dx=torch.empty((T, d), dtype=dev[0].dtype, device=device),
-                 dWg=torch.empty((E, d), dtype=f32, device=device), dW1=torch.empty((E, F, d), dtype=f32, device=device),
-                 dW3=torch.empty((E, F, d), dtype=f32, device=device),
-                 dW2=torch.empty((E, d, F), dtype=f32, device=device))
+                 dWg=torch.empty((E, d), dtype=f32, device=device), dW1=torch.empty((E, F, d), dtype=wd, device=device),
+                 dW3=torch.empty((E, F, d), dtype=wd, device=device),
+                 dW2=torch.empty((E, d, F), dtype=wd, device=device))
     idx, _ = moe.moe_route(dev[0], dev[1], k)
     counts = moe.moe_dispatch(idx, E)[0].cpu().numpy()
     acc = accounting(inp, counts)
@@ -623,7 +626,7 @@ def run_train(args, rank, world, local):
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp.dtype, "data": "synthetic",
         "config": {"workload": workload_name(args.config, args.shape) + "+train", "T": T, "d": d, "ffn": F, "E": E,
-                   "k": k, "seed": c["seed"],
+                   "k": k, "seed": c["seed"], "weight_grads": "bf16" if wd == torch.bfloat16 else "fp32",
                    "l2": "touched weights larger than L2 (no flush)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof,

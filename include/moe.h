@@ -342,13 +342,16 @@ MOE_API moe_status moe_route_stats_f32(const float* x, const float* Wg, int T, i
  * a workspace of moe_train_workspace_size() bytes on the same operands, then
  * pass that workspace here unchanged as fwd_workspace (device, read only).
  * The bfloat16 backward reads GEMM1's kept a and b instead of recomputing
- * them; the fp32 backward recomputes them.  workspace: at least moe_backward_workspace_size() bytes
- * (device, 256-byte aligned).  Outputs (device, overwritten): dx [T][d] in
- * the layer's element type; dWg [E][d], dW1 [E][F][d], dW3 [E][F][d] and
- * dW2 [E][d][F] in float; dlogits [T][E] float (optional, NULL allowed): the
- * gradient of the router scores (zero for unselected experts when alpha = 0).  Every sum runs
- * in a fixed order (no float atomics), so results are bitwise repeatable.
- * stage_events (optional) receives MOE_BWD_NUM_STAGES + 1 events as in
+ * them; the fp32 backward recomputes them.  workspace: at least
+ * moe_backward_workspace_size() bytes (device, 256-byte aligned).
+ * Outputs (device, overwritten): dx [T][d] in the layer's element type;
+ * dWg [E][d] in float; dW1 [E][F][d], dW3 [E][F][d] and dW2 [E][d][F] in
+ * wgrad_dtype: MOE_DTYPE_F32, or MOE_DTYPE_BF16 for a bfloat16 layer (the fp32
+ * sums rounded once, half the bytes to write); dlogits [T][E] float
+ * (optional, NULL allowed): the gradient of the router scores (zero for
+ * unselected experts when alpha = 0).  Every sum runs in a fixed order (no
+ * float atomics), so results are bitwise repeatable.  stage_events
+ * (optional) receives MOE_BWD_NUM_STAGES + 1 events as in
  * moe_forward_profiled; launches (optional) the number of kernels launched.
  * ------------------------------------------------------------------------ */
 enum {
@@ -365,9 +368,10 @@ enum {
 MOE_API size_t moe_backward_workspace_size(int T, int d, int ffn, int E, int k, int dtype);
 
 MOE_API moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const void* W3,
-                                   const void* W2, const void* dout, void* dx, float* dWg, float* dW1,
-                                   float* dW3, float* dW2, float* dlogits, float alpha, int T, int d, int ffn,
-                                   int E, int k, int dtype, const void* fwd_workspace, size_t fwd_workspace_bytes,
+                                   const void* W2, const void* dout, void* dx, float* dWg, void* dW1,
+                                   void* dW3, void* dW2, float* dlogits, float alpha, int wgrad_dtype, int T,
+                                   int d, int ffn, int E, int k, int dtype, const void* fwd_workspace,
+                                   size_t fwd_workspace_bytes,
                                    void* workspace, size_t workspace_bytes, cudaEvent_t* stage_events,
                                    int* launches, cudaStream_t stream);
 

@@ -66,7 +66,7 @@ SIGNATURES = {
     "moe_route_stats": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
     "moe_backward_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
     "moe_train_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
-    "moe_backward_ws": (_ci, [_vp] * 12 + [_cf] + [_ci] * 6 + [_vp, _sz, _vp, _sz, _vp, _vp, _vp]),
+    "moe_backward_ws": (_ci, [_vp] * 12 + [_cf] + [_ci] * 7 + [_vp, _sz, _vp, _sz, _vp, _vp, _vp]),
     "moe_route_stats_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
@@ -325,12 +325,13 @@ def moe_backward_workspace_size(T, d, ffn, E, k, dtype=MOE_DTYPE_BF16) -> int:
 
 
 def moe_backward_ws(x, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, grads=None, dlogits=None,
-                    alpha=0.0, events=None, stream=None):
+                    alpha=0.0, wgrad_dtype=torch.float32, events=None, stream=None):
     """Gradients of the layer given dout = dL/dout, after moe_forward_ws(..., path=MOE_PATH_TRAIN,
     workspace=fwd_workspace) on the same operands (fwd_workspace: moe_train_workspace_size bytes).  Returns (grads, launches) with grads a dict of
     dx (layer dtype), dWg, dW1, dW3, dW2 (float32); pass `grads` to reuse buffers, `dlogits` (float32
     [T][E]) to also get the router-score gradient.  alpha != 0 adds the load-balance loss
-    alpha E sum f p of the forward's routing to the loss."""
+    alpha E sum f p of the forward's routing to the loss.  wgrad_dtype=torch.bfloat16 (bf16 layers)
+    returns dW1, dW3, dW2 rounded once to bf16."""
     code = _dtype_code(x)
     for t, n in ((x, "x"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2"), (dout, "dout")):
         _dev(t, x.dtype, n)
@@ -340,12 +341,15 @@ def moe_backward_ws(x, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, g
     dev = x.device
     if grads is None:
         f32 = torch.float32
+        wd = wgrad_dtype
         grads = dict(dx=torch.empty((T, d), dtype=x.dtype, device=dev), dWg=torch.empty((E, d), dtype=f32, device=dev),
-                     dW1=torch.empty((E, F, d), dtype=f32, device=dev), dW3=torch.empty((E, F, d), dtype=f32, device=dev),
-                     dW2=torch.empty((E, d, F), dtype=f32, device=dev))
+                     dW1=torch.empty((E, F, d), dtype=wd, device=dev), dW3=torch.empty((E, F, d), dtype=wd, device=dev),
+                     dW2=torch.empty((E, d, F), dtype=wd, device=dev))
     _dev(grads["dx"], x.dtype, "dx")
-    for n in ("dWg", "dW1", "dW3", "dW2"):
-        _dev(grads[n], torch.float32, n)
+    _dev(grads["dWg"], torch.float32, "dWg")
+    for n in ("dW1", "dW3", "dW2"):
+        _dev(grads[n], grads["dW1"].dtype, n)
+    wcode = _dtype_code(grads["dW1"])
     if dlogits is not None:
         _dev(dlogits, torch.float32, "dlogits")
     _dev(fwd_workspace, torch.uint8, "fwd_workspace")
@@ -356,7 +360,7 @@ def moe_backward_ws(x, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, g
     n = ctypes.c_int(0)
     _check(_lib.moe_backward_ws(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dout), _ptr(grads["dx"]),
                                 _ptr(grads["dWg"]), _ptr(grads["dW1"]), _ptr(grads["dW3"]), _ptr(grads["dW2"]),
-                                _ptr(dlogits), float(alpha), T, d, F, E, k, code, _ptr(fwd_workspace),
+                                _ptr(dlogits), float(alpha), wcode, T, d, F, E, k, code, _ptr(fwd_workspace),
                                 fwd_workspace.numel(),
                                 _ptr(workspace), workspace.numel(), _events(events, MOE_BWD_NUM_STAGES),
                                 ctypes.byref(n), _stream(stream)), "moe_backward_ws")

@@ -77,6 +77,7 @@ enum : int {
     kDgradH = 3,     // dH = dY W2_e (W2 MN-major), SwiGLU backward -> dA | dB bf16 [slots][2N]
     kDgradX = 4,     // dXp = dA W1_e + dB W3_e (MN-major, K = 2F)   -> fp32 [slots][N]
     kWgrad = 5,      // dW_e = A_e^T B_e over the expert's rows       -> fp32 [E][M][N]
+    kWgrad16 = 6,    // kWgrad rounded once to bf16                   -> bf16 [E][M][N]
 };
 
 
@@ -123,9 +124,10 @@ struct Ctrl {
 template <int MODE>
 struct ModeT {
     static constexpr bool GATED = MODE == kFwd1 || MODE == kFwd1Train;   // B halves = W1 / W3 blocks
-    static constexpr bool A_MN = MODE == kWgrad;
-    static constexpr bool B_MN = MODE == kDgradH || MODE == kDgradX || MODE == kWgrad;
-    static constexpr bool KGROUP = MODE == kWgrad;                        // tiles grouped by K, not by rows
+    static constexpr bool A_MN = MODE == kWgrad || MODE == kWgrad16;
+    static constexpr bool B_MN = MODE == kDgradH || MODE == kDgradX || MODE == kWgrad || MODE == kWgrad16;
+    static constexpr bool KGROUP = MODE == kWgrad || MODE == kWgrad16;   // tiles grouped by K, not by rows
+    static constexpr bool OUT16 = MODE == kWgrad16;
     static constexpr int N_PER_TILE = GATED ? BNH : BN;
     static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
     // Grouped-by-K tiles are short (K = one expert's rows), so their fp32 epilogue is staged
@@ -510,12 +512,20 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                             const int m = mbase + rr;
                             if (m < p.M) {
                                 const float4 v = *reinterpret_cast<const float4*>(stg + rr * OUT_PITCH + cc);
-                                float* dst = m < p.split
-                                                 ? static_cast<float*>(p.out) + ((size_t)e * p.split + m) * (size_t)N
-                                                 : static_cast<float*>(p.out_hi) +
-                                                       ((size_t)e * (p.M - p.split) + (m - p.split)) * (size_t)N;
-                                ptx::st_global_v4_hint(dst + col + cc, __float_as_uint(v.x), __float_as_uint(v.y),
-                                                       __float_as_uint(v.z), __float_as_uint(v.w), pol_out);
+                                const size_t orow = m < p.split ? (size_t)e * p.split + m
+                                                                : (size_t)e * (p.M - p.split) + (m - p.split);
+                                void* base = m < p.split ? p.out : p.out_hi;
+                                if (MT::OUT16) {
+                                    uint2 o;
+                                    o.x = pack_bf16x2(v.x, v.y);
+                                    o.y = pack_bf16x2(v.z, v.w);
+                                    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(base) + orow * (size_t)N +
+                                                              col + cc) = o;
+                                } else {
+                                    float* dst = static_cast<float*>(base) + orow * (size_t)N;
+                                    ptx::st_global_v4_hint(dst + col + cc, __float_as_uint(v.x), __float_as_uint(v.y),
+                                                           __float_as_uint(v.z), __float_as_uint(v.w), pol_out);
+                                }
                             }
                         }
                         __syncwarp();
@@ -747,7 +757,8 @@ cudaError_t launch_tc_wgrad2(const TcBwdArgs& a, cudaStream_t s) {
     gp.split = a.d;
     gp.out_hi = a.dW2;
     const size_t tiles = (size_t)a.E * (((a.d + BM - 1) / BM + 1) / 2) * ((a.F + BN - 1) / BN);
-    return launch_pair<kWgrad>(tiles, a.num_sms, mA, mB, mB, gp, s);
+    return a.wgrad_bf16 ? launch_pair<kWgrad16>(tiles, a.num_sms, mA, mB, mB, gp, s)
+                        : launch_pair<kWgrad>(tiles, a.num_sms, mA, mB, mB, gp, s);
 }
 
 cudaError_t launch_tc_wgrad13(const TcBwdArgs& a, cudaStream_t s) {
@@ -760,7 +771,8 @@ cudaError_t launch_tc_wgrad13(const TcBwdArgs& a, cudaStream_t s) {
     gp.split = a.F;
     gp.out_hi = a.dW3;
     const size_t tiles = (size_t)a.E * (((2 * a.F + BM - 1) / BM + 1) / 2) * ((a.d + BN - 1) / BN);
-    return launch_pair<kWgrad>(tiles, a.num_sms, mA, mB, mB, gp, s);
+    return a.wgrad_bf16 ? launch_pair<kWgrad16>(tiles, a.num_sms, mA, mB, mB, gp, s)
+                        : launch_pair<kWgrad>(tiles, a.num_sms, mA, mB, mB, gp, s);
 }
 
 }  // namespace moe

@@ -358,8 +358,9 @@ BwdPlan make_bwd_plan(int T, int d, int F, int E, int k, int dtype) {
 }
 
 moe_status run_backward(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2,
-                        const void* dout, void* dx, float* dWg, float* dW1, float* dW3, float* dW2, float* dlogits,
-                        float alpha, int T, int d, int F, int E, int k, int dtype, const uint8_t* fws, uint8_t* bws,
+                        const void* dout, void* dx, float* dWg, void* dW1, void* dW3, void* dW2, float* dlogits,
+                        float alpha, int wgrad_dtype, int T, int d, int F, int E, int k, int dtype, const uint8_t* fws,
+                        uint8_t* bws,
                         const DeviceState& dev, cudaStream_t s, cudaEvent_t* ev, int* launches) {
     const Plan p = make_plan(T, d, F, E, k, dtype, false, true);
     const BwdPlan b = make_bwd_plan(T, d, F, E, k, dtype);
@@ -395,9 +396,9 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
     a.dwg_part = reinterpret_cast<float*>(bws + b.dwg);
     a.dx = dx;
     a.dWg = dWg;
-    a.dW1 = dW1;
-    a.dW3 = dW3;
-    a.dW2 = dW2;
+    a.dW1 = static_cast<float*>(dW1);   // the CUDA-core (fp32) path: fp32 gradients only
+    a.dW3 = static_cast<float*>(dW3);
+    a.dW2 = static_cast<float*>(dW2);
     a.T = T;
     a.d = d;
     a.F = F;
@@ -426,6 +427,7 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
         t.dW1 = dW1;
         t.dW3 = dW3;
         t.dW2 = dW2;
+        t.wgrad_bf16 = wgrad_dtype == MOE_DTYPE_BF16;
         t.meta = a.meta;
         t.E = E;
         t.d = d;
@@ -725,8 +727,9 @@ size_t moe_backward_workspace_size(int T, int d, int ffn, int E, int k, int dtyp
 }
 
 moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const void* W3, const void* W2,
-                           const void* dout, void* dx, float* dWg, float* dW1, float* dW3, float* dW2, float* dlogits,
-                           float alpha, int T, int d, int ffn, int E, int k, int dtype, const void* fwd_workspace,
+                           const void* dout, void* dx, float* dWg, void* dW1, void* dW3, void* dW2, float* dlogits,
+                           float alpha, int wgrad_dtype, int T, int d, int ffn, int E, int k, int dtype,
+                           const void* fwd_workspace,
                            size_t fwd_workspace_bytes, void* workspace, size_t workspace_bytes,
                            cudaEvent_t* stage_events, int* launches, cudaStream_t stream) {
     if (launches) *launches = 0;
@@ -738,13 +741,16 @@ moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const 
         if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
     if (dlogits && (reinterpret_cast<uintptr_t>(dlogits) & 3u) != 0) return MOE_ERR_INVALID_ARG;
     if (!(alpha == alpha) || !(alpha - alpha == 0.f)) return MOE_ERR_INVALID_ARG;
+    if (wgrad_dtype != MOE_DTYPE_F32 && wgrad_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (wgrad_dtype == MOE_DTYPE_BF16 && dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
     if (!fwd_workspace || (reinterpret_cast<uintptr_t>(fwd_workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (fwd_workspace_bytes < make_plan(T, d, ffn, E, k, dtype, false, true).total) return MOE_ERR_WORKSPACE;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (workspace_bytes < make_bwd_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
     DeviceState dev;
     if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
-    return run_backward(x, Wg, W1, W3, W2, dout, dx, dWg, dW1, dW3, dW2, dlogits, alpha, T, d, ffn, E, k, dtype,
+    return run_backward(x, Wg, W1, W3, W2, dout, dx, dWg, dW1, dW3, dW2, dlogits, alpha, wgrad_dtype, T, d, ffn, E,
+                        k, dtype,
                         static_cast<const uint8_t*>(fwd_workspace), static_cast<uint8_t*>(workspace), dev, stream,
                         stage_events, launches);
 }

@@ -227,9 +227,10 @@ struct TcBwdArgs {
     const void* dy;     // [slots][d] bf16: g * dout scattered to the slots (padding rows zero)
     void* dab;          // [slots][2F] bf16: dA | dB
     float* dxp;         // [slots][d] fp32
-    float* dW1;         // [E][F][d] fp32
-    float* dW3;
-    float* dW2;         // [E][d][F] fp32
+    void* dW1;          // [E][F][d] fp32, or bf16 when wgrad_bf16
+    void* dW3;
+    void* dW2;          // [E][d][F] fp32, or bf16 when wgrad_bf16
+    bool wgrad_bf16;    // weight gradients rounded once to bf16 in the epilogue
     Meta* meta;
     int E, d, F;
     size_t slots;

@@ -25,7 +25,8 @@ from . import (MOE_DTYPE_BF16, MOE_DTYPE_F32, MOE_PATH_TRAIN, moe_backward_ws, m
 class MoEFunction(torch.autograd.Function):
     """out = MoE(x) with weights (Wg, W1, W3, W2); gradients for x and every weight.
 
-    Weight gradients are computed in fp32 and returned in each weight's dtype.
+    Weight gradients are summed in fp32 and rounded once to each weight's dtype
+    (for bf16 weights, inside the GEMM epilogue).
     """
 
     @staticmethod
@@ -42,7 +43,8 @@ class MoEFunction(torch.autograd.Function):
     @staticmethod
     def backward(ctx, dout):
         x, Wg, W1, W3, W2 = ctx.saved_tensors
-        g, _ = moe_backward_ws(x, Wg, W1, W3, W2, dout.contiguous(), ctx.k, ctx.ws, alpha=ctx.alpha)
+        wd = torch.bfloat16 if W1.dtype == torch.bfloat16 else torch.float32
+        g, _ = moe_backward_ws(x, Wg, W1, W3, W2, dout.contiguous(), ctx.k, ctx.ws, alpha=ctx.alpha, wgrad_dtype=wd)
         ctx.ws = None
         return (g["dx"], g["dWg"].to(Wg.dtype), g["dW1"].to(W1.dtype), g["dW3"].to(W3.dtype), g["dW2"].to(W2.dtype),
                 None, None)

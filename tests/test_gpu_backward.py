@@ -96,6 +96,23 @@ def test_backward_small(moe, dtype, T, d, F, E, k):
     print(dtype, T, d, F, E, k, {a: f"{b:.2e}" for a, b in rel.items()})
 
 
+def test_bf16_weight_gradients_are_the_fp32_ones_rounded(moe):
+    """wgrad_dtype = bf16 rounds the same fp32 sums once in the epilogue: equal to the fp32
+    gradients rounded to nearest even, bit for bit; dx and dWg are unchanged."""
+    inp = moe_inputs.make_inputs(400, 256, 384, 8, 2, "bf16", seed=45)
+    dev = upload(inp)
+    dout = to_dev(moe_inputs.make_dout(400, 256, "bf16", seed=45), "bf16")
+    ws = torch.empty(moe.moe_train_workspace_size(400, 256, 384, 8, 2), dtype=torch.uint8, device="cuda")
+    moe.moe_forward_ws(*dev, 2, path=moe.MOE_PATH_TRAIN, workspace=ws)
+    g32, _ = moe.moe_backward_ws(*dev, dout, 2, ws, alpha=0.1)
+    g16, _ = moe.moe_backward_ws(*dev, dout, 2, ws, alpha=0.1, wgrad_dtype=torch.bfloat16)
+    _status_clear(moe)
+    for n in ("dW1", "dW3", "dW2"):
+        assert g16[n].dtype == torch.bfloat16
+        assert torch.equal(g16[n], g32[n].to(torch.bfloat16)), n
+    assert torch.equal(g16["dx"], g32["dx"]) and torch.equal(g16["dWg"], g32["dWg"])
+
+
 def test_backward_run_to_run_bitwise(moe):
     inp = moe_inputs.make_inputs(300, 256, 256, 8, 2, "bf16", seed=41)
     dev = upload(inp)
