@@ -130,15 +130,21 @@ struct ModeT {
     static constexpr bool OUT16 = MODE == kWgrad16;
     static constexpr int N_PER_TILE = GATED ? BNH : BN;
     static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
-    // Grouped-by-K tiles are short (K = one expert's rows), so their fp32 epilogue is staged
-    // through shared memory for row-contiguous stores; that space comes from one ring stage.
-    // Its fp32 tiles also get two epilogue warps per TMEM lane quarter (each takes half of the
-    // columns), and the ring gives up two stages for both.
+    // An epilogue lane owns one accumulator row, so a lane's 16-byte global access touches
+    // its own 128-byte line and a warp instruction 32 lines.  Epilogues that move several
+    // times the output tile's bytes pass their fp32 chunks (32 rows x 32 columns) through
+    // shared memory instead, and global memory sees 128-byte row segments (8 lanes each):
+    //  * grouped-by-K tiles (K = one expert's rows, so short tiles): the fp32 gradient;
+    //    they also get two epilogue warps per TMEM lane quarter, each taking half the columns;
+    //  * the training forward's kept a, b (written) and the SwiGLU backward's (read), with
+    //    the backward's dA | dB written the same way.
+    // The space comes from the ring, which gives up two stages.
     static constexpr bool STAGED_OUT = KGROUP;
+    static constexpr bool STAGED_AB = MODE == kFwd1Train || MODE == kDgradH;
     static constexpr int EPI_WARPS = STAGED_OUT ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS);
-    static constexpr int STAGES_M = STAGED_OUT ? STAGES - 2 : STAGES;
-    static constexpr int STAGE_OUT_BYTES = STAGED_OUT ? EPI_WARPS * 32 * OUT_PITCH * 4 : 0;
+    static constexpr int STAGES_M = STAGED_OUT || STAGED_AB ? STAGES - 2 : STAGES;
+    static constexpr int STAGE_OUT_BYTES = (STAGED_OUT ? 1 : STAGED_AB ? 2 : 0) * EPI_WARPS * 32 * OUT_PITCH * 4;
     static constexpr int SMEM = STAGES_M * STAGE_BYTES + STAGE_OUT_BYTES + (int)sizeof(Ctrl) + 1024;
 };
 
@@ -401,11 +407,14 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
             const bool live = MT::KGROUP ? m_tile * BM < p.M : m_tile < ctrl->mt[e];
             if (live) {
                 const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+                constexpr int HALVES = MT::EPI_WARPS / NUM_EPI_WARPS;   // warps per TMEM lane quarter
+                const int half = ew / NUM_EPI_WARPS;
                 if (MODE == kFwd1 || MODE == kFwd1Train) {
                     const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
                     __nv_bfloat16* H = static_cast<__nv_bfloat16*>(p.out);
+                    constexpr int CW = BNH / HALVES;
 #pragma unroll 1
-                    for (int c = 0; c < BNH; c += 32) {
+                    for (int c = half * CW; c < (half + 1) * CW; c += 32) {
                         uint32_t ra[32], rb[32];
                         ptx::tmem_ld_32x32b_x32(taddr + c, ra);
                         ptx::tmem_ld_32x32b_x32(taddr + BNH + c, rb);
@@ -423,41 +432,73 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                             ptx::st_global_v4_hint(dst + 16 * v, hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3],
                                                    pol_out);
                         if (MODE == kFwd1Train) {
-                            // keep the pre-activations for the backward
-                            uint8_t* ka = reinterpret_cast<uint8_t*>(p.keep_a + row * (size_t)N + n_blk * BNH + c);
-                            uint8_t* kb = reinterpret_cast<uint8_t*>(p.keep_b + row * (size_t)N + n_blk * BNH + c);
+                            // keep the pre-activations for the backward: the 32 x 32 chunks of a
+                            // and b through shared memory, then 128-byte row segments
+                            float* sa = stage_out + ew * 2 * 32 * OUT_PITCH;
+                            float* sb = sa + 32 * OUT_PITCH;
+                            uint4* wa = reinterpret_cast<uint4*>(sa + lane * OUT_PITCH);
+                            uint4* wb = reinterpret_cast<uint4*>(sb + lane * OUT_PITCH);
 #pragma unroll
                             for (int v = 0; v < 8; ++v) {
-                                ptx::st_global_v4_hint(ka + 16 * v, ra[4 * v], ra[4 * v + 1], ra[4 * v + 2],
-                                                       ra[4 * v + 3], pol_out);
-                                ptx::st_global_v4_hint(kb + 16 * v, rb[4 * v], rb[4 * v + 1], rb[4 * v + 2],
-                                                       rb[4 * v + 3], pol_out);
+                                wa[v] = make_uint4(ra[4 * v], ra[4 * v + 1], ra[4 * v + 2], ra[4 * v + 3]);
+                                wb[v] = make_uint4(rb[4 * v], rb[4 * v + 1], rb[4 * v + 2], rb[4 * v + 3]);
                             }
+                            __syncwarp();
+                            const size_t row0w = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32;
+                            const int cc = (lane & 7) * 4;
+#pragma unroll
+                            for (int it = 0; it < 8; ++it) {
+                                const int rr = it * 4 + (lane >> 3);
+                                const size_t g = (row0w + rr) * (size_t)N + n_blk * BNH + c + cc;
+                                const uint4 va = *reinterpret_cast<const uint4*>(sa + rr * OUT_PITCH + cc);
+                                const uint4 vb = *reinterpret_cast<const uint4*>(sb + rr * OUT_PITCH + cc);
+                                ptx::st_global_v4_hint(p.keep_a + g, va.x, va.y, va.z, va.w, pol_out);
+                                ptx::st_global_v4_hint(p.keep_b + g, vb.x, vb.y, vb.z, vb.w, pol_out);
+                            }
+                            __syncwarp();   // the next chunk reuses the buffers
                         }
                     }
                 } else if (MODE == kDgradH) {
                     // dH tile (TMEM) -> SwiGLU backward with the kept a, b:
                     //     dA = dH b SiLU'(a),  dB = dH SiLU(a)   -> bf16 [slots][2N], dA | dB
-                    const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
+                    // a, b come in and dA | dB go out as 128-byte row segments through shared memory
+                    const size_t row0w = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32;
                     __nv_bfloat16* dAB = static_cast<__nv_bfloat16*>(p.out);
+                    float* sa = stage_out + ew * 2 * 32 * OUT_PITCH;
+                    float* sb = sa + 32 * OUT_PITCH;
+                    const int cc = (lane & 7) * 4;
+                    constexpr int CW = BN / HALVES;
 #pragma unroll 1
-                    for (int c = 0; c < BN; c += 32) {
+                    for (int c = half * CW; c < (half + 1) * CW; c += 32) {
                         const int col = n_blk * BN + c;
                         if (col >= N) break;
-                        const float4* ap = reinterpret_cast<const float4*>(p.aux_a + row * (size_t)N + col);
-                        const float4* bp = reinterpret_cast<const float4*>(p.aux_b + row * (size_t)N + col);
+                        float4 ta[8], tb[8];
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const size_t g = (row0w + it * 4 + (lane >> 3)) * (size_t)N + col + cc;
+                            ta[it] = __ldg(reinterpret_cast<const float4*>(p.aux_a + g));
+                            tb[it] = __ldg(reinterpret_cast<const float4*>(p.aux_b + g));
+                        }
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int rr = it * 4 + (lane >> 3);
+                            *reinterpret_cast<float4*>(sa + rr * OUT_PITCH + cc) = ta[it];
+                            *reinterpret_cast<float4*>(sb + rr * OUT_PITCH + cc) = tb[it];
+                        }
+                        __syncwarp();
                         float av[32], bv[32];
 #pragma unroll
                         for (int v = 0; v < 8; ++v) {
-                            const float4 ta = __ldg(ap + v), tb = __ldg(bp + v);
-                            av[4 * v] = ta.x;
-                            av[4 * v + 1] = ta.y;
-                            av[4 * v + 2] = ta.z;
-                            av[4 * v + 3] = ta.w;
-                            bv[4 * v] = tb.x;
-                            bv[4 * v + 1] = tb.y;
-                            bv[4 * v + 2] = tb.z;
-                            bv[4 * v + 3] = tb.w;
+                            const float4 xa = reinterpret_cast<const float4*>(sa + lane * OUT_PITCH)[v];
+                            const float4 xb = reinterpret_cast<const float4*>(sb + lane * OUT_PITCH)[v];
+                            av[4 * v] = xa.x;
+                            av[4 * v + 1] = xa.y;
+                            av[4 * v + 2] = xa.z;
+                            av[4 * v + 3] = xa.w;
+                            bv[4 * v] = xb.x;
+                            bv[4 * v + 1] = xb.y;
+                            bv[4 * v + 2] = xb.z;
+                            bv[4 * v + 3] = xb.w;
                         }
                         uint32_t r[32];
                         ptx::tmem_ld_32x32b_x32(taddr + c, r);
@@ -472,15 +513,25 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                             pa[i] = pack_bf16x2(da[0], da[1]);
                             pb[i] = pack_bf16x2(dbv[0], dbv[1]);
                         }
-                        uint8_t* dst_a = reinterpret_cast<uint8_t*>(dAB + row * (size_t)(2 * N) + col);
-                        uint8_t* dst_b = dst_a + (size_t)N * 2;
+                        __syncwarp();   // every lane has its row of a, b: the buffer takes dA | dB
+                        uint4* w = reinterpret_cast<uint4*>(sa + lane * OUT_PITCH);
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
-                            ptx::st_global_v4_hint(dst_a + 16 * v, pa[4 * v], pa[4 * v + 1], pa[4 * v + 2],
-                                                   pa[4 * v + 3], pol_out);
-                            ptx::st_global_v4_hint(dst_b + 16 * v, pb[4 * v], pb[4 * v + 1], pb[4 * v + 2],
-                                                   pb[4 * v + 3], pol_out);
+                            w[v] = make_uint4(pa[4 * v], pa[4 * v + 1], pa[4 * v + 2], pa[4 * v + 3]);
+                            w[4 + v] = make_uint4(pb[4 * v], pb[4 * v + 1], pb[4 * v + 2], pb[4 * v + 3]);
                         }
+                        __syncwarp();
+                        // words 0-15 of a staged row are dA's 32 columns, words 16-31 dB's
+                        const int part = cc >> 4;
+                        const int ecol = col + 2 * (cc & 15);
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int rr = it * 4 + (lane >> 3);
+                            const uint4 v = *reinterpret_cast<const uint4*>(sa + rr * OUT_PITCH + cc);
+                            __nv_bfloat16* dst = dAB + (row0w + rr) * (size_t)(2 * N) + (size_t)part * N + ecol;
+                            ptx::st_global_v4_hint(dst, v.x, v.y, v.z, v.w, pol_out);
+                        }
+                        __syncwarp();   // the next chunk reuses the buffers
                     }
                 } else if (MT::STAGED_OUT) {
                     // fp32 gradient tile of expert e, rows m of [M][N] (rows >= split to out_hi):
@@ -489,8 +540,8 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                     float* stg = stage_out + ew * 32 * OUT_PITCH;
                     const bool zero = ctrl->nkb[e] == 0;   // no rows: the accumulator was never written
                     const int mbase = m_tile * BM + q * 32;
-                    constexpr int CW = BN / (MT::EPI_WARPS / NUM_EPI_WARPS);   // columns per warp
-                    const int c0 = (ew / NUM_EPI_WARPS) * CW;
+                    constexpr int CW = BN / HALVES;   // columns per warp
+                    const int c0 = half * CW;
 #pragma unroll 1
                     for (int c = c0; c < c0 + CW; c += 32) {
                         uint32_t r[32];
@@ -531,34 +582,16 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                         __syncwarp();
                     }
                 } else {
-                    // fp32 tile: row-grouped modes write row r of [slots][N]; grouped-by-K writes
-                    // row m of expert e's [M][N] gradient (rows >= split to out_hi)
-                    float* dst_row = nullptr;
-                    bool zero = false;
-                    if (MT::KGROUP) {
-                        const int m = m_tile * BM + q * 32 + lane;
-                        if (m < p.M) {
-                            dst_row = m < p.split
-                                          ? static_cast<float*>(p.out) + ((size_t)e * p.split + m) * (size_t)N
-                                          : static_cast<float*>(p.out_hi) +
-                                                ((size_t)e * (p.M - p.split) + (m - p.split)) * (size_t)N;
-                        }
-                        zero = ctrl->nkb[e] == 0;   // no rows: the accumulator was never written
-                    } else {
-                        const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
-                        dst_row = static_cast<float*>(p.out) + row * (size_t)N;
-                    }
+                    // fp32 tile (kFwd2, kDgradX; grouped-by-K tiles take the staged branch): row r of [slots][N]
+                    const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
+                    float* dst_row = static_cast<float*>(p.out) + row * (size_t)N;
 #pragma unroll 1
                     for (int c = 0; c < BN; c += 32) {
                         uint32_t r[32];
                         ptx::tmem_ld_32x32b_x32(taddr + c, r);
                         ptx::tmem_ld_wait();
                         const int col = n_blk * BN + c;
-                        if (dst_row && col < N) {
-                            if (zero) {
-#pragma unroll
-                                for (int i = 0; i < 32; ++i) r[i] = 0u;
-                            }
+                        if (col < N) {
                             uint8_t* dst = reinterpret_cast<uint8_t*>(dst_row + col);
 #pragma unroll
                             for (int v = 0; v < 8; ++v)

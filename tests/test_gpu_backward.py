@@ -123,6 +123,52 @@ def test_backward_run_to_run_bitwise(moe):
         assert torch.equal(a[n], b[n]), n
 
 
+def _close(name, got, want, rel):
+    """|got - want| <= rel (RMS(want) + |want|) entrywise: sums of the same terms in another order."""
+    got, want = got.double(), want.double()
+    rms = want.pow(2).mean().sqrt()
+    bad = (got - want).abs() > rel * (rms + want.abs())
+    assert not bad.any(), f"{name}: {int(bad.sum())} entries differ by more than {rel:.1e} (RMS + |G|)"
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_token_permutation_equivariance(moe, dtype):
+    """Tokens are independent: permuting x and dout permutes dx and the router-score gradient bit
+    for bit.  The weight gradients sum the same per-token terms in another order (each expert's
+    rows follow token order), so they agree to fp32 reassociation."""
+    T, d, F = 300, 256, 256
+    inp = moe_inputs.make_inputs(T, d, F, 8, 2, dtype, seed=46)
+    dev = upload(inp)
+    dout = to_dev(moe_inputs.make_dout(T, d, dtype, seed=46), dtype)
+    _, a, _ = _run(moe, inp, dev, dout, dlogits=True)
+    p = torch.randperm(T, generator=torch.Generator().manual_seed(1)).cuda()
+    dev_p = (dev[0][p].contiguous(),) + tuple(dev[1:])
+    _, b, _ = _run(moe, inp, dev_p, dout[p].contiguous(), dlogits=True)
+    assert torch.equal(b["dx"], a["dx"][p])
+    assert torch.equal(b["dlogits"], a["dlogits"][p])
+    for n in ("dWg", "dW1", "dW3", "dW2"):
+        _close(n, b[n], a[n], 2e-4)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_expert_relabelling(moe, dtype):
+    """Relabelling the experts (rows of Wg, blocks of W1, W3, W2) permutes every per-expert
+    gradient bit for bit: each expert sees the same tokens in the same order.  dx adds the k
+    router terms in expert-index order, so it agrees to one rounding of its output."""
+    T, d, F = 300, 256, 256
+    inp = moe_inputs.make_inputs(T, d, F, 8, 2, dtype, seed=47)
+    dev = upload(inp)
+    dout = to_dev(moe_inputs.make_dout(T, d, dtype, seed=47), dtype)
+    _, a, _ = _run(moe, inp, dev, dout, dlogits=True)
+    r = torch.tensor([3, 7, 0, 5, 1, 6, 2, 4], device="cuda")
+    dev_r = (dev[0],) + tuple(t[r].contiguous() for t in dev[1:])
+    _, b, _ = _run(moe, inp, dev_r, dout, dlogits=True)
+    for n in ("dWg", "dW1", "dW3", "dW2"):
+        assert torch.equal(b[n], a[n][r]), n
+    assert torch.equal(b["dlogits"], a["dlogits"][:, r])
+    _close("dx", b["dx"], a["dx"], 2.0 ** -7 if dtype == "bf16" else 1e-5)
+
+
 def test_backward_experts_without_tokens(moe):
     """Experts no token chose get exactly zero weight gradients."""
     inp = moe_inputs.make_inputs(100, 128, 256, 8, 2, "bf16", seed=42)
