@@ -32,7 +32,9 @@
  * (cudaMalloc, cudaMallocAsync, torch CUDA tensors); "host" means ordinary or
  * pinned host memory.  Every pointer must be 16-byte aligned.  The caller owns
  * every buffer; the library keeps no pointer past the call.  Outputs are fully
- * overwritten, never accumulated into.
+ * overwritten, never accumulated into.  A call runs on the device that owns its
+ * first device buffer (the current device for the host entry points), and
+ * leaves the calling thread's current device as it found it.
  *
  * Streams: every call is stream-ordered on `stream` (0 = legacy default
  * stream) and returns without synchronising, except moe_forward_host and

@@ -58,20 +58,6 @@ unsigned char* scratch_on(int dev) {
     return g_noalloc_ptr[dev];
 }
 
-// The device that owns `p`, made current; -1 if that fails.
-int owner_device(const void* p) {
-    cudaPointerAttributes at;
-    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
-        cudaGetLastError();
-        return -1;
-    }
-    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return -1;
-    int cur = -1;
-    if (cudaGetDevice(&cur) != cudaSuccess) return -1;
-    if (cur != at.device && cudaSetDevice(at.device) != cudaSuccess) return -1;
-    return at.device;
-}
-
 }  // namespace
 }  // namespace moe
 
@@ -84,7 +70,8 @@ extern "C" moe_status moe_dispatch_noalloc(const int32_t* topk_idx, int T, int E
     if ((long long)T * k + (long long)E * kSegRows >= INT_MAX) return MOE_ERR_UNSUPPORTED;
     if ((size_t)dispatch_blocks(T) * (size_t)E > kNoAllocHistInts) return MOE_ERR_UNSUPPORTED;
     if (!counts || !offsets || (T > 0 && (!topk_idx || !perm || !inv))) return MOE_ERR_INVALID_ARG;
-    const int dev = owner_device(counts);
+    const DeviceScope scope(counts, true);
+    const int dev = scope.device();
     if (dev < 0) return MOE_ERR_INVALID_ARG;
     unsigned char* scratch = scratch_on(dev);
     int* status = status_word(dev);

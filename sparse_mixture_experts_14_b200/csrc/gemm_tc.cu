@@ -285,7 +285,9 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                 const int rowA = ctrl->row0[e] + m_tile * BM;            // row-grouped: A rows
                 const int n0 = n_blk * BN + (int)rank * BNH;             // this CTA's B rows (non-gated)
                 const int nkb = ctrl->nkb[e];
-                if (leader) wave_sync(&meta->waves[p.wave_slot], min(total, (wave + 1) * nclusters));
+                // grouped-by-K tiles are short and their operand blocks stay in L2 across a few
+                // waves of drift: no alignment (it would hold every cluster to the slowest tile)
+                if (leader && !MT::KGROUP) wave_sync(&meta->waves[p.wave_slot], min(total, (wave + 1) * nclusters));
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!ptx::mbar_wait(&ctrl->empty[stage], phase ^ 1u, wc)) {
                         aborted = true;

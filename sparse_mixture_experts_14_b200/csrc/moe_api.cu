@@ -31,22 +31,6 @@ long long wait_limit_ns() {
     return v;
 }
 
-// Make the device that owns `p` current in this library's runtime; returns its id.
-int select_device(const void* p) {
-    int dev = 0;
-    cudaPointerAttributes at;
-    if (p && cudaPointerGetAttributes(&at, p) == cudaSuccess &&
-        (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged)) {
-        dev = at.device;
-        int cur = -1;
-        if (cudaGetDevice(&cur) != cudaSuccess || cur != dev) cudaSetDevice(dev);
-    } else {
-        cudaGetLastError();
-        cudaGetDevice(&dev);
-    }
-    return dev;
-}
-
 struct DeviceState {
     cudaMemPool_t pool;
     int* status;
@@ -263,7 +247,8 @@ moe_status forward_pooled(const void* x, const void* Wg, const void* W1, const v
     moe_status st = check_layer(x, Wg, W1, W3, W2, out, T, d, F, E, k, dtype);
     if (st != MOE_OK || T == 0) return st;
     DeviceState dev;
-    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(x, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     const Plan p = make_plan(T, d, F, E, k, dtype);
     void* ws = nullptr;
     if (cudaMallocFromPoolAsync(&ws, p.total, dev.pool, s) != cudaSuccess) return MOE_ERR_WORKSPACE;
@@ -294,7 +279,8 @@ moe_status block_pooled(const void* h, const void* gamma, float eps, const void*
     if (st == MOE_OK) st = check_block(h, gamma, eps, alpha, stats, out, T, d, dtype);
     if (st != MOE_OK || T == 0) return st;
     DeviceState dev;
-    if (!device_state(select_device(h), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(h, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     const Plan p = make_plan(T, d, F, E, k, dtype, true);
     void* ws = nullptr;
     if (cudaMallocFromPoolAsync(&ws, p.total, dev.pool, s) != cudaSuccess) return MOE_ERR_WORKSPACE;
@@ -314,7 +300,8 @@ moe_status route_stats(const void* x, const void* Wg, int T, int d, int E, int k
     if (T == 0) return MOE_OK;
     if (!x || !Wg || !idx || !w || !stats || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
     DeviceState dev;
-    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(x, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     const size_t lbytes = align_up((size_t)T * E * 4, 256);
     void* scratch = nullptr;
     if (cudaMallocFromPoolAsync(&scratch, lbytes + balance_part_bytes(T, E), dev.pool, s) != cudaSuccess)
@@ -510,7 +497,8 @@ moe_status moe_route(const void* x, const void* Wg, int T, int d, int E, int k, 
     if (T == 0) return MOE_OK;
     if (!x || !Wg || !topk_idx || !topk_w || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
     DeviceState dev;
-    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(x, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     return cuda_status(launch_router_bf16(x, Wg, T, d, E, k, topk_idx, topk_w, dev.num_sms, stream));
 }
 
@@ -522,7 +510,8 @@ moe_status moe_route_f32(const float* x, const float* Wg, int T, int d, int E, i
     if (T == 0) return MOE_OK;
     if (!x || !Wg || !topk_idx || !topk_w || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
     DeviceState dev;
-    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(x, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     return cuda_status(launch_router_f32(x, Wg, T, d, E, k, topk_idx, topk_w, dev.num_sms, stream));
 }
 
@@ -537,7 +526,8 @@ moe_status moe_dispatch(const int32_t* topk_idx, int T, int E, int k, int32_t* c
     if (st != MOE_OK) return st;
     if (!counts || !offsets || (T > 0 && (!topk_idx || !perm || !inv))) return MOE_ERR_INVALID_ARG;
     DeviceState dev;
-    if (!device_state(select_device(counts), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(counts, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     const size_t blk_bytes = align_up((size_t)dispatch_blocks(T) * E * 4 + 1, 256);
     void* scratch = nullptr;
     if (cudaMallocFromPoolAsync(&scratch, blk_bytes + sizeof(Meta), dev.pool, stream) != cudaSuccess)
@@ -586,7 +576,8 @@ moe_status moe_forward_ws(const void* x, const void* Wg, const void* W1, const v
     if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype, false, path == MOE_PATH_TRAIN).total)
         return MOE_ERR_WORKSPACE;
     DeviceState dev;
-    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(x, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     return run_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
                      stream);
 }
@@ -606,7 +597,8 @@ moe_status moe_forward_profiled(const void* x, const void* Wg, const void* W1, c
     if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype, false, path == MOE_PATH_TRAIN).total)
         return MOE_ERR_WORKSPACE;
     DeviceState dev;
-    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(x, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     return run_layer(x, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
                      stream, stage_events, launches);
 }
@@ -616,7 +608,8 @@ moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, 
     moe_status st = check_layer(x_host, Wg, W1, W3, W2, out_host, T, d, ffn, E, k, MOE_DTYPE_BF16);
     if (st != MOE_OK || T == 0) return st;
     DeviceState dev;
-    if (!device_state(select_device(Wg), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(Wg, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     const size_t act = (size_t)T * d * 2;
     const size_t act_al = align_up(act, 256);
     const Plan p = make_plan(T, d, ffn, E, k, MOE_DTYPE_BF16);
@@ -708,7 +701,8 @@ moe_status moe_block_forward_ws(const void* h, const void* gamma, float eps, con
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype, true).total) return MOE_ERR_WORKSPACE;
     DeviceState dev;
-    if (!device_state(select_device(h), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(h, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     const BlockArgs bo{gamma, eps, alpha, stats};
     return run_layer(h, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype, path, static_cast<uint8_t*>(workspace), dev,
                      stream, stage_events, launches, &bo);
@@ -748,7 +742,8 @@ moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const 
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
     if (workspace_bytes < make_bwd_plan(T, d, ffn, E, k, dtype).total) return MOE_ERR_WORKSPACE;
     DeviceState dev;
-    if (!device_state(select_device(x), &dev)) return MOE_ERR_CUDA;
+    const DeviceScope scope(x, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
     return run_backward(x, Wg, W1, W3, W2, dout, dx, dWg, dW1, dW3, dW2, dlogits, alpha, wgrad_dtype, T, d, ffn, E,
                         k, dtype,
                         static_cast<const uint8_t*>(fwd_workspace), static_cast<uint8_t*>(workspace), dev, stream,

@@ -66,6 +66,42 @@ __device__ __forceinline__ void silu_bwd(float a, float b, float dh, float& da, 
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// For the length of one library call: the device that owns p is made current,
+// and the caller's current device is restored on exit.  For a pointer that is
+// not device (or managed) memory, device() is -1 when strict, else the
+// caller's current device.
+class DeviceScope {
+   public:
+    DeviceScope(const void* p, bool strict) {
+        if (cudaGetDevice(&prev_) != cudaSuccess) {
+            cudaGetLastError();
+            prev_ = -1;
+        }
+        cudaPointerAttributes at;
+        if (p && cudaPointerGetAttributes(&at, p) == cudaSuccess &&
+            (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged)) {
+            if (at.device != prev_ && cudaSetDevice(at.device) != cudaSuccess) {
+                cudaGetLastError();
+                return;
+            }
+            dev_ = at.device;
+        } else {
+            cudaGetLastError();
+            if (!strict) dev_ = prev_;
+        }
+    }
+    ~DeviceScope() {
+        if (prev_ >= 0 && dev_ >= 0 && dev_ != prev_) cudaSetDevice(prev_);
+    }
+    DeviceScope(const DeviceScope&) = delete;
+    DeviceScope& operator=(const DeviceScope&) = delete;
+    int device() const { return dev_; }
+
+   private:
+    int prev_ = -1;
+    int dev_ = -1;
+};
+
 // Set-up that CUDA keeps per device (function attributes, occupancy facts):
 // run f once on each device that is current when it is needed.  Concurrent
 // first calls may both run f, which must therefore be idempotent.
