@@ -152,3 +152,54 @@ def test_route_stats_argument_checks(lib):
     assert f(_vp(), _vp(), 4, 128, 8, 2, 1.0, _vp(), _vp(), None, None) == 1   # stats required
     assert f(_vp(), _vp(), 4, 128, 8, 2, float("nan"), _vp(), _vp(), _vp(), None) == 1
     assert f(_vp(), _vp(), 0, 128, 8, 2, 1.0, None, None, None, None) == 0
+
+
+def test_training_workspace_sizes(lib):
+    for name in ("moe_workspace_size", "moe_train_workspace_size", "moe_backward_workspace_size"):
+        getattr(lib, name).restype = ctypes.c_size_t
+    T, d, F, E, k = 4096, 4096, 14336, 8, 2
+    plain = lib.moe_workspace_size(T, d, F, E, k, 1)
+    train = lib.moe_train_workspace_size(T, d, F, E, k, 1)
+    S = (T * k + E * 127 + 127) // 128 * 128               # expert-segment rows
+    assert train >= plain + 2 * S * F * 4 + T * E * 4   # the kept a, b (fp32) and the scores on top
+    bwd = lib.moe_backward_workspace_size(T, d, F, E, k, 1)
+    assert bwd >= S * 2 * F * 2 + S * d * 4              # dA | dB (bf16) and dXp (fp32)
+    assert lib.moe_train_workspace_size(T, d, F, E, k, 7) == 0
+    assert lib.moe_backward_workspace_size(T, d, F, E, 9, 1) == 0   # k > E
+
+
+def _bwd(lib, T=8, d=128, F=256, E=8, k=2, dtype=1, wgrad=0, alpha=0.0, dout=0x7000, dW1=0x8000, dlogits=None,
+         fws=0x10000, fws_bytes=None, ws=0x20000, ws_bytes=None):
+    for name in ("moe_train_workspace_size", "moe_backward_workspace_size"):
+        getattr(lib, name).restype = ctypes.c_size_t
+    if fws_bytes is None:
+        fws_bytes = lib.moe_train_workspace_size(max(T, 1), d, F, E, min(k, E), dtype)
+    if ws_bytes is None:
+        ws_bytes = lib.moe_backward_workspace_size(max(T, 1), d, F, E, min(k, E), dtype)
+    fn = lib.moe_backward_ws
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p] * 12 + [ctypes.c_float] + [ctypes.c_int] * 7 + \
+        [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t] + [ctypes.c_void_p] * 3
+    return fn(_vp(0x1000), _vp(0x2000), _vp(0x3000), _vp(0x4000), _vp(0x5000), _vp(dout) if dout else None,
+              _vp(0x6000), _vp(0x9000), _vp(dW1) if dW1 else None, _vp(0xa000), _vp(0xb000),
+              _vp(dlogits) if dlogits else None, alpha, wgrad, T, d, F, E, k, dtype,
+              _vp(fws) if fws else None, fws_bytes, _vp(ws) if ws else None, ws_bytes, None, None, None)
+
+
+def test_backward_argument_checks(lib):
+    """Every check here returns before the library touches CUDA."""
+    assert _bwd(lib, k=9) == 1                          # k > E
+    assert _bwd(lib, d=100) == 2                        # bf16 needs d % 64 == 0
+    assert _bwd(lib, dout=0) == 1                       # upstream gradient required
+    assert _bwd(lib, dW1=0x8008) == 1                   # misaligned gradient buffer
+    assert _bwd(lib, dlogits=0x9002) == 1               # misaligned score gradient
+    assert _bwd(lib, alpha=float("nan")) == 1
+    assert _bwd(lib, alpha=float("inf")) == 1
+    assert _bwd(lib, wgrad=5) == 1                      # unknown weight-gradient type
+    assert _bwd(lib, dtype=0, d=128, wgrad=1) == 2      # bf16 weight gradients of an fp32 layer
+    assert _bwd(lib, fws=0) == 5                        # no forward workspace
+    assert _bwd(lib, fws=0x10040) == 5                  # not 256-byte aligned
+    assert _bwd(lib, fws_bytes=1024) == 5               # an inference-sized workspace cannot hold a, b
+    assert _bwd(lib, ws=0) == 5
+    assert _bwd(lib, ws_bytes=1024) == 5
+    assert _bwd(lib, T=0) == 0                          # empty batch: no-op
