@@ -90,9 +90,18 @@ def _check(status: int, what: str):
         raise MoEError(status, what)
 
 
-def _stream(stream=None):
+def _stream(stream=None, *tensors):
+    """The stream to launch on: `stream`, else torch's current stream of the device that holds
+    the call's CUDA tensors.  Tensors on several devices (or a stream of another device) raise:
+    a kernel cannot address another device's memory through them."""
+    devs = {t.device for t in tensors if isinstance(t, torch.Tensor) and t.is_cuda}
+    if len(devs) > 1:
+        raise ValueError(f"tensors on several devices: {sorted(str(v) for v in devs)}")
+    dev = devs.pop() if devs else None
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
+    elif dev is not None and stream.device != dev:
+        raise ValueError(f"stream of {stream.device} for tensors on {dev}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -141,7 +150,8 @@ def moe_route(x, Wg, k, topk_idx=None, topk_w=None, stream=None):
     _dev(topk_idx, torch.int32, "topk_idx")
     _dev(topk_w, torch.float32, "topk_w")
     fn = _lib.moe_route if code == MOE_DTYPE_BF16 else _lib.moe_route_f32
-    _check(fn(_ptr(x), _ptr(Wg), T, d, E, k, _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
+    _check(fn(_ptr(x), _ptr(Wg), T, d, E, k, _ptr(topk_idx), _ptr(topk_w),
+              _stream(stream, x, Wg, topk_idx, topk_w)), "moe_route")
     return topk_idx, topk_w
 
 
@@ -159,7 +169,7 @@ def moe_dispatch(topk_idx, E, stream=None):
     perm = torch.empty(max(moe_slots_capacity(T, E, k), 1), dtype=torch.int32, device=dev)
     inv = torch.empty((T, k), dtype=torch.int32, device=dev)
     _check(_lib.moe_dispatch(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
-                             _stream(stream)), "moe_dispatch")
+                             _stream(stream, topk_idx)), "moe_dispatch")
     return counts, offsets, perm, inv
 
 
@@ -171,7 +181,7 @@ def moe_dispatch_noalloc(topk_idx, E, counts, offsets, perm, inv, stream=None):
         _dev(t, torch.int32, n)
     T, k = topk_idx.shape
     _check(_lib.moe_dispatch_noalloc(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
-                                     _stream(stream)), "moe_dispatch_noalloc")
+                                     _stream(stream, topk_idx, counts, offsets, perm, inv)), "moe_dispatch_noalloc")
     return counts, offsets, perm, inv
 
 
@@ -185,8 +195,8 @@ def moe_forward(x, Wg, W1, W3, W2, k, out=None, stream=None):
         out = torch.empty((T, d), dtype=x.dtype, device=x.device)
     _dev(out, x.dtype, "out")
     fn = _lib.moe_forward if code == MOE_DTYPE_BF16 else _lib.moe_forward_f32
-    _check(fn(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, _stream(stream)),
-           "moe_forward")
+    _check(fn(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k,
+              _stream(stream, x, Wg, W1, W3, W2, out)), "moe_forward")
     return out
 
 
@@ -211,7 +221,8 @@ def moe_forward_ws(x, Wg, W1, W3, W2, k, path=MOE_PATH_AUTO, workspace=None, out
         out = torch.empty((T, d), dtype=x.dtype, device=x.device)
     _dev(out, x.dtype, "out")
     _check(_lib.moe_forward_ws(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, code,
-                               path, _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward_ws")
+                               path, _ptr(workspace), workspace.numel(),
+                               _stream(stream, x, Wg, W1, W3, W2, out, workspace)), "moe_forward_ws")
     return out
 
 
@@ -219,12 +230,15 @@ def moe_forward_profiled(x, Wg, W1, W3, W2, k, workspace, out, events=None, path
     """moe_forward_ws recording torch.cuda.Event objects (MOE_NUM_STAGES + 1 of them, timing enabled)
     at the stage boundaries; returns the number of kernels launched."""
     code = _dtype_code(x)
+    for t, n in ((x, "x"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2"), (out, "out")):
+        _dev(t, x.dtype, n)
+    _dev(workspace, torch.uint8, "workspace")
     T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
     ev_arr = _events(events)
     n = ctypes.c_int(0)
     _check(_lib.moe_forward_profiled(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, code,
                                      path, _ptr(workspace), workspace.numel(), ev_arr, ctypes.byref(n),
-                                     _stream(stream)), "moe_forward_profiled")
+                                     _stream(stream, x, Wg, W1, W3, W2, out, workspace)), "moe_forward_profiled")
     return n.value
 
 
@@ -239,7 +253,7 @@ def moe_forward_host(x_host, Wg, W1, W3, W2, k, out_host=None, stream=None):
     if out_host is None:
         out_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
     _check(_lib.moe_forward_host(_ptr(x_host), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out_host), T, d, F, E,
-                                 k, _stream(stream)), "moe_forward_host")
+                                 k, _stream(stream, Wg, W1, W3, W2)), "moe_forward_host")
     return out_host
 
 
@@ -278,7 +292,7 @@ def moe_block_forward(h, gamma, eps, Wg, W1, W3, W2, k, alpha=1.0, stats=None, o
     _dev(out, h.dtype, "out")
     fn = _lib.moe_block_forward if code == MOE_DTYPE_BF16 else _lib.moe_block_forward_f32
     _check(fn(_ptr(h), _ptr(gamma), float(eps), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k,
-              float(alpha), _ptr(stats), _stream(stream)), "moe_block_forward")
+              float(alpha), _ptr(stats), _stream(stream, h, gamma, Wg, W1, W3, W2, stats, out)), "moe_block_forward")
     return out
 
 
@@ -296,7 +310,8 @@ def moe_block_forward_ws(h, gamma, eps, Wg, W1, W3, W2, k, workspace, out, alpha
     _check(_lib.moe_block_forward_ws(_ptr(h), _ptr(gamma), float(eps), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2),
                                      _ptr(out), T, d, F, E, k, float(alpha), _ptr(stats), code, path,
                                      _ptr(workspace), workspace.numel(), _events(events), ctypes.byref(n),
-                                     _stream(stream)), "moe_block_forward_ws")
+                                     _stream(stream, h, gamma, Wg, W1, W3, W2, stats, out, workspace)),
+           "moe_block_forward_ws")
     return n.value
 
 
@@ -311,7 +326,7 @@ def moe_route_stats(x, Wg, k, alpha=1.0, stream=None):
     w = torch.empty((T, k), dtype=torch.float32, device=x.device)
     stats = torch.empty(2 * E + 1, dtype=torch.float32, device=x.device)
     fn = _lib.moe_route_stats if code == MOE_DTYPE_BF16 else _lib.moe_route_stats_f32
-    _check(fn(_ptr(x), _ptr(Wg), T, d, E, k, float(alpha), _ptr(idx), _ptr(w), _ptr(stats), _stream(stream)),
+    _check(fn(_ptr(x), _ptr(Wg), T, d, E, k, float(alpha), _ptr(idx), _ptr(w), _ptr(stats), _stream(stream, x, Wg)),
            "moe_route_stats")
     return idx, w, stats
 
@@ -363,7 +378,9 @@ def moe_backward_ws(x, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, g
                                 _ptr(dlogits), float(alpha), wcode, T, d, F, E, k, code, _ptr(fwd_workspace),
                                 fwd_workspace.numel(),
                                 _ptr(workspace), workspace.numel(), _events(events, MOE_BWD_NUM_STAGES),
-                                ctypes.byref(n), _stream(stream)), "moe_backward_ws")
+                                ctypes.byref(n),
+                                _stream(stream, x, Wg, W1, W3, W2, dout, fwd_workspace, workspace, dlogits,
+                                        *grads.values())), "moe_backward_ws")
     return grads, n.value
 
 
