@@ -31,6 +31,12 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
                            torch autograd of the E=1 dense FFN and of the
                            k=E softmax mixture; slices and token rows equal
                            the full backward
+  block_backward           pinned (tests/test_oracle_pins_block_backward.py):
+                           central finite differences of block() (+ balance()
+                           of block_scores()) on every parameter; torch
+                           autograd of the E=1 dense block and of the k=E
+                           softmax-mixture block; W2 = 0 passes dout to h
+                           unchanged; fp64 operand storage equals fp32
 
 The block and balance steps follow the same page, section "Mixtral 8x7B —
 Sparse MoEの導入" (subsection "Mixtralのアーキテクチャ": RMSNorm, MoE layer,
@@ -51,7 +57,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-DTYPE_CODE = {"f32": 0, "bf16": 1}
+DTYPE_CODE = {"f32": 0, "bf16": 1, "f64": 2}   # f64: operands that are exact fp64 results (block backward)
 
 
 def build(force: bool = False) -> str:
@@ -94,7 +100,7 @@ def _load():
 
 
 def _arr(a, dtype):
-    want = np.uint16 if dtype == "bf16" else np.float32
+    want = {"bf16": np.uint16, "f32": np.float32, "f64": np.float64}[dtype]
     a = np.ascontiguousarray(a)
     if a.dtype != want:
         raise TypeError(f"expected {want} storage for dtype {dtype}, got {a.dtype}")
@@ -309,3 +315,36 @@ def balance_grad(logits, k: int, alpha: float) -> np.ndarray:
     out = np.empty((T, E), dtype=np.float64)
     _check(_load().oracle_balance_grad(T, E, k, s.ctypes.data, float(alpha), out.ctypes.data), "balance_grad")
     return out
+
+
+def _widen(a, dtype) -> np.ndarray:
+    """Exact float64 copy of an operand stored as `dtype`."""
+    a = _arr(a, dtype)
+    if dtype == "bf16":
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def block_backward(h, gamma, eps: float, Wg, W1, W3, W2, dout, k: int, dtype: str, alpha: float = 0.0) -> dict:
+    """Every gradient of L = sum <dout, out> + alpha E sum f p for out = h + MoE(RMSNorm(h)), with the
+    top-k choice held fixed (small shapes): dict(dh, dgamma, dWg, dW1, dW3, dW2, dlogits, idx, g,
+    margin, mingap), all float64.
+
+    The MoE part is backward() at x = u = RMSNorm(h), the exact fp64 rows block() evaluates, which
+    gives du = dL/du (the load-balance part, on the scores Wg u, included).  With
+    rho_t = (mean_i h_ti^2 + eps)^(-1/2) and u_tj = gamma_j h_tj rho_t, d rho_t / d h_ti = -rho_t^3 h_ti / d:
+        dh_ti    = dout_ti + rho_t gamma_i du_ti - (rho_t^3 / d) h_ti sum_j du_tj gamma_j h_tj
+        dgamma_j = sum_t du_tj h_tj rho_t
+    (the residual passes dout to h unchanged).
+    """
+    u = rmsnorm(h, gamma, eps, dtype)
+    h64, g64, dout64 = _widen(h, dtype), _widen(gamma, dtype), _widen(dout, dtype)
+    Wg64, W1_64, W3_64, W2_64 = (_widen(a, dtype) for a in (Wg, W1, W3, W2))
+    r = backward(u, Wg64, W1_64, W3_64, W2_64, dout64, k, "f64", alpha=alpha)
+    du = r.pop("dx")
+    d = h64.shape[1]
+    rho = 1.0 / np.sqrt((h64 * h64).sum(axis=1) / d + eps)
+    proj = (du * g64 * h64).sum(axis=1)
+    r["dh"] = dout64 + rho[:, None] * g64 * du - (rho ** 3 / d)[:, None] * h64 * proj[:, None]
+    r["dgamma"] = (du * h64 * rho[:, None]).sum(axis=0)
+    return r

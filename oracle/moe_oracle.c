@@ -71,8 +71,10 @@
  *                      the router like the rest of ds.
  *
  * Operands are row-major: x[T][d], Wg[E][d], W1[E][F][d], W3[E][F][d],
- * W2[E][d][F].  dtype 0 = float32 storage, 1 = bfloat16 bit patterns; every
- * element is widened exactly to double before use.
+ * W2[E][d][F].  dtype 0 = float32 storage, 1 = bfloat16 bit patterns, 2 =
+ * double (for operands that are themselves exact results, such as the
+ * normalised rows of the block form); every element is widened exactly to
+ * double before use.
  */
 #include <math.h>
 #include <stdint.h>
@@ -85,6 +87,7 @@
 /* exact widening of one stored element to double */
 static double elem(const void* base, int dtype, size_t i) {
     if (dtype == 0) return (double)((const float*)base)[i];
+    if (dtype == 2) return ((const double*)base)[i];
     uint32_t bits = ((uint32_t)((const uint16_t*)base)[i]) << 16;
     float f;
     memcpy(&f, &bits, 4);
