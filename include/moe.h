@@ -159,9 +159,25 @@ MOE_API moe_status moe_dispatch(const int32_t* topk_idx, int T, int E, int k, in
  * GPU (other streams, other host threads) race on it.  The first call on a
  * device, with that device current, looks up the array's device address
  * once; make that call before any stream capture begins.
+ *
+ * One check is stricter than moe_dispatch's: `counts` must be device memory
+ * (it picks the device whose copy of the array is used).  A host or
+ * unregistered `counts` returns MOE_ERR_INVALID_ARG with nothing launched,
+ * where moe_dispatch would launch on the current device and fail later.
  */
 MOE_API moe_status moe_dispatch_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* counts,
                                         int32_t* offsets, int32_t* perm, int32_t* inv, cudaStream_t stream);
+
+/*
+ * Bytes the library's stream-ordered memory pool on `device` holds
+ * (reserved) and has handed out (used) at this moment, as the CUDA pool
+ * attributes report them; both 0 if no call has created that pool yet.  An
+ * observability call (no counterpart on the pages): it launches and
+ * synchronises nothing, so allocations still queued on a stream may not be
+ * counted yet.  reserved, used: host (out).  MOE_ERR_INVALID_ARG for a null
+ * pointer or a device index outside [0, 64).
+ */
+MOE_API moe_status moe_pool_stats(int device, size_t* reserved, size_t* used);
 
 /*
  * The whole layer (route, dispatch, experts, combine) with bfloat16 tensors

@@ -68,6 +68,7 @@ SIGNATURES = {
     "moe_train_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
     "moe_backward_ws": (_ci, [_vp] * 12 + [_cf] + [_ci] * 7 + [_vp, _sz, _vp, _sz, _vp, _vp, _vp]),
     "moe_route_stats_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
+    "moe_pool_stats": (_ci, [_ci, _vp, _vp]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -119,6 +120,14 @@ def _dev(t, dtype, name):
     return t
 
 
+def _room(t, numel, name):
+    """A caller-supplied output must hold at least `numel` elements: the kernels write that many and
+    trust the pointer.  Checked before the device and dtype checks, and before anything launches."""
+    if isinstance(t, torch.Tensor) and t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs {numel}")
+    return t
+
+
 def _dtype_code(t):
     if t.dtype == torch.bfloat16:
         return MOE_DTYPE_BF16
@@ -147,6 +156,8 @@ def moe_route(x, Wg, k, topk_idx=None, topk_w=None, stream=None):
         topk_idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    _room(topk_idx, T * k, "topk_idx")
+    _room(topk_w, T * k, "topk_w")
     _dev(topk_idx, torch.int32, "topk_idx")
     _dev(topk_w, torch.float32, "topk_w")
     fn = _lib.moe_route if code == MOE_DTYPE_BF16 else _lib.moe_route_f32
@@ -176,10 +187,16 @@ def moe_dispatch(topk_idx, E, stream=None):
 def moe_dispatch_noalloc(topk_idx, E, counts, offsets, perm, inv, stream=None):
     """moe_dispatch into caller-provided outputs, using the library's fixed scratch array instead of
     any allocation (for callers that may not allocate device memory); raises MoEError above its limit."""
+    if not isinstance(topk_idx, torch.Tensor) or topk_idx.dim() != 2:
+        raise ValueError("topk_idx must be a 2-D [T][k] tensor")
+    T, k = topk_idx.shape
+    for t, numel, n in ((counts, E, "counts"), (offsets, E + 1, "offsets"),
+                        (perm, moe_slots_capacity(T, E, k) if E > 0 and 0 < k <= E else 0, "perm"),
+                        (inv, T * k, "inv")):
+        _room(t, numel, n)
     _dev(topk_idx, torch.int32, "topk_idx")
     for t, n in ((counts, "counts"), (offsets, "offsets"), (perm, "perm"), (inv, "inv")):
         _dev(t, torch.int32, n)
-    T, k = topk_idx.shape
     _check(_lib.moe_dispatch_noalloc(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
                                      _stream(stream, topk_idx, counts, offsets, perm, inv)), "moe_dispatch_noalloc")
     return counts, offsets, perm, inv
@@ -193,6 +210,7 @@ def moe_forward(x, Wg, W1, W3, W2, k, out=None, stream=None):
     T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
     if out is None:
         out = torch.empty((T, d), dtype=x.dtype, device=x.device)
+    _room(out, T * d, "out")
     _dev(out, x.dtype, "out")
     fn = _lib.moe_forward if code == MOE_DTYPE_BF16 else _lib.moe_forward_f32
     _check(fn(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k,
@@ -219,6 +237,7 @@ def moe_forward_ws(x, Wg, W1, W3, W2, k, path=MOE_PATH_AUTO, workspace=None, out
     _dev(workspace, torch.uint8, "workspace")
     if out is None:
         out = torch.empty((T, d), dtype=x.dtype, device=x.device)
+    _room(out, T * d, "out")
     _dev(out, x.dtype, "out")
     _check(_lib.moe_forward_ws(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, code,
                                path, _ptr(workspace), workspace.numel(),
@@ -230,10 +249,11 @@ def moe_forward_profiled(x, Wg, W1, W3, W2, k, workspace, out, events=None, path
     """moe_forward_ws recording torch.cuda.Event objects (MOE_NUM_STAGES + 1 of them, timing enabled)
     at the stage boundaries; returns the number of kernels launched."""
     code = _dtype_code(x)
+    T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
+    _room(out, T * d, "out")
     for t, n in ((x, "x"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2"), (out, "out")):
         _dev(t, x.dtype, n)
     _dev(workspace, torch.uint8, "workspace")
-    T, d, F, E = _layer_shapes(x, Wg, W1, W3, W2)
     ev_arr = _events(events)
     n = ctypes.c_int(0)
     _check(_lib.moe_forward_profiled(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k, code,
@@ -246,9 +266,13 @@ def moe_forward_host(x_host, Wg, W1, W3, W2, k, out_host=None, stream=None):
     """End to end from host memory: x_host / out_host are CPU bf16 tensors (pinned for full speed)."""
     if x_host.is_cuda or x_host.dtype != torch.bfloat16 or not x_host.is_contiguous():
         raise TypeError("x_host must be a contiguous CPU bfloat16 tensor")
+    T, d = x_host.shape
+    if out_host is not None:
+        _room(out_host, T * d, "out_host")
+        if out_host.is_cuda or out_host.dtype != torch.bfloat16 or not out_host.is_contiguous():
+            raise TypeError("out_host must be a contiguous CPU bfloat16 tensor")
     for t, n in ((Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2")):
         _dev(t, torch.bfloat16, n)
-    T, d = x_host.shape
     E, F, _ = W1.shape
     if out_host is None:
         out_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
@@ -289,6 +313,7 @@ def moe_block_forward(h, gamma, eps, Wg, W1, W3, W2, k, alpha=1.0, stats=None, o
     T, d, F, E = _block_args(h, gamma, Wg, W1, W3, W2, stats)
     if out is None:
         out = torch.empty((T, d), dtype=h.dtype, device=h.device)
+    _room(out, T * d, "out")
     _dev(out, h.dtype, "out")
     fn = _lib.moe_block_forward if code == MOE_DTYPE_BF16 else _lib.moe_block_forward_f32
     _check(fn(_ptr(h), _ptr(gamma), float(eps), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), T, d, F, E, k,
@@ -304,6 +329,7 @@ def moe_block_forward_ws(h, gamma, eps, Wg, W1, W3, W2, k, workspace, out, alpha
     """moe_block_forward with an explicit workspace, path and optional stage events; returns the launch count."""
     code = _dtype_code(h)
     T, d, F, E = _block_args(h, gamma, Wg, W1, W3, W2, stats)
+    _room(out, T * d, "out")
     _dev(workspace, torch.uint8, "workspace")
     _dev(out, h.dtype, "out")
     n = ctypes.c_int(0)
@@ -360,6 +386,10 @@ def moe_backward_ws(x, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, g
         grads = dict(dx=torch.empty((T, d), dtype=x.dtype, device=dev), dWg=torch.empty((E, d), dtype=f32, device=dev),
                      dW1=torch.empty((E, F, d), dtype=wd, device=dev), dW3=torch.empty((E, F, d), dtype=wd, device=dev),
                      dW2=torch.empty((E, d, F), dtype=wd, device=dev))
+    for n, numel in (("dx", T * d), ("dWg", E * d), ("dW1", E * F * d), ("dW3", E * F * d), ("dW2", E * d * F)):
+        _room(grads[n], numel, n)
+    if dlogits is not None:
+        _room(dlogits, T * E, "dlogits")
     _dev(grads["dx"], x.dtype, "dx")
     _dev(grads["dWg"], torch.float32, "dWg")
     for n in ("dW1", "dW3", "dW2"):
@@ -391,6 +421,17 @@ def moe_get_device_status(stream=None) -> int:
 
 def moe_selftest_wait_timeout(limit_ns: int, stream=None):
     _check(_lib.moe_selftest_wait_timeout(int(limit_ns), _stream(stream)), "moe_selftest_wait_timeout")
+
+
+def moe_pool_stats(device=None):
+    """(reserved, used) bytes of the library's memory pool on `device` (default: torch's current device)."""
+    if device is None:
+        device = torch.cuda.current_device()
+    elif isinstance(device, torch.device):
+        device = device.index if device.index is not None else torch.cuda.current_device()
+    r, u = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(_lib.moe_pool_stats(int(device), ctypes.byref(r), ctypes.byref(u)), "moe_pool_stats")
+    return r.value, u.value
 
 
 def moe_decode_max_tokens() -> int:

@@ -489,6 +489,27 @@ using namespace moe;
 
 extern "C" {
 
+moe_status moe_pool_stats(int device, size_t* reserved, size_t* used) {
+    if (!reserved || !used || device < 0 || device >= kMaxDevices) return MOE_ERR_INVALID_ARG;
+    *reserved = 0;
+    *used = 0;
+    cudaMemPool_t pool;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        pool = g_pools[device];
+    }
+    if (!pool) return MOE_OK;
+    uint64_t r = 0, u = 0;
+    if (cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReservedMemCurrent, &r) != cudaSuccess ||
+        cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemCurrent, &u) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    *reserved = (size_t)r;
+    *used = (size_t)u;
+    return MOE_OK;
+}
+
 moe_status moe_route(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* topk_idx, float* topk_w,
                      cudaStream_t stream) {
     moe_status st = check_sizes(T, d, E, k);

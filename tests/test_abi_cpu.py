@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moe.h")
@@ -203,3 +204,51 @@ def test_backward_argument_checks(lib):
     assert _bwd(lib, ws=0) == 5
     assert _bwd(lib, ws_bytes=1024) == 5
     assert _bwd(lib, T=0) == 0                          # empty batch: no-op
+
+
+def _noalloc_outputs(T, E, k, m, short=None):
+    """CPU int32 tensors sized as moe_dispatch_noalloc needs them, one of them a single element short."""
+    need = {"counts": E, "offsets": E + 1, "perm": m.moe_slots_capacity(T, E, k), "inv": T * k}
+    return [torch.zeros(need[n] - (1 if n == short else 0), dtype=torch.int32)
+            for n in ("counts", "offsets", "perm", "inv")]
+
+
+def test_noalloc_binding_rejects_undersized_outputs():
+    """The wrapper checks the room in every caller buffer before anything reaches the library: a
+    buffer one element short raises ValueError; buffers of the right size pass the size checks and
+    only then meet the device check (CPU tensors here)."""
+    import sparse_mixture_experts_14_b200 as m
+    T, E, k = 3000, 8, 2
+    idx = torch.zeros((T, k), dtype=torch.int32)
+    for short in ("counts", "offsets", "perm", "inv"):
+        with pytest.raises(ValueError, match=short):
+            m.moe_dispatch_noalloc(idx, E, *_noalloc_outputs(T, E, k, m, short))
+    with pytest.raises(ValueError, match="2-D"):
+        m.moe_dispatch_noalloc(idx.reshape(-1), E, *_noalloc_outputs(T, E, k, m))
+    with pytest.raises(TypeError, match="CUDA"):
+        m.moe_dispatch_noalloc(idx, E, *_noalloc_outputs(T, E, k, m))
+
+
+def test_binding_rejects_undersized_layer_outputs():
+    import sparse_mixture_experts_14_b200 as m
+    T, d, F, E, k = 8, 64, 128, 4, 2
+    bf = torch.bfloat16
+    x, Wg = torch.zeros((T, d), dtype=bf), torch.zeros((E, d), dtype=bf)
+    W1, W3, W2 = torch.zeros((E, F, d), dtype=bf), torch.zeros((E, F, d), dtype=bf), torch.zeros((E, d, F), dtype=bf)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="out"):
+        m.moe_forward_profiled(x, Wg, W1, W3, W2, k, ws, torch.zeros(T * d - 1, dtype=bf))
+    with pytest.raises(ValueError, match="out_host"):
+        m.moe_forward_host(x, Wg, W1, W3, W2, k, out_host=torch.zeros(T * d - 1, dtype=bf))
+
+
+def test_pool_stats_argument_checks(lib):
+    fn = lib.moe_pool_stats
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    r, u = ctypes.c_size_t(7), ctypes.c_size_t(7)
+    assert fn(0, None, ctypes.byref(u)) == 1
+    assert fn(-1, ctypes.byref(r), ctypes.byref(u)) == 1
+    assert fn(64, ctypes.byref(r), ctypes.byref(u)) == 1
+    assert fn(0, ctypes.byref(r), ctypes.byref(u)) == 0     # no pool created in this process: zeros
+    assert (r.value, u.value) == (0, 0)

@@ -2,8 +2,11 @@
 
 It must give exactly what moe_dispatch gives (integer outputs: bit for bit),
 on two calls in a row that leave different contents in the shared fixed
-scratch array, and refuse sizes past that array's limit.  This file is
-collected last so a stop-at-first-failure run has already run everything else.
+scratch array, and refuse sizes past that array's limit.  It must leave the
+library's memory pool exactly as it found it, and an empty batch (T = 0) must
+give all-zero counts and offsets even after an earlier call left data in the
+array.  This file is collected last so a stop-at-first-failure run has
+already run everything else.
 """
 import ctypes
 
@@ -71,3 +74,34 @@ def test_noalloc_refuses_past_its_limit(moe):
     assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
     assert int(outs[0][0]) == -7            # nothing launched
     _compare(moe, 126976, 32, 2, seed=5)    # the largest accepted size still matches
+
+
+def test_noalloc_empty_batch_after_a_full_one(moe):
+    _compare(moe, 3000, 8, 2, seed=11)      # leaves counts and offsets of 6000 assignments in the array
+    E, k = 8, 2
+    idx = torch.empty((0, k), dtype=torch.int32, device="cuda")
+    counts, offsets, perm, inv = _outputs(0, E, k, moe)
+    moe.moe_dispatch_noalloc(idx, E, counts, offsets, perm, inv)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    assert torch.equal(counts.cpu(), torch.zeros(E, dtype=torch.int32))
+    assert torch.equal(offsets.cpu(), torch.zeros(E + 1, dtype=torch.int32))
+
+
+def test_noalloc_leaves_the_pool_untouched(moe):
+    T, E, k = 9000, 8, 2
+    idx = _routing(T, E, k, seed=3)
+    outs = _outputs(T, E, k, moe)
+    moe.moe_dispatch(idx, E)                # the pooled call may create or grow the pool
+    moe.moe_dispatch_noalloc(idx, E, *outs)  # a first call loads the array's module (lazy loading)
+    torch.cuda.synchronize()
+    pool_before = moe.moe_pool_stats()
+    torch_before = torch.cuda.memory_reserved()
+    free_before = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        moe.moe_dispatch_noalloc(idx, E, *outs)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    assert moe.moe_pool_stats() == pool_before
+    assert torch.cuda.memory_reserved() == torch_before
+    assert torch.cuda.mem_get_info()[0] == free_before
