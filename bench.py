@@ -3,6 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
+The default workload is the largest one, the 8x22B-shape prefill layer
+(T=16384, d=6144, ffn=16384, E=8, k=2, bf16); --config 2 is the Mixtral-shape
+decode layer (T=16), --config 3 / 4 the Mixtral-shape prefill and skewed ones.
+
 A step is one call of the whole layer (route, dispatch, gather, expert GEMMs,
 combine) over one batch of T tokens of the chosen workload, with inputs and
 weights already resident in HBM.  The timed region is K steps bracketed by a
@@ -50,14 +54,17 @@ BLOCK_METRIC = ("MoE sub-layer (RMSNorm + MoE + residual, load-balance statistic
 BLOCK_ALPHA = 0.01
 TRAIN_METRIC = "MoE-layer training step (forward + backward) tokens/sec at 1 B200; achieved % of roofline"
 L2_BYTES = 126 * 1000 * 1000
-DEFAULT_CONFIG = 2   # the Mixtral-shape decode layer (T=16, d=4096, ffn=14336, E=8, k=2)
+# the largest workload: the 8x22B-shape prefill layer (T=16384, d=6144, ffn=16384, E=8, k=2)
+DEFAULT_CONFIG = 5
+# timed steps when --steps is not given: about half a second of layer calls per workload
+DEFAULT_STEPS = {1: 200, 2: 200, 3: 60, 4: 40, 5: 30}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default: by workload, ~0.5 s)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(moe_inputs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -78,7 +85,10 @@ def parse_args():
     ap.add_argument("--stage-every", type=int, default=8,
                     help="record per-stage events on every n-th timed step (events between launches "
                          "break the overlap of dependent launches, so most steps run without them)")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 8 if args.train else DEFAULT_STEPS[args.config]
+    return args
 
 
 def load_peaks():
