@@ -66,3 +66,46 @@ def sample_tokens(T, n, seed=0):
     s = set(rng.choice(T, size=min(n, T), replace=False).tolist())
     s.update({0, T - 1})
     return np.array(sorted(s), dtype=np.int32)
+
+
+def stratified_tokens(idx, E, n_random=8, boundaries=3, odd_tail=8, seed=0, tile=128):
+    """Tokens that reach every tile case of the grouped GEMMs, chosen from a routing idx [T][k]
+    (the oracle's, so the choice never depends on the CUDA path).
+
+    Within expert e's segment the rows are the tokens that chose e, in increasing token order
+    (the dispatch is a stable counting sort), so row r of the segment is the r-th such token.
+    For every expert with tokens this takes:
+      * its first and last row;
+      * the rows on both sides of up to `boundaries` of its 128-row m-tile boundaries, always
+        including the first and the last boundary;
+      * up to `odd_tail` rows spread over its last m-tile when it has an odd number of m-tiles
+        (the CTA pair's second half is then empty);
+    plus `n_random` tokens drawn uniformly, and tokens 0 and T - 1.
+    """
+    idx = np.asarray(idx)
+    T = idx.shape[0]
+    picked = {0, T - 1}
+    for e in range(E):
+        rows = np.nonzero((idx == e).any(axis=1))[0]
+        n = len(rows)
+        if n == 0:
+            continue
+        want = {0, n - 1}
+        mt = (n + tile - 1) // tile
+        bnds = list(range(tile, n, tile))
+        if bnds:
+            sel = sorted({bnds[0], bnds[-1], bnds[len(bnds) // 2]})[:max(boundaries, 2)]
+            for b in sel:
+                want.update({b - 1, b})
+        if mt % 2 == 1:
+            lo = (mt - 1) * tile
+            want.update(np.linspace(lo, n - 1, min(odd_tail, n - lo)).astype(np.int64).tolist())
+        picked.update(int(rows[r]) for r in want)
+    rng = np.random.default_rng(seed)
+    picked.update(rng.choice(T, size=min(n_random, T), replace=False).tolist())
+    return np.array(sorted(picked), dtype=np.int32)
+
+
+def experts_reached(idx, tokens):
+    """Experts chosen by at least one of `tokens` (routing idx [T][k])."""
+    return set(np.unique(np.asarray(idx)[tokens]).tolist())

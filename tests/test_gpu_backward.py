@@ -25,7 +25,7 @@ import torch
 
 import moe_inputs
 import oracle
-from moe_testlib import MARGIN, out_to_f64, sample_tokens, to_dev, upload
+from moe_testlib import MARGIN, experts_reached, out_to_f64, stratified_tokens, to_dev, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -188,11 +188,12 @@ def test_backward_experts_without_tokens(moe):
     _check("dx", _f64(g["dx"]), ref["dx"], "bf16")
 
 
-@pytest.mark.parametrize("cfg,n_tok,alpha", [(1, 0, 0.0), (1, 0, 0.5), (3, 12, 0.0), (3, 8, 0.01), (5, 6, 0.0)])
+@pytest.mark.parametrize("cfg,n_tok,alpha", [(1, 0, 0.0), (1, 0, 0.5), (3, 1, 0.0), (3, 1, 0.01), (5, 1, 0.0)])
 def test_backward_configs(moe, cfg, n_tok, alpha):
     """Full-size workloads (in the launch configuration bench.py --train times): dx and dlogits on
-    sampled tokens, slices of the weight gradients of two experts, and dWg against the GPU's own
-    dlogits reduced on the host; alpha != 0 includes the load-balance loss."""
+    a stratified token sample (every expert's first and last row, its m-tile boundaries, odd last
+    m-tiles), slices of the weight gradients of two experts; alpha != 0 includes the load-balance
+    loss.  dWg at full size is pinned by test_backward_dwg_full_size."""
     inp = moe_inputs.make_config(cfg)
     dtype = inp.dtype
     dout = moe_inputs.make_dout(inp.T, inp.d, dtype, seed=inp.seed)
@@ -204,7 +205,9 @@ def test_backward_configs(moe, cfg, n_tok, alpha):
         for n in ("dx", "dlogits", "dWg", "dW1", "dW3", "dW2"):
             _check(n, _f64(g[n]), ref[n], dtype, K)
         return
-    toks = sample_tokens(inp.T, n_tok, seed=cfg)
+    r_idx = oracle.route(inp.x, inp.Wg, inp.k, dtype)[0]
+    toks = stratified_tokens(r_idx, inp.E, n_random=4, boundaries=2, odd_tail=3, seed=cfg)
+    assert experts_reached(r_idx, toks) == set(range(inp.E))
     ref = oracle.backward_tokens(*inp.arrays(), dout, inp.k, dtype, toks, alpha=alpha)
     keep = ref["margin"] >= MARGIN
     _check("dx", _f64(g["dx"])[toks][keep], ref["dx"][keep], dtype)
@@ -219,9 +222,39 @@ def test_backward_configs(moe, cfg, n_tok, alpha):
         _check(f"dW1[{e}]", _f64(g["dW1"][e][fs]), r1, dtype)
         _check(f"dW3[{e}]", _f64(g["dW3"][e][fs]), r3, dtype)
         _check(f"dW2[{e}]", _f64(g["dW2"][e][:, fs]), c2, dtype)
-    # dWg = dlogits^T x: the GPU's reduction of its own router-score gradient
-    want = g["dlogits"].double().T @ dev[0].double()
-    _check("dWg", _f64(g["dWg"]), want.cpu().numpy(), "f32", inp.T)
+    del dev, g
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("cfg", [3, 5])
+def test_backward_dwg_full_size(moe, cfg):
+    """dWg at full size against the oracle.  dout is kept on a stratified sample of tokens and
+    set to zero on every other token, so the loss only sees the sample: the oracle's score
+    gradient of those tokens gives dWg = sum_t ds_t x_t^T exactly, while the GPU still reduces
+    over all T tokens in its full-size launch configuration.  Tokens with dout = 0 get dx = 0
+    and a zero score gradient exactly (dy = 0 and dg = 0)."""
+    inp = moe_inputs.make_config(cfg)
+    dtype = inp.dtype
+    r_idx = oracle.route(inp.x, inp.Wg, inp.k, dtype)[0]
+    toks = stratified_tokens(r_idx, inp.E, n_random=4, boundaries=2, odd_tail=3, seed=cfg + 10)
+    assert experts_reached(r_idx, toks) == set(range(inp.E))
+    dout = moe_inputs.make_dout(inp.T, inp.d, dtype, seed=inp.seed)
+    mask = np.zeros(inp.T, dtype=bool)
+    mask[toks] = True
+    dout[~mask] = 0
+    dev = upload(inp)
+    _, g, _ = _run(moe, inp, dev, to_dev(dout, dtype), dlogits=True)
+    ref = oracle.backward_tokens(*inp.arrays(), dout, inp.k, dtype, toks)
+    if not (ref["margin"] >= MARGIN).all():
+        pytest.skip("a sampled token sits within the routing margin")
+    x_s = moe_inputs.bf16_bits_to_f32(inp.x[toks]).astype(np.float64) if dtype == "bf16" else \
+        inp.x[toks].astype(np.float64)
+    want = ref["dlogits"].T @ x_s
+    _check("dWg", _f64(g["dWg"]), want, dtype, len(toks))
+    _check("dx", _f64(g["dx"])[toks], ref["dx"], dtype)
+    rest = torch.from_numpy(~mask).cuda()
+    assert torch.count_nonzero(g["dx"][rest]) == 0
+    assert torch.count_nonzero(g["dlogits"][rest]) == 0
     del dev, g
     torch.cuda.empty_cache()
 

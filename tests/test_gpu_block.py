@@ -23,7 +23,7 @@ import torch
 
 import moe_inputs
 import oracle
-from moe_testlib import MARGIN, out_to_f64, sample_tokens, to_dev
+from moe_testlib import MARGIN, experts_reached, out_to_f64, stratified_tokens, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -127,8 +127,10 @@ def test_block_long_rows_bf16(moe):
 # ---------------------------------------------------------------- full-size workloads, sampled tokens
 
 
-@pytest.mark.parametrize("cfg,n", [(1, 0), (2, 0), (3, 40), (5, 16)])
+@pytest.mark.parametrize("cfg,n", [(1, 0), (2, 0), (3, 1), (5, 1)])
 def test_block_configs(moe, cfg, n):
+    """n = 0: every token; n = 1: a stratified sample from the oracle's routing of the normalised
+    rows (every expert's first and last row, m-tile boundaries, odd last m-tiles)."""
     inp = moe_inputs.make_block(moe_inputs.make_config(cfg))
     dv = _upload(inp)
     E, k = inp.E, inp.k
@@ -136,7 +138,11 @@ def test_block_configs(moe, cfg, n):
     out = moe.moe_block_forward(dv["x"], dv["gamma"], EPS, dv["Wg"], dv["W1"], dv["W3"], dv["W2"], k,
                                 alpha=0.01, stats=stats)
     _status_clear(moe)
-    toks = sample_tokens(inp.T, n, seed=cfg) if n else None
+    toks = None
+    if n:
+        r_idx = oracle.select(oracle.block_scores(inp.x, inp.gamma, EPS, inp.Wg, inp.dtype), k)[0]
+        toks = stratified_tokens(r_idx, E, seed=cfg)
+        assert experts_reached(r_idx, toks) == set(range(E))
     ref = oracle.block(inp.x, inp.gamma, EPS, inp.Wg, inp.W1, inp.W3, inp.W2, k=k, dtype=inp.dtype, tokens=toks)
     sel = ref["tokens"]
     got = out_to_f64(out)[sel] if inp.dtype == "bf16" else out.double().cpu().numpy()[sel]
