@@ -167,6 +167,21 @@ class ClockSampler:
                 "samples": len(sms), "power_w_max": round(max(s[2] for s in self.samples), 1)}
 
 
+class nvtx_range:
+    """An NVTX range around a harness phase (warm-up, timed steps, e2e); the library adds its own
+    ranges per layer stage.  A no-op without a profiler attached."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        torch.cuda.nvtx.range_pop()
+        return False
+
+
 # ------------------------------------------------------------------ work accounting
 
 
@@ -412,9 +427,10 @@ def run_ours(args, rank, world, local):
     for row in events:          # create the CUDA events before the library records them
         for e in row:
             e.record(stream)
-    for _ in range(W):
-        step()
-    torch.cuda.synchronize()
+    with nvtx_range("bench.warmup"):
+        for _ in range(W):
+            step()
+        torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -423,14 +439,15 @@ def run_ours(args, rank, world, local):
     sampler.start()
     launches = 0
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(K):
-        if flush:
-            flush_buf.zero_()
-            events[i][0].record(stream)
-        launches += step(events=events[i] if i % every == 0 else None)
-    end.record(stream)
-    torch.cuda.synchronize()
+    with nvtx_range("bench.timed"):
+        start.record(stream)
+        for i in range(K):
+            if flush:
+                flush_buf.zero_()
+                events[i][0].record(stream)
+            launches += step(events=events[i] if i % every == 0 else None)
+        end.record(stream)
+        torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -457,10 +474,12 @@ def run_ours(args, rank, world, local):
                 moe.moe_forward_host(x_host, *dev[1:], k, out_host)
             if world > 1:
                 torch.distributed.barrier()
-            t0 = time.perf_counter()
-            for _ in range(K):
-                moe.moe_forward_host(x_host, *dev[1:], k, out_host)
-            wall = reduce_max(time.perf_counter() - t0, world, device)
+            with nvtx_range("bench.e2e"):
+                t0 = time.perf_counter()
+                for _ in range(K):
+                    moe.moe_forward_host(x_host, *dev[1:], k, out_host)
+                wall = time.perf_counter() - t0
+            wall = reduce_max(wall, world, device)
             e2e = {"value": weak_scaling_value(T, K, world, wall * 1000.0), "unit": "tokens/s",
                    "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
                    "timing": "host wall clock around moe_forward_host (synchronises every step)"}
@@ -583,9 +602,10 @@ def run_train(args, rank, world, local):
                                    events=bev[i] if on else None)
         return n + m
 
-    for _ in range(W):
-        step()
-    torch.cuda.synchronize()
+    with nvtx_range("bench.warmup"):
+        for _ in range(W):
+            step()
+        torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -593,11 +613,12 @@ def run_train(args, rank, world, local):
     sampler.start()
     launches = 0
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(K):
-        launches += step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
+    with nvtx_range("bench.timed"):
+        start.record(stream)
+        for i in range(K):
+            launches += step(i)
+        end.record(stream)
+        torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()

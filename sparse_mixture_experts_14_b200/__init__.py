@@ -21,7 +21,12 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe.so")
+# MOE_LIBRARY=debug loads the bounds-checking build (libmoe_debug.so): the same kernels with every
+# index read from another kernel checked; a failed check records MOE_ERR_DEVICE and skips the access
+_VARIANT = os.environ.get("MOE_LIBRARY", "release")
+if _VARIANT not in ("release", "debug"):
+    raise ImportError(f"MOE_LIBRARY must be 'release' or 'debug', got {_VARIANT!r}")
+LIB_PATH = os.path.join(_HERE, "libmoe_debug.so" if _VARIANT == "debug" else "libmoe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python sparse_mixture_experts_14_b200/build.py` "

@@ -7,6 +7,14 @@ would first import the package, which loads the library being rebuilt.)
 
 Each csrc/*.cu compiles to an object under _build/ (parallel nvcc
 processes); the objects link into sparse_mixture_experts_14_b200/libmoe.so.
+
+The debug variant (build(variant="debug"), or `--debug`) compiles the same
+sources with -DMOE_DEBUG=1 into _build_debug/ and libmoe_debug.so: every
+kernel then checks the indices it reads from other kernels (permutation
+rows, assignment slots, segment offsets, tile rows) against the buffers they
+address, and a failed check records MOE_ERR_DEVICE in the status word and
+skips the access instead of faulting.  The package loads it when the
+environment holds MOE_LIBRARY=debug.
 The CUDA runtime is linked statically and the driver's tensor-map encoder is
 fetched at run time, so the library loads on a machine without a GPU driver
 (symbol checks) and needs no libcuda at link time.
@@ -24,6 +32,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
+VARIANTS = {
+    "release": (BUILD, LIB, []),
+    "debug": (os.path.join(PKG, "_build_debug"), os.path.join(PKG, "libmoe_debug.so"), ["-DMOE_DEBUG=1"]),
+}
 ROOT = os.path.dirname(PKG)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -53,15 +65,16 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
+def build(force: bool = False, verbose: bool = False, extra_flags=None, variant: str = "release") -> str:
+    build_dir, lib, vflags = VARIANTS[variant]
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    os.makedirs(build_dir, exist_ok=True)
     headers = _headers()
-    flags = NVCC_FLAGS + list(extra_flags or [])
+    flags = NVCC_FLAGS + vflags + list(extra_flags or [])
     jobs = []
     objs = []
     for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src).replace(".cu", ".o"))
+        obj = os.path.join(build_dir, os.path.basename(src).replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
             jobs.append([nvcc] + flags + ["-c", src, "-o", obj])
@@ -73,16 +86,17 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
                 sys.stderr.write(" ".join(cmd) + "\n" + r.stdout + r.stderr)
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed on {cmd[-3]}")
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [nvcc] + ARCH + ["-shared", "--cudart", "static", "-o", tmp] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(" ".join(cmd) + "\n" + r.stdout + r.stderr)
-            raise RuntimeError("link of libmoe.so failed")
-        os.replace(tmp, LIB)
-    return LIB
+            raise RuntimeError(f"link of {os.path.basename(lib)} failed")
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                variant="debug" if "--debug" in sys.argv else "release"))

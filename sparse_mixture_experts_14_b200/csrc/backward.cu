@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(256) bwd_scatter_kernel(const T* __restrict__ 
                                                           const float* __restrict__ Y, Meta* __restrict__ meta,
                                                           const int32_t* __restrict__ perm, int E, int T_, int k,
                                                           int d, size_t slots, T* __restrict__ dY,
-                                                          float* __restrict__ dg) {
+                                                          float* __restrict__ dg, int* status) {
     pdl_trigger();
     pdl_wait();
     if (blockIdx.x == 0 && threadIdx.x >= kWaveDgradH && threadIdx.x < kWaveSlots) meta->waves[threadIdx.x] = 0;
@@ -60,6 +60,7 @@ __global__ void __launch_bounds__(256) bwd_scatter_kernel(const T* __restrict__ 
     for (size_t r = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < total && r < slots; r += warps) {
         const int a = perm[r];
         T* dst = dY + r * (size_t)d;
+        debug_check(a >= -1 && a < TK, status);   // -1 marks a padding row
         if (a >= 0 && a < TK) {
             const int t = a / k;
             const float g = w[a];
@@ -192,7 +193,8 @@ __global__ void __launch_bounds__(256) dwg_final_kernel(const float* __restrict_
 template <typename T>
 __global__ void __launch_bounds__(256) dx_combine_kernel(const float* __restrict__ dXp, const int32_t* __restrict__ inv,
                                                          const float* __restrict__ ds, const T* __restrict__ Wg, int T_,
-                                                         int d, int E, int k, T* __restrict__ dx) {
+                                                         int d, int E, int k, size_t slots, int* status,
+                                                         T* __restrict__ dx) {
     pdl_trigger();
     pdl_wait();
     const unsigned q = (unsigned)d / 4;
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float* __restrict
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
             const int slot = inv[(size_t)t * k + j];
-            if (slot < 0) continue;
+            if (slot < 0 || !debug_check((size_t)slot < slots, status)) continue;
             const float4 v = __ldg(reinterpret_cast<const float4*>(dXp + (size_t)slot * d) + c);
             acc.x += v.x;
             acc.y += v.y;
@@ -372,7 +374,7 @@ cudaError_t launch_scatter(const BwdArgs& a, cudaStream_t s) {
     if (blocks < 1) blocks = 1;
     return launch_pdl(bwd_scatter_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, s,
                       static_cast<const T*>(a.dout), a.w, a.Y, a.meta, a.perm, a.E, a.T, a.k, a.d, a.slots,
-                      static_cast<T*>(a.dy), a.dg);
+                      static_cast<T*>(a.dy), a.dg, a.status);
 }
 
 template <typename T>
@@ -398,7 +400,7 @@ cudaError_t launch_dx(const BwdArgs& a, cudaStream_t s) {
     if (blocks < 1) blocks = 1;
     return launch_pdl(dx_combine_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const float*>(a.dxp),
                       a.inv, static_cast<const float*>(a.ds), static_cast<const T*>(a.Wg), a.T, a.d, a.E, a.k,
-                      static_cast<T*>(a.dx));
+                      a.slots, a.status, static_cast<T*>(a.dx));
 }
 
 }  // namespace

@@ -16,7 +16,8 @@ namespace {
 template <bool BF16_OUT, bool RESID>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ Y, const float* __restrict__ w,
                                                       const int32_t* __restrict__ inv, int T, int d, int k,
-                                                      void* __restrict__ out, const void* __restrict__ resid) {
+                                                      size_t slots, int* status, void* __restrict__ out,
+                                                      const void* __restrict__ resid) {
     pdl_trigger();
     pdl_wait();
     const int q = d / 4;   // float4 columns per row
@@ -27,7 +28,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
             const int slot = __ldg(inv + (size_t)t * k + j);
-            if (slot < 0) continue;
+            if (slot < 0 || !debug_check((size_t)slot < slots, status)) continue;
             const float g = __ldg(w + (size_t)t * k + j);
             const float4 y = __ldg(reinterpret_cast<const float4*>(Y + (size_t)slot * d) + c);
             acc.x = fmaf(g, y.x, acc.x);
@@ -64,26 +65,26 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }
 
 template <bool BF16_OUT>
-cudaError_t launch_combine_t(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, void* out,
-                             cudaStream_t s, const void* resid) {
+cudaError_t launch_combine_t(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, size_t slots,
+                             int* status, void* out, cudaStream_t s, const void* resid) {
     const size_t n = (size_t)T * (d / 4);
     size_t blocks = (n + 255) / 256;
     if (blocks > 148 * 32) blocks = 148 * 32;
     if (blocks < 1) blocks = 1;
     auto kern = resid ? combine_kernel<BF16_OUT, true> : combine_kernel<BF16_OUT, false>;
-    return launch_pdl(kern, dim3((unsigned)blocks), dim3(256), 0, s, Y, w, inv, T, d, k, out, resid);
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(256), 0, s, Y, w, inv, T, d, k, slots, status, out, resid);
 }
 
 }  // namespace
 
-cudaError_t launch_combine_bf16(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, void* out,
-                                cudaStream_t s, const void* resid) {
-    return launch_combine_t<true>(Y, w, inv, T, d, k, out, s, resid);
+cudaError_t launch_combine_bf16(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, size_t slots,
+                                int* status, void* out, cudaStream_t s, const void* resid) {
+    return launch_combine_t<true>(Y, w, inv, T, d, k, slots, status, out, s, resid);
 }
 
-cudaError_t launch_combine_f32(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, float* out,
-                               cudaStream_t s, const float* resid) {
-    return launch_combine_t<false>(Y, w, inv, T, d, k, out, s, resid);
+cudaError_t launch_combine_f32(const float* Y, const float* w, const int32_t* inv, int T, int d, int k, size_t slots,
+                               int* status, float* out, cudaStream_t s, const float* resid) {
+    return launch_combine_t<false>(Y, w, inv, T, d, k, slots, status, out, s, resid);
 }
 
 }  // namespace moe

@@ -74,7 +74,7 @@ template <bool GATE>
 __global__ void __launch_bounds__(DTHREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap mapWa, const __grid_constant__ CUtensorMap mapWb,
                   const __grid_constant__ CUtensorMap mapX, const Meta* __restrict__ meta, int E, int K, int R,
-                  void* __restrict__ out, int* status, long long wait_ns) {
+                  size_t slots, void* __restrict__ out, int* status, long long wait_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int DSTAGES = Ring<GATE>::STAGES;
@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(DTHREADS, 1)
         for (int e = 0; e < E; ++e) {
             const int n = meta->counts[e];
             if (n < 0 || n > DNMAX) ok = false;
+            if (!debug_check(n <= 0 || (meta->offsets[e] >= 0 && (size_t)meta->offsets[e] + n <= slots), nullptr))
+                ok = false;   // the segment's rows must lie inside the buffers the epilogue writes
             ctrl->ntok[e] = n;
             ctrl->row0[e] = meta->offsets[e];
             ctrl->tile_base[e + 1] = ctrl->tile_base[e] + (n > 0 ? blocks : 0);
@@ -316,8 +318,8 @@ cudaError_t launch_stage(const CUtensorMap& a, const CUtensorMap& b, const CUten
     int grid = (upper + waves - 1) / waves;
     if (grid > sms) grid = sms;
     if (grid < 1) grid = 1;
-    return launch_pdl(decode_kernel<GATE>, dim3(grid), dim3(DTHREADS), dsmem_bytes<GATE>(), s, a, b, x, g.meta, g.E, K, R, out,
-                      g.status, g.wait_ns);
+    return launch_pdl(decode_kernel<GATE>, dim3(grid), dim3(DTHREADS), dsmem_bytes<GATE>(), s, a, b, x, g.meta, g.E, K, R,
+                      g.slots, out, g.status, g.wait_ns);
 }
 
 }  // namespace

@@ -387,19 +387,21 @@ template <int NORM>
 __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ x, size_t row_bytes, int T, int k,
                                                      const Meta* __restrict__ meta, int E,
                                                      const int32_t* __restrict__ perm, uint8_t* __restrict__ xp,
-                                                     size_t slots, const uint4* __restrict__ gam,
+                                                     size_t slots, int* status, const uint4* __restrict__ gam,
                                                      const float* __restrict__ rstd) {
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
     const size_t total = (size_t)meta->offsets[E];
+    debug_check(total <= slots, status);
     const size_t nvec = row_bytes / 16;
     const long long TK = (long long)T * k;
     for (size_t r = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < total && r < slots;
          r += warps) {
         const int a = perm[r];
         uint4* dst = reinterpret_cast<uint4*>(xp + r * row_bytes);
+        debug_check(a >= -1 && a < TK, status);   // -1 marks a padding row
         if (a >= 0 && a < TK) {
             const int t = a / k;
             copy_row<NORM>(reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes), dst, nvec, lane, gam,
@@ -448,14 +450,16 @@ cudaError_t launch_dispatch_gather_small(const int32_t* idx, int T, int E, int k
 }
 
 cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
-                          const int32_t* perm, void* xp, size_t slots, cudaStream_t s, const GatherNorm& nm) {
+                          const int32_t* perm, void* xp, size_t slots, int* status, cudaStream_t s,
+                          const GatherNorm& nm) {
     const size_t rows_per_block = 8;
     size_t blocks = (slots + rows_per_block - 1) / rows_per_block;
     if (blocks > 65535 * 4) blocks = 65535 * 4;
     const uint4* gam = static_cast<const uint4*>(nm.gamma);
     auto kern = !nm.gamma ? gather_kernel<0> : (elem_bytes == 2 ? gather_kernel<1> : gather_kernel<2>);
     return launch_pdl(kern, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const uint8_t*>(x),
-                      (size_t)d * elem_bytes, T, k, meta, E, perm, static_cast<uint8_t*>(xp), slots, gam, nm.rstd);
+                      (size_t)d * elem_bytes, T, k, meta, E, perm, static_cast<uint8_t*>(xp), slots, status, gam,
+                      nm.rstd);
 }
 
 }  // namespace moe

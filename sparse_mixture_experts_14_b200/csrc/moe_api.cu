@@ -5,10 +5,41 @@
 #include <cstdlib>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe_common.cuh"
 #include "ptx_sm100.cuh"
 
 namespace moe {
+
+// NVTX ranges around the layer's host-side stages, nested in one range per
+// call, so a profiler timeline (Nsight Systems) or an ncu --nvtx filter can
+// tell the stages apart.  Without a tool attached every call is a no-op.
+class NvtxStages {
+   public:
+    NvtxStages(const char* call, const char* const* names, int n) : names_(names), n_(n) { nvtxRangePushA(call); }
+    ~NvtxStages() {
+        if (open_) nvtxRangePop();
+        nvtxRangePop();
+    }
+    // close the current stage's range and open stage i's (i == n closes only)
+    void next(int i) {
+        if (open_) nvtxRangePop();
+        open_ = i >= 0 && i < n_;
+        if (open_) nvtxRangePushA(names_[i]);
+    }
+
+   private:
+    const char* const* names_;
+    int n_;
+    bool open_ = false;
+};
+
+const char* const kFwdStageNames[MOE_NUM_STAGES] = {"moe.route", "moe.dispatch", "moe.gather",
+                                                    "moe.expert1", "moe.expert2", "moe.combine"};
+const char* const kBwdStageNames[MOE_BWD_NUM_STAGES] = {"moe.bwd.scatter", "moe.bwd.dgrad_h", "moe.bwd.swiglu",
+                                                        "moe.bwd.dgrad_x", "moe.bwd.wgrad2", "moe.bwd.wgrad13",
+                                                        "moe.bwd.router"};
 
 __device__ int g_status;   // per-device sticky fault word (first fault wins)
 
@@ -181,7 +212,11 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
     void* h = ws + p.h;
     float* y = reinterpret_cast<float*>(ws + p.y);
 
-    auto mark = [&](int stage) -> cudaError_t { return ev ? cudaEventRecord(ev[stage], s) : cudaSuccess; };
+    NvtxStages nvtx(bo ? "moe.block_forward" : "moe.forward", kFwdStageNames, MOE_NUM_STAGES);
+    auto mark = [&](int stage) -> cudaError_t {
+        nvtx.next(stage);
+        return ev ? cudaEventRecord(ev[stage], s) : cudaSuccess;
+    };
     int n = 0;
     MOE_TRY(mark(MOE_STAGE_ROUTE));
     if (dtype == MOE_DTYPE_BF16) {
@@ -207,7 +242,7 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
         MOE_TRY(launch_dispatch(idx, T, E, k, blk, meta, perm, inv, dev.status, s));
         n += dispatch_launches(T);
         MOE_TRY(mark(MOE_STAGE_GATHER));
-        MOE_TRY(launch_gather(x, es, T, d, E, k, meta, perm, xp, p.slots, s, nm));
+        MOE_TRY(launch_gather(x, es, T, d, E, k, meta, perm, xp, p.slots, dev.status, s, nm));
         n += 1;
     }
     if (dtype == MOE_DTYPE_BF16) {
@@ -223,7 +258,7 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
         MOE_TRY(mark(MOE_STAGE_EXPERT2));
         MOE_TRY(decode ? launch_decode(a, 2, s) : launch_tc_gemm2(a, s));
         MOE_TRY(mark(MOE_STAGE_COMBINE));
-        MOE_TRY(launch_combine_bf16(y, w, inv, T, d, k, out, s, resid));
+        MOE_TRY(launch_combine_bf16(y, w, inv, T, d, k, p.slots, dev.status, out, s, resid));
     } else {
         MOE_TRY(mark(MOE_STAGE_EXPERT1));
         MOE_TRY(launch_simt_gemm1_f32(static_cast<const float*>(xp), static_cast<const float*>(W1),
@@ -233,7 +268,7 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
         MOE_TRY(launch_simt_gemm2_f32(static_cast<const float*>(h), static_cast<const float*>(W2), meta, E, d, F, y,
                                       p.slots, s));
         MOE_TRY(mark(MOE_STAGE_COMBINE));
-        MOE_TRY(launch_combine_f32(y, w, inv, T, d, k, static_cast<float*>(out), s,
+        MOE_TRY(launch_combine_f32(y, w, inv, T, d, k, p.slots, dev.status, static_cast<float*>(out), s,
                                    static_cast<const float*>(resid)));
     }
     n += 3;
@@ -392,8 +427,13 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
     a.E = E;
     a.k = k;
     a.slots = p.slots;
+    a.status = dev.status;
 
-    auto mark = [&](int stage) -> cudaError_t { return ev ? cudaEventRecord(ev[stage], s) : cudaSuccess; };
+    NvtxStages nvtx("moe.backward", kBwdStageNames, MOE_BWD_NUM_STAGES);
+    auto mark = [&](int stage) -> cudaError_t {
+        nvtx.next(stage);
+        return ev ? cudaEventRecord(ev[stage], s) : cudaSuccess;
+    };
     int n = 0;
     MOE_TRY(mark(MOE_BWD_STAGE_SCATTER));
     MOE_TRY(launch_bwd_scatter(a, s));

@@ -35,6 +35,26 @@ __device__ __forceinline__ void record_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+#ifndef MOE_DEBUG
+#define MOE_DEBUG 0
+#endif
+// Debug builds (nvcc -DMOE_DEBUG=1, libmoe_debug.so) check the indices a kernel
+// reads from another kernel's output (segment rows, assignment slots, segment
+// offsets, tile rows) against the buffer they address: a failed check records
+// MOE_ERR_DEVICE and returns false, and the caller skips the access.  Release
+// builds compile the check away (it is always true): those indices are in
+// range by construction of the dispatch.
+__device__ __forceinline__ bool debug_check(bool ok, int* status) {
+#if MOE_DEBUG
+    if (!ok) record_status(status, MOE_ERR_DEVICE);
+    return ok;
+#else
+    (void)ok;
+    (void)status;
+    return true;
+#endif
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -218,14 +238,14 @@ cudaError_t launch_dispatch_gather_small(const int32_t* idx, int T, int E, int k
                                          int d, Meta* meta, int32_t* perm, int32_t* inv, void* xp, size_t slots,
                                          int* status, cudaStream_t s, const GatherNorm& nm = GatherNorm());
 cudaError_t launch_gather(const void* x, size_t elem_bytes, int T, int d, int E, int k, const Meta* meta,
-                          const int32_t* perm, void* xp, size_t slots, cudaStream_t s,
+                          const int32_t* perm, void* xp, size_t slots, int* status, cudaStream_t s,
                           const GatherNorm& nm = GatherNorm());
 
 // resid (nullable, [T][d] in the output type) is added after the gate-weighted sum.
 cudaError_t launch_combine_bf16(const float* Y, const float* w, const int32_t* inv, int T, int d, int k,
-                                void* out, cudaStream_t s, const void* resid = nullptr);
+                                size_t slots, int* status, void* out, cudaStream_t s, const void* resid = nullptr);
 cudaError_t launch_combine_f32(const float* Y, const float* w, const int32_t* inv, int T, int d, int k,
-                               float* out, cudaStream_t s, const float* resid = nullptr);
+                               size_t slots, int* status, float* out, cudaStream_t s, const float* resid = nullptr);
 
 cudaError_t launch_simt_gemm1_f32(const float* xp, const float* W1, const float* W3, const Meta* meta, int E,
                                   int d, int F, float* H, size_t slots, cudaStream_t s);
@@ -313,6 +333,7 @@ struct BwdArgs {
     float* dW2;             // [E][d][F]
     int T, d, F, E, k;
     size_t slots;
+    int* status;            // device status word (debug builds record index faults in it)
 };
 size_t dwg_part_bytes(int T, int E, int d);
 cudaError_t launch_bwd_scatter(const BwdArgs& a, cudaStream_t s);      // dY and dg (1 launch)
