@@ -91,6 +91,7 @@ def _load():
             lib.oracle_backward.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, cd] + [vp] * 10
             lib.oracle_backward_tokens.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, cd, vp, ci] + \
                 [vp] * 6 + [ci]
+            lib.oracle_backward_rows.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp] + [vp] * 6 + [ci]
             lib.oracle_balance_grad.argtypes = [ci, ci, ci, vp, cd, vp]
             lib.oracle_weight_grad_slices.argtypes = [ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, ci, vp, ci, vp, ci,
                                                       vp, vp, vp, ci]
@@ -325,6 +326,50 @@ def _widen(a, dtype) -> np.ndarray:
     return a.astype(np.float64)
 
 
+def backward_rows(u, Wg, W1, W3, W2, dout_rows, k: int, dtype: str, nthreads: int = 0) -> dict:
+    """dx and the router-score gradient (output path, alpha = 0) of given input rows u [n][d] held in
+    float64, with Wg, W1, W3, W2 and dout_rows [n][d] stored as `dtype`: dict(dx, dlogits, idx, g, margin,
+    mingap).  The block form's MoE input is the exact normalised row, which no stored dtype holds."""
+    u = np.ascontiguousarray(u, dtype=np.float64)
+    Wg, W1, W3, W2, dout_rows = (_arr(a, dtype) for a in (Wg, W1, W3, W2, dout_rows))
+    n, d = u.shape
+    E, F = W1.shape[0], W1.shape[1]
+    r = dict(dx=np.empty((n, d)), dlogits=np.empty((n, E)), idx=np.empty((n, k), dtype=np.int32),
+             g=np.empty((n, k)), margin=np.empty(n), mingap=np.empty(n))
+    _check(_load().oracle_backward_rows(n, d, F, E, k, u.ctypes.data, Wg.ctypes.data, W1.ctypes.data,
+                                        W3.ctypes.data, W2.ctypes.data, DTYPE_CODE[dtype], dout_rows.ctypes.data,
+                                        *[r[m].ctypes.data for m in ("dx", "dlogits", "idx", "g", "margin",
+                                                                     "mingap")], nthreads), "backward_rows")
+    return r
+
+
+def _block_chain(h64, g64, dout64, du, eps: float):
+    """The RMSNorm and residual part of the block backward (see block_backward): (dh, dgamma)."""
+    d = h64.shape[1]
+    rho = 1.0 / np.sqrt((h64 * h64).sum(axis=1) / d + eps)
+    proj = (du * g64 * h64).sum(axis=1)
+    dh = dout64 + rho[:, None] * g64 * du - (rho ** 3 / d)[:, None] * h64 * proj[:, None]
+    dgamma = (du * h64 * rho[:, None]).sum(axis=0)
+    return dh, dgamma
+
+
+def block_backward_tokens(h, gamma, eps: float, Wg, W1, W3, W2, dout, k: int, dtype: str, tokens,
+                          nthreads: int = 0) -> dict:
+    """block_backward (alpha = 0) restricted to the listed tokens, for full-size layers: dh of those rows
+    and dgamma summed over them, plus their score gradients and routing: dict(dh, dgamma, dlogits, idx, g,
+    margin, mingap, tokens).  Equal to block_backward's dh rows, and to its dgamma when dout is zero on
+    every other token.  Without the load-balance part the tokens are independent."""
+    tok = np.ascontiguousarray(tokens, dtype=np.int64)
+    h_s = _arr(h, dtype)[tok]
+    dout_s = _arr(dout, dtype)[tok]
+    u = rmsnorm(h_s, gamma, eps, dtype)
+    r = backward_rows(u, Wg, W1, W3, W2, dout_s, k, dtype, nthreads)
+    du = r.pop("dx")
+    r["dh"], r["dgamma"] = _block_chain(_widen(h_s, dtype), _widen(gamma, dtype), _widen(dout_s, dtype), du, eps)
+    r["tokens"] = tok
+    return r
+
+
 def block_backward(h, gamma, eps: float, Wg, W1, W3, W2, dout, k: int, dtype: str, alpha: float = 0.0) -> dict:
     """Every gradient of L = sum <dout, out> + alpha E sum f p for out = h + MoE(RMSNorm(h)), with the
     top-k choice held fixed (small shapes): dict(dh, dgamma, dWg, dW1, dW3, dW2, dlogits, idx, g,
@@ -342,9 +387,5 @@ def block_backward(h, gamma, eps: float, Wg, W1, W3, W2, dout, k: int, dtype: st
     Wg64, W1_64, W3_64, W2_64 = (_widen(a, dtype) for a in (Wg, W1, W3, W2))
     r = backward(u, Wg64, W1_64, W3_64, W2_64, dout64, k, "f64", alpha=alpha)
     du = r.pop("dx")
-    d = h64.shape[1]
-    rho = 1.0 / np.sqrt((h64 * h64).sum(axis=1) / d + eps)
-    proj = (du * g64 * h64).sum(axis=1)
-    r["dh"] = dout64 + rho[:, None] * g64 * du - (rho ** 3 / d)[:, None] * h64 * proj[:, None]
-    r["dgamma"] = (du * h64 * rho[:, None]).sum(axis=0)
+    r["dh"], r["dgamma"] = _block_chain(h64, g64, dout64, du, eps)
     return r

@@ -458,16 +458,22 @@ static void scratch_free(struct bwd_scratch* w) {
  * (zero for unselected experts).  When dWg/dW1/dW3/dW2 are non-null the
  * token's contributions are added to them (the caller runs tokens in order).
  */
-static void token_backward(int d, int F, int E, int k, const void* x, const void* Wg, const void* W1, const void* W3,
-                           const void* W2, int dtype, const void* dout, size_t t, struct bwd_scratch* w, double* dx,
-                           double* ds, int32_t* idx, double* g, double* margin, double* mingap, double* dWg,
-                           double* dW1, double* dW3, double* dW2, const double* ds_extra) {
+static void token_backward(int d, int F, int E, int k, const void* x, int xdtype, const void* Wg, const void* W1,
+                           const void* W3, const void* W2, int dtype, const void* dout, size_t t,
+                           struct bwd_scratch* w, double* dx, double* ds, int32_t* idx, double* g, double* margin,
+                           double* mingap, double* dWg, double* dW1, double* dW3, double* dW2,
+                           const double* ds_extra) {
+    /* x is read as xdtype (the layer's dtype, or double for the block form's exact normalised rows) */
     for (int j = 0; j < d; ++j) {
-        w->xv[j] = elem(x, dtype, t * (size_t)d + j);
+        w->xv[j] = elem(x, xdtype, t * (size_t)d + j);
         w->go[j] = elem(dout, dtype, t * (size_t)d + j);
     }
     double s[64], dg[64];
-    token_scores(d, E, x, Wg, dtype, t, s);
+    for (int e = 0; e < E; ++e) {   /* step 1, as token_scores: j ascending */
+        double acc = 0.0;
+        for (int j = 0; j < d; ++j) acc += w->xv[j] * elem(Wg, dtype, (size_t)e * d + j);
+        s[e] = acc;
+    }
     token_select(E, k, s, idx, g, margin, mingap);
     for (int j = 0; j < k; ++j) {
         expert_forward_keep(d, F, w->xv, W1, W3, W2, dtype, idx[j], w->a + (size_t)j * F, w->b + (size_t)j * F,
@@ -598,7 +604,7 @@ int oracle_backward(int T, int d, int F, int E, int k, const void* x, const void
     memset(dW3, 0, sizeof(double) * (size_t)E * F * d);
     memset(dW2, 0, sizeof(double) * (size_t)E * d * F);
     for (int t = 0; t < T; ++t)
-        token_backward(d, F, E, k, x, Wg, W1, W3, W2, dtype, dout, (size_t)t, &w, dx + (size_t)t * d,
+        token_backward(d, F, E, k, x, dtype, Wg, W1, W3, W2, dtype, dout, (size_t)t, &w, dx + (size_t)t * d,
                        dlogits + (size_t)t * E, idx + (size_t)t * k, g + (size_t)t * k, margin + t, mingap + t, dWg,
                        dW1, dW3, dW2, bal ? bal + (size_t)t * E : NULL);
     scratch_free(&w);
@@ -630,7 +636,7 @@ int oracle_backward_tokens(int T, int d, int F, int E, int k, const void* x, con
         } else {
 #pragma omp for schedule(dynamic, 1)
             for (int r = 0; r < n; ++r)
-                token_backward(d, F, E, k, x, Wg, W1, W3, W2, dtype, dout, (size_t)tokens[r], &w,
+                token_backward(d, F, E, k, x, dtype, Wg, W1, W3, W2, dtype, dout, (size_t)tokens[r], &w,
                                dx + (size_t)r * d, dlogits + (size_t)r * E, idx + (size_t)r * k, g + (size_t)r * k,
                                margin + r, mingap + r, NULL, NULL, NULL, NULL,
                                bal ? bal + (size_t)tokens[r] * E : NULL);
@@ -638,6 +644,40 @@ int oracle_backward_tokens(int T, int d, int F, int E, int k, const void* x, con
         scratch_free(&w);
     }
     free(bal);
+    return fail ? 2 : 0;
+}
+
+/*
+ * dx and ds (step 8, output path only: alpha = 0) of n given input rows held in
+ * double, x_rows [n][d], with the operands Wg, W1, W3, W2 and the upstream
+ * gradient rows dout_rows [n][d] stored as dtype.  The block form's backward
+ * needs this: the MoE layer's input there is the exact normalised row u, which
+ * no stored dtype holds, while its weights stay in theirs.  Rows are
+ * independent (without the load-balance part nothing couples them).
+ */
+int oracle_backward_rows(int n, int d, int F, int E, int k, const double* x_rows, const void* Wg, const void* W1,
+                         const void* W3, const void* W2, int dtype, const void* dout_rows, double* dx,
+                         double* dlogits, int32_t* idx, double* g, double* margin, double* mingap, int nthreads) {
+    if (n < 0 || d <= 0 || F <= 0 || E <= 0 || E > 64 || k <= 0 || k > E) return 1;
+    int fail = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        struct bwd_scratch w;
+        if (!scratch_alloc(&w, d, F, k)) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int r = 0; r < n; ++r)
+                token_backward(d, F, E, k, x_rows, 2, Wg, W1, W3, W2, dtype, dout_rows, (size_t)r, &w,
+                               dx + (size_t)r * d, dlogits + (size_t)r * E, idx + (size_t)r * k, g + (size_t)r * k,
+                               margin + r, mingap + r, NULL, NULL, NULL, NULL, NULL);
+        }
+        scratch_free(&w);
+    }
     return fail ? 2 : 0;
 }
 

@@ -139,3 +139,36 @@ def test_zero_w2_passes_dout_through(dtype):
     for n in ("dgamma", "dWg", "dW1", "dW3", "dlogits"):
         assert np.all(g[n] == 0.0), n
     assert np.any(g["dW2"] != 0.0)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_rows_equal_backward_tokens(dtype):
+    """backward_rows reads its input rows as float64: given the exactly widened rows of x it is
+    backward_tokens bit for bit (the same per-token arithmetic)."""
+    inp = moe_inputs.make_inputs(40, 32, 48, 6, 2, dtype, seed=71)
+    dout = moe_inputs.make_dout(40, 32, dtype, 71)
+    toks = np.array([0, 3, 17, 39], dtype=np.int32)
+    a = oracle.backward_tokens(*inp.arrays(), dout, 2, dtype, toks)
+    b = oracle.backward_rows(_f64(inp.x[toks], dtype), inp.Wg, inp.W1, inp.W3, inp.W2, dout[toks], 2, dtype)
+    for n in ("dx", "dlogits", "g", "margin", "mingap"):
+        assert np.array_equal(a[n], b[n]), n
+    assert np.array_equal(a["idx"], b["idx"])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_block_backward_tokens_is_block_backward_restricted(dtype):
+    """With dout zero on every token but the listed ones, the full block backward's dh rows of the
+    listed tokens and its dgamma (a sum in which every other token adds an exact zero) are the
+    token-restricted ones; the other tokens get dh = 0."""
+    blk = _block_inputs(24, 32, 48, 5, 2, dtype, seed=72)
+    dout = moe_inputs.make_dout(24, 32, dtype, 72)
+    toks = np.array([1, 2, 11, 23], dtype=np.int64)
+    mask = np.zeros(24, dtype=bool)
+    mask[toks] = True
+    dout[~mask] = 0
+    full = oracle.block_backward(blk.x, blk.gamma, EPS, blk.Wg, blk.W1, blk.W3, blk.W2, dout, 2, dtype)
+    part = oracle.block_backward_tokens(blk.x, blk.gamma, EPS, blk.Wg, blk.W1, blk.W3, blk.W2, dout, 2, dtype, toks)
+    np.testing.assert_allclose(part["dh"], full["dh"][toks], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(part["dgamma"], full["dgamma"], rtol=1e-12, atol=1e-15)
+    np.testing.assert_array_equal(part["dlogits"], full["dlogits"][toks])
+    assert np.all(full["dh"][~mask] == 0)
