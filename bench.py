@@ -53,6 +53,8 @@ BLOCK_METRIC = ("MoE sub-layer (RMSNorm + MoE + residual, load-balance statistic
                 "achieved % of roofline")
 BLOCK_ALPHA = 0.01
 TRAIN_METRIC = "MoE-layer training step (forward + backward) tokens/sec at 1 B200; achieved % of roofline"
+BLOCK_TRAIN_METRIC = ("MoE sub-layer (RMSNorm + MoE + residual) training step (forward + backward) tokens/sec "
+                      "at 1 B200; achieved % of roofline")
 L2_BYTES = 126 * 1000 * 1000
 # the largest workload: the 8x22B-shape prefill layer (T=16384, d=6144, ffn=16384, E=8, k=2)
 DEFAULT_CONFIG = 5
@@ -243,21 +245,29 @@ def oracle_fn(inp, block):
     return lambda toks, nt: oracle.moe(*inp.arrays(), k=inp.k, dtype=inp.dtype, tokens=toks, nthreads=nt)
 
 
-def oracle_train_run(inp, dout, target_s):
+def oracle_train_run(inp, dout, target_s, block=False):
     """Time the oracle's forward + backward (all gradients) on an evenly spaced token sample of about
-    target_s seconds (the oracle's backward runs on one thread); returns (tokens/s, sample text, seconds)."""
+    target_s seconds (the oracle's backward runs on one thread); returns (tokens/s, sample text, seconds).
+    block: the block form's backward (RMSNorm and residual around the layer, dh and dgamma included)."""
     import oracle
-    sub = lambda toks: [np.ascontiguousarray(inp.x[toks]), inp.Wg, inp.W1, inp.W3, inp.W2,
-                        np.ascontiguousarray(dout[toks])]
+
+    def run(toks):
+        x, d_s = np.ascontiguousarray(inp.x[toks]), np.ascontiguousarray(dout[toks])
+        if block:
+            return oracle.block_backward(x, inp.gamma, moe_inputs.BLOCK_EPS, inp.Wg, inp.W1, inp.W3, inp.W2, d_s,
+                                         inp.k, inp.dtype, alpha=BLOCK_ALPHA)
+        return oracle.backward(x, inp.Wg, inp.W1, inp.W3, inp.W2, d_s, inp.k, inp.dtype, alpha=BLOCK_ALPHA)
+
     t0 = time.perf_counter()
-    oracle.backward(*sub([0]), inp.k, inp.dtype, alpha=BLOCK_ALPHA)
+    run([0])
     per_tok = max(time.perf_counter() - t0, 1e-5)
     n = int(max(1, min(inp.T, round(target_s / per_tok))))
     toks = np.unique(np.linspace(0, inp.T - 1, n).astype(np.int64))
     t0 = time.perf_counter()
-    oracle.backward(*sub(toks), inp.k, inp.dtype, alpha=BLOCK_ALPHA)
+    run(toks)
     dt = time.perf_counter() - t0
-    sample = (f"{len(toks)} of {inp.T} tokens (evenly spaced): forward and every gradient (dx, dWg, dW1, dW3, dW2, "
+    what = "dh, dgamma, dWg, dW1, dW3, dW2" if block else "dx, dWg, dW1, dW3, dW2"
+    sample = (f"{len(toks)} of {inp.T} tokens (evenly spaced): forward and every gradient ({what}, "
               f"load-balance loss included) of those tokens in fp64, one thread")
     return len(toks) / dt, sample, dt
 
@@ -310,18 +320,20 @@ def run_reference(args, rank):
         dout = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
         per_step = max(0.05, min(30.0, args.ref_seconds / max(args.steps + args.warmup, 1)))
         for _ in range(args.warmup):
-            oracle_train_run(inp, dout, per_step)
+            oracle_train_run(inp, dout, per_step, args.block)
         total_tok, total_t = 0.0, 0.0
         for _ in range(args.steps):
-            v, sample, dt = oracle_train_run(inp, dout, per_step)
+            v, sample, dt = oracle_train_run(inp, dout, per_step, args.block)
             total_tok += v * dt
             total_t += dt
         value = total_tok / total_t
         line = {
-            "impl": "reference", "metric": TRAIN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "impl": "reference", "metric": BLOCK_TRAIN_METRIC if args.block else TRAIN_METRIC, "value": value,
+            "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_t / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_name(args.config, args.shape) + "+train", "T": inp.T, "d": inp.d,
+            "config": {"workload": workload_name(args.config, args.shape) + ("+block" if args.block else "") + "+train",
+                       "T": inp.T, "d": inp.d,
                        "ffn": inp.F, "E": inp.E,
                        "k": inp.k, "seed": c["seed"]},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
@@ -550,19 +562,28 @@ def run_ours(args, rank, world, local):
 
 def run_train(args, rank, world, local):
     """One step = moe_forward_profiled (training path) + moe_backward_ws with the load-balance loss
-    (alpha = 0.01) over one batch, inputs resident."""
+    (alpha = 0.01) over one batch, inputs resident.  With --block: the block form, moe_block_forward_ws
+    (training path, statistics on) + moe_block_backward_ws (dh, dgamma and the layer's gradients)."""
     import sparse_mixture_experts_14_b200 as moe
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     c = moe_inputs.WORKLOADS[args.config]
-    inp = make_workload(args.config, False, args.shape)
+    block = args.block
+    inp = make_workload(args.config, block, args.shape)
     dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
     dout_np = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
     dout = to_dev(dout_np, inp.dtype, device)
     T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
     code = moe.MOE_DTYPE_BF16 if inp.dtype == "bf16" else moe.MOE_DTYPE_F32
-    fws = torch.empty(moe.moe_train_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
-    bws = torch.empty(moe.moe_backward_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
+    if block:
+        gamma = to_dev(inp.gamma, inp.dtype, device)
+        stats = torch.empty(2 * E + 1, dtype=torch.float32, device=device)
+        fws = torch.empty(moe.moe_block_train_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
+        bws = torch.empty(moe.moe_block_backward_workspace_size(T, d, F, E, k, code), dtype=torch.uint8,
+                          device=device)
+    else:
+        fws = torch.empty(moe.moe_train_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
+        bws = torch.empty(moe.moe_backward_workspace_size(T, d, F, E, k, code), dtype=torch.uint8, device=device)
     out = torch.empty((T, d), dtype=dev[0].dtype, device=device)
     f32 = torch.float32
     wd = torch.bfloat16 if (args.bf16_wgrad and inp.dtype == "bf16") else f32
@@ -570,9 +591,16 @@ def run_train(args, rank, world, local):
                  dWg=torch.empty((E, d), dtype=f32, device=device), dW1=torch.empty((E, F, d), dtype=wd, device=device),
                  dW3=torch.empty((E, F, d), dtype=wd, device=device),
                  dW2=torch.empty((E, d, F), dtype=wd, device=device))
-    idx, _ = moe.moe_route(dev[0], dev[1], k)
-    counts = moe.moe_dispatch(idx, E)[0].cpu().numpy()
-    acc = accounting(inp, counts)
+    if block:
+        grads["dh"] = grads.pop("dx")
+        grads["dgamma"] = torch.empty(d, dtype=f32, device=device)
+        moe.moe_block_forward_ws(dev[0], gamma, moe_inputs.BLOCK_EPS, *dev[1:], k, fws, out, alpha=BLOCK_ALPHA,
+                                 stats=stats, path=moe.MOE_PATH_TRAIN)
+        counts = np.rint(stats[:E].double().cpu().numpy() * T).astype(np.int64)
+    else:
+        idx, _ = moe.moe_route(dev[0], dev[1], k)
+        counts = moe.moe_dispatch(idx, E)[0].cpu().numpy()
+    acc = accounting(inp, counts, block)
     kT = k * T
     # executed FLOPs of each backward GEMM stage (bf16: the SwiGLU backward is fused into dgrad_h and
     # reads GEMM1's kept pre-activations; fp32 recomputes GEMM1 in the swiglu_bwd stage)
@@ -597,6 +625,13 @@ def run_train(args, rank, world, local):
 
     def step(i=None):
         on = i is not None and i % every == 0
+        if block:
+            n = moe.moe_block_forward_ws(dev[0], gamma, moe_inputs.BLOCK_EPS, *dev[1:], k, fws, out,
+                                         alpha=BLOCK_ALPHA, stats=stats, path=moe.MOE_PATH_TRAIN,
+                                         events=fev[i] if on else None)
+            _, m = moe.moe_block_backward_ws(dev[0], gamma, *dev[1:], dout, k, fws, workspace=bws, grads=grads,
+                                             alpha=BLOCK_ALPHA, events=bev[i] if on else None)
+            return n + m
         n = moe.moe_forward_profiled(*dev, k, fws, out, events=fev[i] if on else None, path=moe.MOE_PATH_TRAIN)
         _, m = moe.moe_backward_ws(*dev, dout, k, fws, workspace=bws, grads=grads, alpha=BLOCK_ALPHA,
                                    events=bev[i] if on else None)
@@ -650,13 +685,14 @@ def run_train(args, rank, world, local):
                  "flops": step_flops}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, sample, _ = oracle_train_run(inp, dout_np, args.cpu_seconds)
+        v, sample, _ = oracle_train_run(inp, dout_np, args.cpu_seconds, block)
         cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
     line = {
-        "metric": TRAIN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "metric": BLOCK_TRAIN_METRIC if block else TRAIN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp.dtype, "data": "synthetic",
-        "config": {"workload": workload_name(args.config, args.shape) + "+train", "T": T, "d": d, "ffn": F, "E": E,
+        "config": {"workload": workload_name(args.config, args.shape) + ("+block" if block else "") + "+train",
+                   "T": T, "d": d, "ffn": F, "E": E,
                    "k": k, "seed": c["seed"], "weight_grads": "bf16" if wd == torch.bfloat16 else "fp32",
                    "l2": "touched weights larger than L2 (no flush)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},

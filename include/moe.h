@@ -320,6 +320,9 @@ MOE_API moe_status moe_block_forward_f32(const float* h, const float* gamma, flo
  * bytes (device, 256-byte aligned, not in use by another call in flight), an
  * explicit path and dtype, and the optional stage events and launch count of
  * moe_forward_profiled (the statistics, when asked for, run in the route stage).
+ * MOE_PATH_TRAIN also keeps what moe_block_backward_ws needs (the row factors,
+ * the router scores and, bfloat16, GEMM1's a and b); it then needs
+ * moe_block_train_workspace_size() bytes.
  */
 MOE_API moe_status moe_block_forward_ws(const void* h, const void* gamma, float eps, const void* Wg,
                                         const void* W1, const void* W3, const void* W2, void* out, int T,
@@ -392,6 +395,70 @@ MOE_API moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1
                                    size_t fwd_workspace_bytes,
                                    void* workspace, size_t workspace_bytes, cudaEvent_t* stage_events,
                                    int* launches, cudaStream_t stream);
+
+/*
+ * Backward of the block form out = h + MoE(u), u = RMSNorm(h) (section
+ * "Mixtral 8x7B — Sparse MoEの導入", subsection "Mixtralのアーキテクチャ", with
+ * the training loss of subsection "ロードバランス損失").  With du = dL/du (the
+ * layer backward above at x = u) and r = (mean_i h_i^2 + eps)^(-1/2) per row:
+ *
+ *   dh_i     = dout_i + r gamma_i du_i - (r^3 / d) h_i sum_j du_j gamma_j h_j
+ *   dgamma_j = sum_t du_tj h_tj r_t
+ *   dWg      = sum_t ds_t u_t^T   (u unrounded, as the router saw it)
+ *
+ * and dW1, dW3, dW2 as above with the experts' input u (rounded once to the
+ * operand type, as the forward's experts saw it).  The residual passes dout to
+ * h unchanged.  Use: moe_block_forward_ws with MOE_PATH_TRAIN and a workspace
+ * of moe_block_train_workspace_size() bytes, then pass that workspace here as
+ * fwd_workspace with the same h, gamma and weights.  Outputs (device,
+ * overwritten): dh [T][d] in the layer's element type (must not overlap h or
+ * dout), dgamma [d] float, the weight gradients and dlogits as in
+ * moe_backward_ws.  d <= 8192 (MOE_ERR_UNSUPPORTED above: the dh pass keeps
+ * one row of du in a thread block's registers).  Fixed-order sums throughout:
+ * bitwise repeatable.  workspace: moe_block_backward_workspace_size() bytes.
+ */
+MOE_API size_t moe_block_train_workspace_size(int T, int d, int ffn, int E, int k, int dtype);
+MOE_API size_t moe_block_backward_workspace_size(int T, int d, int ffn, int E, int k, int dtype);
+MOE_API moe_status moe_block_backward_ws(const void* h, const void* gamma, const void* Wg, const void* W1,
+                                         const void* W3, const void* W2, const void* dout, void* dh,
+                                         float* dgamma, float* dWg, void* dW1, void* dW3, void* dW2,
+                                         float* dlogits, float alpha, int wgrad_dtype, int T, int d, int ffn,
+                                         int E, int k, int dtype, const void* fwd_workspace,
+                                         size_t fwd_workspace_bytes, void* workspace, size_t workspace_bytes,
+                                         cudaEvent_t* stage_events, int* launches, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Expert parallelism, the dispatch plan (host).  The summary page ("Mixtral of
+ * Experts", its limitations lists) names expert parallelism: experts spread
+ * over GPUs, each token's rows sent to the GPU that holds its chosen experts
+ * and the outputs sent back, one all-to-all each way.  Experts are split into
+ * R contiguous groups: rank s owns experts [s E / R, (s+1) E / R).
+ *
+ * counts_all [R][E] int32 (host, in): every rank's assignments per expert
+ *   (each rank's moe_dispatch counts, gathered).
+ * For rank `rank` (host, out; the caller owns every array):
+ *   send_counts [R], send_offsets [R+1]: rows it sends to each rank, in its
+ *     send order = its assignments sorted by expert, stable in token order
+ *     (moe_dispatch's order without segment padding);
+ *   recv_counts [R], recv_offsets [R+1]: rows it receives from each rank, the
+ *     receive buffer ordered by source rank, each source's run as sent;
+ *   expert_range [2]: its experts [lo, hi); with EL = hi - lo,
+ *   seg_counts [EL], seg_offsets [EL+1]: its expert segments, padded to 128
+ *     rows each (arrays of E and E+1 entries are always large enough);
+ *   block_recv [R][EL], block_seg [R][EL]: the rows of source s for local
+ *     expert l start at block_recv[s][l] in the receive buffer and at
+ *     block_seg[s][l] in the segments; there are counts_all[s][lo + l] of them
+ *     (arrays of R x E entries are always large enough).
+ * Segment l holds source 0's rows, then source 1's, ...: with tokens numbered
+ * source-major, each segment equals the single-GPU dispatch's segment of the
+ * concatenated batch.  MOE_ERR_INVALID_ARG for a null pointer, R or E <= 0, a
+ * rank outside [0, R) or a negative count; MOE_ERR_UNSUPPORTED for E > 32 or
+ * more than 2^31 rows.
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_ep_plan(const int32_t* counts_all, int R, int E, int rank, int32_t* send_counts,
+                               int32_t* send_offsets, int32_t* recv_counts, int32_t* recv_offsets,
+                               int32_t* expert_range, int32_t* seg_counts, int32_t* seg_offsets,
+                               int32_t* block_recv, int32_t* block_seg);
 
 #ifdef __cplusplus
 }

@@ -74,6 +74,10 @@ SIGNATURES = {
     "moe_backward_ws": (_ci, [_vp] * 12 + [_cf] + [_ci] * 7 + [_vp, _sz, _vp, _sz, _vp, _vp, _vp]),
     "moe_route_stats_f32": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp]),
     "moe_pool_stats": (_ci, [_ci, _vp, _vp]),
+    "moe_block_train_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
+    "moe_block_backward_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
+    "moe_block_backward_ws": (_ci, [_vp] * 14 + [_cf] + [_ci] * 7 + [_vp, _sz, _vp, _sz, _vp, _vp, _vp]),
+    "moe_ep_plan": (_ci, [_vp, _ci, _ci, _ci] + [_vp] * 9),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -417,6 +421,86 @@ def moe_backward_ws(x, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, g
                                 _stream(stream, x, Wg, W1, W3, W2, dout, fwd_workspace, workspace, dlogits,
                                         *grads.values())), "moe_backward_ws")
     return grads, n.value
+
+
+def moe_block_train_workspace_size(T, d, ffn, E, k, dtype=MOE_DTYPE_BF16) -> int:
+    return int(_lib.moe_block_train_workspace_size(T, d, ffn, E, k, dtype))
+
+
+def moe_block_backward_workspace_size(T, d, ffn, E, k, dtype=MOE_DTYPE_BF16) -> int:
+    return int(_lib.moe_block_backward_workspace_size(T, d, ffn, E, k, dtype))
+
+
+def moe_block_backward_ws(h, gamma, Wg, W1, W3, W2, dout, k, fwd_workspace, workspace=None, grads=None,
+                          dlogits=None, alpha=0.0, wgrad_dtype=torch.float32, events=None, stream=None):
+    """Gradients of the block out = h + MoE(RMSNorm(h)) given dout, after moe_block_forward_ws(...,
+    path=MOE_PATH_TRAIN, workspace=fwd_workspace) on the same h, gamma and weights.  Returns (grads,
+    launches) with grads a dict of dh (layer dtype), dgamma, dWg (float32), dW1, dW3, dW2 (wgrad_dtype)."""
+    code = _dtype_code(h)
+    T, d, F, E = _layer_shapes(h, Wg, W1, W3, W2)
+    if dout.shape != (T, d) or gamma.shape != (d,):
+        raise ValueError("dout must have the shape of h and gamma shape (d,)")
+    dev = h.device
+    if grads is None:
+        f32, wd = torch.float32, wgrad_dtype
+        grads = dict(dh=torch.empty((T, d), dtype=h.dtype, device=dev), dgamma=torch.empty(d, dtype=f32, device=dev),
+                     dWg=torch.empty((E, d), dtype=f32, device=dev), dW1=torch.empty((E, F, d), dtype=wd, device=dev),
+                     dW3=torch.empty((E, F, d), dtype=wd, device=dev), dW2=torch.empty((E, d, F), dtype=wd, device=dev))
+    for n, numel in (("dh", T * d), ("dgamma", d), ("dWg", E * d), ("dW1", E * F * d), ("dW3", E * F * d),
+                     ("dW2", E * d * F)):
+        _room(grads[n], numel, n)
+    if dlogits is not None:
+        _room(dlogits, T * E, "dlogits")
+    for t, n in ((h, "h"), (gamma, "gamma"), (Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2"), (dout, "dout")):
+        _dev(t, h.dtype, n)
+    _dev(grads["dh"], h.dtype, "dh")
+    _dev(grads["dgamma"], torch.float32, "dgamma")
+    _dev(grads["dWg"], torch.float32, "dWg")
+    for n in ("dW1", "dW3", "dW2"):
+        _dev(grads[n], grads["dW1"].dtype, n)
+    wcode = _dtype_code(grads["dW1"])
+    if dlogits is not None:
+        _dev(dlogits, torch.float32, "dlogits")
+    _dev(fwd_workspace, torch.uint8, "fwd_workspace")
+    if workspace is None:
+        workspace = torch.empty(max(moe_block_backward_workspace_size(T, d, F, E, k, code), 1), dtype=torch.uint8,
+                                device=dev)
+    _dev(workspace, torch.uint8, "workspace")
+    n = ctypes.c_int(0)
+    _check(_lib.moe_block_backward_ws(_ptr(h), _ptr(gamma), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dout),
+                                      _ptr(grads["dh"]), _ptr(grads["dgamma"]), _ptr(grads["dWg"]),
+                                      _ptr(grads["dW1"]), _ptr(grads["dW3"]), _ptr(grads["dW2"]), _ptr(dlogits),
+                                      float(alpha), wcode, T, d, F, E, k, code, _ptr(fwd_workspace),
+                                      fwd_workspace.numel(), _ptr(workspace), workspace.numel(),
+                                      _events(events, MOE_BWD_NUM_STAGES), ctypes.byref(n),
+                                      _stream(stream, h, gamma, Wg, W1, W3, W2, dout, fwd_workspace, workspace,
+                                              dlogits, *grads.values())), "moe_block_backward_ws")
+    return grads, n.value
+
+
+def moe_ep_plan(counts_all, rank):
+    """Expert-parallel dispatch plan of `rank` from every rank's expert counts (int array [R][E]):
+    dict(send_counts, send_offsets, recv_counts, recv_offsets, experts (lo, hi), seg_counts, seg_offsets,
+    block_recv [R][EL], block_seg [R][EL]) as numpy int32 arrays.  Host only: no device is touched."""
+    import numpy as np
+    c = np.ascontiguousarray(counts_all, dtype=np.int32)
+    if c.ndim != 2:
+        raise ValueError("counts_all must be [R][E]")
+    R, E = c.shape
+    a = {n: np.zeros(sz, dtype=np.int32) for n, sz in (("send_counts", R), ("send_offsets", R + 1),
+                                                         ("recv_counts", R), ("recv_offsets", R + 1),
+                                                         ("experts", 2), ("seg_counts", E), ("seg_offsets", E + 1),
+                                                         ("block_recv", R * E), ("block_seg", R * E))}
+    p = lambda n: ctypes.c_void_p(a[n].ctypes.data)
+    _check(_lib.moe_ep_plan(ctypes.c_void_p(c.ctypes.data), R, E, int(rank), p("send_counts"), p("send_offsets"),
+                            p("recv_counts"), p("recv_offsets"), p("experts"), p("seg_counts"), p("seg_offsets"),
+                            p("block_recv"), p("block_seg")), "moe_ep_plan")
+    EL = int(a["experts"][1] - a["experts"][0])
+    a["seg_counts"] = a["seg_counts"][:EL]
+    a["seg_offsets"] = a["seg_offsets"][:EL + 1]
+    a["block_recv"] = a["block_recv"][:R * EL].reshape(R, EL)
+    a["block_seg"] = a["block_seg"][:R * EL].reshape(R, EL)
+    return a
 
 
 def moe_get_device_status(stream=None) -> int:

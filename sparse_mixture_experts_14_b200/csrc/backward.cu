@@ -136,13 +136,18 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const int32_t* __restri
 
 constexpr int kWgChunk = 64;    // tokens per dWg partial sum
 
-// part[c][e][j] = sum over tokens t of chunk c (ascending) of ds[t][e] x[t][j]
-template <typename T, int EB>
+// part[c][e][j] = sum over tokens t of chunk c (ascending) of ds[t][e] x[t][j].
+// NORM (the block form): the router's input is the normalised row
+// u[t][j] = (h[t][j] gamma[j]) r[t], formed here in fp32 from h (passed as x),
+// gamma and the forward's row factors r.
+template <typename T, int EB, bool NORM>
 __global__ void __launch_bounds__(256) dwg_part_kernel(const T* __restrict__ x, const float* __restrict__ ds, int T_,
-                                                       int d, int E, float* __restrict__ part) {
+                                                       int d, int E, float* __restrict__ part,
+                                                       const T* __restrict__ gamma, const float* __restrict__ rstd) {
     pdl_trigger();
     pdl_wait();
     __shared__ float sds[kWgChunk][EB];
+    __shared__ float srow[kWgChunk];
     const int c = blockIdx.y;
     const int t0 = c * kWgChunk;
     const int nt = min(kWgChunk, T_ - t0);
@@ -150,9 +155,12 @@ __global__ void __launch_bounds__(256) dwg_part_kernel(const T* __restrict__ x, 
         const int t = i / EB, e = i - t * EB;
         sds[t][e] = e < E ? ds[(size_t)(t0 + t) * E + e] : 0.f;
     }
+    if (NORM)
+        for (int i = threadIdx.x; i < nt; i += blockDim.x) srow[i] = rstd[t0 + i];
     __syncthreads();
     const int j = blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= d) return;
+    const float gj = NORM ? Elt<T>::get(gamma, j) : 1.f;
     float acc[EB];
 #pragma unroll
     for (int e = 0; e < EB; ++e) acc[e] = 0.f;
@@ -161,13 +169,18 @@ __global__ void __launch_bounds__(256) dwg_part_kernel(const T* __restrict__ x, 
         float xv[8];   // eight rows in flight before the arithmetic
 #pragma unroll
         for (int u = 0; u < 8; ++u) xv[u] = Elt<T>::get(x, (size_t)(t0 + t + u) * d + j);
+        if (NORM) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) xv[u] = (xv[u] * gj) * srow[t + u];
+        }
 #pragma unroll
         for (int u = 0; u < 8; ++u)
 #pragma unroll
             for (int e = 0; e < EB; ++e) acc[e] = fmaf(sds[t + u][e], xv[u], acc[e]);
     }
     for (; t < nt; ++t) {
-        const float xv = Elt<T>::get(x, (size_t)(t0 + t) * d + j);
+        float xv = Elt<T>::get(x, (size_t)(t0 + t) * d + j);
+        if (NORM) xv = (xv * gj) * srow[t];
 #pragma unroll
         for (int e = 0; e < EB; ++e) acc[e] = fmaf(sds[t][e], xv, acc[e]);
     }
@@ -243,6 +256,165 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float* __restrict
         } else {
             *reinterpret_cast<float4*>(out) = acc;
         }
+    }
+}
+
+// Block form: the MoE layer's input is u = RMSNorm(h), u[t][j] = gamma[j] h[t][j] r[t] with
+// r[t] = (mean_i h[t][i]^2 + eps)^(-1/2) (section "Mixtral 8x7B — Sparse MoEの導入",
+// subsection "Mixtralのアーキテクチャ": RMSNorm, the MoE layer, then the residual add).  With
+// du = dL/du (the MoE backward's input gradient: expert rows in selection order, then the router
+// term over experts in ascending order, the dx_combine sum) and dr/dh_i = -r^3 h_i / d:
+//     dh[t][i]    = dout[t][i] + r gamma[i] du[t][i] - (r^3 / d) h[t][i] <du[t], gamma . h[t]>
+//     dgamma[j]   = sum_t du[t][j] h[t][j] r[t]
+// (the residual passes dout to h unchanged).  One block per chunk of kBlkChunk tokens, taken in
+// token order, its threads spanning the row (VPT float4 columns each), the chunk's slots and score
+// gradients staged in shared memory first, so a token's row loads all go out at once:
+// per token the block holds du's row in registers, reduces the projection in a fixed order
+// (thread columns ascending, warp butterfly, warp order), writes dh rounded once, and adds
+// du h r to its per-column dgamma partial, written once per chunk.  dgamma = the chunk partials
+// summed in chunk order (dwg_final_kernel with one row).
+constexpr int kBlkChunk = 8;
+
+// Four consecutive elements of a row as one vector load, widened to fp32.
+template <typename T>
+struct V4;
+template <>
+struct V4<float> {
+    using Raw = float4;
+    __device__ __forceinline__ static Raw load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+    __device__ __forceinline__ static float4 widen(const Raw& r) { return r; }
+};
+template <>
+struct V4<__nv_bfloat16> {
+    using Raw = uint2;
+    __device__ __forceinline__ static Raw load(const __nv_bfloat16* p) {
+        return __ldg(reinterpret_cast<const uint2*>(p));
+    }
+    __device__ __forceinline__ static float4 widen(const Raw& r) {
+        return make_float4(bf16_lo(r.x), bf16_hi(r.x), bf16_lo(r.y), bf16_hi(r.y));
+    }
+};
+
+template <typename T, int VPT>
+__global__ void __launch_bounds__(512, 2) block_dx_kernel(const float* __restrict__ dXp, const int32_t* __restrict__ inv,
+                                                          const float* __restrict__ ds, const T* __restrict__ Wg,
+                                                          const T* __restrict__ h, const T* __restrict__ gamma,
+                                                          const float* __restrict__ rstd, const T* __restrict__ dout,
+                                                          int T_, int d, int E, int k, size_t slots, int* status,
+                                                          T* __restrict__ dh, float* __restrict__ dgam_part) {
+    pdl_trigger();
+    pdl_wait();
+    __shared__ float red[2][32];
+    __shared__ int sslot[kBlkChunk][kMaxExperts];    // the chunk's assignment slots (k <= E <= 32)
+    __shared__ float sds[kBlkChunk][kMaxExperts];     // and its score gradients
+    const int q = d / 4;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int t0 = blockIdx.x * kBlkChunk;
+    const int t1 = min(T_, t0 + kBlkChunk);
+    for (int i = threadIdx.x; i < (t1 - t0) * kMaxExperts; i += blockDim.x) {
+        const int tt = i / kMaxExperts, j = i - tt * kMaxExperts;
+        sslot[tt][j] = j < k ? __ldg(inv + (size_t)(t0 + tt) * k + j) : -1;
+        sds[tt][j] = j < E ? __ldg(ds + (size_t)(t0 + tt) * E + j) : 0.f;
+    }
+    __syncthreads();
+    float4 dgp[VPT];
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) dgp[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t = t0; t < t1; ++t) {
+        const int tt = t - t0;
+        const int buf = tt & 1;
+        float4 du[VPT];
+        float proj = 0.f;
+#pragma unroll
+        for (int v = 0; v < VPT; ++v) {
+            const int c = threadIdx.x + v * blockDim.x;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c < q) {
+                const size_t o = (size_t)t * d + 4 * (size_t)c;
+                // the token's loads go out before the arithmetic that needs them
+                const typename V4<T>::Raw hr = V4<T>::load(h + o);
+                const typename V4<T>::Raw gr = V4<T>::load(gamma + 4 * (size_t)c);
+                // expert rows in selection order
+                for (int j = 0; j < k; ++j) {
+                    const int slot = sslot[tt][j];
+                    if (slot < 0 || !debug_check((size_t)slot < slots, status)) continue;
+                    const float4 x4 = __ldg(reinterpret_cast<const float4*>(dXp + (size_t)slot * d) + c);
+                    acc.x += x4.x;
+                    acc.y += x4.y;
+                    acc.z += x4.z;
+                    acc.w += x4.w;
+                }
+                // then the router term in expert order, nonzero gradients only (dx_combine's sum);
+                // the Wg columns of 8 experts are loaded before their FMAs
+#pragma unroll 1
+                for (int e0 = 0; e0 < E; e0 += 8) {
+                    typename V4<T>::Raw wr[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (e0 + u < E && sds[tt][e0 + u] != 0.f)
+                            wr[u] = V4<T>::load(Wg + (size_t)(e0 + u) * d + 4 * (size_t)c);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float sv = e0 + u < E ? sds[tt][e0 + u] : 0.f;
+                        if (sv == 0.f) continue;
+                        const float4 w4 = V4<T>::widen(wr[u]);
+                        acc.x = fmaf(sv, w4.x, acc.x);
+                        acc.y = fmaf(sv, w4.y, acc.y);
+                        acc.z = fmaf(sv, w4.z, acc.z);
+                        acc.w = fmaf(sv, w4.w, acc.w);
+                    }
+                }
+                const float4 hv = V4<T>::widen(hr), gv = V4<T>::widen(gr);
+                proj = fmaf(acc.x, gv.x * hv.x, proj);
+                proj = fmaf(acc.y, gv.y * hv.y, proj);
+                proj = fmaf(acc.z, gv.z * hv.z, proj);
+                proj = fmaf(acc.w, gv.w * hv.w, proj);
+            }
+            du[v] = acc;
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) proj += __shfl_xor_sync(0xffffffffu, proj, m);
+        if (lane == 0) red[buf][warp] = proj;
+        // one barrier per token: the buffers alternate, so a token's partials are written only after
+        // every thread has passed the previous token's barrier and read the buffer of two tokens back
+        __syncthreads();
+        float tot = 0.f;
+        for (int w = 0; w < nwarps; ++w) tot += red[buf][w];
+        const float r = __ldg(rstd + t);
+        const float c3 = r * r * r / (float)d * tot;
+#pragma unroll
+        for (int v = 0; v < VPT; ++v) {
+            const int c = threadIdx.x + v * blockDim.x;
+            if (c >= q) continue;
+            const size_t o = (size_t)t * d + 4 * (size_t)c;
+            // h, gamma and dout again: the row was just read, so these come from L1
+            const float4 hv = V4<T>::widen(V4<T>::load(h + o));
+            const float4 gv = V4<T>::widen(V4<T>::load(gamma + 4 * (size_t)c));
+            const float4 go = V4<T>::widen(V4<T>::load(dout + o));
+            float outv[4];
+            outv[0] = go.x + r * gv.x * du[v].x - c3 * hv.x;
+            outv[1] = go.y + r * gv.y * du[v].y - c3 * hv.y;
+            outv[2] = go.z + r * gv.z * du[v].z - c3 * hv.z;
+            outv[3] = go.w + r * gv.w * du[v].w - c3 * hv.w;
+            if (sizeof(T) == 2) {
+                uint2 pk;
+                pk.x = pack_bf16x2(outv[0], outv[1]);
+                pk.y = pack_bf16x2(outv[2], outv[3]);
+                *reinterpret_cast<uint2*>(dh + o) = pk;
+            } else {
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(dh) + o) =
+                    make_float4(outv[0], outv[1], outv[2], outv[3]);
+            }
+            dgp[v].x = fmaf(du[v].x * hv.x, r, dgp[v].x);
+            dgp[v].y = fmaf(du[v].y * hv.y, r, dgp[v].y);
+            dgp[v].z = fmaf(du[v].z * hv.z, r, dgp[v].z);
+            dgp[v].w = fmaf(du[v].w * hv.w, r, dgp[v].w);
+        }
+    }
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+        const int c = threadIdx.x + v * blockDim.x;
+        if (c < q) reinterpret_cast<float4*>(dgam_part + (size_t)blockIdx.x * d)[c] = dgp[v];
     }
 }
 
@@ -377,20 +549,63 @@ cudaError_t launch_scatter(const BwdArgs& a, cudaStream_t s) {
                       static_cast<T*>(a.dy), a.dg, a.status);
 }
 
+template <typename T, bool NORM>
+cudaError_t launch_dwg_part(const BwdArgs& a, cudaStream_t s, dim3 grid) {
+    const T* x = static_cast<const T*>(a.x);
+    const T* g = static_cast<const T*>(a.gamma);
+    if (a.E <= 8)
+        return launch_pdl(dwg_part_kernel<T, 8, NORM>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part, g,
+                          a.rstd);
+    if (a.E <= 16)
+        return launch_pdl(dwg_part_kernel<T, 16, NORM>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part, g,
+                          a.rstd);
+    return launch_pdl(dwg_part_kernel<T, 32, NORM>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part, g,
+                      a.rstd);
+}
+
 template <typename T>
 cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s) {
     const int chunks = (a.T + kWgChunk - 1) / kWgChunk;
     const dim3 grid((a.d + 255) / 256, chunks);
-    const T* x = static_cast<const T*>(a.x);
-    cudaError_t e;
-    if (a.E <= 8) e = launch_pdl(dwg_part_kernel<T, 8>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part);
-    else if (a.E <= 16) e = launch_pdl(dwg_part_kernel<T, 16>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part);
-    else e = launch_pdl(dwg_part_kernel<T, 32>, grid, dim3(256), 0, s, x, a.ds, a.T, a.d, a.E, a.dwg_part);
+    cudaError_t e = a.gamma ? launch_dwg_part<T, true>(a, s, grid) : launch_dwg_part<T, false>(a, s, grid);
     if (e != cudaSuccess) return e;
     size_t blocks = ((size_t)a.E * a.d + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     return launch_pdl(dwg_final_kernel, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const float*>(a.dwg_part),
                       chunks, a.E, a.d, a.dWg);
+}
+
+template <typename T>
+cudaError_t launch_block_dx(const BwdArgs& a, cudaStream_t s) {
+    const int chunks = (a.T + kBlkChunk - 1) / kBlkChunk;
+    const int q = a.d / 4;
+    const float* dxp = static_cast<const float*>(a.dxp);
+    const T* Wg = static_cast<const T*>(a.Wg);
+    const T* h = static_cast<const T*>(a.x);
+    const T* g = static_cast<const T*>(a.gamma);
+    const T* dout = static_cast<const T*>(a.dout);
+    T* dh = static_cast<T*>(a.dx);
+    cudaError_t e;
+    // threads span the row, at most 512 per block (two blocks per SM): one float4 column each up to
+    // d = 2048, two up to d = 4096, four up to d = 8192
+    auto go = [&](auto kern, int vpt) {
+        const unsigned nt = (unsigned)(((q + vpt - 1) / vpt + 31) / 32 * 32);
+        return launch_pdl(kern, dim3(chunks), dim3(nt), 0, s, dxp, a.inv, a.ds, Wg, h, g, a.rstd, dout, a.T, a.d,
+                          a.E, a.k, a.slots, a.status, dh, a.dgamma_part);
+    };
+    if (q > 2048) return cudaErrorInvalidValue;   // rows longer than 8192: refused by the entry point
+    if (q <= 512) {
+        e = go(block_dx_kernel<T, 1>, 1);
+    } else if (q <= 1024) {
+        e = go(block_dx_kernel<T, 2>, 2);
+    } else {
+        e = go(block_dx_kernel<T, 4>, 4);
+    }
+    if (e != cudaSuccess) return e;
+    size_t blocks = ((size_t)a.d + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    return launch_pdl(dwg_final_kernel, dim3((unsigned)blocks), dim3(256), 0, s,
+                      static_cast<const float*>(a.dgamma_part), chunks, 1, a.d, a.dgamma);
 }
 
 template <typename T>
@@ -425,7 +640,13 @@ cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_dx_combine(const BwdArgs& a, cudaStream_t s) {
+    if (a.gamma) return a.bf16 ? launch_block_dx<__nv_bfloat16>(a, s) : launch_block_dx<float>(a, s);
     return a.bf16 ? launch_dx<__nv_bfloat16>(a, s) : launch_dx<float>(a, s);
+}
+
+size_t block_dgamma_part_bytes(int T, int d) {
+    const size_t chunks = (size_t)(T > 0 ? (T + kBlkChunk - 1) / kBlkChunk : 1);
+    return chunks * (size_t)d * 4;
 }
 
 cudaError_t launch_simt_bwd_gemms(const BwdArgs& a, cudaStream_t s) {

@@ -191,6 +191,8 @@ moe_status run_layer(const void* x, const void* Wg, const void* W1, const void* 
     const bool train = path == MOE_PATH_TRAIN;
     const Plan p = make_plan(T, d, F, E, k, dtype, bo != nullptr, train);
     RouteExtras ex;
+    ex.status = dev.status;
+    ex.wait_ns = wait_limit_ns();
     GatherNorm nm;
     if (bo) {
         ex.gamma = bo->gamma;
@@ -343,6 +345,8 @@ moe_status route_stats(const void* x, const void* Wg, int T, int d, int E, int k
         return MOE_ERR_WORKSPACE;
     RouteExtras ex;
     ex.logits = static_cast<float*>(scratch);
+    ex.status = dev.status;
+    ex.wait_ns = wait_limit_ns();
     cudaError_t e = dtype == MOE_DTYPE_BF16
                         ? launch_router_bf16(x, Wg, T, d, E, k, idx, w, dev.num_sms, s, ex)
                         : launch_router_f32(static_cast<const float*>(x), static_cast<const float*>(Wg), T, d, E, k,
@@ -355,10 +359,10 @@ moe_status route_stats(const void* x, const void* Wg, int T, int d, int E, int k
 
 // Backward workspace layout (on top of the forward's workspace, which it reads).
 struct BwdPlan {
-    size_t dy, dg, ds, dh, dab, dxp, dwg, total;
+    size_t dy, dg, ds, dh, dab, dxp, dwg, dgam, total;
 };
 
-BwdPlan make_bwd_plan(int T, int d, int F, int E, int k, int dtype) {
+BwdPlan make_bwd_plan(int T, int d, int F, int E, int k, int dtype, bool block = false) {
     BwdPlan b{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -375,6 +379,7 @@ BwdPlan make_bwd_plan(int T, int d, int F, int E, int k, int dtype) {
     b.dab = take(S * 2 * (size_t)F * es);
     b.dxp = take(S * d * 4);
     b.dwg = take(dwg_part_bytes(T, E, d));
+    if (block) b.dgam = take(block_dgamma_part_bytes(T, d));
     b.total = off;
     return b;
 }
@@ -383,9 +388,11 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
                         const void* dout, void* dx, float* dWg, void* dW1, void* dW3, void* dW2, float* dlogits,
                         float alpha, int wgrad_dtype, int T, int d, int F, int E, int k, int dtype, const uint8_t* fws,
                         uint8_t* bws,
-                        const DeviceState& dev, cudaStream_t s, cudaEvent_t* ev, int* launches) {
-    const Plan p = make_plan(T, d, F, E, k, dtype, false, true);
-    const BwdPlan b = make_bwd_plan(T, d, F, E, k, dtype);
+                        const DeviceState& dev, cudaStream_t s, cudaEvent_t* ev, int* launches,
+                        const void* gamma = nullptr, float* dgamma = nullptr) {
+    const bool block = gamma != nullptr;
+    const Plan p = make_plan(T, d, F, E, k, dtype, block, true);
+    const BwdPlan b = make_bwd_plan(T, d, F, E, k, dtype, block);
     uint8_t* fw = const_cast<uint8_t*>(fws);
     BwdArgs a{};
     a.bf16 = dtype == MOE_DTYPE_BF16;
@@ -416,6 +423,12 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
     a.dab = bws + b.dab;
     a.dxp = reinterpret_cast<float*>(bws + b.dxp);
     a.dwg_part = reinterpret_cast<float*>(bws + b.dwg);
+    if (block) {
+        a.gamma = gamma;
+        a.rstd = reinterpret_cast<const float*>(fw + p.rstd);
+        a.dgamma = dgamma;
+        a.dgamma_part = reinterpret_cast<float*>(bws + b.dgam);
+    }
     a.dx = dx;
     a.dWg = dWg;
     a.dW1 = static_cast<float*>(dW1);   // the CUDA-core (fp32) path: fp32 gradients only
@@ -485,7 +498,7 @@ moe_status run_backward(const void* x, const void* Wg, const void* W1, const voi
     MOE_TRY(mark(MOE_BWD_STAGE_ROUTER));
     MOE_TRY(launch_dwg(a, s));
     MOE_TRY(launch_dx_combine(a, s));
-    n += 3;
+    n += block ? 4 : 3;
     MOE_TRY(mark(MOE_BWD_NUM_STAGES));
     if (launches) *launches = n;
     return MOE_OK;
@@ -560,7 +573,10 @@ moe_status moe_route(const void* x, const void* Wg, int T, int d, int E, int k, 
     DeviceState dev;
     const DeviceScope scope(x, false);
     if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
-    return cuda_status(launch_router_bf16(x, Wg, T, d, E, k, topk_idx, topk_w, dev.num_sms, stream));
+    RouteExtras ex;
+    ex.status = dev.status;
+    ex.wait_ns = wait_limit_ns();
+    return cuda_status(launch_router_bf16(x, Wg, T, d, E, k, topk_idx, topk_w, dev.num_sms, stream, ex));
 }
 
 moe_status moe_route_f32(const float* x, const float* Wg, int T, int d, int E, int k, int32_t* topk_idx,
@@ -756,11 +772,13 @@ moe_status moe_block_forward_ws(const void* h, const void* gamma, float eps, con
     moe_status st = check_layer(h, Wg, W1, W3, W2, out, T, d, ffn, E, k, dtype);
     if (st == MOE_OK) st = check_block(h, gamma, eps, alpha, stats, out, T, d, dtype);
     if (st != MOE_OK) return st;
-    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE) return MOE_ERR_INVALID_ARG;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE && path != MOE_PATH_TRAIN)
+        return MOE_ERR_INVALID_ARG;
     if (path == MOE_PATH_DECODE && (dtype != MOE_DTYPE_BF16 || T > kDecodeMaxTokens)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
-    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype, true).total) return MOE_ERR_WORKSPACE;
+    if (workspace_bytes < make_plan(T, d, ffn, E, k, dtype, true, path == MOE_PATH_TRAIN).total)
+        return MOE_ERR_WORKSPACE;
     DeviceState dev;
     const DeviceScope scope(h, false);
     if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
@@ -809,6 +827,55 @@ moe_status moe_backward_ws(const void* x, const void* Wg, const void* W1, const 
                         k, dtype,
                         static_cast<const uint8_t*>(fwd_workspace), static_cast<uint8_t*>(workspace), dev, stream,
                         stage_events, launches);
+}
+
+size_t moe_block_train_workspace_size(int T, int d, int ffn, int E, int k, int dtype) {
+    if (check_sizes(T, d, E, k) != MOE_OK || ffn <= 0) return 0;
+    if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_F32) return 0;
+    return make_plan(T, d, ffn, E, k, dtype, true, true).total;
+}
+
+size_t moe_block_backward_workspace_size(int T, int d, int ffn, int E, int k, int dtype) {
+    if (check_sizes(T, d, E, k) != MOE_OK || ffn <= 0) return 0;
+    if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_F32) return 0;
+    return make_bwd_plan(T, d, ffn, E, k, dtype, true).total;
+}
+
+moe_status moe_block_backward_ws(const void* h, const void* gamma, const void* Wg, const void* W1, const void* W3,
+                                 const void* W2, const void* dout, void* dh, float* dgamma, float* dWg, void* dW1,
+                                 void* dW3, void* dW2, float* dlogits, float alpha, int wgrad_dtype, int T, int d,
+                                 int ffn, int E, int k, int dtype, const void* fwd_workspace,
+                                 size_t fwd_workspace_bytes, void* workspace, size_t workspace_bytes,
+                                 cudaEvent_t* stage_events, int* launches, cudaStream_t stream) {
+    if (launches) *launches = 0;
+    moe_status st = check_layer(h, Wg, W1, W3, W2, dh, T, d, ffn, E, k, dtype);
+    if (st != MOE_OK) return st;
+    if (d > 8192) return MOE_ERR_UNSUPPORTED;   // the dh pass holds a row of du in one block's registers
+    if (T == 0) return MOE_OK;
+    const void* ptrs[7] = {dout, dWg, dW1, dW3, dW2, gamma, dgamma};
+    for (const void* q : ptrs)
+        if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (dlogits && (reinterpret_cast<uintptr_t>(dlogits) & 3u) != 0) return MOE_ERR_INVALID_ARG;
+    if (!(alpha == alpha) || !(alpha - alpha == 0.f)) return MOE_ERR_INVALID_ARG;
+    if (wgrad_dtype != MOE_DTYPE_F32 && wgrad_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (wgrad_dtype == MOE_DTYPE_BF16 && dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+    // dh is written row by row while dout and h of the same row are read: no overlap with either
+    const size_t row = (size_t)d * (dtype == MOE_DTYPE_BF16 ? 2 : 4);
+    const uintptr_t ob = reinterpret_cast<uintptr_t>(dh), oe = ob + row * (size_t)T;
+    for (const void* q : {h, dout}) {
+        const uintptr_t b = reinterpret_cast<uintptr_t>(q), e = b + row * (size_t)T;
+        if (ob < e && b < oe) return MOE_ERR_INVALID_ARG;
+    }
+    if (!fwd_workspace || (reinterpret_cast<uintptr_t>(fwd_workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (fwd_workspace_bytes < make_plan(T, d, ffn, E, k, dtype, true, true).total) return MOE_ERR_WORKSPACE;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (workspace_bytes < make_bwd_plan(T, d, ffn, E, k, dtype, true).total) return MOE_ERR_WORKSPACE;
+    DeviceState dev;
+    const DeviceScope scope(h, false);
+    if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
+    return run_backward(h, Wg, W1, W3, W2, dout, dh, dWg, dW1, dW3, dW2, dlogits, alpha, wgrad_dtype, T, d, ffn, E,
+                        k, dtype, static_cast<const uint8_t*>(fwd_workspace), static_cast<uint8_t*>(workspace), dev,
+                        stream, stage_events, launches, gamma, dgamma);
 }
 
 moe_status moe_route_stats(const void* x, const void* Wg, int T, int d, int E, int k, float alpha,

@@ -1,89 +1,14 @@
-// Shared device/host definitions of the MoE layer's kernels (sm_100a).
+// Host-side definitions shared by the MoE layer's translation units: device
+// selection and per-device set-up, the launch helper, buffer sizes and the
+// launcher declarations.  Device code lives in moe_device.cuh (included here),
+// so edits to these host declarations leave every kernel's device code as it is.
 #pragma once
-
-#include <cuda_runtime.h>
-#include <cuda_bf16.h>
-#include <stdint.h>
 
 #include <atomic>
 
-#include "../../include/moe.h"
+#include "moe_device.cuh"
 
 namespace moe {
-
-// Rows per expert segment granule: every expert's rows are padded to this, so
-// a 128-row tensor-core tile never straddles two experts.
-constexpr int kSegRows = 128;
-constexpr int kMaxExperts = 32;
-// wave counters in Meta: forward GEMM1, GEMM2, then the backward GEMMs (dH,
-// SwiGLU backward, dX, dW2, dW1/dW3)
-constexpr int kWaveSlots = 8;
-enum WaveSlot : int { kWaveFwd1 = 0, kWaveFwd2 = 1, kWaveDgradH = 2, kWaveSwigluBwd = 3, kWaveDgradX = 4,
-                      kWaveWgrad2 = 5, kWaveWgrad13 = 6 };
-// Tokens handled by one dispatch block (histogram / scatter).
-constexpr int kDispatchTokens = 1024;
-
-// Small per-call table written by the dispatch scan, read by every later kernel.
-struct Meta {
-    int32_t counts[kMaxExperts];        // assignments per expert
-    int32_t offsets[kMaxExperts + 1];   // padded segment start rows; offsets[E] = padded total
-    int32_t waves[kWaveSlots];          // wave counters of the expert GEMMs (zeroed by dispatch / backward)
-};
-
-// Per-device sticky status word (first fault wins).
-__device__ __forceinline__ void record_status(int* status, int code) {
-    if (status) atomicCAS(status, 0, code);
-}
-
-#ifndef MOE_DEBUG
-#define MOE_DEBUG 0
-#endif
-// Debug builds (nvcc -DMOE_DEBUG=1, libmoe_debug.so) check the indices a kernel
-// reads from another kernel's output (segment rows, assignment slots, segment
-// offsets, tile rows) against the buffer they address: a failed check records
-// MOE_ERR_DEVICE and returns false, and the caller skips the access.  Release
-// builds compile the check away (it is always true): those indices are in
-// range by construction of the dispatch.
-__device__ __forceinline__ bool debug_check(bool ok, int* status) {
-#if MOE_DEBUG
-    if (!ok) record_status(status, MOE_ERR_DEVICE);
-    return ok;
-#else
-    (void)ok;
-    (void)status;
-    return true;
-#endif
-}
-
-__device__ __forceinline__ uint64_t global_timer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// SiLU(a) * b with SiLU(a) = a / (1 + e^-a).  For a < -88 the denominator is
-// +inf and the fast division gives the correct limit 0.
-__device__ __forceinline__ float silu_mul(float a, float b) {
-    return __fdividef(a, 1.0f + __expf(-a)) * b;
-}
-
-// Backward of h = SiLU(a) b for the upstream gradient dh:
-//     da = dh b SiLU'(a),  db = dh SiLU(a),  SiLU'(a) = s (1 + a (1 - s)),  s = 1 / (1 + e^-a).
-// For a < -88, e^-a is +inf, s is 0 and both gradients are 0.
-__device__ __forceinline__ void silu_bwd(float a, float b, float dh, float& da, float& db) {
-    const float s = __fdividef(1.0f, 1.0f + __expf(-a));
-    db = dh * a * s;
-    da = dh * b * s * (1.0f + a * (1.0f - s));
-}
-
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // For the length of one library call: the device that owns p is made current,
@@ -165,16 +90,6 @@ class PerDeviceInt {
     std::atomic<int> val_[kSlots];
 };
 
-// Programmatic dependent launch.  Every kernel of the layer is launched with
-// programmatic stream serialisation: it lets the next kernel in the stream be
-// scheduled once all of its own CTAs have started (pdl_trigger at entry),
-// and it does no global-memory access before pdl_wait, which returns once
-// the previous grid in the stream has completed and its writes are visible.
-// The next kernel's launch latency and prologue (barrier set-up, tensor
-// memory allocation) thereby overlap the tail of the current one.
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
     cudaLaunchConfig_t cfg = {};
@@ -208,6 +123,8 @@ struct RouteExtras {
     float eps = 0.f;
     float* rstd = nullptr;
     float* logits = nullptr;
+    int* status = nullptr;                 // device status word (bounded pipeline waits record here)
+    long long wait_ns = 1000000000LL;      // limit of one pipeline wait
 };
 
 cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx,
@@ -334,12 +251,18 @@ struct BwdArgs {
     int T, d, F, E, k;
     size_t slots;
     int* status;            // device status word (debug builds record index faults in it)
+    // block form (out = h + MoE(RMSNorm(h))): x is h, dx receives dh; null gamma = the plain layer
+    const void* gamma;      // [d]
+    const float* rstd;      // [T] the forward's row factors r
+    float* dgamma;          // [d] fp32
+    float* dgamma_part;     // block_dgamma_part_bytes(T, d)
 };
 size_t dwg_part_bytes(int T, int E, int d);
+size_t block_dgamma_part_bytes(int T, int d);
 cudaError_t launch_bwd_scatter(const BwdArgs& a, cudaStream_t s);      // dY and dg (1 launch)
 cudaError_t launch_router_bwd(const BwdArgs& a, cudaStream_t s);       // ds (1 launch)
 cudaError_t launch_dwg(const BwdArgs& a, cudaStream_t s);              // dWg (2 launches)
-cudaError_t launch_dx_combine(const BwdArgs& a, cudaStream_t s);       // dx (1 launch)
+cudaError_t launch_dx_combine(const BwdArgs& a, cudaStream_t s);       // dx (1 launch; block form: dh, dgamma: 2)
 cudaError_t launch_simt_bwd_gemms(const BwdArgs& a, cudaStream_t s);   // fp32 expert GEMMs (5 launches)
 
 cudaError_t launch_tc_dgrad_h(const TcBwdArgs& a, cudaStream_t s);      // dH = dY W2_e -> dA, dB

@@ -3,8 +3,12 @@
 // "Mistral/Mixtral architecture" page (score, Top-2 and gate equations) and its
 // MoERouter.forward in "簡易MoEルーターの実装", fused into one pass over x.
 //
-// Large bf16 batches: scores on the tensor cores (router_mma_kernel, 16
-// tokens per block, warps split d).  Small batches and fp32 inputs: CUDA-core
+// Large bf16 batches (plain layer, E a multiple of 8): router_tc_kernel, the
+// scores as a tcgen05 GEMM of 128-token tiles against Wg (N = E rounded up to
+// 16), operands streamed by TMA, one tile per CTA; when there are fewer tiles
+// than SMs the CTAs of a cluster split d and rank 0 adds their partial scores
+// in rank order through distributed shared memory.  Block form and other E:
+// router_mma_kernel (mma.sync, 16 tokens per block, warps split d).  Small batches and fp32 inputs: CUDA-core
 // dot products (router_kernel, one block per token or per few tokens, every
 // 16-byte chunk a thread needs in flight before the arithmetic; rows longer
 // than 1024 chunks loop, router_loop_kernel).  Partial sums are reduced in a
@@ -20,7 +24,11 @@
 // gamma * x is exact in fp32 for bf16 operands; on the tensor cores it enters
 // as two bf16 operands, hi = bf16(gamma x) and lo = gamma x - hi, which are
 // exact too, so the scores see the unrounded normalised row.
+#include <cuda.h>
+
 #include "moe_common.cuh"
+#include "ptx_sm100.cuh"
+#include "tma_map.cuh"
 
 namespace moe {
 namespace {
@@ -424,6 +432,275 @@ __global__ void __launch_bounds__(256) router_mma_kernel(const __nv_bfloat16* __
     }
 }
 
+// ---------------------------------------------------------------- tcgen05 router
+
+constexpr int RT_M = 128;                          // tokens per tile (MMA M, TMEM lanes)
+constexpr int RT_BK = 64;                          // K per stage (one 128-byte swizzle row)
+constexpr int RT_A_BYTES = RT_M * RT_BK * 2;       // 16 KiB of x
+constexpr int RT_MAX_STAGES = 10;
+// Ring of one kernel instance: A (x) and B (EP rows of Wg) per stage, about 180 KiB of x in
+// flight per SM (the only CTA on it), enough to keep HBM busy from 128 SMs.
+template <int EP>
+struct RtRing {
+    static constexpr int STAGE_BYTES = RT_A_BYTES + EP * RT_BK * 2;   // 18 or 20 KiB, 1 KiB aligned
+    static constexpr int STAGES = EP == 16 ? 10 : 9;
+};
+constexpr int RT_CHUNK_KB = 4;                     // stages per fp32 flush (K = 256)
+constexpr int RT_THREADS = 128;
+
+struct RtCtrl {
+    uint64_t full[RT_MAX_STAGES];
+    uint64_t empty[RT_MAX_STAGES];
+    uint64_t done;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int EP>
+constexpr int rt_smem_bytes() {
+    return RtRing<EP>::STAGES * RtRing<EP>::STAGE_BYTES + RT_M * 33 * 4 + (int)sizeof(RtCtrl) + 1024;
+}
+
+// One 128-token tile per CTA (cluster rank = the K split it reads).  Warp 0
+// lane 0 streams x (128 rows x 64) and Wg (EL rows x 64, EL = E) into a
+// 9- or 10-stage ring; warp 1 lane 0 issues tcgen05.mma M = 128, N = EP (E rounded up
+// to 16; the B rows past E hold zeros), accumulating every 256 of K into its
+// own TMEM column block, so no accumulation inside the tensor core runs longer
+// than K = 256; then all four warps read their 32 rows, add the blocks in
+// order in fp32 and, with one split, finish the token (scores, top-k, gates).
+// With several splits each CTA leaves its partial scores in shared memory and
+// rank 0 adds them in rank order.
+template <int EP>
+__global__ void __launch_bounds__(RT_THREADS, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW, int T,
+                     int d, int E, int k, int tmem_cols, RouterIO<__nv_bfloat16> io, int* status,
+                     long long wait_ns) {
+    constexpr int RT_STAGES = RtRing<EP>::STAGES;
+    constexpr int RT_STAGE_BYTES = RtRing<EP>::STAGE_BYTES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* part = reinterpret_cast<float*>(smem + RT_STAGES * RT_STAGE_BYTES);   // [128][33]
+    RtCtrl* ctrl = reinterpret_cast<RtCtrl*>(smem + RT_STAGES * RT_STAGE_BYTES + RT_M * 33 * 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t nsplit;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(nsplit));
+    const uint32_t split = ptx::cluster_ctarank();
+    const int m0 = (int)(blockIdx.x / nsplit) * RT_M;
+    const int nkb = d / RT_BK / (int)nsplit;            // stages of this CTA's K range
+    const int kb0 = (int)split * nkb;
+    const int chunks = (nkb + RT_CHUNK_KB - 1) / RT_CHUNK_KB;
+    const int EL = E;                                    // Wg rows loaded (E % 8 == 0)
+    const uint32_t tx = RT_A_BYTES + (uint32_t)EL * RT_BK * 2;
+
+    pdl_trigger();
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < RT_STAGES; ++st) {
+            ptx::mbar_init(&ctrl->full[st], 1);
+            ptx::mbar_init(&ctrl->empty[st], 1);
+        }
+        ptx::mbar_init(&ctrl->done, 1);
+        ptx::mbar_init(&ctrl->drain, 1);
+        ctrl->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    // B rows past E are never written by TMA: zero them once, so the MMA columns past E hold zeros
+    if (EP > EL) {
+        for (int st = 0; st < RT_STAGES; ++st) {
+            uint32_t* b = reinterpret_cast<uint32_t*>(smem + st * RT_STAGE_BYTES + RT_A_BYTES + EL * RT_BK * 2);
+            for (int i = threadIdx.x; i < (EP - EL) * RT_BK / 2; i += blockDim.x) b[i] = 0u;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::tma_prefetch_desc(&mapX);
+        ptx::tma_prefetch_desc(&mapW);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&ctrl->tmem_base, (uint32_t)tmem_cols);
+        ptx::tmem_relinquish();
+    }
+    pdl_wait();   // global memory only after the previous kernel has completed
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem_base = ctrl->tmem_base;
+    const ptx::WaitCtl wc{&ctrl->abort, status, (uint64_t)wait_ns};
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_x = ptx::policy_evict_first();   // x is read once
+            const uint64_t pol_w = ptx::policy_evict_last();    // Wg is read by every tile
+            bool armed[RT_STAGES];
+            uint32_t armed_phase[RT_STAGES];
+#pragma unroll
+            for (int st = 0; st < RT_STAGES; ++st) {
+                armed[st] = false;
+                armed_phase[st] = 0;
+            }
+            int stage = 0;
+            uint32_t phase = 0;
+            bool aborted = false;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!ptx::mbar_wait(&ctrl->empty[stage], phase ^ 1u, wc)) {
+                    aborted = true;
+                    break;
+                }
+                uint8_t* sa = smem + stage * RT_STAGE_BYTES;
+                ptx::mbar_arrive_expect_tx(&ctrl->full[stage], tx);
+                ptx::tma_load_2d(sa, &mapX, &ctrl->full[stage], (kb0 + kb) * RT_BK, m0, pol_x);
+                ptx::tma_load_2d(sa + RT_A_BYTES, &mapW, &ctrl->full[stage], (kb0 + kb) * RT_BK, 0, pol_w);
+#pragma unroll
+                for (int st = 0; st < RT_STAGES; ++st)
+                    if (st == stage) {
+                        armed[st] = true;
+                        armed_phase[st] = phase;
+                    }
+                if (++stage == RT_STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (aborted || ctrl->abort) {
+#pragma unroll
+                for (int st = 0; st < RT_STAGES; ++st)
+                    if (armed[st]) ptx::mbar_wait_drain(&ctrl->full[st], armed_phase[st], 100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC = ptx::idesc_bf16_f32(RT_M, EP);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool issued = false, aborted = false;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!ptx::mbar_wait(&ctrl->full[stage], phase, wc)) {
+                    aborted = true;
+                    break;
+                }
+                ptx::tc_fence_after_sync();
+                const uint32_t a0 = ptx::smem_addr(smem + stage * RT_STAGE_BYTES);
+                const uint32_t b0 = a0 + RT_A_BYTES;
+                const uint32_t dcol = tmem_base + (uint32_t)((kb / RT_CHUNK_KB) * EP);
+#pragma unroll
+                for (int kk = 0; kk < RT_BK / 16; ++kk)
+                    ptx::tc_mma_bf16(dcol, ptx::desc_kmajor_sw128(a0 + kk * 32), ptx::desc_kmajor_sw128(b0 + kk * 32),
+                                     IDESC, ((kb % RT_CHUNK_KB) | kk) != 0);
+                ptx::tc_commit(&ctrl->empty[stage]);
+                issued = true;
+                if (++stage == RT_STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!aborted) {
+                ptx::tc_commit(&ctrl->done);
+            } else if (issued) {
+                ptx::tc_commit(&ctrl->drain);
+                ptx::mbar_wait_drain(&ctrl->drain, 0, 100000000ull);
+            }
+        }
+    }
+    __syncwarp();
+
+    // epilogue: every warp reads its 32 TMEM lanes (rows m0 + 32 warp + lane)
+    bool ok = ptx::mbar_wait(&ctrl->done, 0, wc);
+    ok = __all_sync(0xffffffffu, ok);
+    const int row = warp * 32 + lane;
+    float sc[EP];
+#pragma unroll
+    for (int e = 0; e < EP; ++e) sc[e] = 0.f;
+    if (ok) {
+        ptx::tc_fence_after_sync();
+        const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16);
+        for (int c = 0; c < chunks; ++c) {
+            uint32_t r[EP];
+            if constexpr (EP == 16) {
+                ptx::tmem_ld_32x32b_x16(taddr + (uint32_t)(c * EP), r);
+            } else {
+                ptx::tmem_ld_32x32b_x32(taddr + (uint32_t)(c * EP), r);
+            }
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < EP; ++e) sc[e] += __uint_as_float(r[e]);
+        }
+    }
+    if (nsplit > 1) {
+#pragma unroll
+        for (int e = 0; e < EP; ++e) part[row * 33 + e] = sc[e];
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after_sync();
+        ptx::tmem_dealloc(tmem_base, (uint32_t)tmem_cols);
+    }
+    if (nsplit > 1) {
+        ptx::cluster_sync();   // every split's partial scores are in its shared memory
+        if (split == 0) {
+            const uint32_t base = ptx::smem_addr(part + row * 33);
+#pragma unroll
+            for (int e = 0; e < EP; ++e) sc[e] = 0.f;
+            for (uint32_t r = 0; r < nsplit; ++r) {
+                const uint32_t peer = ptx::map_to_rank(base, r);
+#pragma unroll
+                for (int e = 0; e < EP; ++e) {
+                    float v;
+                    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(peer + 4u * e) : "memory");
+                    sc[e] += v;
+                }
+            }
+        }
+        ptx::cluster_sync();   // no CTA leaves while rank 0 still reads its partials
+        if (split != 0) return;
+    }
+    if (!ok || m0 + row >= T) return;
+    finish_token<__nv_bfloat16, EP, false>(sc, 0.f, m0 + row, d, E, k, io);
+}
+
+template <int EP>
+cudaError_t launch_router_tc_t(const __nv_bfloat16* x, const __nv_bfloat16* Wg, int T, int d, int E, int k,
+                               const RouterIO<__nv_bfloat16>& io, int num_sms, int* status, long long wait_ns,
+                               cudaStream_t s) {
+    static PerDeviceOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(router_tc_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    rt_smem_bytes<EP>());
+    });
+    if (e != cudaSuccess) return e;
+    const int tiles = (T + RT_M - 1) / RT_M;
+    const int kbs = d / RT_BK;
+    // split d over a cluster while that still leaves every CTA on its own SM, and until the
+    // 256-wide accumulator blocks of one CTA fit the 512 TMEM columns
+    int splits = 1;
+    while (splits < 8 && kbs % (2 * splits) == 0 &&
+           (tiles * 2 * splits <= num_sms || ((kbs / splits + RT_CHUNK_KB - 1) / RT_CHUNK_KB) * EP > 512))
+        splits *= 2;
+    const int chunks = (kbs / splits + RT_CHUNK_KB - 1) / RT_CHUNK_KB;
+    if (chunks * EP > 512) return cudaErrorInvalidValue;
+    int cols = 32;
+    while (cols < chunks * EP) cols *= 2;
+    CUtensorMap mx, mw;
+    if (!map_matrix(&mx, x, (size_t)T, d, RT_BK, RT_M) || !map_matrix(&mw, Wg, (size_t)E, d, RT_BK, E))
+        return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles * splits), 1, 1);
+    cfg.blockDim = dim3(RT_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = rt_smem_bytes<EP>();
+    cfg.stream = s;
+    cudaLaunchAttribute attr2[2];
+    attr2[0].id = cudaLaunchAttributeClusterDimension;
+    attr2[0].val.clusterDim.x = (unsigned)splits;
+    attr2[0].val.clusterDim.y = 1;
+    attr2[0].val.clusterDim.z = 1;
+    attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr2[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr2;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, router_tc_kernel<EP>, mx, mw, T, d, E, k, cols, io, status, wait_ns);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 // Chunks per thread the kernels are compiled for: 16-byte chunks x 256 threads x RMAX
 // cover d <= 8192 (bf16) / 4096 (fp32) with RMAX = 4; longer rows take the looping form.
 template <typename In, int EB, int TB, bool NORM>
@@ -482,6 +759,10 @@ cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int 
     const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(Wg);
     const RouterIO<__nv_bfloat16> io = make_io<__nv_bfloat16>(idx, w, ex);
     // tensor-core scores for large batches; small batches spread one token per block instead
+    if (!ex.gamma && E % 8 == 0 && d % RT_BK == 0 && T > 4 * num_sms) {
+        return E <= 16 ? launch_router_tc_t<16>(xb, wb, T, d, E, k, io, num_sms, ex.status, ex.wait_ns, s)
+                       : launch_router_tc_t<32>(xb, wb, T, d, E, k, io, num_sms, ex.status, ex.wait_ns, s);
+    }
     if (d % 32 == 0 && T > 4 * num_sms) {
         return ex.gamma ? launch_router_mma<true>(xb, wb, T, d, E, k, io, num_sms, s)
                         : launch_router_mma<false>(xb, wb, T, d, E, k, io, num_sms, s);

@@ -21,7 +21,8 @@ def test_small_suite_passes_under_the_debug_build():
     env = dict(os.environ, MOE_LIBRARY="debug")
     cmd = [sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
            "-k", "not configs and not full_size",
-           "tests/test_gpu_parity.py", "tests/test_gpu_block.py", "tests/test_gpu_backward.py"]
+           "tests/test_gpu_parity.py", "tests/test_gpu_block.py", "tests/test_gpu_backward.py",
+           "tests/test_gpu_block_backward.py"]
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=1200)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
     assert " passed" in r.stdout
