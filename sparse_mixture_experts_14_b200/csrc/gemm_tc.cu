@@ -67,7 +67,7 @@ constexpr int NUM_EPI_WARPS = 4;                 // epilogue warps of the row-gr
 constexpr int MN_BOX = 64;                     // MN-major operands: two 64-wide boxes per 128 rows
 constexpr uint32_t MN_LBO = MN_BOX * BK * 2;   // bytes between the two boxes (atoms along M/N)
 constexpr uint32_t MN_SBO = 1024;              // bytes between 8-row groups along K
-constexpr int OUT_PITCH = 36;                  // floats per staged output row (16-byte aligned, no bank conflicts)
+constexpr int OUT_PITCH = 32;                  // floats per staged 32 x 32 chunk row (8 float4 slots, swizzled)
 
 // What one instantiation computes.
 enum : int {
@@ -138,12 +138,15 @@ struct ModeT {
     //    they also get two epilogue warps per TMEM lane quarter, each taking half the columns;
     //  * the training forward's kept a, b (written) and the SwiGLU backward's (read), with
     //    the backward's dA | dB written the same way.
-    // The space comes from the ring, which gives up two stages.
+    // The space comes from the ring, which gives up one stage: each warp's 32 x 32 fp32 chunk
+    // (4 KiB, two of them in the SwiGLU modes) is stored unpadded with its 16-byte slots
+    // XOR-swizzled by row (stage_slot), so both the row-per-lane and the 8-lanes-per-row
+    // accesses run at one 128-byte wavefront per 8 lanes without padding.
     static constexpr bool STAGED_OUT = KGROUP;
     static constexpr bool STAGED_AB = MODE == kFwd1Train || MODE == kDgradH;
     static constexpr int EPI_WARPS = STAGED_OUT ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS);
-    static constexpr int STAGES_M = STAGED_OUT || STAGED_AB ? STAGES - 2 : STAGES;
+    static constexpr int STAGES_M = STAGED_OUT || STAGED_AB ? STAGES - 1 : STAGES;
     static constexpr int STAGE_OUT_BYTES = (STAGED_OUT ? 1 : STAGED_AB ? 2 : 0) * EPI_WARPS * 32 * OUT_PITCH * 4;
     static constexpr int SMEM = STAGES_M * STAGE_BYTES + STAGE_OUT_BYTES + (int)sizeof(Ctrl) + 1024;
 };
@@ -163,6 +166,13 @@ __device__ __forceinline__ void decode_tile(const Ctrl* c, int tile, int& e, int
         n_blk = local / c->pt[e];
         pair = local - n_blk * c->pt[e];
     }
+}
+
+// Float4 slot j (0..7) of row r of a staged 32 x 32 fp32 chunk: rows are 128 bytes with no
+// padding and the slots of row r are permuted by j ^ (r & 7), so that 8 lanes writing slot j of
+// 8 consecutive rows, or 8 lanes reading the 8 slots of one row, touch 8 different bank groups.
+__device__ __forceinline__ float* stage_slot(float* buf, int r, int j) {
+    return buf + r * OUT_PITCH + 4 * (j ^ (r & 7));
 }
 
 // Soft per-wave alignment of the clusters.  CTA pairs that share a block of
@@ -438,12 +448,12 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                             // and b through shared memory, then 128-byte row segments
                             float* sa = stage_out + ew * 2 * 32 * OUT_PITCH;
                             float* sb = sa + 32 * OUT_PITCH;
-                            uint4* wa = reinterpret_cast<uint4*>(sa + lane * OUT_PITCH);
-                            uint4* wb = reinterpret_cast<uint4*>(sb + lane * OUT_PITCH);
 #pragma unroll
                             for (int v = 0; v < 8; ++v) {
-                                wa[v] = make_uint4(ra[4 * v], ra[4 * v + 1], ra[4 * v + 2], ra[4 * v + 3]);
-                                wb[v] = make_uint4(rb[4 * v], rb[4 * v + 1], rb[4 * v + 2], rb[4 * v + 3]);
+                                *reinterpret_cast<uint4*>(stage_slot(sa, lane, v)) =
+                                    make_uint4(ra[4 * v], ra[4 * v + 1], ra[4 * v + 2], ra[4 * v + 3]);
+                                *reinterpret_cast<uint4*>(stage_slot(sb, lane, v)) =
+                                    make_uint4(rb[4 * v], rb[4 * v + 1], rb[4 * v + 2], rb[4 * v + 3]);
                             }
                             __syncwarp();
                             const size_t row0w = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32;
@@ -452,8 +462,8 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                             for (int it = 0; it < 8; ++it) {
                                 const int rr = it * 4 + (lane >> 3);
                                 const size_t g = (row0w + rr) * (size_t)N + n_blk * BNH + c + cc;
-                                const uint4 va = *reinterpret_cast<const uint4*>(sa + rr * OUT_PITCH + cc);
-                                const uint4 vb = *reinterpret_cast<const uint4*>(sb + rr * OUT_PITCH + cc);
+                                const uint4 va = *reinterpret_cast<const uint4*>(stage_slot(sa, rr, lane & 7));
+                                const uint4 vb = *reinterpret_cast<const uint4*>(stage_slot(sb, rr, lane & 7));
                                 ptx::st_global_v4_hint(p.keep_a + g, va.x, va.y, va.z, va.w, pol_out);
                                 ptx::st_global_v4_hint(p.keep_b + g, vb.x, vb.y, vb.z, vb.w, pol_out);
                             }
@@ -484,15 +494,15 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
 #pragma unroll
                         for (int it = 0; it < 8; ++it) {
                             const int rr = it * 4 + (lane >> 3);
-                            *reinterpret_cast<float4*>(sa + rr * OUT_PITCH + cc) = ta[it];
-                            *reinterpret_cast<float4*>(sb + rr * OUT_PITCH + cc) = tb[it];
+                            *reinterpret_cast<float4*>(stage_slot(sa, rr, lane & 7)) = ta[it];
+                            *reinterpret_cast<float4*>(stage_slot(sb, rr, lane & 7)) = tb[it];
                         }
                         __syncwarp();
                         float av[32], bv[32];
 #pragma unroll
                         for (int v = 0; v < 8; ++v) {
-                            const float4 xa = reinterpret_cast<const float4*>(sa + lane * OUT_PITCH)[v];
-                            const float4 xb = reinterpret_cast<const float4*>(sb + lane * OUT_PITCH)[v];
+                            const float4 xa = *reinterpret_cast<const float4*>(stage_slot(sa, lane, v));
+                            const float4 xb = *reinterpret_cast<const float4*>(stage_slot(sb, lane, v));
                             av[4 * v] = xa.x;
                             av[4 * v + 1] = xa.y;
                             av[4 * v + 2] = xa.z;
@@ -516,11 +526,12 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                             pb[i] = pack_bf16x2(dbv[0], dbv[1]);
                         }
                         __syncwarp();   // every lane has its row of a, b: the buffer takes dA | dB
-                        uint4* w = reinterpret_cast<uint4*>(sa + lane * OUT_PITCH);
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
-                            w[v] = make_uint4(pa[4 * v], pa[4 * v + 1], pa[4 * v + 2], pa[4 * v + 3]);
-                            w[4 + v] = make_uint4(pb[4 * v], pb[4 * v + 1], pb[4 * v + 2], pb[4 * v + 3]);
+                            *reinterpret_cast<uint4*>(stage_slot(sa, lane, v)) =
+                                make_uint4(pa[4 * v], pa[4 * v + 1], pa[4 * v + 2], pa[4 * v + 3]);
+                            *reinterpret_cast<uint4*>(stage_slot(sa, lane, 4 + v)) =
+                                make_uint4(pb[4 * v], pb[4 * v + 1], pb[4 * v + 2], pb[4 * v + 3]);
                         }
                         __syncwarp();
                         // words 0-15 of a staged row are dA's 32 columns, words 16-31 dB's
@@ -529,7 +540,7 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
 #pragma unroll
                         for (int it = 0; it < 8; ++it) {
                             const int rr = it * 4 + (lane >> 3);
-                            const uint4 v = *reinterpret_cast<const uint4*>(sa + rr * OUT_PITCH + cc);
+                            const uint4 v = *reinterpret_cast<const uint4*>(stage_slot(sa, rr, lane & 7));
                             __nv_bfloat16* dst = dAB + (row0w + rr) * (size_t)(2 * N) + (size_t)part * N + ecol;
                             ptx::st_global_v4_hint(dst, v.x, v.y, v.z, v.w, pol_out);
                         }
@@ -551,12 +562,12 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                         ptx::tmem_ld_wait();
                         const int col = n_blk * BN + c;
                         if (col >= N) continue;
-                        float4* srow = reinterpret_cast<float4*>(stg + lane * OUT_PITCH);
 #pragma unroll
                         for (int v = 0; v < 8; ++v)
-                            srow[v] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                           : make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                            *reinterpret_cast<float4*>(stage_slot(stg, lane, v)) =
+                                zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                     : make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
                         __syncwarp();
 #pragma unroll
                         for (int it = 0; it < 8; ++it) {
@@ -564,7 +575,7 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                             const int cc = (lane & 7) * 4;
                             const int m = mbase + rr;
                             if (m < p.M) {
-                                const float4 v = *reinterpret_cast<const float4*>(stg + rr * OUT_PITCH + cc);
+                                const float4 v = *reinterpret_cast<const float4*>(stage_slot(stg, rr, lane & 7));
                                 const size_t orow = m < p.split ? (size_t)e * p.split + m
                                                                 : (size_t)e * (p.M - p.split) + (m - p.split);
                                 void* base = m < p.split ? p.out : p.out_hi;
