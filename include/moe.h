@@ -460,6 +460,46 @@ MOE_API moe_status moe_ep_plan(const int32_t* counts_all, int R, int E, int rank
                                int32_t* expert_range, int32_t* seg_counts, int32_t* seg_offsets,
                                int32_t* block_recv, int32_t* block_seg);
 
+/*
+ * Expert parallelism, the data plane (bfloat16): one rank's share of the layer
+ * between its two all-to-alls, which the caller runs (NCCL through
+ * torch.distributed, say) with the counts of moe_ep_plan.
+ *
+ * moe_ep_dispatch (route side, after moe_route): the counting sort of this
+ * rank's assignments and its token rows copied into send order.
+ *   x [T][d] bf16, topk_idx [T][k] int32 (device, in);
+ *   send [T*k][d] bf16 (device, out): row p = the token row of the p-th
+ *     assignment in send order (assignments sorted by expert, stable in token
+ *     order; the rows for rank s are send[send_offsets[s] .. send_offsets[s+1]));
+ *   send_pos [T][k] int32 (device, out): the send row of assignment (t, j);
+ *   counts_host [E] int32 (host, out): assignments per expert, this rank's row
+ *     of counts_all.  The call synchronises `stream` to return them.
+ * moe_ep_experts (expert side): recv [recv_rows][d] bf16 (device, in) holds the
+ *   rows this rank received, in the plan's receive order (recv_rows =
+ *   recv_offsets[R]); counts_all [R][E] (host); W1, W3 [EL][F][d] and W2
+ *   [EL][d][F] (device) are the weights of this rank's experts [lo, hi) only.
+ *   The rows go into padded expert segments (each equal to the single-GPU
+ *   dispatch's segment of the concatenated batch), the tensor-core grouped
+ *   GEMMs run on them, and yrecv [recv_rows][d] float (device, out) receives
+ *   each row's expert output in the receive order, ready to be sent back.
+ *   Scratch comes from the library's pool; the call synchronises `stream` once
+ *   (its small block tables are copied from host memory).
+ * moe_ep_combine (route side, after the return all-to-all): ysend
+ *   [T*k][d] float (device) in send order; out[t] = sum_j topk_w[t][j] *
+ *   ysend[send_pos[t][j]], j ascending, in fp32, rounded once to bf16 (device,
+ *   out [T][d]): the single-GPU combine's arithmetic.
+ * Every output equals the single-GPU layer's bit for bit.  Sizes as the
+ * bfloat16 layer: d % 64 == 0, ffn % 128 == 0, E <= 32; R <= 64.  The pages
+ * describe the scheme (the summary page's limitations lists) without code.
+ */
+MOE_API moe_status moe_ep_dispatch(const void* x, const int32_t* topk_idx, int T, int d, int E, int k, void* send,
+                                   int32_t* send_pos, int32_t* counts_host, cudaStream_t stream);
+MOE_API moe_status moe_ep_experts(const void* recv, const int32_t* counts_all, int R, int E, int rank,
+                                  const void* W1, const void* W3, const void* W2, int d, int ffn, float* yrecv,
+                                  cudaStream_t stream);
+MOE_API moe_status moe_ep_combine(const float* ysend, const float* topk_w, const int32_t* send_pos, int T, int d,
+                                  int k, void* out, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

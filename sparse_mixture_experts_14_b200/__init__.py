@@ -78,6 +78,9 @@ SIGNATURES = {
     "moe_block_backward_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci]),
     "moe_block_backward_ws": (_ci, [_vp] * 14 + [_cf] + [_ci] * 7 + [_vp, _sz, _vp, _sz, _vp, _vp, _vp]),
     "moe_ep_plan": (_ci, [_vp, _ci, _ci, _ci] + [_vp] * 9),
+    "moe_ep_dispatch": (_ci, [_vp, _vp, _ci, _ci, _ci, _ci, _vp, _vp, _vp, _vp]),
+    "moe_ep_experts": (_ci, [_vp, _vp, _ci, _ci, _ci, _vp, _vp, _vp, _ci, _ci, _vp, _vp]),
+    "moe_ep_combine": (_ci, [_vp, _vp, _vp, _ci, _ci, _ci, _vp, _vp]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -501,6 +504,71 @@ def moe_ep_plan(counts_all, rank):
     a["block_recv"] = a["block_recv"][:R * EL].reshape(R, EL)
     a["block_seg"] = a["block_seg"][:R * EL].reshape(R, EL)
     return a
+
+
+def moe_ep_dispatch(x, topk_idx, E, send=None, send_pos=None, stream=None):
+    """Route side of expert parallelism: (send [T*k][d] bf16 rows in send order, send_pos int32 [T][k],
+    counts numpy int32 [E]).  Synchronises the stream (the counts come back to the host)."""
+    import numpy as np
+    T, k = topk_idx.shape
+    d = x.shape[1]
+    if send is None:
+        send = torch.empty((T * k, d), dtype=x.dtype, device=x.device)
+    if send_pos is None:
+        send_pos = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    _room(send, T * k * d, "send")
+    _room(send_pos, T * k, "send_pos")
+    _dev(x, torch.bfloat16, "x")
+    _dev(topk_idx, torch.int32, "topk_idx")
+    _dev(send, torch.bfloat16, "send")
+    _dev(send_pos, torch.int32, "send_pos")
+    counts = np.zeros(E, dtype=np.int32)
+    _check(_lib.moe_ep_dispatch(_ptr(x), _ptr(topk_idx), T, d, E, k, _ptr(send), _ptr(send_pos),
+                                ctypes.c_void_p(counts.ctypes.data), _stream(stream, x, topk_idx, send, send_pos)),
+           "moe_ep_dispatch")
+    return send, send_pos, counts
+
+
+def moe_ep_experts(recv, counts_all, rank, W1, W3, W2, yrecv=None, stream=None):
+    """Expert side: the received rows (receive order of moe_ep_plan) through this rank's experts
+    (W1, W3 [EL][F][d], W2 [EL][d][F]); returns yrecv float32 [rows][d] in the receive order."""
+    import numpy as np
+    c = np.ascontiguousarray(counts_all, dtype=np.int32)
+    R, E = c.shape
+    EL, F, d = W1.shape
+    plan = moe_ep_plan(c, rank)
+    rows = int(plan["recv_offsets"][-1])
+    if recv.shape[0] < rows or recv.shape[1] != d:
+        raise ValueError(f"recv must hold {rows} rows of {d}")
+    if int(plan["experts"][1] - plan["experts"][0]) != EL or W3.shape != W1.shape or W2.shape != (EL, d, F):
+        raise ValueError("W1, W3, W2 must hold exactly this rank's experts")
+    if yrecv is None:
+        yrecv = torch.empty((rows, d), dtype=torch.float32, device=recv.device)
+    _room(yrecv, rows * d, "yrecv")
+    for t, n in ((recv, "recv"), (W1, "W1"), (W3, "W3"), (W2, "W2")):
+        _dev(t, torch.bfloat16, n)
+    _dev(yrecv, torch.float32, "yrecv")
+    _check(_lib.moe_ep_experts(_ptr(recv), ctypes.c_void_p(c.ctypes.data), R, E, int(rank), _ptr(W1), _ptr(W3),
+                               _ptr(W2), d, F, _ptr(yrecv), _stream(stream, recv, W1, W3, W2, yrecv)),
+           "moe_ep_experts")
+    return yrecv
+
+
+def moe_ep_combine(ysend, topk_w, send_pos, out=None, stream=None):
+    """Route side, after the return all-to-all: out[t] = sum_j topk_w[t][j] ysend[send_pos[t][j]] (bf16)."""
+    T, k = send_pos.shape
+    d = ysend.shape[1]
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=ysend.device)
+    _room(out, T * d, "out")
+    _room(ysend, T * k * d, "ysend")
+    _dev(ysend, torch.float32, "ysend")
+    _dev(topk_w, torch.float32, "topk_w")
+    _dev(send_pos, torch.int32, "send_pos")
+    _dev(out, torch.bfloat16, "out")
+    _check(_lib.moe_ep_combine(_ptr(ysend), _ptr(topk_w), _ptr(send_pos), T, d, k, _ptr(out),
+                               _stream(stream, ysend, topk_w, send_pos, out)), "moe_ep_combine")
+    return out
 
 
 def moe_get_device_status(stream=None) -> int:

@@ -536,6 +536,21 @@ int* status_word(int dev) {
     return ptrs[dev];
 }
 
+// The library's stream-ordered pool on device `dev` (current), created on first use; null on failure.
+cudaMemPool_t library_pool(int dev) {
+    DeviceState st;
+    return device_state(dev, &st) ? st.pool : nullptr;
+}
+
+// SM count of device `dev` (0 if unknown: launchers then assume 148).
+int device_sms(int dev) {
+    DeviceState st;
+    return device_state(dev, &st) ? st.num_sms : 0;
+}
+
+// Time limit of one pipeline wait (MOE_WAIT_LIMIT_MS, default 1 s).
+long long pipeline_wait_ns() { return wait_limit_ns(); }
+
 }  // namespace moe
 
 using namespace moe;

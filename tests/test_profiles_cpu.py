@@ -29,7 +29,7 @@ def _entries():
 def test_recorded_traffic_belongs_to_a_capture_of_the_current_sources():
     bench = _bench()
     for key, ent in _entries().items():
-        kernel, workload = key.split("@")
+        kernel, workload = key.split("@", 1)
         assert ent["source_sha"] == bench.source_sha(ent["sources"]), \
             f"{key}: kernel sources changed since the capture: recapture it, or remove the entry"
         assert bench.recorded_traffic(kernel, workload) == ent["bytes_per_launch"]
