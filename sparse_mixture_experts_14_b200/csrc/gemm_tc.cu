@@ -277,6 +277,13 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
         // ---------------------------------------------------------------- TMA producer (both CTAs)
         if (lane == 0) {
             const uint64_t pol = ptx::policy_evict_normal();
+            // GEMM1: an expert's gathered rows (A) are read once per n-block, its W1 / W3 blocks (B)
+            // once per wave.  When the rows outgrow what L2 keeps across waves (workload 5: 50 MB
+            // of rows per expert), streaming weights pushed them out and every wave read them
+            // from HBM again (11.6 GB per launch for 4.7 GB of operands).  Weights evict-first,
+            // rows evict-last: 5.6 GB, and GEMM1 4-6% faster at T >= 8192, neutral at T = 4096.
+            const uint64_t polA = MT::GATED ? ptx::policy_evict_last() : pol;
+            const uint64_t polB = MT::GATED ? ptx::policy_evict_first() : pol;
             int stage = 0;
             uint32_t phase = 0;
             bool armed[NST];
@@ -316,7 +323,7 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                         ptx::tma_load_2d_pair(sb, &mapB1, full_leader, n0, krow, pol);
                         ptx::tma_load_2d_pair(sb + MN_LBO, &mapB1, full_leader, n0 + MN_BOX, krow, pol);
                     } else {
-                        ptx::tma_load_2d_pair(sa, &mapA, full_leader, kb * BK, rowA, pol);
+                        ptx::tma_load_2d_pair(sa, &mapA, full_leader, kb * BK, rowA, polA);
                         if (MT::B_MN) {
                             // weights [E][K][N], N contiguous: [64 k][64 n] boxes
                             const bool hi = MODE == kDgradX && kb >= p.kb_split;
@@ -327,7 +334,7 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                         } else {
                             const CUtensorMap* mapB = (MT::GATED && !leader) ? &mapB3 : &mapB1;
                             const int rowB = MT::GATED ? n_blk * BNH : n0;
-                            ptx::tma_load_3d_pair(sb, mapB, full_leader, kb * BK, rowB, e, pol);
+                            ptx::tma_load_3d_pair(sb, mapB, full_leader, kb * BK, rowB, e, polB);
                         }
                     }
 #pragma unroll
