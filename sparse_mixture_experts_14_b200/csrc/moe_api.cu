@@ -46,6 +46,8 @@ __device__ int g_status;   // per-device sticky fault word (first fault wins)
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kHostChunk = 4096;       // tokens per chunk of the host entry point's pipelined path
+constexpr int kMaxHostChunks = 64;     // at most this many chunks (larger batches take larger chunks)
 
 std::mutex g_mu;
 cudaMemPool_t g_pools[kMaxDevices] = {};
@@ -536,6 +538,24 @@ int* status_word(int dev) {
     return ptrs[dev];
 }
 
+// Two copy streams per device for the host entry point (host-to-device, device-to-host), created
+// on first use, non-blocking (they never wait for the legacy default stream).
+bool copy_streams(int dev, cudaStream_t* h2d, cudaStream_t* d2h) {
+    static std::mutex mu;
+    static cudaStream_t streams[kMaxDevices][2] = {};
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < 2; ++i)
+        if (!streams[dev][i] && cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking) != cudaSuccess) {
+            streams[dev][i] = nullptr;
+            cudaGetLastError();
+            return false;
+        }
+    *h2d = streams[dev][0];
+    *d2h = streams[dev][1];
+    return true;
+}
+
 // The library's stream-ordered pool on device `dev` (current), created on first use; null on failure.
 cudaMemPool_t library_pool(int dev) {
     DeviceState st;
@@ -702,19 +722,67 @@ moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, 
     DeviceState dev;
     const DeviceScope scope(Wg, false);
     if (!device_state(scope.device(), &dev)) return MOE_ERR_CUDA;
-    const size_t act = (size_t)T * d * 2;
+    const size_t row = (size_t)d * 2;
+    const size_t act = (size_t)T * row;
     const size_t act_al = align_up(act, 256);
-    const Plan p = make_plan(T, d, ffn, E, k, MOE_DTYPE_BF16);
+    // Large batches run in chunks of at least kHostChunk tokens, so that each chunk's copies
+    // overlap the previous chunk's layer.  Tokens are independent and every kernel of the
+    // chunked path gives a token the bits it gets in one call (the tensor-core router adds its
+    // K chunks in the same order for any batch; a GEMM row's arithmetic does not depend on its
+    // place in a tile), so the result equals the unchunked call bit for bit.
+    const int nch = T >= 2 * kHostChunk ? min(T / kHostChunk, kMaxHostChunks) : 1;
+    const int tc = (T + nch - 1) / nch;
+    const Plan p = make_plan(tc, d, ffn, E, k, MOE_DTYPE_BF16);
     void* buf = nullptr;
     if (cudaMallocFromPoolAsync(&buf, 2 * act_al + p.total, dev.pool, stream) != cudaSuccess)
         return MOE_ERR_WORKSPACE;
     uint8_t* xd = static_cast<uint8_t*>(buf);
     uint8_t* od = xd + act_al;
     uint8_t* ws = od + act_al;
-    cudaError_t e = cudaMemcpyAsync(xd, x_host, act, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess) {
-        st = run_layer(xd, Wg, W1, W3, W2, od, T, d, ffn, E, k, MOE_DTYPE_BF16, MOE_PATH_AUTO, ws, dev, stream);
-        if (st == MOE_OK) e = cudaMemcpyAsync(out_host, od, act, cudaMemcpyDeviceToHost, stream);
+    cudaError_t e = cudaSuccess;
+    if (nch == 1) {
+        e = cudaMemcpyAsync(xd, x_host, act, cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess) {
+            st = run_layer(xd, Wg, W1, W3, W2, od, T, d, ffn, E, k, MOE_DTYPE_BF16, MOE_PATH_AUTO, ws, dev, stream);
+            if (st == MOE_OK) e = cudaMemcpyAsync(out_host, od, act, cudaMemcpyDeviceToHost, stream);
+        }
+    } else {
+        cudaStream_t h2d = nullptr, d2h = nullptr;
+        if (!copy_streams(scope.device(), &h2d, &d2h)) e = cudaErrorUnknown;
+        // events: [0] the buffer exists; then per chunk "copied in" and "computed"; last "copied out"
+        cudaEvent_t ev[2 * kMaxHostChunks + 2] = {};
+        const int nev = 2 * nch + 2;
+        for (int i = 0; i < nev && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[0], stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(h2d, ev[0], 0);
+        for (int c = 0; c < nch && e == cudaSuccess; ++c) {
+            const size_t t0 = (size_t)c * tc, n = (size_t)min(tc, T - c * tc);
+            e = cudaMemcpyAsync(xd + t0 * row, static_cast<const uint8_t*>(x_host) + t0 * row, n * row,
+                                cudaMemcpyHostToDevice, h2d);
+            if (e == cudaSuccess) e = cudaEventRecord(ev[1 + c], h2d);
+        }
+        for (int c = 0; c < nch && e == cudaSuccess && st == MOE_OK; ++c) {
+            const size_t t0 = (size_t)c * tc;
+            const int n = min(tc, T - c * tc);
+            e = cudaStreamWaitEvent(stream, ev[1 + c], 0);
+            if (e != cudaSuccess) break;
+            st = run_layer(xd + t0 * row, Wg, W1, W3, W2, od + t0 * row, n, d, ffn, E, k, MOE_DTYPE_BF16,
+                           MOE_PATH_AUTO, ws, dev, stream);
+            if (st != MOE_OK) break;
+            e = cudaEventRecord(ev[1 + nch + c], stream);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(d2h, ev[1 + nch + c], 0);
+            if (e == cudaSuccess)
+                e = cudaMemcpyAsync(static_cast<uint8_t*>(out_host) + t0 * row, od + t0 * row, (size_t)n * row,
+                                    cudaMemcpyDeviceToHost, d2h);
+        }
+        // the buffer goes back to the pool only after the last copy out
+        if (ev[nev - 1]) {
+            if (cudaEventRecord(ev[nev - 1], d2h) == cudaSuccess) cudaStreamWaitEvent(stream, ev[nev - 1], 0);
+            else cudaStreamSynchronize(d2h);
+        }
+        if (h2d) cudaStreamSynchronize(h2d);
+        for (int i = 0; i < nev; ++i)
+            if (ev[i]) cudaEventDestroy(ev[i]);
     }
     cudaError_t f = cudaFreeAsync(buf, stream);
     cudaError_t g = cudaStreamSynchronize(stream);

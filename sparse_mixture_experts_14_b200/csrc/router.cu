@@ -459,7 +459,7 @@ struct RtCtrl {
 
 template <int EP>
 constexpr int rt_smem_bytes() {
-    return RtRing<EP>::STAGES * RtRing<EP>::STAGE_BYTES + RT_M * 33 * 4 + (int)sizeof(RtCtrl) + 1024;
+    return RtRing<EP>::STAGES * RtRing<EP>::STAGE_BYTES + (int)sizeof(RtCtrl) + 1024;
 }
 
 // One 128-token tile per CTA (cluster rank = the K split it reads).  Warp 0
@@ -469,8 +469,11 @@ constexpr int rt_smem_bytes() {
 // own TMEM column block, so no accumulation inside the tensor core runs longer
 // than K = 256; then all four warps read their 32 rows, add the blocks in
 // order in fp32 and, with one split, finish the token (scores, top-k, gates).
-// With several splits each CTA leaves its partial scores in shared memory and
-// rank 0 adds them in rank order.
+// With several splits each CTA leaves the values of each of its 256-wide K
+// chunks in shared memory (the ring, idle by then) and rank 0 adds all chunks in
+// global K order.  Every split count therefore adds the same chunk values in the
+// same order: the scores, and so the routing, of a token do not depend on the
+// batch it comes in (for every T this kernel serves).
 template <int EP>
 __global__ void __launch_bounds__(RT_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW, int T,
@@ -480,8 +483,9 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     constexpr int RT_STAGE_BYTES = RtRing<EP>::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* part = reinterpret_cast<float*>(smem + RT_STAGES * RT_STAGE_BYTES);   // [128][33]
-    RtCtrl* ctrl = reinterpret_cast<RtCtrl*>(smem + RT_STAGES * RT_STAGE_BYTES + RT_M * 33 * 4);
+    // after the main loop the ring holds each chunk's scores for the cluster reduction: [chunk][row][EP + 1]
+    float* part = reinterpret_cast<float*>(smem);
+    RtCtrl* ctrl = reinterpret_cast<RtCtrl*>(smem + RT_STAGES * RT_STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t nsplit;
     asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(nsplit));
@@ -621,13 +625,15 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                 ptx::tmem_ld_32x32b_x32(taddr + (uint32_t)(c * EP), r);
             }
             ptx::tmem_ld_wait();
+            if (nsplit > 1) {
+                float* dst = part + ((size_t)c * RT_M + row) * (EP + 1);
 #pragma unroll
-            for (int e = 0; e < EP; ++e) sc[e] += __uint_as_float(r[e]);
+                for (int e = 0; e < EP; ++e) dst[e] = __uint_as_float(r[e]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < EP; ++e) sc[e] += __uint_as_float(r[e]);
+            }
         }
-    }
-    if (nsplit > 1) {
-#pragma unroll
-        for (int e = 0; e < EP; ++e) part[row * 33 + e] = sc[e];
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
@@ -636,22 +642,23 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         ptx::tmem_dealloc(tmem_base, (uint32_t)tmem_cols);
     }
     if (nsplit > 1) {
-        ptx::cluster_sync();   // every split's partial scores are in its shared memory
+        ptx::cluster_sync();   // every split's chunk scores are in its shared memory
         if (split == 0) {
-            const uint32_t base = ptx::smem_addr(part + row * 33);
-#pragma unroll
-            for (int e = 0; e < EP; ++e) sc[e] = 0.f;
+            // all chunks in global K order: split r holds chunks r * chunks .. (r + 1) * chunks - 1
             for (uint32_t r = 0; r < nsplit; ++r) {
-                const uint32_t peer = ptx::map_to_rank(base, r);
+                for (int c = 0; c < chunks; ++c) {
+                    const uint32_t peer =
+                        ptx::map_to_rank(ptx::smem_addr(part + ((size_t)c * RT_M + row) * (EP + 1)), r);
 #pragma unroll
-                for (int e = 0; e < EP; ++e) {
-                    float v;
-                    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(peer + 4u * e) : "memory");
-                    sc[e] += v;
+                    for (int e = 0; e < EP; ++e) {
+                        float v;
+                        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(peer + 4u * e) : "memory");
+                        sc[e] += v;
+                    }
                 }
             }
         }
-        ptx::cluster_sync();   // no CTA leaves while rank 0 still reads its partials
+        ptx::cluster_sync();   // no CTA leaves while rank 0 still reads its chunks
         if (split != 0) return;
     }
     if (!ok || m0 + row >= T) return;
@@ -670,14 +677,26 @@ cudaError_t launch_router_tc_t(const __nv_bfloat16* x, const __nv_bfloat16* Wg, 
     if (e != cudaSuccess) return e;
     const int tiles = (T + RT_M - 1) / RT_M;
     const int kbs = d / RT_BK;
-    // split d over a cluster while that still leaves every CTA on its own SM, and until the
-    // 256-wide accumulator blocks of one CTA fit the 512 TMEM columns
-    int splits = 1;
-    while (splits < 8 && kbs % (2 * splits) == 0 &&
-           (tiles * 2 * splits <= num_sms || ((kbs / splits + RT_CHUNK_KB - 1) / RT_CHUNK_KB) * EP > 512))
-        splits *= 2;
+    // A split count is usable when it divides d's K steps into whole 256-wide chunks per CTA (so
+    // every split count adds the same chunks in the same order), the CTA's chunks fit the 512 TMEM
+    // columns and, with a cluster, its chunk scores fit the idle ring.  Take the largest usable one
+    // that keeps one CTA per SM, else the smallest usable one.
+    const long long ring = (long long)RtRing<EP>::STAGES * RtRing<EP>::STAGE_BYTES;
+    auto usable = [&](int sp) {
+        if (kbs % sp != 0) return false;
+        const int per = kbs / sp;
+        if (sp > 1 && per % RT_CHUNK_KB != 0) return false;
+        const int ch = (per + RT_CHUNK_KB - 1) / RT_CHUNK_KB;
+        if (ch * EP > 512) return false;
+        return sp == 1 || (long long)ch * RT_M * (EP + 1) * 4 <= ring;
+    };
+    int splits = 0;
+    for (int sp = 8; sp >= 1 && !splits; sp /= 2)
+        if (usable(sp) && (long long)tiles * sp <= num_sms) splits = sp;
+    for (int sp = 1; sp <= 8 && !splits; sp *= 2)
+        if (usable(sp)) splits = sp;
+    if (!splits) return cudaErrorNotSupported;   // the caller takes the mma.sync router
     const int chunks = (kbs / splits + RT_CHUNK_KB - 1) / RT_CHUNK_KB;
-    if (chunks * EP > 512) return cudaErrorInvalidValue;
     int cols = 32;
     while (cols < chunks * EP) cols *= 2;
     CUtensorMap mx, mw;
@@ -760,8 +779,9 @@ cudaError_t launch_router_bf16(const void* x, const void* Wg, int T, int d, int 
     const RouterIO<__nv_bfloat16> io = make_io<__nv_bfloat16>(idx, w, ex);
     // tensor-core scores for large batches; small batches spread one token per block instead
     if (!ex.gamma && E % 8 == 0 && d % RT_BK == 0 && T > 4 * num_sms) {
-        return E <= 16 ? launch_router_tc_t<16>(xb, wb, T, d, E, k, io, num_sms, ex.status, ex.wait_ns, s)
-                       : launch_router_tc_t<32>(xb, wb, T, d, E, k, io, num_sms, ex.status, ex.wait_ns, s);
+        const cudaError_t e = E <= 16 ? launch_router_tc_t<16>(xb, wb, T, d, E, k, io, num_sms, ex.status, ex.wait_ns, s)
+                                      : launch_router_tc_t<32>(xb, wb, T, d, E, k, io, num_sms, ex.status, ex.wait_ns, s);
+        if (e != cudaErrorNotSupported) return e;   // else: no usable split of d, the mma.sync router below
     }
     if (d % 32 == 0 && T > 4 * num_sms) {
         return ex.gamma ? launch_router_mma<true>(xb, wb, T, d, E, k, io, num_sms, s)

@@ -371,3 +371,31 @@ def test_forward_ws_graph_capture(moe, T):
     _status_clear(moe)
     assert torch.equal(out, want)
     del g
+
+
+@pytest.mark.parametrize("d,E,k", [(1024, 8, 2), (4096, 8, 2), (2048, 32, 2), (6144, 16, 4)])
+def test_route_is_batch_invariant(moe, d, E, k):
+    """The tensor-core router adds its 256-wide K chunks in the same order whatever cluster split a
+    batch size picks: a token's gates and experts are the same bits in a batch of 1000 and of 9000."""
+    inp = moe_inputs.make_inputs(9000, d, 128, E, k, "bf16", seed=d + E, weights=False)
+    x, Wg = upload(inp)[:2]
+    idx_big, w_big = moe.moe_route(x, Wg, k)
+    idx_small, w_small = moe.moe_route(x[:1000].contiguous(), Wg, k)
+    _status_clear(moe)
+    assert torch.equal(idx_small, idx_big[:1000])
+    assert torch.equal(w_small, w_big[:1000])
+
+
+@pytest.mark.parametrize("T", [8192, 10001])
+def test_chunked_host_entry_matches_device(moe, T):
+    """Batches of 8192 tokens and more go through the host entry point in pipelined chunks; the
+    result equals the one-call device path bit for bit, from pinned and from pageable buffers."""
+    inp = moe_inputs.make_inputs(T, 256, 512, 8, 2, "bf16", seed=T)
+    dev = upload(inp)
+    a = moe.moe_forward(*dev, 2).cpu()
+    b = moe.moe_forward_host(dev[0].cpu().pin_memory(), *dev[1:], 2)
+    assert torch.equal(a, b)
+    out = torch.empty_like(a)
+    c = moe.moe_forward_host(dev[0].cpu(), *dev[1:], 2, out_host=out)
+    assert torch.equal(a, c)
+    _status_clear(moe)
