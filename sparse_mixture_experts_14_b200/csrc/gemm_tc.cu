@@ -28,21 +28,10 @@
 //              quarter, gating / fp32 stores; then one arrival per warp on the
 //              leader's "accumulator free" barrier
 // Pair tiles are (expert, n-block, m-tile pair) with pairs fastest, so the
-// CTAs at work share one block of expert weights through L2.  The tile list is
-// derived on the device from the dispatch offsets and counts: no host
-// synchronisation.
-//
-// The last rows of an expert.  The pair MMA multiplies 256 rows by one B block
-// shared by both CTAs, so a 256-row tile over an expert's last r < 256 rows would
-// spend 256 - r rows of tensor time on padding (at 4096 tokens, 9% of GEMM1 and
-// GEMM2).  In the forward GEMMs that remainder runs with the operands' roles
-// swapped instead: the weights are the M = 256 side (each CTA's 128 weight rows,
-// the B block of a full tile) and the remainder the N side, N = r rounded up to 16,
-// each CTA holding N/2 of those rows, so the MMAs cost what the r rows need.  The
-// accumulator is then [weight row][token]: in GEMM1 each CTA's 128 weight rows are
-// 64 features of W1 then the same 64 of W3, so the W1 and W3 results of a feature
-// sit in lanes of two different warps, which trade half of each 32-column chunk
-// through shared memory for the gating.
+// CTAs at work share one block of expert weights through L2.  When an expert
+// has an odd number of m-tiles, the peer of its last pair computes rows past
+// the expert's segment and stores nothing.  The tile list is derived on the
+// device from the dispatch offsets: no host synchronisation.
 //
 // The same kernel runs the layer's backward GEMMs (gradients of the expert
 // equations, the training the page's "ロードバランス損失" subsection closes with):
@@ -120,7 +109,6 @@ struct Ctrl {
     uint64_t tfull[2];          // each CTA: accumulator b holds a finished tile
     uint64_t tempty[2];         // leader: both CTAs' epilogues released accumulator b
     uint64_t drain;
-    uint64_t xfull[2][2];       // SWAP_XCHG: [warp pair][buffer]: both warps' halves of a chunk are staged
     uint32_t tmem_base;
     int abort;
     int total;
@@ -129,8 +117,6 @@ struct Ctrl {
     int pt[kMaxExperts];        // pairs of m-tiles of expert e
     int row0[kMaxExperts];      // first row of expert e's segment
     int nkb[kMaxExperts];       // K blocks of expert e (grouped-by-K tiles)
-    int pf[kMaxExperts];        // SWAP_REM: full 256-row pairs of expert e; pair pf[e] is the swapped tile
-    int nrem[kMaxExperts];      // SWAP_REM: its N (the r remaining rows rounded up to 16; 0: no such tile)
     int ntn;                    // n-blocks per expert
     int n_fast;                 // tile order (decode_tile)
 };
@@ -158,14 +144,10 @@ struct ModeT {
     // accesses run at one 128-byte wavefront per 8 lanes without padding.
     static constexpr bool STAGED_OUT = KGROUP;
     static constexpr bool STAGED_AB = MODE == kFwd1Train || MODE == kDgradH;
-    // an expert's last r < 256 rows as one swapped tile (see the file comment); GEMM1's gating
-    // then trades accumulator halves between warps through shared memory
-    static constexpr bool SWAP_REM = MODE == kFwd1 || MODE == kFwd2;
-    static constexpr bool SWAP_XCHG = MODE == kFwd1;
     static constexpr int EPI_WARPS = STAGED_OUT ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS);
-    static constexpr int STAGES_M = STAGED_OUT || STAGED_AB || SWAP_XCHG ? STAGES - 1 : STAGES;
-    static constexpr int STAGE_OUT_BYTES = (STAGED_OUT || SWAP_XCHG ? 1 : STAGED_AB ? 2 : 0) * EPI_WARPS * 32 * OUT_PITCH * 4;
+    static constexpr int STAGES_M = STAGED_OUT || STAGED_AB ? STAGES - 1 : STAGES;
+    static constexpr int STAGE_OUT_BYTES = (STAGED_OUT ? 1 : STAGED_AB ? 2 : 0) * EPI_WARPS * 32 * OUT_PITCH * 4;
     static constexpr int SMEM = STAGES_M * STAGE_BYTES + STAGE_OUT_BYTES + (int)sizeof(Ctrl) + 1024;
 };
 
@@ -213,10 +195,7 @@ __device__ __forceinline__ void wave_sync(int* counter, int target) {
 template <int MODE>
 __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB1,
-                   const __grid_constant__ CUtensorMap mapB3, const __grid_constant__ CUtensorMap mapB1s,
-                   const __grid_constant__ CUtensorMap mapB3s, const __grid_constant__ CUtensorMap mapA16,
-                   const __grid_constant__ CUtensorMap mapA32, const __grid_constant__ CUtensorMap mapA64,
-                   const GemmParams p) {
+                   const __grid_constant__ CUtensorMap mapB3, const GemmParams p) {
     using MT = ModeT<MODE>;
     constexpr int NST = MT::STAGES_M;
     extern __shared__ uint8_t smem_raw[];
@@ -244,7 +223,6 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
             ptx::mbar_init(&ctrl->tempty[b], 2 * MT::EPI_WARPS);
         }
         ptx::mbar_init(&ctrl->drain, 1);
-        for (int i = 0; i < 4; ++i) ptx::mbar_init(&ctrl->xfull[i >> 1][i & 1], 64);
         ctrl->abort = 0;
         ptx::fence_mbar_init();
     }
@@ -252,15 +230,6 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
         ptx::tma_prefetch_desc(&mapA);
         ptx::tma_prefetch_desc(&mapB1);
         if (MT::GATED || MODE == kDgradX) ptx::tma_prefetch_desc(&mapB3);
-        if (MT::SWAP_REM && MT::GATED) {
-            ptx::tma_prefetch_desc(&mapB1s);
-            ptx::tma_prefetch_desc(&mapB3s);
-        }
-        if (MT::SWAP_REM) {
-            ptx::tma_prefetch_desc(&mapA16);
-            ptx::tma_prefetch_desc(&mapA32);
-            ptx::tma_prefetch_desc(&mapA64);
-        }
     }
     if (warp == 1) {
         ptx::tmem_alloc_pair(&ctrl->tmem_base, TMEM_COLS);
@@ -289,16 +258,6 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                 ctrl->mt[e] = mt;
                 ctrl->pt[e] = (mt + 1) / 2;
                 ctrl->nkb[e] = (p.K + BK - 1) / BK;
-                if (MT::SWAP_REM) {
-                    // the first counts[e] rows of the segment are the expert's; the rest is padding
-                    const int cnt = meta->counts[e];
-                    if (cnt < 0 || cnt > rows) ok = false;
-                    const int c = ok ? cnt : 0;
-                    const int rem = c % (2 * BM);
-                    ctrl->pf[e] = c / (2 * BM);
-                    ctrl->nrem[e] = (rem + 15) & ~15;
-                    ctrl->pt[e] = ctrl->pf[e] + (rem != 0);
-                }
             }
             ctrl->row0[e] = r0;
             ctrl->tile_base[e + 1] = ctrl->tile_base[e] + ctrl->pt[e] * ntn;
@@ -343,15 +302,6 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                 const int rowA = ctrl->row0[e] + m_tile * BM;            // row-grouped: A rows
                 const int n0 = n_blk * BN + (int)rank * BNH;             // this CTA's B rows (non-gated)
                 const int nkb = ctrl->nkb[e];
-                // swapped remainder tile: this CTA's nrem / 2 rows come in the smallest box of
-                // 16 / 32 / 64 / 128 rows that holds them (the tile is bound by operand delivery,
-                // the weights block being the same as a full tile's)
-                const bool swap = MT::SWAP_REM && pair == ctrl->pf[e];
-                const int half_rows = swap ? ctrl->nrem[e] >> 1 : BM;
-                const int box_rows = half_rows <= 16 ? 16 : half_rows <= 32 ? 32 : half_rows <= 64 ? 64 : BM;
-                const CUtensorMap* mapAsw = box_rows == 16 ? &mapA16 : box_rows == 32 ? &mapA32
-                                          : box_rows == 64 ? &mapA64 : &mapA;
-                const uint32_t tx = swap ? 2u * (uint32_t)(B_BYTES + box_rows * BK * 2) : PAIR_TX_BYTES;
                 // grouped-by-K tiles are short and their operand blocks stay in L2 across a few
                 // waves of drift: no alignment (it would hold every cluster to the slowest tile)
                 if (leader && !MT::KGROUP) wave_sync(&meta->waves[p.wave_slot], min(total, (wave + 1) * nclusters));
@@ -363,7 +313,7 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                     uint8_t* sa = smem + stage * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
                     const uint32_t full_leader = ptx::map_to_rank(ptx::smem_addr(&ctrl->full[stage]), 0);
-                    if (leader) ptx::mbar_arrive_expect_tx(&ctrl->full[stage], tx);
+                    if (leader) ptx::mbar_arrive_expect_tx(&ctrl->full[stage], PAIR_TX_BYTES);
                     if (MT::KGROUP) {
                         // A^T and B^T tiles of the expert's rows: [64 k][64 m] boxes, m / n contiguous
                         const int krow = ctrl->row0[e] + kb * BK;
@@ -372,18 +322,6 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                         ptx::tma_load_2d_pair(sa + MN_LBO, &mapA, full_leader, m0 + MN_BOX, krow, pol);
                         ptx::tma_load_2d_pair(sb, &mapB1, full_leader, n0, krow, pol);
                         ptx::tma_load_2d_pair(sb + MN_LBO, &mapB1, full_leader, n0 + MN_BOX, krow, pol);
-                    } else if (swap) {
-                        // swapped remainder tile: this CTA's nrem / 2 rows and its 128 weight rows
-                        const int tok = ctrl->row0[e] + pair * 2 * BM + (int)rank * half_rows;
-                        ptx::tma_load_2d_pair(sa, mapAsw, full_leader, kb * BK, tok, polA);
-                        if (MT::GATED) {
-                            // rows 0-63: W1 features f0 + [0, 64), rows 64-127: W3's
-                            const int f0 = n_blk * BNH + (int)rank * (BNH / 2);
-                            ptx::tma_load_3d_pair(sb, &mapB1s, full_leader, kb * BK, f0, e, polB);
-                            ptx::tma_load_3d_pair(sb + B_BYTES / 2, &mapB3s, full_leader, kb * BK, f0, e, polB);
-                        } else {
-                            ptx::tma_load_3d_pair(sb, &mapB1, full_leader, kb * BK, n0, e, polB);
-                        }
                     } else {
                         ptx::tma_load_2d_pair(sa, &mapA, full_leader, kb * BK, rowA, polA);
                         if (MT::B_MN) {
@@ -436,8 +374,6 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                 }
                 ptx::tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                const bool swap = MT::SWAP_REM && pair == ctrl->pf[e];
-                const uint32_t idesc = swap ? ptx::idesc_bf16_f32(2 * BM, ctrl->nrem[e]) : MT::IDESC;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!ptx::mbar_wait(&ctrl->full[stage], phase, wc)) {
                         aborted = true;
@@ -453,11 +389,7 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                                                      : ptx::desc_kmajor_sw128(a0 + kk * 32);
                         const uint64_t db = MT::B_MN ? ptx::desc_mnmajor_sw128(b0 + kk * 2048, MN_LBO, MN_SBO)
                                                      : ptx::desc_kmajor_sw128(b0 + kk * 32);
-                        // swapped tile: the weights (B slot) are the M side, the rows (A slot) the N side
-                        if (swap)
-                            ptx::tc_mma_bf16_pair(d_tmem, db, da, idesc, (kb | kk) != 0);
-                        else
-                            ptx::tc_mma_bf16_pair(d_tmem, da, db, idesc, (kb | kk) != 0);
+                        ptx::tc_mma_bf16_pair(d_tmem, da, db, MT::IDESC, (kb | kk) != 0);
                     }
                     ptx::tc_commit_pair_multicast(&ctrl->empty[stage], 0x3);
                     issued = true;
@@ -483,9 +415,7 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
         const uint64_t pol_out = ptx::policy_evict_first();
         int acc = 0;
         uint32_t acc_phase = 0;
-        int xchunk = 0;       // SWAP_XCHG: chunks traded so far (buffer parity, barrier phase)
-        bool xfail = false;   // a trade's wait gave up (abort raised)
-        for (int tile = cluster; tile < total && !xfail; tile += nclusters) {
+        for (int tile = cluster; tile < total; tile += nclusters) {
             int e, pair, n_blk;
             decode_tile(ctrl, tile, e, pair, n_blk);
             const int m_tile = 2 * pair + (int)rank;
@@ -493,72 +423,12 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             ptx::tc_fence_after_sync();
-            // a swapped tile has output in both CTAs; elsewhere the peer of an odd expert's last
-            // pair holds rows past the segment
-            const bool live = MT::KGROUP                              ? m_tile * BM < p.M
-                              : MT::SWAP_REM && pair == ctrl->pf[e] ? true
-                                                                    : m_tile < ctrl->mt[e];
+            const bool live = MT::KGROUP ? m_tile * BM < p.M : m_tile < ctrl->mt[e];
             if (live) {
                 const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
                 constexpr int HALVES = MT::EPI_WARPS / NUM_EPI_WARPS;   // warps per TMEM lane quarter
                 const int half = ew / NUM_EPI_WARPS;
-                if (MT::SWAP_REM && pair == ctrl->pf[e]) {
-                    // swapped remainder tile: lane = weight row, column t = row t of the remainder
-                    const int nrem = ctrl->nrem[e];
-                    const size_t tok0 = (size_t)ctrl->row0[e] + (size_t)pair * 2 * BM;
-                    if (MT::SWAP_XCHG) {
-                        // quarter pr holds W1 results of features f0 + 32 pr + lane, quarter pr + 2 the W3
-                        // results of the same features.  Per 32-column chunk each warp stages the half
-                        // its partner gates (the W1 warp gates columns 0-15, the W3 warp 16-31) in its
-                        // buffer of the chunk's parity; both warps' lanes arrive on that buffer's barrier
-                        // (its next use is two chunks on, after both have arrived on the other buffer's,
-                        // so after the partner read this one)
-                        const int pr = q & 1;
-                        const bool is_b = q >= 2;
-                        const int f = n_blk * BNH + (int)rank * (BNH / 2) + pr * 32 + lane;
-                        __nv_bfloat16* H = static_cast<__nv_bfloat16*>(p.out);
-#pragma unroll 1
-                        for (int c = 0; c < nrem; c += 32) {
-                            uint32_t r[32];
-                            ptx::tmem_ld_32x32b_x32(taddr + c, r);
-                            ptx::tmem_ld_wait();
-                            const int xb = xchunk & 1;
-                            const uint32_t ph = (uint32_t)(xchunk >> 1) & 1u;
-                            ++xchunk;
-                            float* mine = stage_out + (q * 2 + xb) * 16 * 32;
-                            const float* theirs = stage_out + ((q ^ 2) * 2 + xb) * 16 * 32;
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) mine[i * 32 + lane] = __uint_as_float(is_b ? r[i] : r[16 + i]);
-                            ptx::mbar_arrive(&ctrl->xfull[pr][xb]);
-                            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&ctrl->xfull[pr][xb], ph, wc))) {
-                                xfail = true;
-                                break;
-                            }
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const float o = theirs[i * 32 + lane];
-                                const float a = is_b ? o : __uint_as_float(r[i]);
-                                const float b = is_b ? __uint_as_float(r[16 + i]) : o;
-                                const int t = c + i + (is_b ? 16 : 0);
-                                if (t < nrem) H[(tok0 + t) * (size_t)N + f] = __float2bfloat16_rn(silu_mul(a, b));
-                            }
-                        }
-                    } else {
-                        const int col = n_blk * BN + (int)rank * BNH + q * 32 + lane;
-                        float* Y = static_cast<float*>(p.out);
-#pragma unroll 1
-                        for (int c = 0; c < nrem; c += 32) {
-                            uint32_t r[32];
-                            ptx::tmem_ld_32x32b_x32(taddr + c, r);
-                            ptx::tmem_ld_wait();
-                            if (col < N) {
-#pragma unroll
-                                for (int i = 0; i < 32; ++i)
-                                    if (c + i < nrem) Y[(tok0 + c + i) * (size_t)N + col] = __uint_as_float(r[i]);
-                            }
-                        }
-                    }
-                } else if (MODE == kFwd1 || MODE == kFwd1Train) {
+                if (MODE == kFwd1 || MODE == kFwd1Train) {
                     const size_t row = (size_t)ctrl->row0[e] + (size_t)m_tile * BM + q * 32 + lane;
                     __nv_bfloat16* H = static_cast<__nv_bfloat16*>(p.out);
                     constexpr int CW = BNH / HALVES;
@@ -836,13 +706,9 @@ size_t row_pair_tiles(size_t slots, int E, int n_tiles) {
     return ((slots / BM + (size_t)E) / 2 + 1) * (size_t)n_tiles;
 }
 
-// Boxes of the swapped remainder tiles (other modes: unused): mB1s / mB3s GEMM1's 64-row weight
-// boxes, mAr[0..2] 16-, 32- and 64-row boxes of the rows.
 template <int MODE>
 cudaError_t launch_pair(size_t pair_tiles, int num_sms, const CUtensorMap& mA, const CUtensorMap& mB1,
-                        const CUtensorMap& mB3, const GemmParams& gp, cudaStream_t s,
-                        const CUtensorMap* mB1s = nullptr, const CUtensorMap* mB3s = nullptr,
-                        const CUtensorMap* mAr = nullptr) {
+                        const CUtensorMap& mB3, const GemmParams& gp, cudaStream_t s) {
     cudaError_t e = ensure_smem_attr<MODE>();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -859,8 +725,7 @@ cudaError_t launch_pair(size_t pair_tiles, int num_sms, const CUtensorMap& mA, c
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<MODE>, mA, mB1, mB3, mB1s ? *mB1s : mB1, mB3s ? *mB3s : mB3,
-                           mAr ? mAr[0] : mA, mAr ? mAr[1] : mA, mAr ? mAr[2] : mA, gp);
+    e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<MODE>, mA, mB1, mB3, gp);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -882,18 +747,13 @@ GemmParams params(Meta* meta, int E, int N, int K, int wave_slot, size_t slots, 
 }  // namespace
 
 cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s) {
-    CUtensorMap mA, mB1, mB3, mB1s, mB3s;
+    CUtensorMap mA, mB1, mB3;
     if (!map_rows(&mA, a.xp, a.slots, a.d, BM) || !map_weights(&mB1, a.W1, a.E, a.F, a.d, BNH) ||
-        !map_weights(&mB3, a.W3, a.E, a.F, a.d, BNH) || !map_weights(&mB1s, a.W1, a.E, a.F, a.d, BNH / 2) ||
-        !map_weights(&mB3s, a.W3, a.E, a.F, a.d, BNH / 2))
+        !map_weights(&mB3, a.W3, a.E, a.F, a.d, BNH))
         return cudaErrorInvalidValue;
-    CUtensorMap mAr[3];
-    for (int i = 0; i < 3; ++i)
-        if (!map_rows(&mAr[i], a.xp, a.slots, a.d, 16 << i)) return cudaErrorInvalidValue;
     const GemmParams gp = params(const_cast<Meta*>(a.meta), a.E, a.F, a.d, kWaveFwd1, a.slots, a.H, a.status,
                                  a.wait_ns);
-    return launch_pair<kFwd1>(row_pair_tiles(a.slots, a.E, (a.F + BNH - 1) / BNH), a.num_sms, mA, mB1, mB3, gp, s,
-                              &mB1s, &mB3s, mAr);
+    return launch_pair<kFwd1>(row_pair_tiles(a.slots, a.E, (a.F + BNH - 1) / BNH), a.num_sms, mA, mB1, mB3, gp, s);
 }
 
 cudaError_t launch_tc_gemm1_train(const TcGemmArgs& a, float* keep_a, float* keep_b, cudaStream_t s) {
@@ -909,15 +769,12 @@ cudaError_t launch_tc_gemm1_train(const TcGemmArgs& a, float* keep_a, float* kee
 }
 
 cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s) {
-    CUtensorMap mA, mB, mAr[3];
+    CUtensorMap mA, mB;
     if (!map_rows(&mA, a.H, a.slots, a.F, BM) || !map_weights(&mB, a.W2, a.E, a.d, a.F, BNH))
         return cudaErrorInvalidValue;
-    for (int i = 0; i < 3; ++i)
-        if (!map_rows(&mAr[i], a.H, a.slots, a.F, 16 << i)) return cudaErrorInvalidValue;
     const GemmParams gp = params(const_cast<Meta*>(a.meta), a.E, a.d, a.F, kWaveFwd2, a.slots, a.Y, a.status,
                                  a.wait_ns);
-    return launch_pair<kFwd2>(row_pair_tiles(a.slots, a.E, (a.d + BN - 1) / BN), a.num_sms, mA, mB, mB, gp, s,
-                              nullptr, nullptr, mAr);
+    return launch_pair<kFwd2>(row_pair_tiles(a.slots, a.E, (a.d + BN - 1) / BN), a.num_sms, mA, mB, mB, gp, s);
 }
 
 cudaError_t launch_tc_dgrad_h(const TcBwdArgs& a, cudaStream_t s) {

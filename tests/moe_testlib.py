@@ -79,10 +79,7 @@ def stratified_tokens(idx, E, n_random=8, boundaries=3, odd_tail=8, seed=0, tile
       * the rows on both sides of up to `boundaries` of its 128-row m-tile boundaries, always
         including the first and the last boundary;
       * up to `odd_tail` rows spread over its last m-tile when it has an odd number of m-tiles
-        (in the training forward the CTA pair's second half is then empty);
-      * the rows after its last full 256-row pair (the forward's swapped remainder tile): the
-        first and last of them, both sides of the split between the pair's two CTAs (half of
-        the remainder rounded up to 16), and up to `odd_tail` rows spread over them;
+        (the CTA pair's second half is then empty);
     plus `n_random` tokens drawn uniformly, and tokens 0 and T - 1.
     """
     idx = np.asarray(idx)
@@ -102,12 +99,6 @@ def stratified_tokens(idx, E, n_random=8, boundaries=3, odd_tail=8, seed=0, tile
                 want.update({b - 1, b})
         if mt % 2 == 1:
             lo = (mt - 1) * tile
-            want.update(np.linspace(lo, n - 1, min(odd_tail, n - lo)).astype(np.int64).tolist())
-        lo = (n // (2 * tile)) * 2 * tile
-        if lo < n:
-            split = lo + ((n - lo + 15) // 16 * 16) // 2
-            want.update({lo, n - 1})
-            want.update(r for r in (split - 1, split) if r < n)
             want.update(np.linspace(lo, n - 1, min(odd_tail, n - lo)).astype(np.int64).tolist())
         picked.update(int(rows[r]) for r in want)
     rng = np.random.default_rng(seed)

@@ -1,14 +1,14 @@
-"""The last rows of each expert in the forward grouped GEMMs.
+"""The last rows of each expert in the expert GEMMs.
 
-An expert's rows run as full 256-row CTA-pair tiles, then its last r < 256 rows
-as one tile with the operands' roles swapped (the weights on the MMA's M side,
-the r rows, rounded up to 16, on its N side).  The expert counts are set
-directly through the expert-side entry point of expert parallelism on one rank
-(rows arrive grouped by expert), so every remainder size of interest is reached:
-r = 1, a multiple of 16, one past it, 128, 129, 255 and none at all.  Every row
-is compared with the oracle's expert (subsection "各エキスパートの構造" of the
-Mistral/Mixtral architecture page); a row's result must not depend on which
-kind of tile computed it.
+An expert's rows run as 256-row CTA-pair tiles (two 128-row m-tiles); its last
+r = n mod 256 rows share a tile with padding rows, and when its 128-row m-tiles
+are odd in number the pair's second CTA holds padding only.  The expert counts
+are set directly through the expert-side entry point of expert parallelism on
+one rank (rows arrive grouped by expert), so every remainder of interest is
+reached: r = 1, a multiple of 16, one past it, 128, 129, 255 and none at all.
+Every row is compared with the oracle's expert (subsection "各エキスパートの構造"
+of the Mistral/Mixtral architecture page), and a row's result must not depend
+on where in a tile it lands.
 """
 import numpy as np
 import pytest
@@ -64,7 +64,7 @@ def test_remainder_rows_match_oracle(moe, counts, d, F):
 @pytest.mark.parametrize("n", [16, 100, 200, 255])
 def test_row_result_does_not_depend_on_the_tile_kind(moe, n):
     """The same n rows of one expert, once inside a full 256-row pair tile (the expert holds 256
-    rows) and once as the expert's swapped remainder tile (it holds only these n): equal bits."""
+    rows) and once as the expert's only, partly padded tile (it holds just these n): equal bits."""
     d, F = 256, 512
     inp = moe_inputs.make_inputs(256, d, F, 1, 2, "bf16", seed=n)
     x, _, W1, W3, W2 = upload(inp)
