@@ -46,8 +46,12 @@ __device__ int g_status;   // per-device sticky fault word (first fault wins)
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kHostChunk = 4096;       // tokens per chunk of the host entry point's pipelined path
-constexpr int kMaxHostChunks = 64;     // at most this many chunks (larger batches take larger chunks)
+// Chunks of the host entry point's pipelined path: a short first chunk (its copy in is the only
+// one the layer waits for), a short last one (its copy out is the only one that follows the
+// layer) and middle chunks of up to kHostMid tokens.
+constexpr int kHostEdge = 2048;
+constexpr int kHostMid = 6144;
+constexpr int kMaxHostChunks = 64;     // at most this many chunks (larger batches take larger middle chunks)
 
 std::mutex g_mu;
 cudaMemPool_t g_pools[kMaxDevices] = {};
@@ -725,13 +729,36 @@ moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, 
     const size_t row = (size_t)d * 2;
     const size_t act = (size_t)T * row;
     const size_t act_al = align_up(act, 256);
-    // Large batches run in chunks of at least kHostChunk tokens, so that each chunk's copies
-    // overlap the previous chunk's layer.  Tokens are independent and every kernel of the
-    // chunked path gives a token the bits it gets in one call (the tensor-core router adds its
-    // K chunks in the same order for any batch; a GEMM row's arithmetic does not depend on its
-    // place in a tile), so the result equals the unchunked call bit for bit.
-    const int nch = T >= 2 * kHostChunk ? min(T / kHostChunk, kMaxHostChunks) : 1;
-    const int tc = (T + nch - 1) / nch;
+    // Batches of 2 kHostEdge tokens or more run in chunks, so that each chunk's copies overlap
+    // another chunk's layer.  Tokens are independent and every kernel of the chunked path gives a
+    // token the bits it gets in one call (the tensor-core router adds its K chunks in the same
+    // order for any batch; a GEMM row's arithmetic does not depend on its place in a tile), so
+    // the result equals the unchunked call bit for bit.
+    int cstart[kMaxHostChunks + 1];
+    int nch = 1, tc = T;
+    cstart[0] = 0;
+    // Every chunk holds at least kHostEdge tokens, so every chunk takes the prefill kernels.
+    if (T >= 2 * kHostEdge) {
+        const int mid = T - 2 * kHostEdge;
+        if (mid < kHostEdge) {
+            nch = 2;                       // two halves
+            cstart[1] = T / 2;
+            tc = T - T / 2;
+        } else {
+            const int nmid = min((mid + kHostMid - 1) / kHostMid, kMaxHostChunks - 2);
+            nch = nmid + 2;
+            cstart[1] = kHostEdge;
+            tc = kHostEdge;
+            for (int c = 0; c < nmid; ++c) {
+                const int n = mid / nmid + (c < mid % nmid ? 1 : 0);
+                cstart[2 + c] = cstart[1 + c] + n;
+                tc = max(tc, n);
+            }
+        }
+        cstart[nch] = T;
+    } else {
+        cstart[1] = T;
+    }
     const Plan p = make_plan(tc, d, ffn, E, k, MOE_DTYPE_BF16);
     void* buf = nullptr;
     if (cudaMallocFromPoolAsync(&buf, 2 * act_al + p.total, dev.pool, stream) != cudaSuccess)
@@ -756,14 +783,14 @@ moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, 
         if (e == cudaSuccess) e = cudaEventRecord(ev[0], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(h2d, ev[0], 0);
         for (int c = 0; c < nch && e == cudaSuccess; ++c) {
-            const size_t t0 = (size_t)c * tc, n = (size_t)min(tc, T - c * tc);
+            const size_t t0 = (size_t)cstart[c], n = (size_t)(cstart[c + 1] - cstart[c]);
             e = cudaMemcpyAsync(xd + t0 * row, static_cast<const uint8_t*>(x_host) + t0 * row, n * row,
                                 cudaMemcpyHostToDevice, h2d);
             if (e == cudaSuccess) e = cudaEventRecord(ev[1 + c], h2d);
         }
         for (int c = 0; c < nch && e == cudaSuccess && st == MOE_OK; ++c) {
-            const size_t t0 = (size_t)c * tc;
-            const int n = min(tc, T - c * tc);
+            const size_t t0 = (size_t)cstart[c];
+            const int n = cstart[c + 1] - cstart[c];
             e = cudaStreamWaitEvent(stream, ev[1 + c], 0);
             if (e != cudaSuccess) break;
             st = run_layer(xd + t0 * row, Wg, W1, W3, W2, od + t0 * row, n, d, ffn, E, k, MOE_DTYPE_BF16,
