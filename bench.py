@@ -524,7 +524,9 @@ def run_ours(args, rank, world, local):
     elif T <= moe.moe_decode_max_tokens():
         kname = {"expert1": "decode_kernel<true>", "expert2": "decode_kernel<false>"}[dom]
     else:
-        kname = {"expert1": "tc_gemm_kernel<kFwd1>", "expert2": "tc_gemm_kernel<kFwd2>"}[dom]
+        # the forward GEMMs run on 256 x 512 tiles when their reduction is 5120 or longer
+        kname = {"expert1": "tc_gemm_kernel<kFwd1W>" if d >= 5120 else "tc_gemm_kernel<kFwd1>",
+                 "expert2": "tc_gemm_kernel<kFwd2W>" if F >= 5120 else "tc_gemm_kernel<kFwd2>"}[dom]
     roof["traffic"] = recorded_traffic(kname, workload_name(args.config, args.shape))
     roof["kernel"] = kname
     roof["per_launch"] = {"flops": fl, "bytes": by, "ms": stages[dom]}

@@ -141,6 +141,27 @@ def test_forward_bf16_small(moe, T, d, F, E, k):
     compare_outputs(out_to_f64(out), ref["out"], keep, "bf16")
 
 
+@pytest.mark.parametrize("T,d,F,E,k", [(517, 5120, 5120, 8, 2), (300, 6144, 1024, 8, 2), (301, 1024, 6144, 6, 2)])
+def test_forward_wide_tiles(moe, T, d, F, E, k):
+    """Reductions of 5120 and more run on 256 x 512 tiles (GEMM1 when d >= 5120, GEMM2 when
+    ffn >= 5120): both wide, GEMM1 only, GEMM2 only (ffn = 6144 is 12 wide n-blocks, d = 1024
+    two of GEMM2's), ragged expert counts.  Rows this long are compared on the stratified token
+    sample of the full-size workloads (every expert's first and last rows, its m-tile boundaries
+    and odd last m-tile): over every token of these shapes (1.5-1.8 M outputs, the largest at
+    5.5 x RMS) rounding the exact result to bf16 alone costs up to 1.8% of the 2% bound."""
+    inp = moe_inputs.make_inputs(T, d, F, E, k, "bf16", seed=T + d + F)
+    dev = upload(inp)
+    out = moe.moe_forward(*dev, k)
+    _status_clear(moe)
+    r_idx = oracle.route(inp.x, inp.Wg, k, inp.dtype)[0]
+    toks = stratified_tokens(r_idx, E, seed=T)
+    ref = oracle.moe(*inp.arrays(), k=k, dtype="bf16", tokens=toks, nthreads=oracle.max_threads())
+    idx, w = moe.moe_route(dev[0], dev[1], k)
+    keep = compare_routing(idx.cpu().numpy()[toks], w.cpu().numpy()[toks], ref)
+    rel = compare_outputs(out_to_f64(out)[toks], ref["out"], keep, "bf16")
+    print(f"wide {T}x{d}x{F}: max|err|/RMS = {rel:.3e} over {keep.sum()} tokens")
+
+
 @pytest.mark.parametrize("T,d,F,E,k", [(64, 128, 256, 8, 2), (1, 4, 1, 1, 1), (37, 12, 20, 3, 2),
                                        (200, 64, 100, 8, 8), (129, 132, 70, 6, 1)])
 def test_forward_f32_small(moe, T, d, F, E, k):
