@@ -510,6 +510,13 @@ def run_ours(args, rank, world, local):
     roof_tps = T / max(layer_t_tensor, layer_t_hbm)
     layer_roof = {"bound": layer_bound, "roofline_tokens_per_s": roof_tps, "frac": (value / world) / roof_tps,
                   "flops": acc["layer_flops"], "bytes": acc["layer_bytes"], "touched_experts": acc["touched"]}
+    if layer_bound == "tensor":
+        # the same fraction against the other dense bf16 denominators: the measured burst and
+        # sustained (power-capped) rates, and the 2.25 PFLOP/s datasheet figure
+        achieved = acc["layer_flops"] * (value / world) / T / 1e12
+        layer_roof["frac_vs"] = {"burst": achieved / peaks["bf16_tflops"],
+                                 "sustained": achieved / peaks["bf16_tflops_sustained"],
+                                 "datasheet": achieved / 2250.0}
 
     dom = max(("expert1", "expert2"), key=lambda s: stages[s])
     fl, by = acc[f"{dom}_flops"], acc[f"{dom}_bytes"]
