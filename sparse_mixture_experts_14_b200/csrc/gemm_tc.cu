@@ -82,6 +82,7 @@ enum : int {
     kWgrad16 = 6,    // kWgrad rounded once to bf16                   -> bf16 [E][M][N]
     kFwd1W = 7,      // kFwd1 on 256 x 512 tiles (two N = 256 MMAs per A stage)
     kFwd2W = 8,      // kFwd2 on 256 x 512 tiles
+    kDgradXW = 9,    // kDgradX on 256 x 512 tiles
 };
 
 
@@ -132,8 +133,11 @@ struct ModeT {
     // fewer operand bytes per MMA).  The accumulator takes all 512 TMEM columns (one buffer: the
     // epilogue of a tile is not overlapped with the next tile's MMAs, so it gets two warps per
     // TMEM lane quarter, one per 256-column half) and the ring has 4 stages.
-    static constexpr bool WIDE = MODE == kFwd1W || MODE == kFwd2W;
-    static constexpr int BASE = MODE == kFwd1W ? kFwd1 : MODE == kFwd2W ? kFwd2 : MODE;   // what it computes
+    static constexpr bool WIDE = MODE == kFwd1W || MODE == kFwd2W || MODE == kDgradXW;
+    static constexpr int BASE = MODE == kFwd1W    ? kFwd1
+                                : MODE == kFwd2W  ? kFwd2
+                                : MODE == kDgradXW ? kDgradX
+                                                   : MODE;   // what it computes
     static constexpr int NW = WIDE ? 2 : 1;             // N = 256 MMAs per K = 16 slice
     static constexpr int ACCS = WIDE ? 1 : 2;           // accumulator buffers in the 512 TMEM columns
     static constexpr int B_ROWS = NW * BNH;             // B rows each CTA holds per stage
@@ -142,7 +146,7 @@ struct ModeT {
     static constexpr uint32_t PAIR_TX = 2u * STAGE;
     static constexpr bool GATED = BASE == kFwd1 || BASE == kFwd1Train;   // B halves = W1 / W3 blocks
     static constexpr bool A_MN = MODE == kWgrad || MODE == kWgrad16;
-    static constexpr bool B_MN = MODE == kDgradH || MODE == kDgradX || MODE == kWgrad || MODE == kWgrad16;
+    static constexpr bool B_MN = MODE == kDgradH || BASE == kDgradX || MODE == kWgrad || MODE == kWgrad16;
     static constexpr bool KGROUP = MODE == kWgrad || MODE == kWgrad16;   // tiles grouped by K, not by rows
     static constexpr bool OUT16 = MODE == kWgrad16;
     static constexpr int N_PER_TILE = GATED ? NW * BNH : NW * BN;
@@ -347,8 +351,12 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                             const bool hi = MT::BASE == kDgradX && kb >= p.kb_split;
                             const CUtensorMap* mapB = hi ? &mapB3 : &mapB1;
                             const int kk = (hi ? kb - p.kb_split : kb) * BK;
-                            ptx::tma_load_3d_pair(sb, mapB, full_leader, n0, kk, e, pol);
-                            ptx::tma_load_3d_pair(sb + MN_LBO, mapB, full_leader, n0 + MN_BOX, kk, e, pol);
+#pragma unroll
+                            for (int h = 0; h < MT::NW; ++h) {
+                                ptx::tma_load_3d_pair(sb + h * B_BYTES, mapB, full_leader, n0 + h * BN, kk, e, pol);
+                                ptx::tma_load_3d_pair(sb + h * B_BYTES + MN_LBO, mapB, full_leader, n0 + h * BN + MN_BOX,
+                                                      kk, e, pol);
+                            }
                         } else {
                             // 128-row blocks h = 0 .. NW-1 of this CTA's B rows (gated: features
                             // n_blk * NW * 128 + h * 128 of W1 in the leader, of W3 in the peer)
@@ -413,9 +421,12 @@ __global__ void __launch_bounds__(ModeT<MODE>::THREADS, 1)
                         const uint64_t db = MT::B_MN ? ptx::desc_mnmajor_sw128(b0 + kk * 2048, MN_LBO, MN_SBO)
                                                      : ptx::desc_kmajor_sw128(b0 + kk * 32);
                         ptx::tc_mma_bf16_pair(d_tmem, da, db, MT::IDESC, (kb | kk) != 0);
-                        if (MT::WIDE)   // B rows 128-255 of each CTA: accumulator columns 256-511
-                            ptx::tc_mma_bf16_pair(d_tmem + BN, da, ptx::desc_kmajor_sw128(b0 + B_BYTES + kk * 32),
-                                                  MT::IDESC, (kb | kk) != 0);
+                        if (MT::WIDE) {   // B rows 128-255 of each CTA: accumulator columns 256-511
+                            const uint64_t db2 = MT::B_MN
+                                                     ? ptx::desc_mnmajor_sw128(b0 + B_BYTES + kk * 2048, MN_LBO, MN_SBO)
+                                                     : ptx::desc_kmajor_sw128(b0 + B_BYTES + kk * 32);
+                            ptx::tc_mma_bf16_pair(d_tmem + BN, da, db2, MT::IDESC, (kb | kk) != 0);
+                        }
                     }
                     ptx::tc_commit_pair_multicast(&ctrl->empty[stage], 0x3);
                     issued = true;
@@ -843,6 +854,9 @@ cudaError_t launch_tc_dgrad_x(const TcBwdArgs& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     GemmParams gp = params(a.meta, a.E, a.d, 2 * a.F, kWaveDgradX, a.slots, a.dxp, a.status, a.wait_ns);
     gp.kb_split = a.F / BK;
+    if (2 * a.F >= kWideMinK)
+        return launch_pair<kDgradXW>(row_pair_tiles(a.slots, a.E, (a.d + 2 * BN - 1) / (2 * BN)), a.num_sms, mA, mB1,
+                                     mB3, gp, s);
     return launch_pair<kDgradX>(row_pair_tiles(a.slots, a.E, (a.d + BN - 1) / BN), a.num_sms, mA, mB1, mB3, gp,
                                 s);
 }

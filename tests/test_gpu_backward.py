@@ -76,6 +76,7 @@ def _check(name, got, want, dtype, K=256):
 
 @pytest.mark.parametrize("dtype,T,d,F,E,k", [("bf16", 200, 256, 512, 8, 2), ("bf16", 700, 192, 384, 4, 2),
                                              ("bf16", 90, 128, 256, 16, 4), ("bf16", 40, 256, 128, 8, 8),
+                                             ("bf16", 160, 512, 2560, 8, 2),   # dXp on 256 x 512 tiles (K = 2F)
                                              ("f32", 64, 128, 256, 8, 2), ("f32", 150, 96, 160, 5, 3)])
 def test_backward_small(moe, dtype, T, d, F, E, k):
     inp = moe_inputs.make_inputs(T, d, F, E, k, dtype, seed=T + d + E + k)
