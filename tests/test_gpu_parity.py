@@ -141,11 +141,13 @@ def test_forward_bf16_small(moe, T, d, F, E, k):
     compare_outputs(out_to_f64(out), ref["out"], keep, "bf16")
 
 
-@pytest.mark.parametrize("T,d,F,E,k", [(517, 5120, 5120, 8, 2), (300, 6144, 1024, 8, 2), (301, 1024, 6144, 6, 2)])
+@pytest.mark.parametrize("T,d,F,E,k", [(517, 5120, 5120, 8, 2), (300, 6144, 1024, 8, 2), (301, 1024, 6144, 6, 2),
+                                       (257, 5184, 5248, 8, 2)])
 def test_forward_wide_tiles(moe, T, d, F, E, k):
     """Reductions of 5120 and more run on 256 x 512 tiles (GEMM1 when d >= 5120, GEMM2 when
     ffn >= 5120): both wide, GEMM1 only, GEMM2 only (ffn = 6144 is 12 wide n-blocks, d = 1024
-    two of GEMM2's), ragged expert counts.  Rows this long are compared on the stratified token
+    two of GEMM2's), and both wide with ragged last n-blocks (ffn = 5248: GEMM1's last 256
+    features half past ffn; d = 5184: GEMM2's last 512 columns mostly past d); ragged expert counts.  Rows this long are compared on the stratified token
     sample of the full-size workloads (every expert's first and last rows, its m-tile boundaries
     and odd last m-tile): over every token of these shapes (1.5-1.8 M outputs, the largest at
     5.5 x RMS) rounding the exact result to bf16 alone costs up to 1.8% of the 2% bound."""
