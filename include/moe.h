@@ -242,10 +242,10 @@ MOE_API moe_status moe_forward_profiled(const void* x, const void* Wg, const voi
  * device, runs moe_forward with the device-resident weights (device), copies
  * the result back into out_host [T][d] (host, bf16) and synchronises
  * `stream`.  Pinned host buffers give full copy bandwidth; pageable ones work.
- * From 4096 tokens on the batch runs in chunks of at least 2048 tokens (a
- * 2048-token first and last chunk around middle ones of up to 6144) on two
- * library-owned copy streams, so that copies overlap the layer; the result is
- * bit for bit that of one call on the whole batch.
+ * From 4096 tokens on the batch runs in chunks on two library-owned copy
+ * streams, so that copies overlap the layer: two halves below 8192 tokens,
+ * else a 1024-token first and last chunk around middle ones of up to 7168.
+ * The result is bit for bit that of one call on the whole batch.
  */
 MOE_API moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3,
                             const void* W2, void* out_host, int T, int d, int ffn, int E, int k,

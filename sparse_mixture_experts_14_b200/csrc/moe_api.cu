@@ -48,9 +48,12 @@ namespace {
 constexpr int kMaxDevices = 64;
 // Chunks of the host entry point's pipelined path: a short first chunk (its copy in is the only
 // one the layer waits for), a short last one (its copy out is the only one that follows the
-// layer) and middle chunks of up to kHostMid tokens.
-constexpr int kHostEdge = 2048;
-constexpr int kHostMid = 6144;
+// layer) and middle chunks of up to kHostMid tokens.  Every chunk streams all touched expert
+// weights once (about 0.8 ms at the 8x22B shape), so the middle chunks stay few and large;
+// batches below kHostSplit3 run as two halves.
+constexpr int kHostEdge = 1024;
+constexpr int kHostMid = 7168;
+constexpr int kHostSplit3 = 8192;
 constexpr int kMaxHostChunks = 64;     // at most this many chunks (larger batches take larger middle chunks)
 
 std::mutex g_mu;
@@ -729,7 +732,7 @@ moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, 
     const size_t row = (size_t)d * 2;
     const size_t act = (size_t)T * row;
     const size_t act_al = align_up(act, 256);
-    // Batches of 2 kHostEdge tokens or more run in chunks, so that each chunk's copies overlap
+    // Batches of 4096 tokens or more run in chunks, so that each chunk's copies overlap
     // another chunk's layer.  Tokens are independent and every kernel of the chunked path gives a
     // token the bits it gets in one call (the tensor-core router adds its K chunks in the same
     // order for any batch; a GEMM row's arithmetic does not depend on its place in a tile), so
@@ -738,9 +741,9 @@ moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, 
     int nch = 1, tc = T;
     cstart[0] = 0;
     // Every chunk holds at least kHostEdge tokens, so every chunk takes the prefill kernels.
-    if (T >= 2 * kHostEdge) {
+    if (T >= 4096) {
         const int mid = T - 2 * kHostEdge;
-        if (mid < kHostEdge) {
+        if (T < kHostSplit3) {
             nch = 2;                       // two halves
             cstart[1] = T / 2;
             tc = T - T / 2;

@@ -412,8 +412,8 @@ def test_route_is_batch_invariant(moe, d, E, k):
 @pytest.mark.parametrize("T", [4096, 6143, 8192, 10001, 16384])
 def test_chunked_host_entry_matches_device(moe, T):
     """Batches of 4096 tokens and more go through the host entry point in pipelined chunks (two
-    halves, or a 2048-token first and last chunk around middle ones of up to 6144); the result
-    equals the one-call device path bit for bit, from pinned and from pageable buffers."""
+    halves below 8192 tokens, else a 1024-token first and last chunk around middle ones of up to
+    7168); the result equals the one-call device path bit for bit, from pinned and pageable buffers."""
     inp = moe_inputs.make_inputs(T, 256, 512, 8, 2, "bf16", seed=T)
     dev = upload(inp)
     a = moe.moe_forward(*dev, 2).cpu()
