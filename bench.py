@@ -84,10 +84,15 @@ def parse_args():
                     help="time a training step: forward (grouped-GEMM path) + backward with all gradients")
     ap.add_argument("--bf16-wgrad", action="store_true",
                     help="with --train: weight gradients rounded to bf16 in the GEMM epilogue (fp32 otherwise)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: each of the N ranks holds E/N experts and its own batch; route, "
+                         "dispatch, NCCL all-to-all of the rows, this rank's experts, all-to-all back, combine")
     ap.add_argument("--stage-every", type=int, default=8,
                     help="record per-stage events on every n-th timed step (events between launches "
                          "break the overlap of dependent launches, so most steps run without them)")
     args = ap.parse_args()
+    if args.ep and (args.train or args.block or args.impl == "reference"):
+        ap.error("--ep times the plain layer's forward on our kernels")
     if args.steps is None:
         args.steps = 8 if args.train else DEFAULT_STEPS[args.config]
     return args
@@ -717,6 +722,77 @@ def run_train(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+EP_METRIC = ("MoE-layer tokens/sec, expert parallel over the job's GPUs (experts split across ranks, "
+             "all-to-all dispatch and combine)")
+
+
+def run_ep(args, rank, world, local):
+    """One expert-parallel forward per step (sparse_mixture_experts_14_b200.ep.moe_forward_ep): the
+    route, dispatch, expert and combine kernels of the library around torch.distributed's NCCL
+    all-to-alls.  Every rank holds the experts expert_range(E, world, rank) and its own batch of
+    the workload's T tokens; the first step's output is checked against the single-GPU layer on
+    the same tokens, bit for bit.  The plan needs the counts on the host, so each step
+    synchronises twice: the timing is device time between events around whole steps."""
+    import sparse_mixture_experts_14_b200 as moe
+    from sparse_mixture_experts_14_b200.ep import expert_range, moe_forward_ep
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    c = moe_inputs.WORKLOADS[args.config]
+    inp = make_workload(args.config, False, args.shape)
+    if inp.dtype != "bf16":
+        raise SystemExit("--ep runs the bf16 workloads")
+    x, Wg, W1, W3, W2 = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
+    T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
+    lo, hi = expert_range(E, world, rank)
+    W1l, W3l, W2l = W1[lo:hi].contiguous(), W3[lo:hi].contiguous(), W2[lo:hi].contiguous()
+    # the single-GPU check needs the full weights; the timed steps touch only this rank's experts
+    ref = moe.moe_forward(x, Wg, W1, W3, W2, k)
+    got = moe_forward_ep(x, Wg, W1l, W3l, W2l, k)
+    torch.cuda.synchronize()
+    if not torch.equal(got, ref):
+        raise RuntimeError("expert-parallel output differs from the single-GPU layer")
+    del ref, got, W1, W3, W2
+    torch.cuda.empty_cache()
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        moe_forward_ep(x, Wg, W1l, W3l, W2l, k)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    stream = torch.cuda.current_stream(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with nvtx_range("bench.timed"):
+        start.record(stream)
+        for _ in range(K):
+            moe_forward_ep(x, Wg, W1l, W3l, W2l, k)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if moe.moe_get_device_status() != moe.MOE_OK:
+        raise RuntimeError("device fault during the timed region")
+    total_ms = reduce_max(start.elapsed_time(end), world, device)
+    value = weak_scaling_value(T, K, world, total_ms)
+    if rank != 0:
+        return
+    line = {
+        "metric": EP_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": inp.dtype, "data": "synthetic",
+        "config": {"workload": workload_name(args.config, args.shape) + "+ep", "T": T, "d": d, "ffn": F, "E": E,
+                   "k": k, "seed": c["seed"], "experts_per_rank": hi - lo,
+                   "parallelism": f"expert parallel x{world}" if world > 1 else "expert parallel x1 (one-rank group)",
+                   "check": "first step equal to the single-GPU layer bit for bit"},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -725,14 +801,24 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
-    if world > 1:
+    dist = world > 1 or args.ep
+    if dist:
         torch.cuda.set_device(local)
+        if world == 1:
+            # a one-rank NCCL group for the expert-parallel data plane on one GPU
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(29500 + os.getpid() % 1000))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
                                              device_id=torch.device("cuda", local))
     try:
-        (run_train if args.train else run_ours)(args, rank, world, local)
+        if args.ep:
+            run_ep(args, rank, world, local)
+        else:
+            (run_train if args.train else run_ours)(args, rank, world, local)
     finally:
-        if world > 1:
+        if dist:
             torch.distributed.destroy_process_group()
 
 
