@@ -87,6 +87,8 @@ def parse_args():
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: each of the N ranks holds E/N experts and its own batch; route, "
                          "dispatch, NCCL all-to-all of the rows, this rank's experts, all-to-all back, combine")
+    ap.add_argument("--seed", type=int, default=None,
+                    help="the workload's recipe with another seed (inputs, weights and routing change with it)")
     ap.add_argument("--stage-every", type=int, default=8,
                     help="record per-stage events on every n-th timed step (events between launches "
                          "break the overlap of dependent launches, so most steps run without them)")
@@ -277,19 +279,20 @@ def oracle_train_run(inp, dout, target_s, block=False):
     return len(toks) / dt, sample, dt
 
 
-def make_workload(cfg, block, shape=None):
-    if shape:
+def make_workload(cfg, block, shape=None, seed=None):
+    if shape or seed is not None:
         c = moe_inputs.WORKLOADS[cfg]
-        T, d, F = (int(v) for v in shape.split(","))
-        inp = moe_inputs.make_inputs(T, d, F, c["E"], c["k"], c["dtype"], c["seed"], c["skew"])
+        T, d, F = (int(v) for v in shape.split(",")) if shape else (c["T"], c["d"], c["F"])
+        inp = moe_inputs.make_inputs(T, d, F, c["E"], c["k"], c["dtype"], c["seed"] if seed is None else seed,
+                                     c["skew"])
     else:
         inp = moe_inputs.make_config(cfg)
     return moe_inputs.make_block(inp) if block else inp
 
 
-def workload_name(cfg, shape=None):
+def workload_name(cfg, shape=None, seed=None):
     c = moe_inputs.WORKLOADS[cfg]
-    return c["name"] + (f"@shape={shape}" if shape else "")
+    return c["name"] + (f"@shape={shape}" if shape else "") + (f"@seed={seed}" if seed is not None else "")
 
 
 def cpu_oracle_run(inp, target_s, threads, block=False):
@@ -320,7 +323,7 @@ def run_reference(args, rank):
     if rank != 0:
         return
     c = moe_inputs.WORKLOADS[args.config]
-    inp = make_workload(args.config, args.block, args.shape)
+    inp = make_workload(args.config, args.block, args.shape, args.seed)
     if args.train:
         dout = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
         per_step = max(0.05, min(30.0, args.ref_seconds / max(args.steps + args.warmup, 1)))
@@ -337,10 +340,10 @@ def run_reference(args, rank):
             "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_t / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_name(args.config, args.shape) + ("+block" if args.block else "") + "+train",
+            "config": {"workload": workload_name(args.config, args.shape, args.seed) + ("+block" if args.block else "") + "+train",
                        "T": inp.T, "d": inp.d,
                        "ffn": inp.F, "E": inp.E,
-                       "k": inp.k, "seed": c["seed"]},
+                       "k": inp.k, "seed": inp.seed},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
@@ -367,9 +370,9 @@ def run_reference(args, rank):
         "impl": "reference", "metric": BLOCK_METRIC if args.block else METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt / max(args.steps, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_name(args.config, args.shape) + ("+block" if args.block else ""),
+        "config": {"workload": workload_name(args.config, args.shape, args.seed) + ("+block" if args.block else ""),
                    "T": inp.T, "d": inp.d,
-                   "ffn": inp.F, "E": inp.E, "k": inp.k, "seed": c["seed"],
+                   "ffn": inp.F, "E": inp.E, "k": inp.k, "seed": inp.seed,
                    "sample_tokens_per_step": int(len(toks))},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -405,7 +408,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.set_device(device)
     c = moe_inputs.WORKLOADS[args.config]
     block = args.block
-    inp = make_workload(args.config, block, args.shape)
+    inp = make_workload(args.config, block, args.shape, args.seed)
     dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
     tdt = dev[0].dtype
     T, d, F, E, k = inp.T, inp.d, inp.F, inp.E, inp.k
@@ -539,7 +542,7 @@ def run_ours(args, rank, world, local):
         # the forward GEMMs run on 256 x 512 tiles when their reduction is 5120 or longer
         kname = {"expert1": "tc_gemm_kernel<kFwd1W>" if d >= 5120 else "tc_gemm_kernel<kFwd1>",
                  "expert2": "tc_gemm_kernel<kFwd2W>" if F >= 5120 else "tc_gemm_kernel<kFwd2>"}[dom]
-    roof["traffic"] = recorded_traffic(kname, workload_name(args.config, args.shape))
+    roof["traffic"] = recorded_traffic(kname, workload_name(args.config, args.shape, args.seed))
     roof["kernel"] = kname
     roof["per_launch"] = {"flops": fl, "bytes": by, "ms": stages[dom]}
     roof["peak_source"] = f"{peak_src} ({'sustained' if long_run and roof['unit'] == 'TFLOP/s' else 'burst'})"
@@ -555,9 +558,9 @@ def run_ours(args, rank, world, local):
         "steps": K, "warmup": W,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp.dtype, "data": "synthetic",
-        "config": {"workload": workload_name(args.config, args.shape) + ("+block" if block else ""), "T": T, "d": d,
+        "config": {"workload": workload_name(args.config, args.shape, args.seed) + ("+block" if block else ""), "T": T, "d": d,
                    "ffn": F, "E": E, "k": k,
-                   "seed": c["seed"],
+                   "seed": inp.seed,
                    "routing": "zipf1.2-skewed" if c["skew"] else "near-uniform",
                    "l2": "L2 flushed between steps" if flush else "touched weights larger than L2 (no flush)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
@@ -583,7 +586,7 @@ def run_train(args, rank, world, local):
     torch.cuda.set_device(device)
     c = moe_inputs.WORKLOADS[args.config]
     block = args.block
-    inp = make_workload(args.config, block, args.shape)
+    inp = make_workload(args.config, block, args.shape, args.seed)
     dev = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
     dout_np = moe_inputs.make_dout(inp.T, inp.d, inp.dtype, seed=inp.seed)
     dout = to_dev(dout_np, inp.dtype, device)
@@ -689,7 +692,7 @@ def run_train(args, rank, world, local):
     dom = max(bwd_flops, key=lambda n: bst[n])
     sec = bst[dom] / 1000.0
     roof = {"bound": "tensor", "achieved": bwd_flops[dom] / sec / 1e12, "peak": tflops_peak, "unit": "TFLOP/s",
-            "traffic": recorded_traffic(f"tc_gemm_kernel ({dom})", workload_name(args.config, args.shape)),
+            "traffic": recorded_traffic(f"tc_gemm_kernel ({dom})", workload_name(args.config, args.shape, args.seed)),
             "kernel": f"tc_gemm_kernel ({dom})",
             "per_launch": {"flops": bwd_flops[dom], "ms": bst[dom]},
             "peak_source": f"{peak_src} ({'sustained' if long_run else 'burst'})"}
@@ -705,9 +708,9 @@ def run_train(args, rank, world, local):
         "metric": BLOCK_TRAIN_METRIC if block else TRAIN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp.dtype, "data": "synthetic",
-        "config": {"workload": workload_name(args.config, args.shape) + ("+block" if block else "") + "+train",
+        "config": {"workload": workload_name(args.config, args.shape, args.seed) + ("+block" if block else "") + "+train",
                    "T": T, "d": d, "ffn": F, "E": E,
-                   "k": k, "seed": c["seed"], "weight_grads": "bf16" if wd == torch.bfloat16 else "fp32",
+                   "k": k, "seed": inp.seed, "weight_grads": "bf16" if wd == torch.bfloat16 else "fp32",
                    "l2": "touched weights larger than L2 (no flush)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof,
@@ -738,7 +741,7 @@ def run_ep(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     c = moe_inputs.WORKLOADS[args.config]
-    inp = make_workload(args.config, False, args.shape)
+    inp = make_workload(args.config, False, args.shape, args.seed)
     if inp.dtype != "bf16":
         raise SystemExit("--ep runs the bf16 workloads")
     x, Wg, W1, W3, W2 = [to_dev(a, inp.dtype, device) for a in inp.arrays()]
@@ -784,8 +787,8 @@ def run_ep(args, rank, world, local):
         "metric": EP_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp.dtype, "data": "synthetic",
-        "config": {"workload": workload_name(args.config, args.shape) + "+ep", "T": T, "d": d, "ffn": F, "E": E,
-                   "k": k, "seed": c["seed"], "experts_per_rank": hi - lo,
+        "config": {"workload": workload_name(args.config, args.shape, args.seed) + "+ep", "T": T, "d": d, "ffn": F, "E": E,
+                   "k": k, "seed": inp.seed, "experts_per_rank": hi - lo,
                    "parallelism": f"expert parallel x{world}" if world > 1 else "expert parallel x1 (one-rank group)",
                    "check": "first step equal to the single-GPU layer bit for bit"},
         "clocks": clocks,
