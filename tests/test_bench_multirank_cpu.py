@@ -112,3 +112,25 @@ def test_reference_arm_json_contract():
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_seed_option_changes_the_inputs_and_tags_the_workload():
+    """--seed runs a workload's recipe with another seed; the workload name carries it, so a
+    traffic figure recorded for the standard seed is never looked up for it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = bench.make_workload(1, False)
+    b = bench.make_workload(1, False, seed=7)
+    assert b.seed == 7 and a.seed != 7
+    assert (a.T, a.d, a.F, a.E, a.k) == (b.T, b.d, b.F, b.E, b.k)
+    assert not (a.x == b.x).all()
+    assert bench.workload_name(1) != bench.workload_name(1, seed=7)
+    assert bench.workload_name(3, "4096,4096,4096", 5).endswith("@shape=4096,4096,4096@seed=5")
+
+
+@pytest.mark.parametrize("extra", [["--train"], ["--block"], ["--impl", "reference"]])
+def test_ep_mode_refuses_other_modes(extra):
+    """--ep times the plain layer's forward on the library's kernels only."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--ep"] + extra
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert r.returncode != 0 and "--ep" in r.stderr
