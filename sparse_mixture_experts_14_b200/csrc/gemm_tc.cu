@@ -50,6 +50,8 @@
 // described to tcgen05.mma as MN-major, so no operand is ever transposed in HBM.
 #include <cuda.h>
 
+#include <cstdlib>
+
 #include "moe_common.cuh"
 #include "ptx_sm100.cuh"
 #include "tma_map.cuh"
@@ -795,8 +797,17 @@ GemmParams params(Meta* meta, int E, int N, int K, int wave_slot, size_t slots, 
 
 // Wide (256 x 512) tiles when the reduction is long enough to hide their unoverlapped epilogue:
 // measured A/B (one box, libraries alternating), GEMM2 (K = ffn = 14336 / 16384) ran 5-7% faster
-// at every workload, GEMM1 4% faster at K = d = 6144 and 2% slower at K = 4096.
-constexpr int kWideMinK = 5120;
+// at every workload, GEMM1 4% faster at K = d = 6144 and 2% slower at K = 4096.  The environment
+// variable MOE_WIDE_MIN_K (read once per process) moves the threshold; a value past every K keeps
+// all tiles 256 x 256, which gives the same output bits (each output element sees the same MMAs
+// in the same K order).
+int wide_min_k() {
+    static const int v = [] {
+        const char* s = std::getenv("MOE_WIDE_MIN_K");
+        return s && *s ? std::atoi(s) : 5120;
+    }();
+    return v;
+}
 
 cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s) {
     CUtensorMap mA, mB1, mB3;
@@ -805,7 +816,7 @@ cudaError_t launch_tc_gemm1(const TcGemmArgs& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     const GemmParams gp = params(const_cast<Meta*>(a.meta), a.E, a.F, a.d, kWaveFwd1, a.slots, a.H, a.status,
                                  a.wait_ns);
-    if (a.d >= kWideMinK)
+    if (a.d >= wide_min_k())
         return launch_pair<kFwd1W>(row_pair_tiles(a.slots, a.E, (a.F + 2 * BNH - 1) / (2 * BNH)), a.num_sms, mA, mB1,
                                    mB3, gp, s);
     return launch_pair<kFwd1>(row_pair_tiles(a.slots, a.E, (a.F + BNH - 1) / BNH), a.num_sms, mA, mB1, mB3, gp, s);
@@ -829,7 +840,7 @@ cudaError_t launch_tc_gemm2(const TcGemmArgs& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     const GemmParams gp = params(const_cast<Meta*>(a.meta), a.E, a.d, a.F, kWaveFwd2, a.slots, a.Y, a.status,
                                  a.wait_ns);
-    if (a.F >= kWideMinK)
+    if (a.F >= wide_min_k())
         return launch_pair<kFwd2W>(row_pair_tiles(a.slots, a.E, (a.d + 2 * BN - 1) / (2 * BN)), a.num_sms, mA, mB, mB,
                                    gp, s);
     return launch_pair<kFwd2>(row_pair_tiles(a.slots, a.E, (a.d + BN - 1) / BN), a.num_sms, mA, mB, mB, gp, s);
@@ -855,7 +866,7 @@ cudaError_t launch_tc_dgrad_x(const TcBwdArgs& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     GemmParams gp = params(a.meta, a.E, a.d, 2 * a.F, kWaveDgradX, a.slots, a.dxp, a.status, a.wait_ns);
     gp.kb_split = a.F / BK;
-    if (2 * a.F >= kWideMinK)
+    if (2 * a.F >= wide_min_k())
         return launch_pair<kDgradXW>(row_pair_tiles(a.slots, a.E, (a.d + 2 * BN - 1) / (2 * BN)), a.num_sms, mA, mB1,
                                      mB3, gp, s);
     return launch_pair<kDgradX>(row_pair_tiles(a.slots, a.E, (a.d + BN - 1) / BN), a.num_sms, mA, mB1, mB3, gp,
