@@ -108,3 +108,23 @@ def test_config_table(cfg):
     c = moe_inputs.WORKLOADS[cfg]
     assert c["k"] == 2 and c["E"] == 8
     assert c["dtype"] == ("f32" if cfg == 1 else "bf16")
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_mixtral_shapes_match_printed_parameter_counts(cfg):
+    """The Mixtral 8x7B workloads' sizes against the figures the Mistral/Mixtral page prints.
+
+    "各エキスパートの構造": W1, W3 are d_ff x d_model and W2 d_model x d_ff with d_ff = 14336;
+    the GQA section: d_model = 4096 with L = 32 layers; "パラメータ数と推論コスト": about 46.7B
+    parameters in all and 12.9B active per token, total = attn + 8 P_FFN and active = attn + 2 P_FFN,
+    whence P_FFN of about 5.63B.  A SwiGLU expert holds three d x F matrices in each of the 32 layers.
+    """
+    c = moe_inputs.WORKLOADS[cfg]
+    d, F, E, k = c["d"], c["F"], c["E"], c["k"]
+    assert (d, F, E, k) == (4096, 14336, 8, 2)
+    p_ffn = 32 * 3 * d * F
+    from_totals = (46.7e9 - 12.9e9) / (E - k)     # the two printed totals solved for one expert
+    assert abs(p_ffn - from_totals) / from_totals < 0.005
+    assert abs(p_ffn - 5.63e9) / 5.63e9 < 0.005
+    # the pin separates: two matrices per expert instead of three would be a third short
+    assert abs(32 * 2 * d * F - from_totals) / from_totals > 0.3
