@@ -252,6 +252,21 @@ MOE_API moe_status moe_forward_host(const void* x_host, const void* Wg, const vo
                             cudaStream_t stream);
 
 /*
+ * The chunk plan moe_forward_host uses for a batch of T tokens (host only, no
+ * device needed): writes the first token of each chunk to starts[0..n-1] and T
+ * to starts[n] (starts: host, max_chunks + 1 ints, caller-owned) and returns
+ * the chunk count n: 1 below 4096 tokens, 2 (halves) below 8192, else a
+ * 1024-token first and last chunk around near-equal middle ones of up to 7168
+ * tokens (at most 64 chunks in all; past that the middle ones grow).  Returns
+ * 0 with nothing written if T < 0, starts is NULL or n would exceed
+ * max_chunks.  Chunks are runs of consecutive tokens; tokens are independent
+ * (each token's routing and expert rows depend on that token alone, per the
+ * Top-2 gating and expert equations of the Mistral/Mixtral page), which is why
+ * the chunked call returns the bits of one call.
+ */
+MOE_API int moe_host_chunk_plan(int T, int* starts, int max_chunks);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word: MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE (the first fault recorded
  * since the last read), or MOE_ERR_CUDA if the synchronisation itself failed.

@@ -58,6 +58,7 @@ SIGNATURES = {
     "moe_forward_profiled": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _vp, _sz, _vp,
                                    _vp, _vp]),
     "moe_forward_host": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _vp]),
+    "moe_host_chunk_plan": (_ci, [_ci, _vp, _ci]),
     "moe_get_device_status": (_ci, [_vp]),
     "moe_selftest_wait_timeout": (_ci, [_ll, _vp]),
     "moe_status_string": (ctypes.c_char_p, [_ci]),
@@ -593,6 +594,15 @@ def moe_pool_stats(device=None):
 
 def moe_decode_max_tokens() -> int:
     return int(_lib.moe_decode_max_tokens())
+
+
+def moe_host_chunk_plan(T: int, max_chunks: int = 64) -> list:
+    """Token boundaries [0, ..., T] of the chunks moe_forward_host runs a T-token batch in."""
+    starts = (ctypes.c_int * (max_chunks + 1))()
+    n = int(_lib.moe_host_chunk_plan(int(T), starts, int(max_chunks)))
+    if n < 1:
+        raise ValueError(f"no chunk plan for T={T} within {max_chunks} chunks")
+    return list(starts[: n + 1])
 
 
 def loaded_library_path() -> str:

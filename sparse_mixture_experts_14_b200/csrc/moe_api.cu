@@ -51,6 +51,7 @@ constexpr int kMaxDevices = 64;
 // layer) and middle chunks of up to kHostMid tokens.  Every chunk streams all touched expert
 // weights once (about 0.8 ms at the 8x22B shape), so the middle chunks stay few and large;
 // batches below kHostSplit3 run as two halves.
+constexpr int kHostChunkMin = 4096;   // smaller batches run in one piece
 constexpr int kHostEdge = 1024;
 constexpr int kHostMid = 7168;
 constexpr int kHostSplit3 = 8192;
@@ -722,6 +723,30 @@ moe_status moe_forward_profiled(const void* x, const void* Wg, const void* W1, c
                      stream, stage_events, launches);
 }
 
+// Every chunk of a split batch holds at least kHostEdge tokens, so every chunk takes the
+// prefill kernels (the decode path would give its tokens other bits than one call does).
+int moe_host_chunk_plan(int T, int* starts, int max_chunks) {
+    if (T < 0 || !starts || max_chunks < 1) return 0;
+    int n = 1;
+    if (T >= kHostSplit3) {
+        // a kHostEdge-token first and last chunk around near-equal middle ones of up to
+        // kHostMid tokens (more middle tokens per chunk once the chunk count is at its cap)
+        const int mid = T - 2 * kHostEdge;
+        const int nmid = min((mid + kHostMid - 1) / kHostMid, kMaxHostChunks - 2);
+        n = nmid + 2;
+        if (n > max_chunks) return 0;
+        starts[1] = kHostEdge;
+        for (int c = 0; c < nmid; ++c) starts[2 + c] = starts[1 + c] + mid / nmid + (c < mid % nmid ? 1 : 0);
+    } else if (T >= kHostChunkMin) {
+        n = 2;   // two halves
+        if (n > max_chunks) return 0;
+        starts[1] = T / 2;
+    }
+    starts[0] = 0;
+    starts[n] = T;
+    return n;
+}
+
 moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3, const void* W2,
                             void* out_host, int T, int d, int ffn, int E, int k, cudaStream_t stream) {
     moe_status st = check_layer(x_host, Wg, W1, W3, W2, out_host, T, d, ffn, E, k, MOE_DTYPE_BF16);
@@ -738,30 +763,10 @@ moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, 
     // order for any batch; a GEMM row's arithmetic does not depend on its place in a tile), so
     // the result equals the unchunked call bit for bit.
     int cstart[kMaxHostChunks + 1];
-    int nch = 1, tc = T;
-    cstart[0] = 0;
-    // Every chunk holds at least kHostEdge tokens, so every chunk takes the prefill kernels.
-    if (T >= 4096) {
-        const int mid = T - 2 * kHostEdge;
-        if (T < kHostSplit3) {
-            nch = 2;                       // two halves
-            cstart[1] = T / 2;
-            tc = T - T / 2;
-        } else {
-            const int nmid = min((mid + kHostMid - 1) / kHostMid, kMaxHostChunks - 2);
-            nch = nmid + 2;
-            cstart[1] = kHostEdge;
-            tc = kHostEdge;
-            for (int c = 0; c < nmid; ++c) {
-                const int n = mid / nmid + (c < mid % nmid ? 1 : 0);
-                cstart[2 + c] = cstart[1 + c] + n;
-                tc = max(tc, n);
-            }
-        }
-        cstart[nch] = T;
-    } else {
-        cstart[1] = T;
-    }
+    const int nch = moe_host_chunk_plan(T, cstart, kMaxHostChunks);
+    if (nch < 1) return MOE_ERR_INVALID_ARG;
+    int tc = 0;   // the largest chunk sizes the workspace
+    for (int c = 0; c < nch; ++c) tc = max(tc, cstart[c + 1] - cstart[c]);
     const Plan p = make_plan(tc, d, ffn, E, k, MOE_DTYPE_BF16);
     void* buf = nullptr;
     if (cudaMallocFromPoolAsync(&buf, 2 * act_al + p.total, dev.pool, stream) != cudaSuccess)

@@ -252,3 +252,39 @@ def test_pool_stats_argument_checks(lib):
     assert fn(64, ctypes.byref(r), ctypes.byref(u)) == 1
     assert fn(0, ctypes.byref(r), ctypes.byref(u)) == 0     # no pool created in this process: zeros
     assert (r.value, u.value) == (0, 0)
+
+
+def test_host_chunk_plan(lib):
+    """The host entry point's chunk plan: runs of consecutive tokens covering [0, T), each split
+    batch's chunks large enough for the prefill kernels, short first and last chunks around
+    near-equal middle ones."""
+    import numpy as np
+    import sparse_mixture_experts_14_b200 as m
+    plan = m.moe_host_chunk_plan
+    assert plan(0) == [0, 0]
+    assert plan(4095) == [0, 4095]
+    assert plan(4096) == [0, 2048, 4096]
+    assert plan(8191) == [0, 4095, 8191]
+    assert plan(8192) == [0, 1024, 7168, 8192]
+    assert plan(16384) == [0, 1024, 8192, 15360, 16384]
+    decode_max = m.moe_decode_max_tokens()
+    for T in [4096, 4097, 6143, 8191, 8192, 8193, 10001, 16385, 30000, 100_000, 1 << 20, 2_000_000]:
+        s = plan(T)
+        sizes = np.diff(s)
+        assert s[0] == 0 and s[-1] == T and len(s) - 1 <= 64
+        assert sizes.min() >= 1024 and sizes.min() > decode_max
+        if T < 8192:
+            assert len(sizes) == 2 and abs(int(sizes[0]) - int(sizes[1])) <= 1
+        else:
+            assert sizes[0] == 1024 and sizes[-1] == 1024
+            mids = sizes[1:-1]
+            assert mids.max() - mids.min() <= 1
+            if len(sizes) < 64:
+                assert mids.max() <= 7168
+    buf = (ctypes.c_int * 65)()
+    lib.moe_host_chunk_plan.restype = ctypes.c_int
+    assert lib.moe_host_chunk_plan(-1, buf, 64) == 0
+    assert lib.moe_host_chunk_plan(16384, None, 64) == 0
+    assert lib.moe_host_chunk_plan(16384, buf, 3) == 0          # four chunks do not fit in three
+    assert lib.moe_host_chunk_plan(16384, buf, 4) == 4
+    assert list(buf[:5]) == [0, 1024, 8192, 15360, 16384]
