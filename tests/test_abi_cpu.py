@@ -288,3 +288,38 @@ def test_host_chunk_plan(lib):
     assert lib.moe_host_chunk_plan(16384, buf, 3) == 0          # four chunks do not fit in three
     assert lib.moe_host_chunk_plan(16384, buf, 4) == 4
     assert list(buf[:5]) == [0, 1024, 8192, 15360, 16384]
+
+
+def test_header_serves_a_plain_c_program(lib, tmp_path):
+    """include/moe.h compiles as C99 with warnings as errors, and a C program links libmoe.so and
+    calls its host-only entry points (no device is touched)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    cuda_inc = next((p for p in ("/usr/local/cuda/include", os.path.join(os.environ.get("CUDA_HOME", ""), "include"))
+                     if os.path.exists(os.path.join(p, "cuda_runtime_api.h"))), None)
+    if cuda_inc is None:
+        pytest.skip("no CUDA headers")
+    src = tmp_path / "client.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+int main(void) {
+    int s[65];
+    if (moe_host_chunk_plan(16384, s, 64) != 4 || s[1] != 1024 || s[4] != 16384) return 1;
+    if (moe_slots_capacity(16, 8, 2) % 128 != 0) return 2;
+    if (strcmp(moe_status_string(MOE_ERR_TIMEOUT), "device wait timed out") != 0) return 3;
+    if (moe_forward(NULL, NULL, NULL, NULL, NULL, NULL, 8, 128, 256, 8, 9, 0) != MOE_ERR_INVALID_ARG) return 4;
+    printf("ok\n");
+    return 0;
+}
+''')
+    libdir = os.path.dirname(lib._name)
+    exe = tmp_path / "client"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+                    str(src), "-L", libdir, "-lmoe", "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
