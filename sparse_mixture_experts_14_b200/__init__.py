@@ -149,7 +149,16 @@ def _dtype_code(t):
     raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
 
 
+def _router_shapes(x, Wg):
+    """Tokens x [T][d] and router weights Wg [E][d]: the kernels trust these sizes."""
+    if x.dim() != 2 or Wg.dim() != 2 or Wg.shape[1] != x.shape[1]:
+        raise ValueError(f"inconsistent shapes x{tuple(x.shape)} Wg{tuple(Wg.shape)}")
+    return x.shape[0], x.shape[1], Wg.shape[0]
+
+
 def _layer_shapes(x, Wg, W1, W3, W2):
+    if x.dim() != 2 or W1.dim() != 3:
+        raise ValueError(f"x must be [T][d] and W1 [E][F][d], got x{tuple(x.shape)} W1{tuple(W1.shape)}")
     T, d = x.shape
     E, F, d1 = W1.shape
     if Wg.shape != (E, d) or d1 != d or W3.shape != (E, F, d) or W2.shape != (E, d, F):
@@ -160,11 +169,10 @@ def _layer_shapes(x, Wg, W1, W3, W2):
 
 def moe_route(x, Wg, k, topk_idx=None, topk_w=None, stream=None):
     """Router scores, top-k (lowest index on ties), softmax over the k: (topk_idx int32 [T][k], topk_w f32 [T][k])."""
+    T, d, E = _router_shapes(x, Wg)
     code = _dtype_code(x)
     _dev(x, x.dtype, "x")
     _dev(Wg, x.dtype, "Wg")
-    T, d = x.shape
-    E = Wg.shape[0]
     if topk_idx is None:
         topk_idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
     if topk_w is None:
@@ -279,14 +287,13 @@ def moe_forward_host(x_host, Wg, W1, W3, W2, k, out_host=None, stream=None):
     """End to end from host memory: x_host / out_host are CPU bf16 tensors (pinned for full speed)."""
     if x_host.is_cuda or x_host.dtype != torch.bfloat16 or not x_host.is_contiguous():
         raise TypeError("x_host must be a contiguous CPU bfloat16 tensor")
-    T, d = x_host.shape
+    T, d, F, E = _layer_shapes(x_host, Wg, W1, W3, W2)
     if out_host is not None:
         _room(out_host, T * d, "out_host")
         if out_host.is_cuda or out_host.dtype != torch.bfloat16 or not out_host.is_contiguous():
             raise TypeError("out_host must be a contiguous CPU bfloat16 tensor")
     for t, n in ((Wg, "Wg"), (W1, "W1"), (W3, "W3"), (W2, "W2")):
         _dev(t, torch.bfloat16, n)
-    E, F, _ = W1.shape
     if out_host is None:
         out_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
     _check(_lib.moe_forward_host(_ptr(x_host), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out_host), T, d, F, E,
@@ -356,11 +363,10 @@ def moe_block_forward_ws(h, gamma, eps, Wg, W1, W3, W2, k, workspace, out, alpha
 
 def moe_route_stats(x, Wg, k, alpha=1.0, stream=None):
     """moe_route plus load-balance statistics: (topk_idx, topk_w, stats [2E+1] = f, p, loss)."""
+    T, d, E = _router_shapes(x, Wg)
     code = _dtype_code(x)
     _dev(x, x.dtype, "x")
     _dev(Wg, x.dtype, "Wg")
-    T, d = x.shape
-    E = Wg.shape[0]
     idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
     w = torch.empty((T, k), dtype=torch.float32, device=x.device)
     stats = torch.empty(2 * E + 1, dtype=torch.float32, device=x.device)
@@ -512,6 +518,8 @@ def moe_ep_dispatch(x, topk_idx, E, send=None, send_pos=None, stream=None):
     counts numpy int32 [E]).  Synchronises the stream (the counts come back to the host)."""
     import numpy as np
     T, k = topk_idx.shape
+    if x.dim() != 2 or x.shape[0] != T:
+        raise ValueError(f"x must be [T][d] with T = {T} rows (topk_idx), got {tuple(x.shape)}")
     d = x.shape[1]
     if send is None:
         send = torch.empty((T * k, d), dtype=x.dtype, device=x.device)
@@ -563,6 +571,7 @@ def moe_ep_combine(ysend, topk_w, send_pos, out=None, stream=None):
         out = torch.empty((T, d), dtype=torch.bfloat16, device=ysend.device)
     _room(out, T * d, "out")
     _room(ysend, T * k * d, "ysend")
+    _room(topk_w, T * k, "topk_w")
     _dev(ysend, torch.float32, "ysend")
     _dev(topk_w, torch.float32, "topk_w")
     _dev(send_pos, torch.int32, "send_pos")

@@ -242,6 +242,30 @@ def test_binding_rejects_undersized_layer_outputs():
         m.moe_forward_host(x, Wg, W1, W3, W2, k, out_host=torch.zeros(T * d - 1, dtype=bf))
 
 
+def test_binding_rejects_inconsistent_shapes():
+    """The sizes the kernels trust come from the tensors' shapes: the wrappers refuse shapes that do
+    not fit together (ValueError, CPU tensors, nothing reaches the library)."""
+    import sparse_mixture_experts_14_b200 as m
+    T, d, F, E, k = 8, 64, 128, 4, 2
+    bf = torch.bfloat16
+    x, Wg = torch.zeros((T, d), dtype=bf), torch.zeros((E, d), dtype=bf)
+    W1, W3, W2 = torch.zeros((E, F, d), dtype=bf), torch.zeros((E, F, d), dtype=bf), torch.zeros((E, d, F), dtype=bf)
+    short_Wg = torch.zeros((E, d // 2), dtype=bf)
+    for route in (m.moe_route, m.moe_route_stats):
+        with pytest.raises(ValueError, match="inconsistent"):
+            route(x, short_Wg, k)
+        with pytest.raises(ValueError, match="inconsistent"):
+            route(x.reshape(-1), Wg, k)
+    for bad in ((short_Wg, W1, W3, W2), (Wg, W1[:, :, : d // 2], W3, W2), (Wg, W1, W3[:, : F // 2], W2),
+                (Wg, W1, W3, W2.transpose(1, 2).contiguous())):
+        with pytest.raises(ValueError, match="inconsistent"):
+            m.moe_forward_host(x, *bad, k)
+    with pytest.raises(ValueError, match="rows"):
+        m.moe_ep_dispatch(x[: T - 1], torch.zeros((T, k), dtype=torch.int32), E)
+    with pytest.raises(ValueError, match="topk_w"):
+        m.moe_ep_combine(torch.zeros((T * k, d)), torch.zeros((T, k - 1)), torch.zeros((T, k), dtype=torch.int32))
+
+
 def test_pool_stats_argument_checks(lib):
     fn = lib.moe_pool_stats
     fn.restype = ctypes.c_int
