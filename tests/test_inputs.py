@@ -112,19 +112,19 @@ def test_config_table(cfg):
 
 @pytest.mark.parametrize("cfg", [2, 3, 4])
 def test_mixtral_shapes_match_printed_parameter_counts(cfg):
-    """The Mixtral 8x7B workloads' sizes against the figures the Mistral/Mixtral page prints.
-
-    "各エキスパートの構造": W1, W3 are d_ff x d_model and W2 d_model x d_ff with d_ff = 14336;
-    the GQA section: d_model = 4096 with L = 32 layers; "パラメータ数と推論コスト": about 46.7B
-    parameters in all and 12.9B active per token, total = attn + 8 P_FFN and active = attn + 2 P_FFN,
-    whence P_FFN of about 5.63B.  A SwiGLU expert holds three d x F matrices in each of the 32 layers.
-    """
+    """The Mixtral 8x7B workloads' sizes against the figures the Mistral/Mixtral page prints
+    (tests/golden/mixtral_8x7b_printed_sizes.json, each figure with its section): d_ff, d_model,
+    the layer count, 8 experts with top-2, and the parameter totals, from which one expert's
+    parameters over all layers follow as (total - active) / (experts - top_k).  A SwiGLU expert
+    holds three d x F matrices in each layer."""
+    with open(os.path.join(os.path.dirname(__file__), "golden", "mixtral_8x7b_printed_sizes.json")) as f:
+        g = json.load(f)
     c = moe_inputs.WORKLOADS[cfg]
     d, F, E, k = c["d"], c["F"], c["E"], c["k"]
-    assert (d, F, E, k) == (4096, 14336, 8, 2)
-    p_ffn = 32 * 3 * d * F
-    from_totals = (46.7e9 - 12.9e9) / (E - k)     # the two printed totals solved for one expert
+    assert (d, F, E, k) == (g["d_model"], g["d_ff"], g["experts"], g["top_k"])
+    p_ffn = g["layers"] * 3 * d * F
+    from_totals = (g["total_params"] - g["active_params"]) / (E - k)
     assert abs(p_ffn - from_totals) / from_totals < 0.005
-    assert abs(p_ffn - 5.63e9) / 5.63e9 < 0.005
+    assert abs(p_ffn - g["p_ffn_estimate"]) / g["p_ffn_estimate"] < 0.005
     # the pin separates: two matrices per expert instead of three would be a third short
-    assert abs(32 * 2 * d * F - from_totals) / from_totals > 0.3
+    assert abs(g["layers"] * 2 * d * F - from_totals) / from_totals > 0.3
