@@ -243,8 +243,7 @@ MOE_API moe_status moe_forward_profiled(const void* x, const void* Wg, const voi
  * the result back into out_host [T][d] (host, bf16) and synchronises
  * `stream`.  Pinned host buffers give full copy bandwidth; pageable ones work.
  * From 4096 tokens on the batch runs in chunks on two library-owned copy
- * streams, so that copies overlap the layer: two halves below 8192 tokens,
- * else a 1024-token first and last chunk around middle ones of up to 7168.
+ * streams, so that copies overlap the layer (moe_host_chunk_plan gives them).
  * The result is bit for bit that of one call on the whole batch.
  */
 MOE_API moe_status moe_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3,
@@ -255,9 +254,11 @@ MOE_API moe_status moe_forward_host(const void* x_host, const void* Wg, const vo
  * The chunk plan moe_forward_host uses for a batch of T tokens (host only, no
  * device needed): writes the first token of each chunk to starts[0..n-1] and T
  * to starts[n] (starts: host, max_chunks + 1 ints, caller-owned) and returns
- * the chunk count n: 1 below 4096 tokens, 2 (halves) below 8192, else a
+ * the chunk count n: 1 below 4096 tokens, 2 (halves) below 8192, then a
  * 1024-token first and last chunk around near-equal middle ones of up to 7168
- * tokens (at most 64 chunks in all; past that the middle ones grow).  Returns
+ * tokens below 12288, else 2560-token first and last chunks around middle
+ * ones of up to 11264 (at most 64 chunks in all; past that the middle ones
+ * grow).  Returns
  * 0 with nothing written if T < 0, starts is NULL or n would exceed
  * max_chunks.  Chunks are runs of consecutive tokens; tokens are independent
  * (each token's routing and expert rows depend on that token alone, per the

@@ -48,13 +48,19 @@ namespace {
 constexpr int kMaxDevices = 64;
 // Chunks of the host entry point's pipelined path: a short first chunk (its copy in is the only
 // one the layer waits for), a short last one (its copy out is the only one that follows the
-// layer) and middle chunks of up to kHostMid tokens.  Every chunk streams all touched expert
-// weights once (about 0.8 ms at the 8x22B shape), so the middle chunks stay few and large;
-// batches below kHostSplit3 run as two halves.
+// layer) and middle chunks in between.  Every chunk streams all touched expert weights once and
+// pads each expert's rows to whole tiles, so the middle chunks stay few and large; the first
+// chunk's layer has to last about as long as the copy in of the first middle chunk, which is why
+// large batches take a longer first chunk (measured at the 8x22B shape, 16384 tokens: 1024-token
+// edges around two 7168-token middles 17.6 ms per call, 2560-token edges around one 11264-token
+// middle 16.9 ms).  Batches below kHostSplit3 run as two halves.
 constexpr int kHostChunkMin = 4096;   // smaller batches run in one piece
-constexpr int kHostEdge = 1024;
-constexpr int kHostMid = 7168;
 constexpr int kHostSplit3 = 8192;
+constexpr int kHostEdge = 1024;       // kHostSplit3 <= T < kHostLarge
+constexpr int kHostMid = 7168;
+constexpr int kHostLarge = 12288;
+constexpr int kHostEdgeL = 2560;      // T >= kHostLarge
+constexpr int kHostMidL = 11264;
 constexpr int kMaxHostChunks = 64;     // at most this many chunks (larger batches take larger middle chunks)
 
 std::mutex g_mu;
@@ -729,13 +735,15 @@ int moe_host_chunk_plan(int T, int* starts, int max_chunks) {
     if (T < 0 || !starts || max_chunks < 1) return 0;
     int n = 1;
     if (T >= kHostSplit3) {
-        // a kHostEdge-token first and last chunk around near-equal middle ones of up to
-        // kHostMid tokens (more middle tokens per chunk once the chunk count is at its cap)
-        const int mid = T - 2 * kHostEdge;
-        const int nmid = min((mid + kHostMid - 1) / kHostMid, kMaxHostChunks - 2);
+        // an edge-token first and last chunk around near-equal middle ones of up to mid_max
+        // tokens (more middle tokens per chunk once the chunk count is at its cap)
+        const int edge = T >= kHostLarge ? kHostEdgeL : kHostEdge;
+        const int mid_max = T >= kHostLarge ? kHostMidL : kHostMid;
+        const int mid = T - 2 * edge;
+        const int nmid = min((mid + mid_max - 1) / mid_max, kMaxHostChunks - 2);
         n = nmid + 2;
         if (n > max_chunks) return 0;
-        starts[1] = kHostEdge;
+        starts[1] = edge;
         for (int c = 0; c < nmid; ++c) starts[2 + c] = starts[1 + c] + mid / nmid + (c < mid % nmid ? 1 : 0);
     } else if (T >= kHostChunkMin) {
         n = 2;   // two halves

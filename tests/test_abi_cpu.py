@@ -290,9 +290,12 @@ def test_host_chunk_plan(lib):
     assert plan(4096) == [0, 2048, 4096]
     assert plan(8191) == [0, 4095, 8191]
     assert plan(8192) == [0, 1024, 7168, 8192]
-    assert plan(16384) == [0, 1024, 8192, 15360, 16384]
+    assert plan(12287) == [0, 1024, 6144, 11263, 12287]
+    assert plan(12288) == [0, 2560, 9728, 12288]
+    assert plan(16384) == [0, 2560, 13824, 16384]
     decode_max = m.moe_decode_max_tokens()
-    for T in [4096, 4097, 6143, 8191, 8192, 8193, 10001, 16385, 30000, 100_000, 1 << 20, 2_000_000]:
+    for T in [4096, 4097, 6143, 8191, 8192, 8193, 10001, 12287, 12288, 16385, 30000, 100_000, 1 << 20,
+              2_000_000]:
         s = plan(T)
         sizes = np.diff(s)
         assert s[0] == 0 and s[-1] == T and len(s) - 1 <= 64
@@ -300,18 +303,19 @@ def test_host_chunk_plan(lib):
         if T < 8192:
             assert len(sizes) == 2 and abs(int(sizes[0]) - int(sizes[1])) <= 1
         else:
-            assert sizes[0] == 1024 and sizes[-1] == 1024
+            edge, mid_max = (1024, 7168) if T < 12288 else (2560, 11264)
+            assert sizes[0] == edge and sizes[-1] == edge
             mids = sizes[1:-1]
             assert mids.max() - mids.min() <= 1
             if len(sizes) < 64:
-                assert mids.max() <= 7168
+                assert mids.max() <= mid_max
     buf = (ctypes.c_int * 65)()
     lib.moe_host_chunk_plan.restype = ctypes.c_int
     assert lib.moe_host_chunk_plan(-1, buf, 64) == 0
     assert lib.moe_host_chunk_plan(16384, None, 64) == 0
-    assert lib.moe_host_chunk_plan(16384, buf, 3) == 0          # four chunks do not fit in three
-    assert lib.moe_host_chunk_plan(16384, buf, 4) == 4
-    assert list(buf[:5]) == [0, 1024, 8192, 15360, 16384]
+    assert lib.moe_host_chunk_plan(8192, buf, 2) == 0           # three chunks do not fit in two
+    assert lib.moe_host_chunk_plan(8192, buf, 3) == 3
+    assert list(buf[:4]) == [0, 1024, 7168, 8192]
 
 
 def test_header_serves_a_plain_c_program(lib, tmp_path):
@@ -333,7 +337,7 @@ def test_header_serves_a_plain_c_program(lib, tmp_path):
 #include "moe.h"
 int main(void) {
     int s[65];
-    if (moe_host_chunk_plan(16384, s, 64) != 4 || s[1] != 1024 || s[4] != 16384) return 1;
+    if (moe_host_chunk_plan(16384, s, 64) != 3 || s[1] != 2560 || s[3] != 16384) return 1;
     if (moe_slots_capacity(16, 8, 2) % 128 != 0) return 2;
     if (strcmp(moe_status_string(MOE_ERR_TIMEOUT), "device wait timed out") != 0) return 3;
     if (moe_forward(NULL, NULL, NULL, NULL, NULL, NULL, 8, 128, 256, 8, 9, 0) != MOE_ERR_INVALID_ARG) return 4;

@@ -409,11 +409,12 @@ def test_route_is_batch_invariant(moe, d, E, k):
     assert torch.equal(w_small, w_big[:1000])
 
 
-@pytest.mark.parametrize("T", [4096, 6143, 8192, 10001, 16384])
+@pytest.mark.parametrize("T", [4096, 6143, 8192, 10001, 12288, 16384, 30000])
 def test_chunked_host_entry_matches_device(moe, T):
     """Batches of 4096 tokens and more go through the host entry point in pipelined chunks (two
-    halves below 8192 tokens, else a 1024-token first and last chunk around middle ones of up to
-    7168); the result equals the one-call device path bit for bit, from pinned and pageable buffers."""
+    halves below 8192 tokens, then short first and last chunks around middle ones, by
+    moe_host_chunk_plan); the result equals the one-call device path bit for bit, from pinned and
+    pageable buffers."""
     inp = moe_inputs.make_inputs(T, 256, 512, 8, 2, "bf16", seed=T)
     dev = upload(inp)
     a = moe.moe_forward(*dev, 2).cpu()
